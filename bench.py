@@ -1,0 +1,398 @@
+"""Throughput of the SVDQuant W4A4 linear (+ AWQ W4A16 projection) on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+  K1  activation quantize + low-rank down-projection   X [4608 x 3072] bf16
+  K2  tcgen05 NVFP4 GEMM + low-rank up-projection      -> Y [4608 x 9216] bf16
+  K3  AWQ W4A16 projection                             [2 x 3072] -> [2 x 18432]
+(the attention-QKV-shaped layer of a 12B-class DiT at 1024x1024: 4096 image +
+512 text tokens, rank 32; and its adaLN modulation projection).
+
+value = algorithmic FLOPs of the step / step time (TFLOP/s, all ranks).
+Inputs rotate over buffer sets that together exceed twice the L2 cache, so no
+step reads what the previous one left in L2.  Multi-GPU runs are independent
+replicas (the layer needs no exchange between GPUs): weak scaling.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K, N, RANK = 4608, 3072, 9216, 32
+AM, AK, AN = 2, 3072, 18432
+WORKLOAD = ("attention-QKV SVDQ W4A4 linear 4608x3072->9216 rank 32 (NVFP4, group 16) "
+            "+ AWQ W4A16 adaLN projection 2x3072->18432 (INT4, group 64)")
+METRIC = "SVDQ W4A4 linear TFLOPS and % of B200 dense-FP4 peak; W4A16 GB/s vs HBM"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / dense bf16 ratio (9 / 2.25 PFLOP/s)
+
+W4A4_FLOPS = 2 * M * K * N                # 4-bit main branch
+LOWRANK_FLOPS = 2 * M * K * RANK + 2 * M * RANK * N
+AWQ_FLOPS = 2 * AM * AK * AN
+STEP_FLOPS = W4A4_FLOPS + LOWRANK_FLOPS + AWQ_FLOPS
+# Algorithmic bytes per launch (each byte the kernel must move once).
+K1_BYTES = (M * K * 2 + K * RANK * 2 + K * 4          # X, L1T, inv_lambda
+            + M * K // 2 + M * K // 16 + M * 64 * 2)  # codes, scales, U
+K2_BYTES = (M * K // 2 + M * K // 16 + M * 64 * 2     # activation codes, scales, U
+            + N * K // 2 + N * K // 16 + N * 64 * 2   # weight codes, scales, L2T
+            + N * 2 + M * N * 2)                      # bias, Y
+K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
+            + AM * AK * 2 + AK * 4 + AN * 2 + AM * AN * 2)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return PEAKS_FALLBACK, "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu):
+        self.gpu = gpu
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows]
+        smax = max(float(r[2]) for r in rows)
+        loaded = [float(r[1]) for r in rows if float(r[3]) > 250.0] or sm
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ------------------------------------------------------------------ our arm
+def setup(device, sets):
+    import torch
+
+    from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
+
+    lib.svdq_init(device.index)
+    c = synthetic.QKV
+    xb, wb, bb = c.make()
+    x = synthetic.bf16_bits_to_f32(xb)
+    amax = np.max(np.abs(x), axis=0).astype(np.float32)
+    packed = lib.svdq_pack_weights(wb, amax, RANK, seed=c.seed)
+    a = synthetic.AWQ
+    axb, awb, abb, asc = a.make()
+    apk = lib.awq_pack_weights(awb, asc)
+
+    def bf(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+
+    def t(arr):
+        return torch.from_numpy(np.ascontiguousarray(arr))
+
+    host = dict(X=bf(xb).pin_memory(), AX=bf(axb).pin_memory())
+    sz = lib.svdq_act_sizes(M, K)
+    S = []
+    for _ in range(sets):
+        S.append(dict(
+            X=bf(xb).to(device), inv_lambda=t(packed["inv_lambda"]).to(device), l1t=bf(packed["l1t"]).to(device),
+            l2t=bf(packed["l2t"]).to(device), w_codes=t(packed["w_codes"]).to(device),
+            w_scales=t(packed["w_scales"]).to(device), s_w=t(packed["s_w"]).to(device),
+            s_a=t(packed["s_a"]).to(device), bias=bf(bb).to(device),
+            codes=torch.empty((M, K // 2), dtype=torch.uint8, device=device),
+            scales=torch.empty(sz["scales"], dtype=torch.uint8, device=device),
+            U=torch.empty((M, 64), dtype=torch.bfloat16, device=device),
+            Y=torch.empty((M, N), dtype=torch.bfloat16, device=device),
+            AX=bf(axb).to(device), qweight=t(apk["qweight"]).to(device), ascales=bf(apk["scales"]).to(device),
+            azeros=bf(apk["zeros"]).to(device), inv_awq=t(apk["inv_awq"]).to(device), abias=bf(abb).to(device),
+            AY=torch.empty((AM, AN), dtype=torch.bfloat16, device=device)))
+    set_bytes = sum(v.numel() * v.element_size() for v in S[0].values())
+    return S, host, set_bytes
+
+
+def step(S, i, ev=None):
+    from bit_w4a4_diffusion_smooth_b200 import lib
+    s = S[i % len(S)]
+    if ev is not None:
+        ev[0].record()
+    lib.svdq_quantize_act(s["X"], s["inv_lambda"], s["l1t"], RANK, s["s_a"], s["s_w"], s["codes"], s["scales"],
+                          s["U"])
+    if ev is not None:
+        ev[1].record()
+    lib.svdq_linear_w4a4(s["codes"], s["scales"], s["U"], s["s_a"], s["w_codes"], s["w_scales"], s["l2t"], s["s_w"],
+                         s["bias"], M, N, K, RANK, 0, 0, s["Y"])
+    if ev is not None:
+        ev[2].record()
+    lib.awq_linear_w4a16(s["AX"], s["inv_awq"], s["qweight"], s["ascales"], s["azeros"], s["abias"], AN, s["AY"])
+    if ev is not None:
+        ev[3].record()
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from bit_w4a4_diffusion_smooth_b200 import lib
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    sets = 4
+    S, host, set_bytes = setup(device, sets)
+    while sets * set_bytes < 2 * l2:
+        sets += 1
+        S, host, set_bytes = setup(device, sets)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(S, i)
+    rc = lib.svdq_check_status()
+    if rc != lib.OK:
+        raise RuntimeError(f"device status after warm-up: {lib.status_name(rc)}")
+
+    # ---- device-timed region: K steps, per-kernel events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        step(S, i, evs[i])
+    t1.record()
+    barrier()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    k1 = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    k2 = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    k3 = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    rc = lib.svdq_check_status()
+    if rc != lib.OK:
+        raise RuntimeError(f"device status after timing: {lib.status_name(rc)}")
+
+    # ---- end to end through the public API, host buffers in and out
+    yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    ayh = torch.empty((AM, AN), dtype=torch.bfloat16, pin_memory=True)
+    e_steps = max(3, min(args.steps, 20))
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e_steps):
+        s = S[i % len(S)]
+        s["X"].copy_(host["X"], non_blocking=True)
+        s["AX"].copy_(host["AX"], non_blocking=True)
+        step(S, i)
+        yh.copy_(s["Y"], non_blocking=True)
+        ayh.copy_(s["AY"], non_blocking=True)
+    e1.record()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+
+    # ---- max over ranks
+    vals = torch.tensor([ms, k1, k2, k3, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms, k1, k2, k3, e2e_ms = vals.tolist()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    pk, how = peaks()
+    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    ms_step = ms / args.steps
+    k2_tflops = (W4A4_FLOPS + 2 * M * RANK * N) / (k2 * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(STEP_FLOPS * world / (ms_step * 1e-3) / 1e12, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3-scaled, fp32 accumulate); bf16 low-rank; int4 x bf16",
+        "data": "synthetic (seeded; outlier channels/rows as in the workload)",
+        "config": {"workload": WORKLOAD, "parallelism": f"replicas x{world}",
+                   "l2": f"{len(S)} rotating input/output sets, {len(S) * set_bytes / 1e6:.0f} MB > 2x L2",
+                   "flops_per_step": STEP_FLOPS},
+        "roofline": {"bound": "tensor", "kernel": "svdq_linear_w4a4 (K2)",
+                     "achieved": round(k2_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(k2_tflops / fp4_peak, 4), "traffic": None,
+                     "peak_source": f"{how} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16)"},
+        "kernels": {
+            "K1_quantize_act": {"us": round(k1 * 1e3, 2), "GB/s": round(K1_BYTES / (k1 * 1e-3) / 1e9, 1),
+                                "frac_hbm": round(K1_BYTES / (k1 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+            "K2_linear_w4a4": {"us": round(k2 * 1e3, 2), "TFLOP/s": round(k2_tflops, 1),
+                               "frac_fp4": round(k2_tflops / fp4_peak, 4)},
+            "K3_awq_w4a16": {"us": round(k3 * 1e3, 2), "GB/s": round(K3_BYTES / (k3 * 1e-3) / 1e9, 1),
+                             "frac_hbm": round(K3_BYTES / (k3 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+            "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how,
+        },
+        "e2e": {"value": round(STEP_FLOPS * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * K * 2 + AM * AK * 2, "d2h_bytes_per_step": M * N * 2 + AM * AN * 2},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(rows=64, reps=2)
+    print(json.dumps(line))
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(rows, x, packed, bb, awq_case):
+    """One bounded sample of the step on the CPU oracle; returns (flops, seconds)."""
+    from oracle import awq as oawq
+    from oracle import formats, svdquant
+
+    def bf(bits):
+        return formats.bf16_bits_to_float(np.asarray(bits, np.uint16))
+
+    l1 = bf(packed["l1t"]).T
+    l2 = bf(packed["l2t"])[:, :RANK].T
+    w_codes = np.empty((N, K), np.uint8)
+    w_codes[:, 0::2], w_codes[:, 1::2] = packed["w_codes"] & 15, packed["w_codes"] >> 4
+    m_i = np.arange(N)[:, None]
+    kb = np.arange(K // 16)[None, :]
+    w_sf = packed["w_scales"][((m_i // 128) * (K // 64) + kb // 4) * 512 + (m_i % 32) * 16 + ((m_i % 128) // 32) * 4
+                              + kb % 4]
+    axb, ainv, aq, as_, az, abias = awq_case
+    t = time.perf_counter()
+    codes, sf, u = svdquant.quantize_act(x[:rows], packed["inv_lambda"], l1, packed["s_a"][0], packed["s_w"][0])
+    svdquant.w4a4_linear(codes, sf, packed["s_a"][0], w_codes, w_sf, packed["s_w"][0], u, l2, bf(bb))
+    oawq.linear(axb, ainv, aq, as_, az, abias)
+    dt = time.perf_counter() - t
+    flops = rows / M * (W4A4_FLOPS + LOWRANK_FLOPS) + AWQ_FLOPS
+    return flops, dt
+
+
+def _oracle_inputs():
+    from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
+    from oracle import awq as oawq
+    from oracle import formats
+
+    c = synthetic.QKV
+    xb, wb, bb = c.make()
+    x = formats.bf16_bits_to_float(xb)
+    packed = lib.svdq_pack_weights(wb, np.max(np.abs(x), axis=0).astype(np.float32), RANK, seed=c.seed)
+    a = synthetic.AWQ
+    axb, awb, abb, asc = a.make()
+    ap = oawq.pack(formats.bf16_bits_to_float(awb), asc)
+    awq_case = (formats.bf16_bits_to_float(axb), ap["inv_a"], ap["q"], ap["s"], ap["z"], formats.bf16_bits_to_float(abb))
+    return x, packed, bb, awq_case
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(rows=64, reps=2):
+    x, packed, bb, awq_case = _oracle_inputs()
+    flops = secs = 0.0
+    for _ in range(reps):
+        f, s = oracle_sample(rows, x, packed, bb, awq_case)
+        flops += f
+        secs += s
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"{rows} of {M} rows of the QKV layer (quantize + two-branch float64 GEMM) + the full "
+                      f"2x3072->18432 AWQ projection, {reps} repetitions"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    x, packed, bb, awq_case = _oracle_inputs()
+    rows = 32
+    for _ in range(args.warmup):
+        oracle_sample(rows, x, packed, bb, awq_case)
+    flops = secs = 0.0
+    for _ in range(args.steps):
+        f, s = oracle_sample(rows, x, packed, bb, awq_case)
+        flops += f
+        secs += s
+    v = round(flops / secs / 1e12, 6)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (CPU oracle)",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "single host process"},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+                         "sample": f"{rows} of {M} rows of the QKV layer + the full AWQ projection per step"},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

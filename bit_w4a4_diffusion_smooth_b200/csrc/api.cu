@@ -1,0 +1,194 @@
+// C ABI plumbing: device selection and validation, per-thread error text,
+// the per-device status word written by bounded waits, and two probes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "device_common.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+
+namespace {
+thread_local std::string g_last_error;
+std::mutex g_state_mutex;
+std::vector<DeviceState> g_states;
+}  // namespace
+
+int fail(int status, const std::string &msg) {
+  g_last_error = msg;
+  return status;
+}
+int ok() {
+  g_last_error.clear();
+  return SVDQ_OK;
+}
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// One status word per device: the first error code a kernel's bounded wait
+// recorded since the last svdq_check_status.
+__device__ unsigned int g_status_word;
+
+DeviceState *current_device_state() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    fail(SVDQ_ERR_CUDA, "cudaGetDevice failed");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_state_mutex);
+  if (dev < 0 || dev >= static_cast<int>(g_states.size()) || !g_states[dev].initialized) {
+    fail(SVDQ_ERR_NOT_INITIALIZED, "svdq_init() was not called for device " + std::to_string(dev));
+    return nullptr;
+  }
+  return &g_states[dev];
+}
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      p = nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+}  // namespace
+
+int encode_tmap_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = fn(out, dtype, 2, const_cast<void *>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string(static_cast<int>(r)) + ")");
+  return SVDQ_OK;
+}
+
+namespace {
+__global__ void wait_timeout_kernel(unsigned long long limit_ns, unsigned int *status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    dev::mbar_init(&bar, 1);
+    dev::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: the wait has to run out.
+    if (!dev::mbar_wait(&bar, 0, limit_ns, nullptr)) dev::report(status, SVDQ_ERR_TIMEOUT);
+  }
+  __syncthreads();
+}
+
+__global__ void convert_probe_kernel(const float *in, int n, uint8_t *e2m1_out, uint8_t *e4m3_out) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) e4m3_out[i] = static_cast<uint8_t>(dev::cvt_e4m3(in[i]));
+  if (i < n / 2) e2m1_out[i] = static_cast<uint8_t>(dev::cvt_e2m1x2(in[2 * i], in[2 * i + 1]));
+}
+}  // namespace
+
+}  // namespace svdq
+
+using namespace svdq;
+
+extern "C" int svdq_version(void) { return 10000; }
+
+extern "C" const char *svdq_last_error_string(void) { return g_last_error.c_str(); }
+
+extern "C" const char *svdq_status_string(int status) {
+  switch (status) {
+    case SVDQ_OK: return "SVDQ_OK";
+    case SVDQ_ERR_INVALID_ARG: return "SVDQ_ERR_INVALID_ARG";
+    case SVDQ_ERR_SHAPE: return "SVDQ_ERR_SHAPE";
+    case SVDQ_ERR_ALIGNMENT: return "SVDQ_ERR_ALIGNMENT";
+    case SVDQ_ERR_UNSUPPORTED_DEVICE: return "SVDQ_ERR_UNSUPPORTED_DEVICE";
+    case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
+    case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT";
+    case SVDQ_ERR_NOT_INITIALIZED: return "SVDQ_ERR_NOT_INITIALIZED";
+    default: return "SVDQ_ERR_UNKNOWN";
+  }
+}
+
+extern "C" int svdq_init(int device) {
+  int count = 0;
+  cudaError_t e = cudaGetDeviceCount(&count);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SVDQ_ERR_CUDA, std::string("cudaGetDeviceCount: ") + cudaGetErrorString(e));
+  }
+  if (device < 0 || device >= count) return fail(SVDQ_ERR_INVALID_ARG, "svdq_init: no such device");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, device);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("cudaGetDeviceProperties: ") + cudaGetErrorString(e));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(SVDQ_ERR_UNSUPPORTED_DEVICE, "svdq_init: device " + std::to_string(device) + " (" + prop.name +
+                                                 ") has compute capability " + std::to_string(prop.major) + "." +
+                                                 std::to_string(prop.minor) + "; this library runs on 10.0 (B200) only");
+  e = cudaSetDevice(device);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("cudaSetDevice: ") + cudaGetErrorString(e));
+  void *status = nullptr;
+  e = cudaGetSymbolAddress(&status, g_status_word);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lock(g_state_mutex);
+  if (static_cast<int>(g_states.size()) < count) g_states.resize(count);
+  DeviceState &st = g_states[device];
+  st.sm_count = prop.multiProcessorCount;
+  st.max_smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+  st.status_word = static_cast<unsigned int *>(status);
+  st.initialized = true;
+  return ok();
+}
+
+extern "C" int svdq_check_status(svdq_stream_t stream) {
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("stream failed: ") + cudaGetErrorString(e));
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word));
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("reading status: ") + cudaGetErrorString(e));
+  unsigned int zero = 0;
+  e = cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("clearing status: ") + cudaGetErrorString(e));
+  if (word != 0) return fail(static_cast<int>(word), "a kernel's bounded wait ran out");
+  return ok();
+}
+
+extern "C" int svdq_debug_wait_timeout(uint64_t limit_ns, svdq_stream_t stream) {
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  if (limit_ns > 10ull * 1000 * 1000 * 1000) return fail(SVDQ_ERR_INVALID_ARG, "limit above 10 s");
+  wait_timeout_kernel<<<1, 32, 0, stream>>>(limit_ns, st->status_word);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return ok();
+}
+
+extern "C" int svdq_debug_convert(const float *in, int n, uint8_t *e2m1_out, uint8_t *e4m3_out,
+                                  svdq_stream_t stream) {
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  if (!in || !e2m1_out || !e4m3_out) return fail(SVDQ_ERR_INVALID_ARG, "svdq_debug_convert: null pointer");
+  if (n < 2 || n % 2) return fail(SVDQ_ERR_SHAPE, "svdq_debug_convert: n must be even and >= 2");
+  convert_probe_kernel<<<(n + 255) / 256, 256, 0, stream>>>(in, n, e2m1_out, e4m3_out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return ok();
+}

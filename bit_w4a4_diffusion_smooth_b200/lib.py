@@ -1,0 +1,248 @@
+"""ctypes binding of libsvdq_b200.so: the same entry points as include/svdq.h.
+
+Argument marshalling only: every computation happens inside the library (its
+CUDA kernels, or its host pack code).  Device arguments are torch CUDA
+tensors (torch supplies device memory and streams); host arguments are numpy
+arrays.  A missing library raises immediately: there is no fallback path.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq_b200.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_SHAPE = 2
+ERR_ALIGNMENT = 3
+ERR_UNSUPPORTED_DEVICE = 4
+ERR_CUDA = 5
+ERR_TIMEOUT = 6
+ERR_NOT_INITIALIZED = 7
+
+EPILOGUE_NONE = 0
+EPILOGUE_GELU_ERF = 1
+EPILOGUE_GELU_TANH = 2
+LR_STRIDE = 64
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.POINTER(ctypes.c_size_t)
+_SIGNATURES = {
+    "svdq_version": (_I, []),
+    "svdq_last_error_string": (ctypes.c_char_p, []),
+    "svdq_status_string": (ctypes.c_char_p, [_I]),
+    "svdq_init": (_I, [_I]),
+    "svdq_weight_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ, _SZ]),
+    "svdq_act_sizes": (_I, [_I, _I, _SZ, _SZ, _SZ]),
+    "svdq_pack_weights": (_I, [_P, _I, _I, _P, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "svdq_quantize_host": (_I, [_P, _I, _I, ctypes.c_float, _P, _P]),
+    "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
+    "svdq_linear_w4a4": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
+    "awq_pack_weights": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P]),
+    "awq_linear_w4a16": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P]),
+    "svdq_check_status": (_I, [_P]),
+    "svdq_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
+    "svdq_debug_convert": (_I, [_P, _I, _P, _P, _P]),
+}
+EXPORTS = tuple(_SIGNATURES)
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, name, status, text):
+        self.status = status
+        super().__init__(f"{name}: {status_name(status)}: {text}")
+
+
+def load():
+    """Loads the library once; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m bit_w4a4_diffusion_smooth_b200.build_lib`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_name(status):
+    return load().svdq_status_string(int(status)).decode()
+
+
+def _check(name, rc):
+    if rc != OK:
+        raise SvdqError(name, rc, load().svdq_last_error_string().decode())
+
+
+# ---------------------------------------------------------------- marshalling
+
+def _dptr(t, name, dtype=None, allow_none=False):
+    """Device pointer of a CUDA tensor (checked: on a GPU, contiguous rows)."""
+    if t is None:
+        if allow_none:
+            return None
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if t.dim() >= 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must have unit stride in its last dimension")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _hptr(a, dtype, name):
+    if not isinstance(a, np.ndarray) or a.dtype != dtype or not a.flags.c_contiguous:
+        raise ValueError(f"{name} must be a C-contiguous numpy array of {np.dtype(dtype).name}")
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+# ---------------------------------------------------------------- entry points
+
+def svdq_version():
+    return load().svdq_version()
+
+
+def svdq_init(device=0):
+    _check("svdq_init", load().svdq_init(int(device)))
+
+
+def svdq_weight_sizes(K, N, rank):
+    s = [ctypes.c_size_t() for _ in range(5)]
+    _check("svdq_weight_sizes", load().svdq_weight_sizes(K, N, rank, *[ctypes.byref(x) for x in s]))
+    return dict(zip(("inv_lambda", "l1t", "l2t", "w_codes", "w_scales"), (x.value for x in s)))
+
+
+def svdq_act_sizes(M, K):
+    s = [ctypes.c_size_t() for _ in range(3)]
+    _check("svdq_act_sizes", load().svdq_act_sizes(M, K, *[ctypes.byref(x) for x in s]))
+    return dict(zip(("codes", "scales", "u"), (x.value for x in s)))
+
+
+def svdq_pack_weights(W_bits, act_absmax, rank, num_threads=0, seed=0, want_residual=False):
+    """Host pack.  W_bits: uint16 [K, N] bf16 patterns; act_absmax: float32 [K].
+
+    Returns numpy arrays: inv_lambda [K] f32, l1t [rank, K] u16, l2t [N, 64] u16,
+    w_codes [N, K/2] u8, w_scales (tile order) u8, s_w, s_a (float32 scalars),
+    residual [K, N] f32 if asked.
+    """
+    K, N = W_bits.shape
+    sz = svdq_weight_sizes(K, N, rank)
+    out = dict(
+        inv_lambda=np.zeros(K, np.float32),
+        l1t=np.zeros((rank, K), np.uint16),
+        l2t=np.zeros((N, LR_STRIDE), np.uint16),
+        w_codes=np.zeros((N, K // 2), np.uint8),
+        w_scales=np.zeros(sz["w_scales"], np.uint8),
+        s_w=np.zeros(1, np.float32),
+        s_a=np.zeros(1, np.float32),
+    )
+    residual = np.zeros((K, N), np.float32) if want_residual else None
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    act_absmax = np.ascontiguousarray(act_absmax, dtype=np.float32)
+    rc = load().svdq_pack_weights(
+        _hptr(W_bits, np.uint16, "W"), K, N, _hptr(act_absmax, np.float32, "act_absmax"), rank,
+        num_threads, seed, _hptr(out["inv_lambda"], np.float32, "inv_lambda"),
+        _hptr(out["l1t"], np.uint16, "l1t") if rank else None, _hptr(out["l2t"], np.uint16, "l2t"),
+        _hptr(out["w_codes"], np.uint8, "w_codes"), _hptr(out["w_scales"], np.uint8, "w_scales"),
+        _hptr(out["s_w"], np.float32, "s_w"), _hptr(out["s_a"], np.float32, "s_a"),
+        _hptr(residual, np.float32, "residual") if want_residual else None)
+    _check("svdq_pack_weights", rc)
+    if want_residual:
+        out["residual"] = residual
+    return out
+
+
+def svdq_quantize_host(T, s_t):
+    """Host NVFP4 of float32 rows T [rows, K]: (codes [rows, K/2] u8, scales tile order u8)."""
+    T = np.ascontiguousarray(T, dtype=np.float32)
+    rows, K = T.shape
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros(svdq_act_sizes(rows, K)["scales"], np.uint8)
+    _check("svdq_quantize_host", load().svdq_quantize_host(
+        _hptr(T, np.float32, "T"), rows, K, ctypes.c_float(float(s_t)),
+        _hptr(codes, np.uint8, "codes"), _hptr(scales, np.uint8, "scales")))
+    return codes, scales
+
+
+def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, codes, scales, U, M=None, K=None, stream=None):
+    """Enqueues the activation kernel.  X: bf16 CUDA [M, ldx] (row stride ldx)."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    ldx = X.stride(0)
+    _check("svdq_quantize_act", load().svdq_quantize_act(
+        _dptr(X, "X", torch.bfloat16), M, K, ldx, _dptr(inv_lambda, "inv_lambda", torch.float32),
+        _dptr(l1t, "l1t", allow_none=rank == 0), rank, _dptr(s_a, "s_a", torch.float32),
+        _dptr(s_w, "s_w", torch.float32), _dptr(codes, "codes", torch.uint8),
+        _dptr(scales, "scales", torch.uint8), _dptr(U, "U"), _stream(stream)))
+
+
+def svdq_linear_w4a4(a_codes, a_scales, U, s_a, w_codes, w_scales, l2t, s_w, bias, M, N, K, rank,
+                     epilogue, gelu_col_begin, Y, stream=None):
+    """Enqueues the W4A4 GEMM.  Y: bf16 CUDA [M, ldy]."""
+    import torch
+    _check("svdq_linear_w4a4", load().svdq_linear_w4a4(
+        _dptr(a_codes, "a_codes", torch.uint8), _dptr(a_scales, "a_scales", torch.uint8),
+        _dptr(U, "U", allow_none=rank == 0), _dptr(s_a, "s_a", torch.float32),
+        _dptr(w_codes, "w_codes", torch.uint8), _dptr(w_scales, "w_scales", torch.uint8),
+        _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
+        _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue, gelu_col_begin,
+        _dptr(Y, "Y", torch.bfloat16), Y.stride(0), _stream(stream)))
+
+
+def awq_pack_weights(W_bits, awq_scale, group=64):
+    """Host AWQ pack: returns qweight (u32, fragment order), scales, zeros (u16 [N, K/g]), inv_awq."""
+    W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    awq_scale = np.ascontiguousarray(awq_scale, dtype=np.float32)
+    K, N = W_bits.shape
+    out = dict(qweight=np.zeros(N * K // 8, np.uint32), scales=np.zeros((N, K // group), np.uint16),
+               zeros=np.zeros((N, K // group), np.uint16), inv_awq=np.zeros(K, np.float32))
+    _check("awq_pack_weights", load().awq_pack_weights(
+        _hptr(W_bits, np.uint16, "W"), K, N, _hptr(awq_scale, np.float32, "awq_scale"), group,
+        _hptr(out["qweight"], np.uint32, "qweight"), _hptr(out["scales"], np.uint16, "scales"),
+        _hptr(out["zeros"], np.uint16, "zeros"), _hptr(out["inv_awq"], np.float32, "inv_awq")))
+    return out
+
+
+def awq_linear_w4a16(X, inv_awq, qweight, scales, zeros, bias, N, Y, group=64, M=None, K=None, stream=None):
+    """Enqueues the W4A16 GEMV.  X: bf16 CUDA [M, ldx]; Y: bf16 CUDA [M, ldy]."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    _check("awq_linear_w4a16", load().awq_linear_w4a16(
+        _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_awq, "inv_awq", allow_none=True),
+        _dptr(qweight, "qweight"), _dptr(scales, "scales"), _dptr(zeros, "zeros"), group,
+        _dptr(bias, "bias", allow_none=True), N, _dptr(Y, "Y", torch.bfloat16), Y.stride(0),
+        _stream(stream)))
+
+
+def svdq_check_status(stream=None):
+    """Synchronizes `stream`, returns the status code and clears it (no raise)."""
+    return load().svdq_check_status(_stream(stream))
+
+
+def svdq_debug_wait_timeout(limit_ns, stream=None):
+    _check("svdq_debug_wait_timeout", load().svdq_debug_wait_timeout(int(limit_ns), _stream(stream)))
+
+
+def svdq_debug_convert(x, e2m1_out, e4m3_out, stream=None):
+    import torch
+    _check("svdq_debug_convert", load().svdq_debug_convert(
+        _dptr(x, "x", torch.float32), x.numel(), _dptr(e2m1_out, "e2m1_out", torch.uint8),
+        _dptr(e4m3_out, "e4m3_out", torch.uint8), _stream(stream)))

@@ -1,0 +1,253 @@
+/*
+ * svdq.h - C ABI of the B200 (sm_100a) SVDQuant W4A4 linear layer and the AWQ
+ * W4A16 projection.
+ *
+ * The layer (web page "Nunchaku Diffusers 支持降低显存占用，但硬件仍决定适用范围",
+ * remio.ai, section "SVDQuant 将棘手数值移出 4 位路径"; and "Diffusers × Nunchaku
+ * 4-bit", donmalab.com, section "量化的核心挑戰：為什麼 4-bit 很難？"):
+ *
+ *     Y = (X^ . L1) . L2 + Q(X^) . Q(R) + b,   X^ = X . diag(lambda)^-1,
+ *     W' = diag(lambda) . W,  L1 . L2 = top-r SVD of W',  R = W' - L1 . L2
+ *
+ * with Q() the NVFP4 format (e2m1 elements, one e4m3 scale per 16 elements
+ * along K, one fp32 scale per tensor).  The same pages assign 4-bit-weight,
+ * 16-bit-activation AWQ layers to the modulation / adaptive-norm projections
+ * (remio.ai, section "Nunchaku Diffusers 支持改变了加载路径").
+ *
+ * Conventions for every call
+ *   - Return value: an svdq_status.  On failure svdq_last_error_string()
+ *     (per calling thread) describes the first problem found.  Argument checks
+ *     happen on the host before anything is enqueued; a failed check enqueues
+ *     nothing.
+ *   - Device calls take device pointers and are asynchronous on the caller's
+ *     CUDA stream (cudaStream_t passed as svdq_stream_t; NULL = legacy default
+ *     stream).  They never synchronize and never allocate device memory.
+ *   - Host calls (the *_pack_* and *_sizes calls) take host pointers and run
+ *     on the calling thread; they need no GPU.
+ *   - The caller owns every buffer.  Buffers must not overlap unless stated.
+ *   - bf16 tensors are passed as raw 16-bit patterns (uint16_t / void*).
+ *   - Every device pointer must be 16-byte aligned and every row stride a
+ *     multiple of 16 bytes (SVDQ_ERR_ALIGNMENT otherwise).
+ *   - Device waits inside the kernels are bounded (about one second); a wait
+ *     that runs out records SVDQ_ERR_TIMEOUT in a per-device status word that
+ *     svdq_check_status() returns.  Kernels never trap.
+ *
+ * Packed layouts (all produced by this library; documented so callers can
+ * move them around as opaque bytes):
+ *   codes   NVFP4 element codes, row-major [rows][K/2] bytes; element 2j of a
+ *           row is the low nibble of byte j, element 2j+1 the high nibble.
+ *           Code = sign bit 3 | e2m1 magnitude code 0..7.
+ *   scales  ue4m3 block scales in the tcgen05 scale-factor tile order:
+ *           rows padded to a multiple of 128, K/16 scales per row grouped in
+ *           atoms of 128 rows x 4 scales (512 bytes).  Scale (row m, block kb)
+ *           lives at byte
+ *             ((m/128)*(K/64) + kb/4)*512 + (m%32)*16 + ((m%128)/32)*4 + kb%4.
+ *           Scales of padding rows are 0.
+ *   L1T     low-rank down-projection, transposed: [rank][K] bf16.
+ *   U, L2T  low-rank activations [M][64] and up-projection [N][64] bf16, row
+ *           stride fixed at SVDQ_LR_STRIDE (64) elements; columns >= rank are 0.
+ *   AWQ     qweight: N*K/8 uint32 words in the fragment order of the W4A16
+ *           kernel's tensor-core tiles.  Columns go in blocks of 16 and K in
+ *           groups of 64; block b, group G owns words [(b*(K/64)+G)*128, +128):
+ *           32 lanes x 4 words, word j of lane 4g+t covering k = 64G+16j+kq.
+ *           Its nibbles (bits 4i..4i+3) hold, for column c of the block:
+ *             i = 0 / 4: c = g,   kq = 2t / 2t+1;   i = 1 / 5: c = g+8, kq = 2t / 2t+1
+ *             i = 2 / 6: c = g,   kq = 2t+8/2t+9;   i = 3 / 7: c = g+8, kq = 2t+8/2t+9
+ *           scales, zeros [N][K/group] bf16 (zeros are integers 0..15).
+ */
+#ifndef SVDQ_B200_H
+#define SVDQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *svdq_stream_t; /* identical to cudaStream_t */
+
+enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size */
+  SVDQ_ERR_SHAPE = 2,             /* a shape rule below is violated */
+  SVDQ_ERR_ALIGNMENT = 3,         /* pointer or stride not 16-byte aligned */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 4,/* not a compute capability 10.0 GPU */
+  SVDQ_ERR_CUDA = 5,              /* a CUDA runtime / driver call failed */
+  SVDQ_ERR_TIMEOUT = 6,           /* a bounded device wait ran out */
+  SVDQ_ERR_NOT_INITIALIZED = 7    /* svdq_init() was not called for the device */
+};
+
+enum svdq_epilogue {
+  SVDQ_EPILOGUE_NONE = 0,
+  SVDQ_EPILOGUE_GELU_ERF = 1,     /* 0.5 y (1 + erf(y / sqrt 2)) */
+  SVDQ_EPILOGUE_GELU_TANH = 2     /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+};
+
+#define SVDQ_LR_STRIDE 64  /* row stride (elements) of U and L2T; max rank */
+#define SVDQ_GROUP 16      /* NVFP4 block size along K */
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int svdq_version(void);
+
+/* Text of the last error raised on the calling thread ("" if none). */
+const char *svdq_last_error_string(void);
+
+/* Name of a status code. */
+const char *svdq_status_string(int status);
+
+/*
+ * Select and validate a GPU.  The pages require that an unsupported
+ * GPU / kernel combination is reported as an error instead of running
+ * silently (remio.ai, section "硬件支持划分了最快路径与最广泛路径"); here that
+ * means anything but compute capability 10.0 (sm_100a: B200) returns
+ * SVDQ_ERR_UNSUPPORTED_DEVICE.  Makes `device` current on the calling thread
+ * and caches its properties.  Must precede the device calls below for that
+ * device.  Idempotent.
+ */
+int svdq_init(int device);
+
+/*
+ * Byte sizes of the packed buffers of one SVDQ layer (host, no GPU).
+ * Rules: K % 64 == 0, N % 8 == 0, 0 <= rank <= 64, rank % 16 == 0.
+ *   inv_lambda [K] f32, L1T [rank][K] bf16, L2T [N][64] bf16,
+ *   w_codes [N][K/2] u8, w_scales (tile order, rows padded to 128) u8.
+ */
+int svdq_weight_sizes(int K, int N, int rank, size_t *inv_lambda_bytes, size_t *l1t_bytes,
+                      size_t *l2t_bytes, size_t *w_codes_bytes, size_t *w_scales_bytes);
+
+/* Byte sizes of the activation-side buffers: codes [M][K/2], scales (tile
+ * order, rows padded to 128), U [M][64] bf16.  Rules: M >= 1, K % 64 == 0. */
+int svdq_act_sizes(int M, int K, size_t *codes_bytes, size_t *scales_bytes, size_t *u_bytes);
+
+/*
+ * Offline quantization of one layer on the host (the pages' quantize step:
+ * "diffuse-compressor" turns the weights into 4 bits and produces the
+ * low-rank branch; donmalab.com, section "自行量化模型的流程").
+ *
+ *   W          [K][N] bf16, host.  Input features by output features.
+ *   act_absmax [K] f32, host: per-input-channel max |X| over calibration
+ *              data (the pages: calibration samples decide the scales and
+ *              the low-rank correction, remio.ai, section
+ *              "基准测试展示了性能提升，但并非普遍结论").
+ *   rank       0..64, multiple of 16.
+ *   num_threads host threads for the SVD (<= 0: all cores).
+ * Outputs (host buffers of the sizes from svdq_weight_sizes):
+ *   inv_lambda [K]  f32(1 / lambda_j), lambda_j = sqrt(absmaxX_j / absmaxW_j)
+ *                   (1 when either is 0);
+ *   l1t        [rank][K] bf16 = (U_r Sigma_r)^T of W' = W / inv_lambda;
+ *   l2t        [N][64] bf16 = V_r (the rows of V_r^T, transposed), zero-padded;
+ *   w_codes, w_scales: NVFP4 of R = W' - L1 L2 (f32-rounded), blocks along K;
+ *   s_w        fp32 tensor scale of R: f32(max|R|) / 2688 (1 if R == 0);
+ *   s_a        static activation tensor scale:
+ *              max_j f32(absmaxX_j * inv_lambda_j) / 2688.
+ *   residual   optional [K][N] f32 copy of f32(R) (NULL to skip).
+ * The top-r SVD is a seeded randomized subspace iteration (deterministic for
+ * a given seed and thread count).
+ */
+int svdq_pack_weights(const uint16_t *W, int K, int N, const float *act_absmax, int rank,
+                      int num_threads, uint64_t seed, float *inv_lambda, uint16_t *l1t,
+                      uint16_t *l2t, uint8_t *w_codes, uint8_t *w_scales, float *s_w, float *s_a,
+                      float *residual);
+
+/*
+ * NVFP4 quantization of a host float32 matrix T [rows][K] (host, no GPU),
+ * blocks of 16 along K under tensor scale s_t, into the packed codes and
+ * tile-order scales above.  Used by the pack; exposed for tooling and tests.
+ */
+int svdq_quantize_host(const float *T, int rows, int K, float s_t, uint8_t *codes,
+                       uint8_t *scales);
+
+/*
+ * Activation side of one SVDQ layer (the first fused kernel on the pages:
+ * the low-rank down-projection combined with the quantization of the input,
+ * remio.ai, section "SVDQuant 将棘手数值移出 4 位路径").  One pass over X:
+ *   x^      = f32(x * inv_lambda[k])
+ *   per block of 16 along K:  sb = e4m3_rne_sat(f32(amax|x^|) / f32(6 s_a)),
+ *                             q  = e2m1_rne_sat(x^ * f32(1 / f32(sb * s_a)))
+ *   U[m][j] = bf16( sum_k bf16(x^[m][k]) * L1T[j][k] / f32(s_a * s_w) )
+ * Args: X [M][ldx] bf16 (device), ldx >= K; inv_lambda [K] f32; l1t
+ * [rank][K] bf16 (ignored when rank == 0); s_a, s_w device scalars (f32);
+ * outputs codes, scales, U as laid out above (U columns rank..63 are zeroed).
+ * Rules: K % 64 == 0, ldx % 8 == 0, 0 <= rank <= 64, rank % 16 == 0, M >= 1.
+ */
+int svdq_quantize_act(const void *X, int M, int K, int ldx, const float *inv_lambda,
+                      const void *l1t, int rank, const float *s_a, const float *s_w,
+                      uint8_t *codes, uint8_t *scales, void *U, svdq_stream_t stream);
+
+/*
+ * The W4A4 GEMM with the low-rank up-projection fused in (the second fused
+ * kernel on the pages, remio.ai, section "SVDQuant 将棘手数值移出 4 位路径"):
+ *   acc = U . L2T^T + sum_k qa sa qw sw     (tcgen05 block-scaled FP4, fp32)
+ *   Y   = bf16( epilogue( f32(s_a s_w) * acc + bias ) )
+ * epilogue: svdq_epilogue; GELU applies to output columns >= gelu_col_begin
+ * only (a fused QKV + MLP-in projection activates just its MLP part).
+ * Args: activation codes/scales/U from svdq_quantize_act; weight codes,
+ * scales, L2T and scalars from svdq_pack_weights (uploaded); bias [N] bf16 or
+ * NULL; Y [M][ldy] bf16, ldy >= N.
+ * Rules: K % 64 == 0, N % 8 == 0, ldy % 8 == 0, 0 <= rank <= 64,
+ * rank % 16 == 0, M >= 1, 0 <= gelu_col_begin <= N.
+ */
+int svdq_linear_w4a4(const uint8_t *a_codes, const uint8_t *a_scales, const void *U,
+                     const float *s_a, const uint8_t *w_codes, const uint8_t *w_scales,
+                     const void *l2t, const float *s_w, const void *bias, int M, int N, int K,
+                     int rank, int epilogue, int gelu_col_begin, void *Y, int ldy,
+                     svdq_stream_t stream);
+
+/*
+ * Offline AWQ quantization on the host (asymmetric INT4 per group along K):
+ *   W_a = diag(awq_scale) W;  per group and output column:
+ *   lo = min(0, min W_a), hi = max(0, max W_a), s = bf16((hi - lo) / 15),
+ *   z = clamp(rne(-lo / s), 0, 15), q = clamp(rne(W_a / s) + z, 0, 15);
+ *   an all-zero group takes s = 1, z = 0.  inv_awq[k] = f32(1 / awq_scale[k]).
+ * Args: W [K][N] bf16 host; awq_scale [K] f32 (> 0); group 64 (K % group == 0);
+ * N % 16 == 0; outputs qweight (N*K/8 u32, fragment order above),
+ * scales/zeros [N][K/group] bf16, inv_awq [K].
+ */
+int awq_pack_weights(const uint16_t *W, int K, int N, const float *awq_scale, int group,
+                     uint32_t *qweight, uint16_t *scales, uint16_t *zeros, float *inv_awq);
+
+/*
+ * AWQ W4A16 projection for small row counts (the modulation / adaLN layers):
+ *   Y[m][n] = bf16( sum_g s[n][g] * sum_{k in g} f32(x[m][k] inv_awq[k]) (q - z[n][g]) + bias[n] )
+ * in fp32.  X [M][ldx] bf16; inv_awq [K] f32 or NULL (= 1); bias [N] or NULL.
+ * The products run on tensor cores with X^ split into bf16 hi + lo parts
+ * (relative error of the split ~2^-17).
+ * Rules: 1 <= M <= 16, group == 64, K % 64 == 0, N % 16 == 0, ldx >= K,
+ * ldy >= N, ldx % 8 == 0, ldy % 8 == 0.
+ */
+int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq,
+                     const uint32_t *qweight, const void *scales, const void *zeros, int group,
+                     const void *bias, int N, void *Y, int ldy, svdq_stream_t stream);
+
+/*
+ * Waits for `stream`, then returns and clears the device status word of the
+ * current device: SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel's bounded wait ran
+ * out since the last check (SVDQ_ERR_CUDA if the stream itself failed).
+ */
+int svdq_check_status(svdq_stream_t stream);
+
+/*
+ * Self-test of the bounded wait used by every kernel: launches one block that
+ * waits on a shared-memory barrier nothing will ever complete, with a limit
+ * of `limit_ns` nanoseconds.  The status word then holds SVDQ_ERR_TIMEOUT.
+ * Exists so that the timeout path can be tested without a fault.
+ */
+int svdq_debug_wait_timeout(uint64_t limit_ns, svdq_stream_t stream);
+
+/*
+ * Conversion probe (device buffers, n even):
+ *   e2m1_out[i] = e2m1(in[2i+1]) << 4 | e2m1(in[2i])   for i < n/2
+ *   e4m3_out[i] = e4m3(in[i])                           for i < n
+ * both round-to-nearest-even with saturation, through the same conversion
+ * instructions the kernels use.  Lets the tests check those conversions
+ * against the format definitions.
+ */
+int svdq_debug_convert(const float *in, int n, uint8_t *e2m1_out, uint8_t *e4m3_out,
+                       svdq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_B200_H */

@@ -1,0 +1,86 @@
+"""The C-ABI library on the CPU: it loads, exports every declared entry point,
+and its host-side argument checks and size queries behave (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_w4a4_diffusion_smooth_b200 import lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    so = lib.load()
+    declared = _declared_functions()
+    assert len(declared) >= 15
+    for name in declared:
+        assert hasattr(so, name), name
+    assert set(lib.EXPORTS) == set(declared)
+    assert lib.svdq_version() == 10000
+
+
+def test_status_strings():
+    assert lib.status_name(0) == "SVDQ_OK"
+    assert lib.status_name(lib.ERR_TIMEOUT) == "SVDQ_ERR_TIMEOUT"
+    assert lib.status_name(99) == "SVDQ_ERR_UNKNOWN"
+
+
+def test_sizes():
+    s = lib.svdq_weight_sizes(3072, 9216, 32)
+    assert s["w_codes"] == 9216 * 1536
+    assert s["w_scales"] == 9216 * 192
+    assert s["l1t"] == 32 * 3072 * 2 and s["l2t"] == 9216 * 64 * 2
+    a = lib.svdq_act_sizes(200, 256)
+    assert a["codes"] == 200 * 128 and a["scales"] == 256 * 16 and a["u"] == 200 * 128
+    with pytest.raises(lib.SvdqError) as e:
+        lib.svdq_weight_sizes(100, 256, 16)
+    assert e.value.status == lib.ERR_SHAPE
+    with pytest.raises(lib.SvdqError) as e:
+        lib.svdq_weight_sizes(256, 256, 24)
+    assert e.value.status == lib.ERR_SHAPE
+
+
+def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
+    so = lib.load()
+    null = ctypes.c_void_p(0)
+    rc = so.svdq_quantize_act(null, 64, 256, 256, null, null, 16, null, null, null, null, null, null)
+    assert rc == lib.ERR_INVALID_ARG
+    p = ctypes.c_void_p(16)  # never dereferenced: the shape check fails first
+    rc = so.svdq_linear_w4a4(p, p, p, p, p, p, p, p, None, 64, 256, 100, 16, 0, 0, p, 256, None)
+    assert rc == lib.ERR_SHAPE
+    assert b"K % 64" in so.svdq_last_error_string()
+    rc = so.svdq_linear_w4a4(p, p, p, p, p, p, p, p, None, 64, 256, 256, 16, 7, 0, p, 256, None)
+    assert rc == lib.ERR_INVALID_ARG
+    rc = so.awq_linear_w4a16(p, 17, 256, 256, None, p, p, p, 64, None, 256, p, 256, None)
+    assert rc == lib.ERR_SHAPE
+    odd = ctypes.c_void_p(24)
+    rc = so.svdq_linear_w4a4(odd, p, p, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None)
+    assert rc == lib.ERR_ALIGNMENT
+
+
+def test_init_without_a_b200_is_an_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(lib.SvdqError) as e:
+        lib.svdq_init(0)
+    assert e.value.status in (lib.ERR_CUDA, lib.ERR_INVALID_ARG)
+
+
+def test_pack_argument_checks():
+    w = np.zeros((100, 64), np.uint16)
+    with pytest.raises(lib.SvdqError):
+        lib.svdq_pack_weights(w, np.ones(100, np.float32), 16)
+    with pytest.raises(lib.SvdqError):
+        lib.awq_pack_weights(np.zeros((64, 24), np.uint16), np.ones(64, np.float32))
+    with pytest.raises(lib.SvdqError):
+        lib.awq_pack_weights(np.zeros((64, 32), np.uint16), np.zeros(64, np.float32))

@@ -1,0 +1,63 @@
+"""GPU parity of the AWQ W4A16 projection (K3) against the oracle, through the
+C ABI.  The weights are the oracle's AWQ pack, put in the library's fragment
+layout by the test-side writer; bar: max |got - want| / RMS of the oracle's
+row <= 1e-2 (the kernel reaches ~1e-5 before the bf16 output rounding)."""
+import numpy as np
+import pytest
+
+from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
+from oracle import awq as oawq
+from oracle import formats
+from tests import gpu_util as G
+from tests import layouts as L
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _init():
+    G.init()
+
+
+def _run(m, k, n, seed, with_bias=True, use_inv=True):
+    xb, _ = synthetic.activation(m, k, seed)
+    wb, _ = synthetic.weight(k, n, seed, 0.02)
+    a = synthetic.awq_scales(k, seed) if use_inv else np.ones(k, np.float32)
+    bb = synthetic.bias(n, seed)
+    p = oawq.pack(formats.bf16_bits_to_float(wb), a)
+    Y = G.poisoned_bf16(m, n)
+    lib.awq_linear_w4a16(G.bf16_dev(xb), G.dev(p["inv_a"]) if use_inv else None, G.dev(L.awq_pack(p["q"])),
+                         G.bf16_dev(L.bf16_bits(p["s"].T)), G.bf16_dev(L.bf16_bits(p["z"].T)),
+                         G.bf16_dev(bb) if with_bias else None, n, Y)
+    G.check_ok()
+    x = formats.bf16_bits_to_float(xb)
+    want = oawq.linear(x, p["inv_a"], p["q"], p["s"], p["z"], formats.bf16_bits_to_float(bb) if with_bias else None)
+    return G.row_rms_error(G.bf16_host(Y), want)
+
+
+@pytest.mark.parametrize("m,k,n", [(1, 64, 16), (2, 192, 48), (5, 1024, 320), (8, 512, 64), (9, 256, 96),
+                                   (16, 3072, 512), (3, 4096, 112)])
+def test_awq_parity(m, k, n):
+    assert _run(m, k, n, seed=m + k + n) <= 1e-2
+
+
+def test_awq_without_bias_and_scales():
+    assert _run(4, 256, 64, 21, with_bias=False, use_inv=False) <= 1e-2
+
+
+def test_awq_full_size_adaln():
+    """The modulation workload: 2 x 3072 -> 18432 (6 x 3072 adaLN outputs)."""
+    c = synthetic.AWQ
+    assert _run(c.m, c.k, c.n, c.seed) <= 1e-2
+
+
+def test_awq_layer_from_host_pack():
+    """The user-facing layer (library host pack + K3) against the oracle."""
+    from bit_w4a4_diffusion_smooth_b200.layer import AWQLinear
+    xb, wb, bb, a = synthetic.AwqCase("awq small", 2, 512, 256, seed=5).make()
+    layer = AWQLinear.from_weight(wb, a, bb)
+    y = G.bf16_host(layer(G.bf16_dev(xb)))
+    p = oawq.pack(formats.bf16_bits_to_float(wb), a)
+    want = oawq.linear(formats.bf16_bits_to_float(xb), p["inv_a"], p["q"], p["s"], p["z"],
+                       formats.bf16_bits_to_float(bb))
+    assert G.row_rms_error(y, want) <= 1e-2

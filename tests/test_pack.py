@@ -1,0 +1,116 @@
+"""Host pack of the library (C++) against the oracle (CPU only).
+
+Bit-exact where the method fixes the result: inverse smoothing factors,
+activation scale, and - stage-wise - the NVFP4 codes and scales of the
+pack's own residual, and every AWQ code, scale and zero point.  The top-r SVD
+is checked by Eckart-Young against the oracle's exact spectrum (singular
+vectors are not unique, so the factors themselves are not compared).
+"""
+import numpy as np
+import pytest
+
+from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
+from oracle import awq as oawq
+from oracle import formats, nvfp4, svdquant
+from tests import layouts
+
+F32 = np.float32
+
+
+def _case(m, k, n, seed, x_out=4, x_fac=30.0, w_out=2, w_fac=8.0):
+    xb, _ = synthetic.activation(m, k, seed, x_out, x_fac)
+    wb, _ = synthetic.weight(k, n, seed, 0.02, w_out, w_fac)
+    x = formats.bf16_bits_to_float(xb)
+    amax = np.max(np.abs(x), axis=0).astype(F32)
+    return xb, wb, x, amax
+
+
+@pytest.mark.parametrize("k,n,rank", [(256, 256, 16), (128, 64, 0), (192, 128, 32)])
+def test_pack_matches_oracle(k, n, rank):
+    xb, wb, x, amax = _case(64, k, n, seed=k + n + rank)
+    p = lib.svdq_pack_weights(wb, amax, rank, want_residual=True)
+    w = formats.bf16_bits_to_float(wb)
+    o = svdquant.pack(w, amax, rank)
+    np.testing.assert_array_equal(p["inv_lambda"], o["inv_lambda"])
+    assert p["s_a"][0] == o["s_a"]
+    # stage-wise: the oracle quantizes the pack's own residual
+    r32 = p["residual"]
+    s_w = nvfp4.tensor_scale(np.max(np.abs(r32)))
+    assert p["s_w"][0] == s_w
+    codes, sf = nvfp4.quantize_blocks(r32.T, s_w)
+    np.testing.assert_array_equal(layouts.unpack_codes(p["w_codes"], k), codes)
+    np.testing.assert_array_equal(layouts.untile_scales(p["w_scales"], n, k), sf)
+    assert (layouts.padding_scales(p["w_scales"], n, k) == 0).all()
+    # the residual is W' - L1 L2 with the pack's bf16 factors
+    l1 = layouts.bf16_bits_to_f64(p["l1t"]).T
+    l2 = layouts.bf16_bits_to_f64(p["l2t"])[:, :rank].T
+    assert (p["l2t"][:, rank:] == 0).all()
+    np.testing.assert_allclose(r32, (o["w_prime"] - l1 @ l2).astype(F32), rtol=0, atol=1e-6)
+    # L1 L2 itself is not compared with the oracle's: with a nearly flat tail
+    # of the spectrum the top-r subspace is not unique (see the Eckart-Young
+    # test for what is).
+
+
+@pytest.mark.parametrize("k,n,rank,tol", [(256, 256, 16, 1e-3), (512, 1536, 32, 1e-3)])
+def test_pack_svd_eckart_young(k, n, rank, tol):
+    xb, wb, x, amax = _case(64, k, n, seed=3, x_out=max(1, k // 64), x_fac=50.0, w_out=max(1, k // 200))
+    w = formats.bf16_bits_to_float(wb)
+    p = lib.svdq_pack_weights(wb, amax, rank, want_residual=True)
+    wp = svdquant.smoothed_weight(w, p["inv_lambda"])
+    sig = np.linalg.svd(wp, compute_uv=False)
+    optimal = np.sum(sig[rank:] ** 2)
+    # the pack's factors before bf16 rounding would reach the optimum; with
+    # bf16 factors the residual grows by at most the rounding of L1 L2
+    got = np.sum(p["residual"].astype(np.float64) ** 2)
+    assert got >= optimal * (1 - 1e-9)
+    assert got <= optimal * (1 + tol) + np.sum(sig[:rank] ** 2) * 2 ** -14, (got / optimal - 1)
+
+
+def test_pack_is_deterministic():
+    xb, wb, x, amax = _case(32, 128, 64, seed=5)
+    a = lib.svdq_pack_weights(wb, amax, 16, num_threads=3, seed=7)
+    b = lib.svdq_pack_weights(wb, amax, 16, num_threads=3, seed=7)
+    for key in a:
+        np.testing.assert_array_equal(a[key], b[key])
+
+
+def test_host_quantizer_matches_oracle_bit_exactly():
+    rng = np.random.default_rng(0)
+    t = (rng.standard_normal((70, 320)) * np.exp2(rng.integers(-8, 8, (70, 1)))).astype(F32)
+    # plant exact ties of the e2m1 grid and of the e4m3 scale
+    t[3, :16] = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -5, -0.25, 0, -0.0, 4, 3, 2, 1], F32)
+    t[5, 16:32] = 0.0
+    s_t = nvfp4.tensor_scale(np.max(np.abs(t)))
+    codes, sf = lib.svdq_quantize_host(t, s_t)
+    oc, osf = nvfp4.quantize_blocks(t, s_t)
+    np.testing.assert_array_equal(layouts.unpack_codes(codes, 320), oc)
+    np.testing.assert_array_equal(layouts.untile_scales(sf, 70, 320), osf)
+    oc1, osf1 = nvfp4.quantize_blocks(t[3:4], F32(1.0))
+    c1, sf1 = lib.svdq_quantize_host(t[3:4].copy(), 1.0)
+    np.testing.assert_array_equal(layouts.unpack_codes(c1, 320), oc1)
+
+
+@pytest.mark.parametrize("k,n", [(64, 16), (192, 48), (3072, 64)])
+def test_awq_pack_matches_oracle(k, n):
+    wb, _ = synthetic.weight(k, n, 11, 0.02)
+    a = synthetic.awq_scales(k, 11)
+    p = lib.awq_pack_weights(wb, a)
+    o = oawq.pack(formats.bf16_bits_to_float(wb), a)
+    np.testing.assert_array_equal(layouts.awq_unpack(p["qweight"], k, n), o["q"])
+    np.testing.assert_array_equal(layouts.bf16_bits_to_f64(p["scales"]).T, o["s"])
+    np.testing.assert_array_equal(layouts.bf16_bits_to_f64(p["zeros"]).T, o["z"])
+    np.testing.assert_array_equal(p["inv_awq"], o["inv_a"])
+
+
+def test_awq_layout_reader_round_trip():
+    """The test-side reader inverts a layout written by hand from the header text."""
+    k, n = 64, 16
+    q = np.random.default_rng(1).integers(0, 16, (k, n)).astype(np.uint8)
+    words = np.zeros(n * k // 8, np.uint32)
+    for kk in range(k):
+        for c in range(n):
+            j, kq = (kk % 64) // 16, kk % 16
+            lane = (c % 8) * 4 + (kq % 8) // 2
+            i = (c // 8) + 2 * (kq // 8) + 4 * (kq % 2)
+            words[((c // 16) * 1 + kk // 64) * 128 + lane * 4 + j] |= np.uint32(q[kk, c]) << np.uint32(4 * i)
+    np.testing.assert_array_equal(layouts.awq_unpack(words, k, n), q)

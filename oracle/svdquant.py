@@ -24,6 +24,9 @@ Readings where the pages are silent (each also in the design notes):
   * The activation tensor scale is static: calibrated from the per-channel
     absolute maxima of X (the pages: calibration samples decide the scales,
     section "基准测试展示了性能提升，但并非普遍结论").
+  * The low-rank branch is a 16-bit branch ("一个小型 16 位低秩分支"): its input
+    is the smoothed activation rounded to bf16 (RNE of the float32 X^), its
+    factors are bf16; products and sums are exact here (float64).
   * The low-rank up-projection enters the 4-bit GEMM's accumulator divided by
     alpha = f32(s_A * s_W), the epilogue multiplies by alpha (the fusion of the
     up-projection into the 4-bit GEMM, section "SVDQuant 将棘手数值移出 4 位路径").
@@ -112,15 +115,15 @@ def quantize_act(x, inv_lambda, l1, s_a, s_w):
     down-projection).
 
     x: float64 [M, K] holding bf16 values.  Returns NVFP4 codes [M, K] and
-    scales [M, K/16] of X^ = f32(x * inv_lambda), and U = (X^ . L1) / alpha in
-    float64 with X^ unrounded.
+    scales [M, K/16] of X^ = f32(x * inv_lambda), and U = (bf16(X^) . L1) /
+    alpha in float64 (the 16-bit branch takes X^ in bf16).
     """
     x = np.asarray(x, dtype=np.float64)
     inv = np.asarray(inv_lambda, dtype=F32)
     x_hat32 = (x.astype(F32) * inv[None, :]).astype(F32)
     codes, sf = nvfp4.quantize_blocks(x_hat32, s_a)
-    x_hat = x * inv.astype(np.float64)[None, :]              # exact in float64
-    u = (x_hat @ np.asarray(l1, dtype=np.float64)) / np.float64(alpha(s_a, s_w))
+    x_hat16 = formats.bf16_round(x_hat32.astype(np.float64))
+    u = (x_hat16 @ np.asarray(l1, dtype=np.float64)) / np.float64(alpha(s_a, s_w))
     return codes, sf, u
 
 

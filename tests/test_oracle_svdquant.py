@@ -82,10 +82,11 @@ def test_exact_rank_r_weight_leaves_only_low_rank_branch():
     p = svdquant.pack(w, np.max(np.abs(x), axis=0).astype(F32), r, round_bf16=False)
     assert np.abs(p["residual"]).max() <= 1e-12 * np.abs(p["w_prime"]).max()
     y = svdquant.forward(x, p)
-    x_hat = x * p["inv_lambda"].astype(np.float64)[None, :]
-    low = (x_hat @ p["l1"]) @ p["l2"]
+    x_hat32 = (x.astype(F32) * p["inv_lambda"][None, :]).astype(F32).astype(np.float64)
+    low = (formats.bf16_round(x_hat32) @ p["l1"]) @ p["l2"]
     np.testing.assert_allclose(y, low, rtol=0, atol=1e-9 * np.abs(low).max())
-    np.testing.assert_allclose(y, x @ w, rtol=0, atol=1e-9 * np.abs(low).max())
+    # the only departure from X W is the bf16 input of the 16-bit branch
+    np.testing.assert_allclose(y, x @ w, rtol=0, atol=2.0 ** -7 * np.abs(low).max())
 
 
 def _brute_gemm(a_codes, a_sf, s_a, w_codes, w_sf, s_w, bias):
@@ -168,7 +169,21 @@ def test_quantize_act_on_grid_activation():
     codes, sf, u = svdquant.quantize_act(x, inv, l1, s_a, s_w)
     assert (sf == 0x38).all()
     np.testing.assert_array_equal(formats.e2m1_decode(codes), np.where(g == 0, 0, g))
-    np.testing.assert_allclose(u, (g @ l1) / 0.5, rtol=1e-13)
+    np.testing.assert_allclose(u, (g @ l1) / 0.5, rtol=1e-13)   # G is exact in bf16
+
+
+def test_low_rank_input_is_bf16():
+    """The 16-bit branch sees X^ rounded to bf16: a value that bf16 cannot hold
+    moves U by exactly its rounding error times L1."""
+    k = 16
+    x = np.zeros((1, k))
+    x[0, 0] = 1.0 + 2.0 ** -7           # exact in bf16
+    x[0, 1] = 1.0
+    inv = np.ones(k, F32)
+    inv[1] = F32(1.0 + 2.0 ** -9)         # X^[1] = 1 + 2^-9 rounds to 1 in bf16 (tie -> even)
+    l1 = np.eye(k)[:, :2]
+    _, _, u = svdquant.quantize_act(x, inv, l1, F32(1.0), F32(1.0))
+    assert u[0, 0] == 1.0 + 2.0 ** -7 and u[0, 1] == 1.0
 
 
 def test_gelu_forms():

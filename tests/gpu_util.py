@@ -48,6 +48,30 @@ def row_rms_error(got, want):
     return float(np.max(np.abs(got - want) / rms[:, None]))
 
 
+def bf16_ulp(v):
+    """Spacing of bf16 numbers just above |v|'s power of two (2^-133 at 0)."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, np.exp2(np.maximum(e, -126) - 7), 2.0 ** -133)
+
+
+def excess_error(got, want):
+    """The parity measure for bf16 outputs: max over a row of
+    max(0, |got - want| - ulp(got) / 2) divided by the RMS of the oracle's row.
+
+    A kernel that returns bf16 cannot be closer to the exact value than half a
+    bf16 spacing of its own result; this measures what the kernel's arithmetic
+    adds beyond that rounding of its output (a lower bound of
+    |pre-rounding result - want|).
+    """
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    rms = np.sqrt(np.mean(want ** 2, axis=1))
+    rms = np.where(rms == 0, 1.0, rms)
+    d = np.maximum(0.0, np.abs(got - want) - 0.5 * bf16_ulp(got))
+    return float(np.max(d / rms[:, None]))
+
+
 def check_ok():
     rc = lib.svdq_check_status()
     assert rc == lib.OK, lib.status_name(rc)

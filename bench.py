@@ -41,11 +41,11 @@ LOWRANK_FLOPS = 2 * M * K * RANK + 2 * M * RANK * N
 AWQ_FLOPS = 2 * AM * AK * AN
 STEP_FLOPS = W4A4_FLOPS + LOWRANK_FLOPS + AWQ_FLOPS
 # Algorithmic bytes per launch (each byte the kernel must move once).
-K1_BYTES = (M * K * 2 + K * RANK * 2 + K * 4          # X, L1T, inv_lambda
-            + M * K // 2 + M * K // 16 + M * 64 * 2)  # codes, scales, U
-K2_BYTES = (M * K // 2 + M * K // 16 + M * 64 * 2     # activation codes, scales, U
-            + N * K // 2 + N * K // 16 + N * 64 * 2   # weight codes, scales, L2T
-            + N * 2 + M * N * 2)                      # bias, Y
+K1_BYTES = (M * K * 2 + K * RANK * 2 + K * 4            # X, L1T, inv_lambda
+            + M * K // 2 + M * K // 16 + M * RANK * 2)  # codes, scales, U
+K2_BYTES = (M * K // 2 + M * K // 16 + M * RANK * 2     # activation codes, scales, U
+            + N * K // 2 + N * K // 16 + N * RANK * 2   # weight codes, scales, L2T
+            + N * 2 + M * N * 2)                        # bias, Y
 K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
             + AM * AK * 2 + AK * 4 + AN * 2 + AM * AN * 2)
 
@@ -136,12 +136,10 @@ def setup(device, sets):
     for _ in range(sets):
         S.append(dict(
             X=bf(xb).to(device), inv_lambda=t(packed["inv_lambda"]).to(device), l1t=bf(packed["l1t"]).to(device),
-            l2t=bf(packed["l2t"]).to(device), w_codes=t(packed["w_codes"]).to(device),
-            w_scales=t(packed["w_scales"]).to(device), s_w=t(packed["s_w"]).to(device),
-            s_a=t(packed["s_a"]).to(device), bias=bf(bb).to(device),
-            codes=torch.empty((M, K // 2), dtype=torch.uint8, device=device),
-            scales=torch.empty(sz["scales"], dtype=torch.uint8, device=device),
-            U=torch.empty((M, 64), dtype=torch.bfloat16, device=device),
+            l2t=t(packed["l2t"]).to(device), w_bundle=t(packed["w_bundle"]).to(device),
+            s_w=t(packed["s_w"]).to(device), s_a=t(packed["s_a"]).to(device), bias=bf(bb).to(device),
+            a_bundle=torch.empty(sz["a_bundle"], dtype=torch.uint8, device=device),
+            U=torch.empty(sz["u"], dtype=torch.uint8, device=device),
             Y=torch.empty((M, N), dtype=torch.bfloat16, device=device),
             AX=bf(axb).to(device), qweight=t(apk["qweight"]).to(device), ascales=bf(apk["scales"]).to(device),
             azeros=bf(apk["zeros"]).to(device), inv_awq=t(apk["inv_awq"]).to(device), abias=bf(abb).to(device),
@@ -155,12 +153,11 @@ def step(S, i, ev=None):
     s = S[i % len(S)]
     if ev is not None:
         ev[0].record()
-    lib.svdq_quantize_act(s["X"], s["inv_lambda"], s["l1t"], RANK, s["s_a"], s["s_w"], s["codes"], s["scales"],
-                          s["U"])
+    lib.svdq_quantize_act(s["X"], s["inv_lambda"], s["l1t"], RANK, s["s_a"], s["s_w"], s["a_bundle"], s["U"])
     if ev is not None:
         ev[1].record()
-    lib.svdq_linear_w4a4(s["codes"], s["scales"], s["U"], s["s_a"], s["w_codes"], s["w_scales"], s["l2t"], s["s_w"],
-                         s["bias"], M, N, K, RANK, 0, 0, s["Y"])
+    lib.svdq_linear_w4a4(s["a_bundle"], s["U"], s["s_a"], s["w_bundle"], s["l2t"], s["s_w"], s["bias"],
+                         M, N, K, RANK, 0, 0, s["Y"])
     if ev is not None:
         ev[2].record()
     lib.awq_linear_w4a16(s["AX"], s["inv_awq"], s["qweight"], s["ascales"], s["azeros"], s["abias"], AN, s["AY"])
@@ -299,18 +296,11 @@ def oracle_sample(rows, x, packed, bb, awq_case):
     def bf(bits):
         return formats.bf16_bits_to_float(np.asarray(bits, np.uint16))
 
-    l1 = bf(packed["l1t"]).T
-    l2 = bf(packed["l2t"])[:, :RANK].T
-    w_codes = np.empty((N, K), np.uint8)
-    w_codes[:, 0::2], w_codes[:, 1::2] = packed["w_codes"] & 15, packed["w_codes"] >> 4
-    m_i = np.arange(N)[:, None]
-    kb = np.arange(K // 16)[None, :]
-    w_sf = packed["w_scales"][((m_i // 128) * (K // 64) + kb // 4) * 512 + (m_i % 32) * 16 + ((m_i % 128) // 32) * 4
-                              + kb % 4]
+    l1, l2, w_codes, w_sf = packed["l1"], packed["l2"], packed["w_codes"], packed["w_sf"]
     axb, ainv, aq, as_, az, abias = awq_case
     t = time.perf_counter()
-    codes, sf, u = svdquant.quantize_act(x[:rows], packed["inv_lambda"], l1, packed["s_a"][0], packed["s_w"][0])
-    svdquant.w4a4_linear(codes, sf, packed["s_a"][0], w_codes, w_sf, packed["s_w"][0], u, l2, bf(bb))
+    codes, sf, u = svdquant.quantize_act(x[:rows], packed["inv_lambda"], l1, packed["s_a"], packed["s_w"])
+    svdquant.w4a4_linear(codes, sf, packed["s_a"], w_codes, w_sf, packed["s_w"], u, l2, bf(bb))
     oawq.linear(axb, ainv, aq, as_, az, abias)
     dt = time.perf_counter() - t
     flops = rows / M * (W4A4_FLOPS + LOWRANK_FLOPS) + AWQ_FLOPS
@@ -318,14 +308,15 @@ def oracle_sample(rows, x, packed, bb, awq_case):
 
 
 def _oracle_inputs():
-    from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
+    from bit_w4a4_diffusion_smooth_b200 import synthetic
     from oracle import awq as oawq
-    from oracle import formats
+    from oracle import formats, svdquant
 
     c = synthetic.QKV
     xb, wb, bb = c.make()
     x = formats.bf16_bits_to_float(xb)
-    packed = lib.svdq_pack_weights(wb, np.max(np.abs(x), axis=0).astype(np.float32), RANK, seed=c.seed)
+    # the oracle's own pack; its cost is not part of the timed sample
+    packed = svdquant.pack(formats.bf16_bits_to_float(wb), np.max(np.abs(x), axis=0).astype(np.float32), RANK)
     a = synthetic.AWQ
     axb, awb, abb, asc = a.make()
     ap = oawq.pack(formats.bf16_bits_to_float(awb), asc)

@@ -276,15 +276,13 @@ void top_r_basis(const double *Wp, int K, int N, int r, int threads, uint64_t se
 }
 }  // namespace
 
-// NVFP4 quantization of float32 rows (see svdq.h).
-static void quantize_rows_f32(const float *T, int rows, int K, float s_t, uint8_t *codes,
-                              uint8_t *scales, int threads) {
+// NVFP4 quantization of float32 rows into a bundle of tile height th (see svdq.h).
+static void quantize_rows_f32(const float *T, int rows, int K, float s_t, int th, uint8_t *bundle, int threads) {
   const float d = 6.0f * s_t;
-  std::memset(scales, 0, sf_bytes(rows, K));
+  std::memset(bundle, 0, bundle_bytes(rows, K, th));
   parallel_for(rows, threads, [&](int b, int e) {
     for (int m = b; m < e; ++m) {
       const float *t = T + static_cast<size_t>(m) * K;
-      uint8_t *c = codes + static_cast<size_t>(m) * (K / 2);
       for (int kb = 0; kb < K / 16; ++kb) {
         float amax = 0.0f;
         for (int i = 0; i < 16; ++i) amax = std::max(amax, std::fabs(t[kb * 16 + i]));
@@ -292,11 +290,12 @@ static void quantize_rows_f32(const float *T, int rows, int K, float s_t, uint8_
         float scale = kE4m3.v[sb] * s_t;
         float inv = scale == 0.0f ? 0.0f : 1.0f / scale;
         for (int i = 0; i < 16; i += 2) {
-          uint8_t lo = e2m1_code(t[kb * 16 + i] * inv);
-          uint8_t hi = e2m1_code(t[kb * 16 + i + 1] * inv);
-          c[(kb * 16 + i) / 2] = static_cast<uint8_t>(lo | (hi << 4));
+          const int k = kb * 16 + i;
+          uint8_t lo = e2m1_code(t[k] * inv);
+          uint8_t hi = e2m1_code(t[k + 1] * inv);
+          bundle[bundle_code_offset(m, k, K, th)] = static_cast<uint8_t>(lo | (hi << 4));
         }
-        scales[sf_offset(m, kb, K)] = sb;
+        bundle[bundle_scale_offset(m, kb * 16, K, th)] = sb;
       }
     }
   });
@@ -312,20 +311,19 @@ static int default_threads(int t) {
 
 using namespace svdq;
 
-extern "C" int svdq_quantize_host(const float *T, int rows, int K, float s_t, uint8_t *codes,
-                                  uint8_t *scales) {
-  if (!T || !codes || !scales) return fail(SVDQ_ERR_INVALID_ARG, "svdq_quantize_host: null pointer");
+extern "C" int svdq_quantize_host(const float *T, int rows, int K, float s_t, int tile_rows, uint8_t *bundle) {
+  if (!T || !bundle) return fail(SVDQ_ERR_INVALID_ARG, "svdq_quantize_host: null pointer");
   if (rows < 1 || K < 64 || K % 64) return fail(SVDQ_ERR_SHAPE, "svdq_quantize_host: need rows >= 1, K % 64 == 0");
+  if (tile_rows != 128 && tile_rows != 256) return fail(SVDQ_ERR_SHAPE, "svdq_quantize_host: tile_rows must be 128 or 256");
   if (!(s_t > 0.0f) || !std::isfinite(s_t)) return fail(SVDQ_ERR_INVALID_ARG, "svdq_quantize_host: s_t must be > 0");
-  quantize_rows_f32(T, rows, K, s_t, codes, scales, default_threads(0));
+  quantize_rows_f32(T, rows, K, s_t, tile_rows, bundle, default_threads(0));
   return ok();
 }
 
 extern "C" int svdq_pack_weights(const uint16_t *W, int K, int N, const float *act_absmax, int rank,
                                  int num_threads, uint64_t seed, float *inv_lambda, uint16_t *l1t,
-                                 uint16_t *l2t, uint8_t *w_codes, uint8_t *w_scales, float *s_w,
-                                 float *s_a, float *residual) {
-  if (!W || !act_absmax || !inv_lambda || !l2t || !w_codes || !w_scales || !s_w || !s_a ||
+                                 uint8_t *l2t, uint8_t *w_bundle, float *s_w, float *s_a, float *residual) {
+  if (!W || !act_absmax || !inv_lambda || !l2t || !w_bundle || !s_w || !s_a ||
       (rank > 0 && !l1t))
     return fail(SVDQ_ERR_INVALID_ARG, "svdq_pack_weights: null pointer");
   if (K < 64 || K % 64 || N < 8 || N % 8)
@@ -372,16 +370,14 @@ extern "C" int svdq_pack_weights(const uint16_t *W, int K, int N, const float *a
       }
     }
   }
+  std::memset(l2t, 0, lowrank_bytes(N, 256));
   for (int n = 0; n < N; ++n)
-    for (int i = 0; i < SVDQ_LR_STRIDE; ++i) {
-      uint16_t b = 0;
-      if (i < rank) {
-        float f = static_cast<float>(L2[static_cast<size_t>(i) * N + n]);
-        uint32_t u;
-        std::memcpy(&u, &f, 4);
-        b = static_cast<uint16_t>(u >> 16);
-      }
-      l2t[static_cast<size_t>(n) * SVDQ_LR_STRIDE + i] = b;
+    for (int i = 0; i < rank; ++i) {
+      float f = static_cast<float>(L2[static_cast<size_t>(i) * N + n]);
+      uint32_t u;
+      std::memcpy(&u, &f, 4);
+      const uint16_t b = static_cast<uint16_t>(u >> 16);
+      std::memcpy(l2t + lowrank_offset(n, i, 256), &b, 2);
     }
 
   // 3. Residual R = W' - L1 L2 in float64, rounded to float32, stored K-major
@@ -412,7 +408,7 @@ extern "C" int svdq_pack_weights(const uint16_t *W, int K, int N, const float *a
 
   // 4. NVFP4 of R (blocks of 16 along K for each output column).
   *s_w = tensor_scale(amax);
-  quantize_rows_f32(Rt.data(), N, K, *s_w, w_codes, w_scales, threads);
+  quantize_rows_f32(Rt.data(), N, K, *s_w, 256, w_bundle, threads);
 
   // 5. Static activation scale from the calibration maxima.
   float xa = 0.0f;
@@ -422,23 +418,21 @@ extern "C" int svdq_pack_weights(const uint16_t *W, int K, int N, const float *a
 }
 
 extern "C" int svdq_weight_sizes(int K, int N, int rank, size_t *inv_lambda_bytes, size_t *l1t_bytes,
-                                 size_t *l2t_bytes, size_t *w_codes_bytes, size_t *w_scales_bytes) {
+                                 size_t *l2t_bytes, size_t *w_bundle_bytes) {
   if (K < 64 || K % 64 || N < 8 || N % 8)
     return fail(SVDQ_ERR_SHAPE, "svdq_weight_sizes: need K % 64 == 0 and N % 8 == 0");
   if (rank < 0 || rank > SVDQ_LR_STRIDE || rank % 16)
     return fail(SVDQ_ERR_SHAPE, "svdq_weight_sizes: rank must be a multiple of 16 in [0, 64]");
   if (inv_lambda_bytes) *inv_lambda_bytes = static_cast<size_t>(K) * 4;
   if (l1t_bytes) *l1t_bytes = static_cast<size_t>(rank) * K * 2;
-  if (l2t_bytes) *l2t_bytes = static_cast<size_t>(N) * SVDQ_LR_STRIDE * 2;
-  if (w_codes_bytes) *w_codes_bytes = static_cast<size_t>(N) * (K / 2);
-  if (w_scales_bytes) *w_scales_bytes = sf_bytes(N, K);
+  if (l2t_bytes) *l2t_bytes = lowrank_bytes(N, 256);
+  if (w_bundle_bytes) *w_bundle_bytes = bundle_bytes(N, K, 256);
   return ok();
 }
 
-extern "C" int svdq_act_sizes(int M, int K, size_t *codes_bytes, size_t *scales_bytes, size_t *u_bytes) {
+extern "C" int svdq_act_sizes(int M, int K, size_t *a_bundle_bytes, size_t *u_bytes) {
   if (M < 1 || K < 64 || K % 64) return fail(SVDQ_ERR_SHAPE, "svdq_act_sizes: need M >= 1 and K % 64 == 0");
-  if (codes_bytes) *codes_bytes = static_cast<size_t>(M) * (K / 2);
-  if (scales_bytes) *scales_bytes = sf_bytes(M, K);
-  if (u_bytes) *u_bytes = static_cast<size_t>(M) * SVDQ_LR_STRIDE * 2;
+  if (a_bundle_bytes) *a_bundle_bytes = bundle_bytes(M, K, 128);
+  if (u_bytes) *u_bytes = lowrank_bytes(M, 128);
   return ok();
 }

@@ -5,20 +5,23 @@
 // page "Nunchaku Diffusers 支持降低显存占用，但硬件仍决定适用范围", remio.ai,
 // section "SVDQuant 将棘手数值移出 4 位路径").  One read of X produces:
 //   * the NVFP4 codes and ue4m3 block scales of X^ = X . diag(inv_lambda),
-//   * U = (bf16(X^) . L1) / (s_a s_w), the low-rank activations the GEMM adds.
+//     written straight into the 128-row operand bundle the GEMM streams;
+//   * U = (bf16(X^) . L1) / (s_a s_w), the low-rank activations the GEMM adds,
+//     written as 128-row swizzled tiles.
 //
 // Design (memory bound: X is read once, ~0.3 B written per byte read):
-//   * one CTA per 32 rows, 8 compute warps + 1 TMA warp; a 4-stage ring of
-//     [32 rows x 256 cols] bf16 tiles of X and [rank x 256] tiles of L1^T,
-//     loaded by TMA with the 128-byte swizzle (conflict-free for both the
-//     row-wise quantize pass and ldmatrix);
-//   * quantize pass: each warp owns 4 rows, each lane 8 consecutive
-//     elements (two lanes per 16-block, one shuffle for the block max),
-//     16-byte shared loads, 128-byte coalesced code stores; X^ is written
-//     back in place as bf16;
-//   * down-projection pass: warp w multiplies its 32-column slice of the
-//     tile with mma.sync (bf16 in, fp32 accumulate), partial sums are added
-//     across warps once at the end;
+//   * one CTA per 32 rows, 16 compute warps + 1 TMA warp; a 4-stage ring of
+//     [32 rows x 256 cols] bf16 tiles of X, [rank x 256] tiles of L1^T and
+//     256-float slices of inv_lambda, loaded by TMA / bulk copies; X and L1^T
+//     land with the 128-byte swizzle (conflict-free for the row-wise pass and
+//     for ldmatrix);
+//   * quantize pass: each warp owns 2 rows, each lane 8 consecutive elements
+//     (two lanes per 16-block, one shuffle for the block max); codes go out
+//     as one 128-byte row segment per warp and row, four block scales per
+//     32-bit store; X^ is written back in place as bf16;
+//   * down-projection pass: warp w multiplies k16-slice w of the tile with
+//     mma.sync (bf16 in, fp32 accumulate); partial sums are added across the
+//     warps once at the end;
 //   * every wait is bounded (mbarrier try_wait + %globaltimer); a wait that
 //     runs out records SVDQ_ERR_TIMEOUT and the block leaves cleanly.
 #include <cuda.h>
@@ -34,26 +37,27 @@ namespace svdq {
 namespace {
 
 constexpr int BM = 32;             // rows per CTA
-constexpr int KC = 256;            // columns per stage
+constexpr int KC = kStageK;        // columns per stage (one bundle k-stage)
 constexpr int STAGES = 4;
-constexpr int CWARPS = 8;          // compute warps
+constexpr int CWARPS = 16;         // compute warps
 constexpr int THREADS = (CWARPS + 1) * 32;
 constexpr int X_BOX = BM * 128;    // one [32 x 64] bf16 box, 128-byte rows
 constexpr int X_STAGE = 4 * X_BOX;
+constexpr int INV_BYTES = KC * 4;
 
 struct Params {
-  int M, K, m_pad;
+  int M, K, KS;
   const float *inv_lambda;
   const float *s_a, *s_w;
-  uint8_t *codes, *scales;
-  uint16_t *U;
+  uint8_t *bundle;
+  uint8_t *U;
   unsigned int *status;
   unsigned long long limit_ns;
 };
 
 template <int RANK>
 __host__ __device__ constexpr int stage_bytes() {
-  return X_STAGE + 4 * RANK * 128;
+  return X_STAGE + 4 * RANK * 128 + INV_BYTES;
 }
 template <int RANK>
 __host__ __device__ constexpr int smem_bytes() {
@@ -66,12 +70,18 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return static_cast<uint32_t>(r * 128 + ((((c >> 3) ^ r) & 7) << 4));
 }
 
+__device__ __forceinline__ void fail_wait(volatile int *abort_flag, unsigned int *status) {
+  *abort_flag = 1;
+  dev::report(status, SVDQ_ERR_TIMEOUT);
+}
+
 template <int RANK>
 __global__ void __launch_bounds__(THREADS, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1, Params p) {
   constexpr int NP = RANK / 16;           // pairs of 8-wide MMA column tiles
   constexpr int L1_BOX = RANK * 128;
   constexpr int STAGE = stage_bytes<RANK>();
+  constexpr int INV_OFF = X_STAGE + 4 * L1_BOX;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -83,7 +93,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
-  const int nchunks = (p.K + KC - 1) / KC;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -103,21 +112,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       dev::prefetch_tmap(&tm_x);
       if (RANK > 0) dev::prefetch_tmap(&tm_l1);
       int issued = 0;
-      for (int c = 0; c < nchunks; ++c) {
+      for (int c = 0; c < p.KS; ++c) {
         const int s = c % STAGES;
-        const uint32_t ph = (c / STAGES) & 1;
-        if (!dev::mbar_wait(&empty[s], ph ^ 1, p.limit_ns, abort_flag)) {
-          *abort_flag = 1;
-          dev::report(p.status, SVDQ_ERR_TIMEOUT);
+        if (!dev::mbar_wait(&empty[s], ((c / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
+          fail_wait(abort_flag, p.status);
           break;
         }
         const int nbox = min(4, (p.K - c * KC) / 64);
-        dev::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * (X_BOX + L1_BOX)));
+        dev::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * (X_BOX + L1_BOX + 256)));
         uint8_t *st = smem + s * STAGE;
         for (int b = 0; b < nbox; ++b) {
           dev::tma_load_2d(st + b * X_BOX, &tm_x, &full[s], c * KC + b * 64, m0);
           if (RANK > 0) dev::tma_load_2d(st + X_STAGE + b * L1_BOX, &tm_l1, &full[s], c * KC + b * 64, 0);
         }
+        dev::bulk_load(st + INV_OFF, p.inv_lambda + c * KC, static_cast<uint32_t>(nbox * 256), &full[s]);
         ++issued;
       }
       if (*abort_flag) {
@@ -140,25 +148,26 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const float s_a = __ldg(p.s_a);
   const float d6 = __fmul_rn(6.0f, s_a);
-  bool ok = true;
+  const int m_blk = m0 / 128;
+  const int r_base = m0 % 128;            // row of this CTA's first row inside its 128-row tile
 
-  for (int c = 0; c < nchunks && ok; ++c) {
+  for (int c = 0; c < p.KS; ++c) {
     const int s = c % STAGES;
     const uint32_t ph = (c / STAGES) & 1;
     if (!dev::mbar_wait(&full[s], ph, p.limit_ns, abort_flag)) {
-      ok = false;
-      break;
+      fail_wait(abort_flag, p.status);
+      return;
     }
     const int nbox = min(4, (p.K - c * KC) / 64);
     uint8_t *st = smem + s * STAGE;
-    const int col = c * KC + 8 * lane;        // first of this lane's 8 columns
     const int box = lane >> 3;
-    const bool col_ok = box < nbox;
+    const bool col_ok = box < nbox;       // columns past K quantize as zeros
+    uint8_t *tile = p.bundle + (static_cast<size_t>(m_blk) * p.KS + c) * bundle_tile_bytes(128);
 
     float inv[8];
     if (col_ok) {
-      const float4 i0 = __ldg(reinterpret_cast<const float4 *>(p.inv_lambda + col));
-      const float4 i1 = __ldg(reinterpret_cast<const float4 *>(p.inv_lambda + col + 4));
+      const float4 i0 = *reinterpret_cast<const float4 *>(st + INV_OFF + 32 * lane);
+      const float4 i1 = *reinterpret_cast<const float4 *>(st + INV_OFF + 32 * lane + 16);
       inv[0] = i0.x; inv[1] = i0.y; inv[2] = i0.z; inv[3] = i0.w;
       inv[4] = i1.x; inv[5] = i1.y; inv[6] = i1.z; inv[7] = i1.w;
     } else {
@@ -166,11 +175,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = 0; i < 8; ++i) inv[i] = 0.0f;
     }
 
-    // ---- quantize pass: rows 4*warp .. 4*warp+3
+    // ---- quantize pass: rows 2*warp, 2*warp+1
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = warp * 4 + i;
-      const int m = m0 + r;
+    for (int i = 0; i < 2; ++i) {
+      const int r = warp * 2 + i;
+      const int rt = r_base + r;          // row inside the 128-row bundle tile
       uint8_t *chunk = st + box * X_BOX + sw_off(r, (8 * lane) & 63);
       uint4 raw = make_uint4(0, 0, 0, 0);
       if (col_ok) raw = *reinterpret_cast<const uint4 *>(chunk);
@@ -192,15 +201,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         packed |= dev::cvt_e2m1x2(__fmul_rn(xh[2 * j], rinv), __fmul_rn(xh[2 * j + 1], rinv)) << (8 * j);
-      if (col_ok && m < p.M)
-        *reinterpret_cast<uint32_t *>(p.codes + static_cast<size_t>(m) * (p.K / 2) + col / 2) = packed;
-      // four consecutive block scales (lanes 8q, 8q+2, 8q+4, 8q+6) -> one word
+      // this lane's 4 code bytes: byte 4*lane of the row, 128-byte swizzle
+      *reinterpret_cast<uint32_t *>(tile + rt * 128 + ((((lane >> 2) ^ rt) & 7) << 4) + (lane & 3) * 4) = packed;
+      // four consecutive block scales (lanes 8q, 8q+2, 8q+4, 8q+6) -> one word of atom q
       const int base = lane & ~7;
       const uint32_t word = __shfl_sync(0xFFFFFFFFu, sb, base) | (__shfl_sync(0xFFFFFFFFu, sb, base + 2) << 8) |
                             (__shfl_sync(0xFFFFFFFFu, sb, base + 4) << 16) |
                             (__shfl_sync(0xFFFFFFFFu, sb, base + 6) << 24);
-      if ((lane & 7) == 0 && col_ok && m < p.m_pad)
-        *reinterpret_cast<uint32_t *>(p.scales + sf_offset(m, col / 16, p.K)) = word;
+      if ((lane & 7) == 0)
+        *reinterpret_cast<uint32_t *>(tile + 128 * 128 + box * 512 + (rt & 31) * 16 + ((rt >> 5) & 3) * 4) = word;
       if (RANK > 0 && col_ok) {
         uint4 o;
         __nv_bfloat162 h0 = __floats2bfloat162_rn(xh[0], xh[1]);
@@ -215,62 +224,52 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
 
-    // ---- down-projection pass: warp w takes columns [32w, 32w+32) of the tile
+    // ---- down-projection pass: warp w takes columns [16w, 16w+16) of the tile
     if (RANK > 0) {
       __syncwarp();
       if (lane == 0) dev::mbar_arrive(&ready[s]);
       if (!dev::mbar_wait(&ready[s], ph, p.limit_ns, abort_flag)) {
-        ok = false;
-        break;
+        fail_wait(abort_flag, p.status);
+        return;
       }
-      const int kbox = warp >> 1;
+      const int kbox = warp >> 2;
       if (kbox < nbox) {
         const uint32_t xbase = dev::smem_u32(st + kbox * X_BOX);
         const uint32_t lbase = dev::smem_u32(st + X_STAGE + kbox * L1_BOX);
+        const int kc = (warp & 3) * 16;
+        uint32_t a[2][4];
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const int kc = (warp & 1) * 32 + ks * 16;
-          uint32_t a[2][4];
+        for (int mt = 0; mt < 2; ++mt) {
+          const int r = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          dev::ldmatrix_x4(xbase + sw_off(r, kc + (lane >> 4) * 8), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+        }
+#pragma unroll
+        for (int np = 0; np < NP; ++np) {
+          const int n = np * 16 + (lane & 7) + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          dev::ldmatrix_x4(lbase + sw_off(n, kc + ((lane >> 3) & 1) * 8), b0, b1, b2, b3);
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt) {
-            const int r = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            dev::ldmatrix_x4(xbase + sw_off(r, kc + (lane >> 4) * 8), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-          }
-#pragma unroll
-          for (int np = 0; np < NP; ++np) {
-            const int n = np * 16 + (lane & 7) + (lane >> 4) * 8;
-            uint32_t b0, b1, b2, b3;
-            dev::ldmatrix_x4(lbase + sw_off(n, kc + ((lane >> 3) & 1) * 8), b0, b1, b2, b3);
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              dev::mma_bf16_16816(acc[mt][2 * np], a[mt], b0, b1);
-              dev::mma_bf16_16816(acc[mt][2 * np + 1], a[mt], b2, b3);
-            }
+            dev::mma_bf16_16816(acc[mt][2 * np], a[mt], b0, b1);
+            dev::mma_bf16_16816(acc[mt][2 * np + 1], a[mt], b2, b3);
           }
         }
       }
+      // the next TMA load into this stage must come after our generic writes
+      dev::fence_proxy_async();
     }
-    // the next TMA load into this stage must come after our generic writes
-    if (RANK > 0) dev::fence_proxy_async();
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(&empty[s]);
   }
 
-  if (!ok) {
-    *abort_flag = 1;
-    dev::report(p.status, SVDQ_ERR_TIMEOUT);
-    return;
-  }
-
-  // ---- U = (sum of the warps' partial products) / (s_a s_w), bf16, [M][64]
-  const int tid = threadIdx.x;  // 0..255
+  // ---- U = (sum of the warps' partial products) / (s_a s_w), bf16, 128-row tiles
+  const int tid = threadIdx.x;  // 0..511
   if (RANK > 0) {
     // every warp is done with the stage buffers -> reuse them for partials
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(sync);
     if (!dev::mbar_wait(sync, 0, p.limit_ns, abort_flag)) {
-      *abort_flag = 1;
-      dev::report(p.status, SVDQ_ERR_TIMEOUT);
+      fail_wait(abort_flag, p.status);
       return;
     }
     float *red = reinterpret_cast<float *>(smem);  // [CWARPS][BM][RANK]
@@ -289,29 +288,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(sync);
     if (!dev::mbar_wait(sync, 1, p.limit_ns, abort_flag)) {
-      *abort_flag = 1;
-      dev::report(p.status, SVDQ_ERR_TIMEOUT);
+      fail_wait(abort_flag, p.status);
       return;
     }
-    const float alpha = __fmul_rn(s_a, __ldg(p.s_w));
-    for (int idx = tid; idx < BM * SVDQ_LR_STRIDE; idx += CWARPS * 32) {
-      const int r = idx / SVDQ_LR_STRIDE, j = idx % SVDQ_LR_STRIDE;
-      const int m = m0 + r;
-      if (m >= p.M) continue;
-      float v = 0.0f;
-      if (j < RANK) {
+  }
+  const float alpha = __fmul_rn(s_a, __ldg(p.s_w));
+  for (int idx = tid; idx < BM * (SVDQ_LR_STRIDE / 8); idx += CWARPS * 32) {
+    const int r = idx >> 3, cc = idx & 7;   // row, 8-column chunk
+    const int m = m0 + r;
+    uint32_t o[4] = {0, 0, 0, 0};
+    if (RANK > 0 && 8 * cc < RANK) {
+      const float *red = reinterpret_cast<const float *>(smem);
+      float v[8];
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) v += red[(w * BM + r) * RANK + j];
-        v = __fdiv_rn(v, alpha);
+      for (int j = 0; j < 8; ++j) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int w = 0; w < CWARPS; ++w) sum += red[(w * BM + r) * RANK + 8 * cc + j];
+        v[j] = __fdiv_rn(sum, alpha);
       }
-      __nv_bfloat16 h = __float2bfloat16_rn(v);
-      p.U[static_cast<size_t>(m) * SVDQ_LR_STRIDE + j] = *reinterpret_cast<uint16_t *>(&h);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        o[j] = *reinterpret_cast<uint32_t *>(&h);
+      }
     }
-  } else {
-    for (int idx = tid; idx < BM * SVDQ_LR_STRIDE; idx += CWARPS * 32) {
-      const int r = idx / SVDQ_LR_STRIDE, j = idx % SVDQ_LR_STRIDE;
-      if (m0 + r < p.M) p.U[static_cast<size_t>(m0 + r) * SVDQ_LR_STRIDE + j] = 0;
-    }
+    *reinterpret_cast<uint4 *>(p.U + lowrank_offset(m, 8 * cc, 128)) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -332,15 +334,15 @@ int launch(const CUtensorMap &tx, const CUtensorMap &tl, const Params &p, int gr
 using namespace svdq;
 
 extern "C" int svdq_quantize_act(const void *X, int M, int K, int ldx, const float *inv_lambda, const void *l1t,
-                                 int rank, const float *s_a, const float *s_w, uint8_t *codes, uint8_t *scales,
-                                 void *U, svdq_stream_t stream) {
-  if (!X || !inv_lambda || !s_a || !s_w || !codes || !scales || !U || (rank > 0 && !l1t))
+                                 int rank, const float *s_a, const float *s_w, uint8_t *a_bundle, void *U,
+                                 svdq_stream_t stream) {
+  if (!X || !inv_lambda || !s_a || !s_w || !a_bundle || !U || (rank > 0 && !l1t))
     return fail(SVDQ_ERR_INVALID_ARG, "svdq_quantize_act: null pointer");
   if (M < 1 || K < 64 || K % 64 || ldx < K || ldx % 8)
     return fail(SVDQ_ERR_SHAPE, "svdq_quantize_act: need M >= 1, K % 64 == 0, ldx >= K, ldx % 8 == 0");
   if (rank < 0 || rank > SVDQ_LR_STRIDE || rank % 16)
     return fail(SVDQ_ERR_SHAPE, "svdq_quantize_act: rank must be a multiple of 16 in [0, 64]");
-  if (!aligned16(X) || !aligned16(inv_lambda) || !aligned16(codes) || !aligned16(scales) || !aligned16(U) ||
+  if (!aligned16(X) || !aligned16(inv_lambda) || !aligned16(a_bundle) || !aligned16(U) ||
       (rank > 0 && !aligned16(l1t)))
     return fail(SVDQ_ERR_ALIGNMENT, "svdq_quantize_act: pointers must be 16-byte aligned");
   DeviceState *st = current_device_state();
@@ -349,13 +351,12 @@ extern "C" int svdq_quantize_act(const void *X, int M, int K, int ldx, const flo
   Params p;
   p.M = M;
   p.K = K;
-  p.m_pad = (M + 127) / 128 * 128;
+  p.KS = bundle_ks(K);
   p.inv_lambda = inv_lambda;
   p.s_a = s_a;
   p.s_w = s_w;
-  p.codes = codes;
-  p.scales = scales;
-  p.U = static_cast<uint16_t *>(U);
+  p.bundle = a_bundle;
+  p.U = static_cast<uint8_t *>(U);
   p.status = st->status_word;
   p.limit_ns = kWaitLimitNs;
 
@@ -371,7 +372,7 @@ extern "C" int svdq_quantize_act(const void *X, int M, int K, int ldx, const flo
   } else {
     tl = tx;
   }
-  const int grid = p.m_pad / BM;
+  const int grid = (M + 127) / 128 * (128 / BM);   // every row of every 128-row tile
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (rank) {
     case 0: return launch<0>(tx, tl, p, grid, s);

@@ -22,19 +22,59 @@ int ok();
 #define SVDQ_HD inline
 #endif
 
-// Byte offset of block scale (row m, 16-block kb) in the tcgen05 scale-factor
-// tile order used for every NVFP4 scale buffer of this library: atoms of
-// 128 rows x 4 scales (512 bytes), atoms ordered K-fastest; inside an atom
-// row m sits at (m % 32) * 16 + ((m % 128) / 32) * 4 and block kb at kb % 4.
-// This is the order in which tcgen05.cp (32x128b, warpx4) moves one atom into
-// four TMEM columns: lane m % 32, column (m % 128) / 32, byte kb % 4.
-SVDQ_HD size_t sf_offset(int m, int kb, int K) {
-  return (static_cast<size_t>(m >> 7) * static_cast<size_t>(K >> 6) + static_cast<size_t>(kb >> 2)) * 512u +
-         static_cast<size_t>(m & 31) * 16u + static_cast<size_t>((m >> 5) & 3) * 4u +
-         static_cast<size_t>(kb & 3);
+// ---------------------------------------------------------------------------
+// Operand bundles: the layout in which NVFP4 operands (codes + block scales)
+// live in memory, built so that one GEMM pipeline stage is one contiguous copy.
+//
+// A matrix of `rows` x K elements is cut into tiles of TH rows (128 for
+// activations, 256 for weights) by 256 K-elements.  Tile (tr, ks) starts at
+//   (tr * KS + ks) * TH * 144 bytes,   KS = ceil(K / 256),
+// and holds
+//   * TH rows x 128 bytes of e2m1 codes, element k of row r in byte k/2 of
+//     the row (low nibble for even k), rows 128 bytes apart, the 16-byte
+//     chunks of a row permuted by the 128-byte swizzle: chunk c of row r at
+//     r*128 + ((c ^ (r % 8)) * 16) - the shared-memory image a tcgen05 MMA
+//     reads with a SWIZZLE_128B K-major descriptor;
+//   * then TH/128 x 4 atoms of 512 bytes of ue4m3 block scales: the scale of
+//     (row r, 16-block j of the tile) at TH*128 + (r/128)*2048 + (j/4)*512 +
+//     (r%32)*16 + ((r%128)/32)*4 + j%4 - the order in which tcgen05.cp
+//     (32x128b, warpx4) moves one atom into four TMEM columns.
+// Rows past `rows` and elements past K are zero (codes and scales).
+constexpr int kStageK = 256;
+
+SVDQ_HD int bundle_ks(int K) { return (K + kStageK - 1) / kStageK; }
+SVDQ_HD size_t bundle_tile_bytes(int th) { return static_cast<size_t>(th) * 144u; }
+SVDQ_HD size_t bundle_bytes(int rows, int K, int th) {
+  return static_cast<size_t>((rows + th - 1) / th) * static_cast<size_t>(bundle_ks(K)) * bundle_tile_bytes(th);
 }
-SVDQ_HD size_t sf_bytes(int rows, int K) {
-  return static_cast<size_t>((rows + 127) / 128) * 128u * static_cast<size_t>(K / 16);
+SVDQ_HD size_t bundle_tile_offset(int m, int k, int K, int th) {
+  return (static_cast<size_t>(m / th) * static_cast<size_t>(bundle_ks(K)) + static_cast<size_t>(k / kStageK)) *
+         bundle_tile_bytes(th);
+}
+// Byte holding the code of element (m, k); the low nibble for even k.
+SVDQ_HD size_t bundle_code_offset(int m, int k, int K, int th) {
+  const int r = m % th, kb = (k % kStageK) / 2;
+  return bundle_tile_offset(m, k, K, th) + static_cast<size_t>(r) * 128u +
+         static_cast<size_t>((((kb >> 4) ^ r) & 7) << 4) + static_cast<size_t>(kb & 15);
+}
+// Byte holding the block scale of element (m, k).
+SVDQ_HD size_t bundle_scale_offset(int m, int k, int K, int th) {
+  const int r = m % th, j = (k % kStageK) / 16;
+  return bundle_tile_offset(m, k, K, th) + static_cast<size_t>(th) * 128u + static_cast<size_t>(r >> 7) * 2048u +
+         static_cast<size_t>(j >> 2) * 512u + static_cast<size_t>(r & 31) * 16u +
+         static_cast<size_t>((r >> 5) & 3) * 4u + static_cast<size_t>(j & 3);
+}
+
+// Low-rank operands: tiles of TH rows x 64 bf16 (TH = 128 for U, 256 for
+// L2T), 128-byte rows with the 128-byte swizzle; element (m, j) at
+//   (m/TH)*TH*128 + (m%TH)*128 + (((j/8) ^ (m%8)) * 16) + (j%8)*2.
+SVDQ_HD size_t lowrank_bytes(int rows, int th) {
+  return static_cast<size_t>((rows + th - 1) / th) * static_cast<size_t>(th) * 128u;
+}
+SVDQ_HD size_t lowrank_offset(int m, int j, int th) {
+  const int r = m % th;
+  return static_cast<size_t>(m / th) * static_cast<size_t>(th) * 128u + static_cast<size_t>(r) * 128u +
+         static_cast<size_t>((((j >> 3) ^ r) & 7) << 4) + static_cast<size_t>(j & 7) * 2u;
 }
 
 // Per-device state filled by svdq_init.

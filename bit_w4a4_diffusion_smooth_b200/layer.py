@@ -30,9 +30,8 @@ class SVDQLinear:
         lib.svdq_init(self.device.index or 0)
         self.inv_lambda = _dev(packed["inv_lambda"], device)
         self.l1t = _dev(packed["l1t"], device, torch.bfloat16) if rank else None
-        self.l2t = _dev(packed["l2t"], device, torch.bfloat16)
-        self.w_codes = _dev(packed["w_codes"], device)
-        self.w_scales = _dev(packed["w_scales"], device)
+        self.l2t = _dev(packed["l2t"], device)
+        self.w_bundle = _dev(packed["w_bundle"], device)
         self.s_w = _dev(np.asarray(packed["s_w"], np.float32).reshape(1), device)
         self.s_a = _dev(np.asarray(packed["s_a"], np.float32).reshape(1), device)
         self.bias = _dev(bias_bits, device, torch.bfloat16) if bias_bits is not None else None
@@ -50,21 +49,19 @@ class SVDQLinear:
         if M not in self._bufs:
             sz = lib.svdq_act_sizes(M, self.K)
             self._bufs[M] = dict(
-                codes=torch.empty((M, self.K // 2), dtype=torch.uint8, device=self.device),
-                scales=torch.empty(sz["scales"], dtype=torch.uint8, device=self.device),
-                U=torch.empty((M, lib.LR_STRIDE), dtype=torch.bfloat16, device=self.device))
+                a_bundle=torch.empty(sz["a_bundle"], dtype=torch.uint8, device=self.device),
+                U=torch.empty(sz["u"], dtype=torch.uint8, device=self.device))
         return self._bufs[M]
 
     def quantize(self, X, stream=None):
         b = self.buffers(X.shape[0])
         lib.svdq_quantize_act(X, self.inv_lambda, self.l1t, self.rank, self.s_a, self.s_w,
-                              b["codes"], b["scales"], b["U"], stream=stream)
+                              b["a_bundle"], b["U"], stream=stream)
         return b
 
     def gemm(self, b, M, Y, stream=None):
-        lib.svdq_linear_w4a4(b["codes"], b["scales"], b["U"], self.s_a, self.w_codes, self.w_scales,
-                             self.l2t, self.s_w, self.bias, M, self.N, self.K, self.rank, self.epilogue,
-                             self.gelu_col_begin, Y, stream=stream)
+        lib.svdq_linear_w4a4(b["a_bundle"], b["U"], self.s_a, self.w_bundle, self.l2t, self.s_w, self.bias,
+                             M, self.N, self.K, self.rank, self.epilogue, self.gelu_col_begin, Y, stream=stream)
         return Y
 
     def __call__(self, X, Y=None, stream=None):

@@ -37,12 +37,12 @@ _SIGNATURES = {
     "svdq_last_error_string": (ctypes.c_char_p, []),
     "svdq_status_string": (ctypes.c_char_p, [_I]),
     "svdq_init": (_I, [_I]),
-    "svdq_weight_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ, _SZ]),
-    "svdq_act_sizes": (_I, [_I, _I, _SZ, _SZ, _SZ]),
-    "svdq_pack_weights": (_I, [_P, _I, _I, _P, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _P, _P]),
-    "svdq_quantize_host": (_I, [_P, _I, _I, ctypes.c_float, _P, _P]),
-    "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
-    "svdq_linear_w4a4": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_weight_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ]),
+    "svdq_act_sizes": (_I, [_I, _I, _SZ, _SZ]),
+    "svdq_pack_weights": (_I, [_P, _I, _I, _P, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _P]),
+    "svdq_quantize_host": (_I, [_P, _I, _I, ctypes.c_float, _I, _P]),
+    "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P]),
+    "svdq_linear_w4a4": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "awq_pack_weights": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "awq_linear_w4a16": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P]),
     "svdq_check_status": (_I, [_P]),
@@ -123,32 +123,31 @@ def svdq_init(device=0):
 
 
 def svdq_weight_sizes(K, N, rank):
-    s = [ctypes.c_size_t() for _ in range(5)]
+    s = [ctypes.c_size_t() for _ in range(4)]
     _check("svdq_weight_sizes", load().svdq_weight_sizes(K, N, rank, *[ctypes.byref(x) for x in s]))
-    return dict(zip(("inv_lambda", "l1t", "l2t", "w_codes", "w_scales"), (x.value for x in s)))
+    return dict(zip(("inv_lambda", "l1t", "l2t", "w_bundle"), (x.value for x in s)))
 
 
 def svdq_act_sizes(M, K):
-    s = [ctypes.c_size_t() for _ in range(3)]
+    s = [ctypes.c_size_t() for _ in range(2)]
     _check("svdq_act_sizes", load().svdq_act_sizes(M, K, *[ctypes.byref(x) for x in s]))
-    return dict(zip(("codes", "scales", "u"), (x.value for x in s)))
+    return dict(zip(("a_bundle", "u"), (x.value for x in s)))
 
 
 def svdq_pack_weights(W_bits, act_absmax, rank, num_threads=0, seed=0, want_residual=False):
     """Host pack.  W_bits: uint16 [K, N] bf16 patterns; act_absmax: float32 [K].
 
-    Returns numpy arrays: inv_lambda [K] f32, l1t [rank, K] u16, l2t [N, 64] u16,
-    w_codes [N, K/2] u8, w_scales (tile order) u8, s_w, s_a (float32 scalars),
-    residual [K, N] f32 if asked.
+    Returns numpy arrays: inv_lambda [K] f32, l1t [rank, K] u16 (bf16), l2t
+    (256-row low-rank tiles, u8), w_bundle (256-row NVFP4 bundle, u8), s_w, s_a
+    (float32 scalars), and residual [K, N] f32 if asked.
     """
     K, N = W_bits.shape
     sz = svdq_weight_sizes(K, N, rank)
     out = dict(
         inv_lambda=np.zeros(K, np.float32),
         l1t=np.zeros((rank, K), np.uint16),
-        l2t=np.zeros((N, LR_STRIDE), np.uint16),
-        w_codes=np.zeros((N, K // 2), np.uint8),
-        w_scales=np.zeros(sz["w_scales"], np.uint8),
+        l2t=np.zeros(sz["l2t"], np.uint8),
+        w_bundle=np.zeros(sz["w_bundle"], np.uint8),
         s_w=np.zeros(1, np.float32),
         s_a=np.zeros(1, np.float32),
     )
@@ -158,8 +157,8 @@ def svdq_pack_weights(W_bits, act_absmax, rank, num_threads=0, seed=0, want_resi
     rc = load().svdq_pack_weights(
         _hptr(W_bits, np.uint16, "W"), K, N, _hptr(act_absmax, np.float32, "act_absmax"), rank,
         num_threads, seed, _hptr(out["inv_lambda"], np.float32, "inv_lambda"),
-        _hptr(out["l1t"], np.uint16, "l1t") if rank else None, _hptr(out["l2t"], np.uint16, "l2t"),
-        _hptr(out["w_codes"], np.uint8, "w_codes"), _hptr(out["w_scales"], np.uint8, "w_scales"),
+        _hptr(out["l1t"], np.uint16, "l1t") if rank else None, _hptr(out["l2t"], np.uint8, "l2t"),
+        _hptr(out["w_bundle"], np.uint8, "w_bundle"),
         _hptr(out["s_w"], np.float32, "s_w"), _hptr(out["s_a"], np.float32, "s_a"),
         _hptr(residual, np.float32, "residual") if want_residual else None)
     _check("svdq_pack_weights", rc)
@@ -168,19 +167,19 @@ def svdq_pack_weights(W_bits, act_absmax, rank, num_threads=0, seed=0, want_resi
     return out
 
 
-def svdq_quantize_host(T, s_t):
-    """Host NVFP4 of float32 rows T [rows, K]: (codes [rows, K/2] u8, scales tile order u8)."""
+def svdq_quantize_host(T, s_t, tile_rows=128):
+    """Host NVFP4 of float32 rows T [rows, K] into a bundle of the given tile height (u8)."""
     T = np.ascontiguousarray(T, dtype=np.float32)
     rows, K = T.shape
-    codes = np.zeros((rows, K // 2), np.uint8)
-    scales = np.zeros(svdq_act_sizes(rows, K)["scales"], np.uint8)
+    ks = (K + 255) // 256
+    bundle = np.zeros(((rows + tile_rows - 1) // tile_rows) * ks * tile_rows * 144, np.uint8)
     _check("svdq_quantize_host", load().svdq_quantize_host(
-        _hptr(T, np.float32, "T"), rows, K, ctypes.c_float(float(s_t)),
-        _hptr(codes, np.uint8, "codes"), _hptr(scales, np.uint8, "scales")))
-    return codes, scales
+        _hptr(T, np.float32, "T"), rows, K, ctypes.c_float(float(s_t)), tile_rows,
+        _hptr(bundle, np.uint8, "bundle")))
+    return bundle
 
 
-def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, codes, scales, U, M=None, K=None, stream=None):
+def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M=None, K=None, stream=None):
     """Enqueues the activation kernel.  X: bf16 CUDA [M, ldx] (row stride ldx)."""
     import torch
     M = X.shape[0] if M is None else M
@@ -189,18 +188,17 @@ def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, codes, scales, U, M=No
     _check("svdq_quantize_act", load().svdq_quantize_act(
         _dptr(X, "X", torch.bfloat16), M, K, ldx, _dptr(inv_lambda, "inv_lambda", torch.float32),
         _dptr(l1t, "l1t", allow_none=rank == 0), rank, _dptr(s_a, "s_a", torch.float32),
-        _dptr(s_w, "s_w", torch.float32), _dptr(codes, "codes", torch.uint8),
-        _dptr(scales, "scales", torch.uint8), _dptr(U, "U"), _stream(stream)))
+        _dptr(s_w, "s_w", torch.float32), _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U"),
+        _stream(stream)))
 
 
-def svdq_linear_w4a4(a_codes, a_scales, U, s_a, w_codes, w_scales, l2t, s_w, bias, M, N, K, rank,
-                     epilogue, gelu_col_begin, Y, stream=None):
+def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue, gelu_col_begin, Y,
+                     stream=None):
     """Enqueues the W4A4 GEMM.  Y: bf16 CUDA [M, ldy]."""
     import torch
     _check("svdq_linear_w4a4", load().svdq_linear_w4a4(
-        _dptr(a_codes, "a_codes", torch.uint8), _dptr(a_scales, "a_scales", torch.uint8),
-        _dptr(U, "U", allow_none=rank == 0), _dptr(s_a, "s_a", torch.float32),
-        _dptr(w_codes, "w_codes", torch.uint8), _dptr(w_scales, "w_scales", torch.uint8),
+        _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U", allow_none=rank == 0),
+        _dptr(s_a, "s_a", torch.float32), _dptr(w_bundle, "w_bundle", torch.uint8),
         _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
         _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue, gelu_col_begin,
         _dptr(Y, "Y", torch.bfloat16), Y.stride(0), _stream(stream)))

@@ -34,18 +34,23 @@
  *
  * Packed layouts (all produced by this library; documented so callers can
  * move them around as opaque bytes):
- *   codes   NVFP4 element codes, row-major [rows][K/2] bytes; element 2j of a
- *           row is the low nibble of byte j, element 2j+1 the high nibble.
- *           Code = sign bit 3 | e2m1 magnitude code 0..7.
- *   scales  ue4m3 block scales in the tcgen05 scale-factor tile order:
- *           rows padded to a multiple of 128, K/16 scales per row grouped in
- *           atoms of 128 rows x 4 scales (512 bytes).  Scale (row m, block kb)
- *           lives at byte
- *             ((m/128)*(K/64) + kb/4)*512 + (m%32)*16 + ((m%128)/32)*4 + kb%4.
- *           Scales of padding rows are 0.
- *   L1T     low-rank down-projection, transposed: [rank][K] bf16.
- *   U, L2T  low-rank activations [M][64] and up-projection [N][64] bf16, row
- *           stride fixed at SVDQ_LR_STRIDE (64) elements; columns >= rank are 0.
+ *   bundle  NVFP4 operand (e2m1 codes + ue4m3 block scales), cut into tiles
+ *           of TH rows x 256 K-elements (TH = 128 for activations, 256 for
+ *           weights).  Tile (tr, ks) starts at (tr * ceil(K/256) + ks) * TH*144
+ *           bytes and holds TH rows x 128 bytes of codes (element k of row r in
+ *           byte k/2 of the row, low nibble for even k; code = sign bit 3 |
+ *           e2m1 magnitude 0..7; the 16-byte chunks of a row permuted by the
+ *           128-byte swizzle: chunk c of row r at r*128 + ((c ^ (r%8)) * 16)),
+ *           then TH/128 x 4 atoms of 512 bytes of block scales (scale of row r,
+ *           16-block j of the tile at TH*128 + (r/128)*2048 + (j/4)*512 +
+ *           (r%32)*16 + ((r%128)/32)*4 + j%4).  Rows past the matrix and
+ *           elements past K are zero.  Each tile is the shared-memory image of
+ *           one GEMM pipeline stage, so a stage is one contiguous copy.
+ *   L1T     low-rank down-projection, transposed: [rank][K] bf16, row-major.
+ *   U, L2T  low-rank activations (M rows) and up-projection (N rows) as tiles
+ *           of TH rows x 64 bf16 (TH = 128 for U, 256 for L2T), 128-byte rows
+ *           with the 128-byte swizzle: element (m, j) at (m/TH)*TH*128 +
+ *           (m%TH)*128 + (((j/8) ^ (m%8)) * 16) + (j%8)*2; columns >= rank are 0.
  *   AWQ     qweight: N*K/8 uint32 words in the fragment order of the W4A16
  *           kernel's tensor-core tiles.  Columns go in blocks of 16 and K in
  *           groups of 64; block b, group G owns words [(b*(K/64)+G)*128, +128):
@@ -110,15 +115,15 @@ int svdq_init(int device);
 /*
  * Byte sizes of the packed buffers of one SVDQ layer (host, no GPU).
  * Rules: K % 64 == 0, N % 8 == 0, 0 <= rank <= 64, rank % 16 == 0.
- *   inv_lambda [K] f32, L1T [rank][K] bf16, L2T [N][64] bf16,
- *   w_codes [N][K/2] u8, w_scales (tile order, rows padded to 128) u8.
+ *   inv_lambda [K] f32, L1T [rank][K] bf16, L2T (256-row tiles),
+ *   w_bundle (256-row tiles).
  */
 int svdq_weight_sizes(int K, int N, int rank, size_t *inv_lambda_bytes, size_t *l1t_bytes,
-                      size_t *l2t_bytes, size_t *w_codes_bytes, size_t *w_scales_bytes);
+                      size_t *l2t_bytes, size_t *w_bundle_bytes);
 
-/* Byte sizes of the activation-side buffers: codes [M][K/2], scales (tile
- * order, rows padded to 128), U [M][64] bf16.  Rules: M >= 1, K % 64 == 0. */
-int svdq_act_sizes(int M, int K, size_t *codes_bytes, size_t *scales_bytes, size_t *u_bytes);
+/* Byte sizes of the activation-side buffers: a_bundle (128-row tiles) and U
+ * (128-row tiles).  Rules: M >= 1, K % 64 == 0. */
+int svdq_act_sizes(int M, int K, size_t *a_bundle_bytes, size_t *u_bytes);
 
 /*
  * Offline quantization of one layer on the host (the pages' quantize step:
@@ -136,8 +141,9 @@ int svdq_act_sizes(int M, int K, size_t *codes_bytes, size_t *scales_bytes, size
  *   inv_lambda [K]  f32(1 / lambda_j), lambda_j = sqrt(absmaxX_j / absmaxW_j)
  *                   (1 when either is 0);
  *   l1t        [rank][K] bf16 = (U_r Sigma_r)^T of W' = W / inv_lambda;
- *   l2t        [N][64] bf16 = V_r (the rows of V_r^T, transposed), zero-padded;
- *   w_codes, w_scales: NVFP4 of R = W' - L1 L2 (f32-rounded), blocks along K;
+ *   l2t        V_r (rows of V_r^T, transposed) as 256-row low-rank tiles;
+ *   w_bundle   NVFP4 of R = W' - L1 L2 (f32-rounded), blocks along K, as a
+ *              256-row bundle (output column n = row n);
  *   s_w        fp32 tensor scale of R: f32(max|R|) / 2688 (1 if R == 0);
  *   s_a        static activation tensor scale:
  *              max_j f32(absmaxX_j * inv_lambda_j) / 2688.
@@ -147,16 +153,15 @@ int svdq_act_sizes(int M, int K, size_t *codes_bytes, size_t *scales_bytes, size
  */
 int svdq_pack_weights(const uint16_t *W, int K, int N, const float *act_absmax, int rank,
                       int num_threads, uint64_t seed, float *inv_lambda, uint16_t *l1t,
-                      uint16_t *l2t, uint8_t *w_codes, uint8_t *w_scales, float *s_w, float *s_a,
-                      float *residual);
+                      uint8_t *l2t, uint8_t *w_bundle, float *s_w, float *s_a, float *residual);
 
 /*
  * NVFP4 quantization of a host float32 matrix T [rows][K] (host, no GPU),
- * blocks of 16 along K under tensor scale s_t, into the packed codes and
- * tile-order scales above.  Used by the pack; exposed for tooling and tests.
+ * blocks of 16 along K under tensor scale s_t, into a bundle of tile height
+ * tile_rows (128 or 256; bundle_bytes from the layout above).  Used by the
+ * pack; exposed for tooling and tests.
  */
-int svdq_quantize_host(const float *T, int rows, int K, float s_t, uint8_t *codes,
-                       uint8_t *scales);
+int svdq_quantize_host(const float *T, int rows, int K, float s_t, int tile_rows, uint8_t *bundle);
 
 /*
  * Activation side of one SVDQ layer (the first fused kernel on the pages:
@@ -168,12 +173,13 @@ int svdq_quantize_host(const float *T, int rows, int K, float s_t, uint8_t *code
  *   U[m][j] = bf16( sum_k bf16(x^[m][k]) * L1T[j][k] / f32(s_a * s_w) )
  * Args: X [M][ldx] bf16 (device), ldx >= K; inv_lambda [K] f32; l1t
  * [rank][K] bf16 (ignored when rank == 0); s_a, s_w device scalars (f32);
- * outputs codes, scales, U as laid out above (U columns rank..63 are zeroed).
+ * outputs a_bundle (128-row bundle, padding rows and columns written as 0)
+ * and U (128-row low-rank tiles, columns rank..63 and padding rows 0).
  * Rules: K % 64 == 0, ldx % 8 == 0, 0 <= rank <= 64, rank % 16 == 0, M >= 1.
  */
 int svdq_quantize_act(const void *X, int M, int K, int ldx, const float *inv_lambda,
                       const void *l1t, int rank, const float *s_a, const float *s_w,
-                      uint8_t *codes, uint8_t *scales, void *U, svdq_stream_t stream);
+                      uint8_t *a_bundle, void *U, svdq_stream_t stream);
 
 /*
  * The W4A4 GEMM with the low-rank up-projection fused in (the second fused
@@ -182,17 +188,16 @@ int svdq_quantize_act(const void *X, int M, int K, int ldx, const float *inv_lam
  *   Y   = bf16( epilogue( f32(s_a s_w) * acc + bias ) )
  * epilogue: svdq_epilogue; GELU applies to output columns >= gelu_col_begin
  * only (a fused QKV + MLP-in projection activates just its MLP part).
- * Args: activation codes/scales/U from svdq_quantize_act; weight codes,
- * scales, L2T and scalars from svdq_pack_weights (uploaded); bias [N] bf16 or
- * NULL; Y [M][ldy] bf16, ldy >= N.
+ * Args: a_bundle and U from svdq_quantize_act; w_bundle, L2T and the
+ * scalars from svdq_pack_weights (uploaded); bias [N] bf16 or NULL;
+ * Y [M][ldy] bf16, ldy >= N.
  * Rules: K % 64 == 0, N % 8 == 0, ldy % 8 == 0, 0 <= rank <= 64,
  * rank % 16 == 0, M >= 1, 0 <= gelu_col_begin <= N.
  */
-int svdq_linear_w4a4(const uint8_t *a_codes, const uint8_t *a_scales, const void *U,
-                     const float *s_a, const uint8_t *w_codes, const uint8_t *w_scales,
-                     const void *l2t, const float *s_w, const void *bias, int M, int N, int K,
-                     int rank, int epilogue, int gelu_col_begin, void *Y, int ldy,
-                     svdq_stream_t stream);
+int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const float *s_a,
+                     const uint8_t *w_bundle, const void *l2t, const float *s_w, const void *bias,
+                     int M, int N, int K, int rank, int epilogue, int gelu_col_begin, void *Y,
+                     int ldy, svdq_stream_t stream);
 
 /*
  * Offline AWQ quantization on the host (asymmetric INT4 per group along K):

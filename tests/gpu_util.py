@@ -81,14 +81,11 @@ def weights_dev(p, rank):
     """An oracle SVDQ pack (oracle.svdquant.pack) in the library's device layout."""
     k = p["inv_lambda"].shape[0]
     n = p["w_codes"].shape[0]
-    l2t = np.zeros((n, lib.LR_STRIDE), np.uint16)
-    l2t[:, :rank] = L.bf16_bits(p["l2"].T)
     return dict(
         inv_lambda=dev(p["inv_lambda"]),
         l1t=bf16_dev(L.bf16_bits(p["l1"].T)) if rank else None,
-        l2t=bf16_dev(l2t),
-        w_codes=dev(L.pack_codes(p["w_codes"])),
-        w_scales=dev(L.tile_scales(p["w_sf"], n, k)),
+        l2t=dev(L.lowrank_pack(L.bf16_bits(p["l2"].T), 256)),
+        w_bundle=dev(L.bundle_pack(p["w_codes"], p["w_sf"], n, k, 256)),
         s_w=dev(np.array([p["s_w"]], np.float32)),
         s_a=dev(np.array([p["s_a"]], np.float32)),
     )
@@ -102,24 +99,27 @@ def run_k1(xb, m, k, rank, d, ldx=None):
         Xp[:, :k] = X
         X = Xp[:, :k]
     sz = lib.svdq_act_sizes(m, k)
-    codes = poisoned_u8(m, k // 2)
-    scales = poisoned_u8(sz["scales"])
-    U = poisoned_bf16(m, lib.LR_STRIDE)
-    lib.svdq_quantize_act(X, d["inv_lambda"], d["l1t"], rank, d["s_a"], d["s_w"], codes, scales, U, M=m, K=k)
+    bundle = poisoned_u8(sz["a_bundle"])
+    U = poisoned_u8(sz["u"])
+    lib.svdq_quantize_act(X, d["inv_lambda"], d["l1t"], rank, d["s_a"], d["s_w"], bundle, U, M=m, K=k)
     check_ok()
-    return codes, scales, U
+    return bundle, U
 
 
 def run_k2(oc, osf, ou, d, bias_bits, m, n, k, rank, epilogue, begin, ldy=None):
     """K2 on the oracle's activation operands (codes, scales, bf16-valued U/alpha)."""
-    U = np.zeros((m, lib.LR_STRIDE), np.uint16)
-    U[:, :rank] = L.bf16_bits(ou)
+    U = L.lowrank_pack(L.bf16_bits(ou), 128)
     ldy = n if ldy is None else ldy
     Yfull = poisoned_bf16(m, ldy)
     Y = Yfull[:, :n]
-    lib.svdq_linear_w4a4(dev(L.pack_codes(oc)), dev(L.tile_scales(osf, m, k)), bf16_dev(U), d["s_a"],
-                         d["w_codes"], d["w_scales"], d["l2t"], d["s_w"],
-                         bf16_dev(bias_bits) if bias_bits is not None else None,
+    lib.svdq_linear_w4a4(dev(L.bundle_pack(oc, osf, m, k, 128)), dev(U), d["s_a"], d["w_bundle"], d["l2t"],
+                         d["s_w"], bf16_dev(bias_bits) if bias_bits is not None else None,
                          m, n, k, rank, epilogue, begin, Y)
     check_ok()
     return Y, Yfull
+
+
+def unpack_act(bundle, U, m, k):
+    """GPU activation outputs -> (codes [m, k], scales [m, k/16], U bf16 bits [m, 64])."""
+    codes, sf = L.bundle_unpack(u8(bundle), m, k, 128)
+    return codes, sf, L.lowrank_unpack(u8(U), m, 128)

@@ -7,34 +7,90 @@ codes [rows, K] (0..15), scales [rows, K/16] (ue4m3 patterns), AWQ q [K, N].
 import numpy as np
 
 
-def unpack_codes(packed, K):
-    """[rows, K/2] bytes -> [rows, K] codes; element 2j = low nibble of byte j."""
-    p = np.asarray(packed, dtype=np.uint8).reshape(-1, K // 2)
-    out = np.empty((p.shape[0], K), dtype=np.uint8)
-    out[:, 0::2] = p & 0x0F
-    out[:, 1::2] = p >> 4
-    return out
+def _ks(K):
+    return (K + 255) // 256
 
 
-def scale_index(rows, K):
-    """Byte offset of scale (m, kb) for all m < rows, kb < K/16 (tile order)."""
+def bundle_size(rows, K, th):
+    return ((rows + th - 1) // th) * _ks(K) * th * 144
+
+
+def _tile(m, k, K, th):
+    return ((m // th) * _ks(K) + k // 256) * th * 144
+
+
+def code_index(rows, K, th):
+    """Byte offsets of the code bytes (elements 2j, 2j+1) of rows x K/2, in bundle order."""
     m = np.arange(rows)[:, None]
-    kb = np.arange(K // 16)[None, :]
-    return ((m // 128) * (K // 64) + kb // 4) * 512 + (m % 32) * 16 + ((m % 128) // 32) * 4 + kb % 4
+    k = np.arange(0, K, 2)[None, :]
+    r = m % th
+    kb = (k % 256) // 2
+    return _tile(m, k, K, th) + r * 128 + ((((kb >> 4) ^ r) & 7) << 4) + (kb & 15)
 
 
-def untile_scales(buf, rows, K):
+def scale_index(rows, K, th):
+    """Byte offsets of the block scales of rows x K/16, in bundle order."""
+    m = np.arange(rows)[:, None]
+    k = np.arange(0, K, 16)[None, :]
+    r = m % th
+    j = (k % 256) // 16
+    return (_tile(m, k, K, th) + th * 128 + (r // 128) * 2048 + (j // 4) * 512 + (r % 32) * 16
+            + ((r % 128) // 32) * 4 + j % 4)
+
+
+def bundle_unpack(buf, rows, K, th):
+    """Bundle bytes -> (codes [rows, K] 0..15, scales [rows, K/16] ue4m3 patterns)."""
     buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
-    return buf[scale_index(rows, K)]
+    cb = buf[code_index(rows, K, th)]
+    codes = np.empty((rows, K), dtype=np.uint8)
+    codes[:, 0::2] = cb & 0x0F
+    codes[:, 1::2] = cb >> 4
+    return codes, buf[scale_index(rows, K, th)]
 
 
-def padding_scales(buf, rows, K):
-    """Scales of the rows between `rows` and the next multiple of 128."""
-    pad = (rows + 127) // 128 * 128
-    if pad == rows:
-        return np.zeros((0, K // 16), np.uint8)
-    idx = scale_index(pad, K)[rows:]
-    return np.asarray(buf, dtype=np.uint8).reshape(-1)[idx]
+def bundle_pack(codes, scales, rows, K, th):
+    """(codes [rows, K], scales [rows, K/16]) -> bundle bytes; padding stays zero."""
+    buf = np.zeros(bundle_size(rows, K, th), dtype=np.uint8)
+    c = np.asarray(codes, dtype=np.uint8)
+    buf[code_index(rows, K, th)] = c[:, 0::2] | (c[:, 1::2] << 4)
+    buf[scale_index(rows, K, th)] = np.asarray(scales, dtype=np.uint8)
+    return buf
+
+
+def bundle_padding_is_zero(buf, rows, K, th):
+    buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    used = np.zeros(buf.size, dtype=bool)
+    used[code_index(rows, K, th)] = True
+    used[scale_index(rows, K, th)] = True
+    return not buf[~used].any()
+
+
+def lowrank_index(rows, th):
+    """Byte offsets of element (m, j), j < 64, of a low-rank tile buffer (bf16, 2 bytes)."""
+    m = np.arange(rows)[:, None]
+    j = np.arange(64)[None, :]
+    r = m % th
+    return (m // th) * th * 128 + r * 128 + ((((j >> 3) ^ r) & 7) << 4) + (j & 7) * 2
+
+
+def lowrank_unpack(buf, rows, th):
+    """Low-rank tile bytes -> bf16 bit patterns [rows, 64] (uint16)."""
+    b = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    idx = lowrank_index(rows, th)
+    return (b[idx].astype(np.uint16) | (b[idx + 1].astype(np.uint16) << 8))
+
+
+def lowrank_pack(bits, th):
+    """bf16 bit patterns [rows, r<=64] -> low-rank tile bytes (columns r.. zero)."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    rows, r = bits.shape
+    full = np.zeros((rows, 64), dtype=np.uint16)
+    full[:, :r] = bits
+    buf = np.zeros(((rows + th - 1) // th) * th * 128, dtype=np.uint8)
+    idx = lowrank_index(rows, th)
+    buf[idx] = (full & 0xFF).astype(np.uint8)
+    buf[idx + 1] = (full >> 8).astype(np.uint8)
+    return buf
 
 
 def awq_unpack(qweight, K, N):
@@ -63,20 +119,6 @@ def bf16_bits_to_f64(bits):
 # ---------------------------------------------------------------- writers
 # (the inverse direction: oracle arrays -> the library's packed layouts, so a
 # kernel can be run on operands that the oracle produced)
-
-def pack_codes(codes):
-    """[rows, K] codes -> [rows, K/2] bytes (element 2j in the low nibble)."""
-    c = np.asarray(codes, dtype=np.uint8)
-    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
-
-
-def tile_scales(sf, rows, K):
-    """[rows, K/16] scales -> tile-order buffer with rows padded to 128 (pad = 0)."""
-    pad = (rows + 127) // 128 * 128
-    buf = np.zeros(pad * (K // 16), dtype=np.uint8)
-    buf[scale_index(rows, K)] = np.asarray(sf, dtype=np.uint8)
-    return buf
-
 
 def awq_pack(q):
     """q [K, N] (0..15) -> fragment-order words (the inverse of awq_unpack)."""

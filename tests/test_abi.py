@@ -36,11 +36,11 @@ def test_status_strings():
 
 def test_sizes():
     s = lib.svdq_weight_sizes(3072, 9216, 32)
-    assert s["w_codes"] == 9216 * 1536
-    assert s["w_scales"] == 9216 * 192
+    assert s["w_bundle"] == 9216 * 1536 + 9216 * 192       # codes + scales, 256-row tiles fit exactly
     assert s["l1t"] == 32 * 3072 * 2 and s["l2t"] == 9216 * 64 * 2
-    a = lib.svdq_act_sizes(200, 256)
-    assert a["codes"] == 200 * 128 and a["scales"] == 256 * 16 and a["u"] == 200 * 128
+    a = lib.svdq_act_sizes(200, 320)
+    assert a["a_bundle"] == 2 * 2 * 128 * 144                # rows padded to 256, K to 512
+    assert a["u"] == 256 * 128
     with pytest.raises(lib.SvdqError) as e:
         lib.svdq_weight_sizes(100, 256, 16)
     assert e.value.status == lib.ERR_SHAPE
@@ -52,18 +52,18 @@ def test_sizes():
 def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
     so = lib.load()
     null = ctypes.c_void_p(0)
-    rc = so.svdq_quantize_act(null, 64, 256, 256, null, null, 16, null, null, null, null, null, null)
+    rc = so.svdq_quantize_act(null, 64, 256, 256, null, null, 16, null, null, null, null, null)
     assert rc == lib.ERR_INVALID_ARG
     p = ctypes.c_void_p(16)  # never dereferenced: the shape check fails first
-    rc = so.svdq_linear_w4a4(p, p, p, p, p, p, p, p, None, 64, 256, 100, 16, 0, 0, p, 256, None)
+    rc = so.svdq_linear_w4a4(p, p, p, p, p, p, None, 64, 256, 100, 16, 0, 0, p, 256, None)
     assert rc == lib.ERR_SHAPE
     assert b"K % 64" in so.svdq_last_error_string()
-    rc = so.svdq_linear_w4a4(p, p, p, p, p, p, p, p, None, 64, 256, 256, 16, 7, 0, p, 256, None)
+    rc = so.svdq_linear_w4a4(p, p, p, p, p, p, None, 64, 256, 256, 16, 7, 0, p, 256, None)
     assert rc == lib.ERR_INVALID_ARG
     rc = so.awq_linear_w4a16(p, 17, 256, 256, None, p, p, p, 64, None, 256, p, 256, None)
     assert rc == lib.ERR_SHAPE
     odd = ctypes.c_void_p(24)
-    rc = so.svdq_linear_w4a4(odd, p, p, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None)
+    rc = so.svdq_linear_w4a4(odd, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None)
     assert rc == lib.ERR_ALIGNMENT
 
 

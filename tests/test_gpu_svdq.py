@@ -49,21 +49,21 @@ _run_k1 = G.run_k1
 _run_k2 = G.run_k2
 
 
-def _check_k1(x, p, rank, codes, scales, U, rows=None):
+def _check_k1(x, p, rank, bundle, U, rows=None):
     M, k = x.shape
     xs = x if rows is None else x[rows]
     oc, osf, ou = svdquant.quantize_act(xs, p["inv_lambda"], p["l1"], p["s_a"], p["s_w"])
-    gc = L.unpack_codes(G.u8(codes), k)
-    gsf = L.untile_scales(G.u8(scales), M, k)
-    gu = G.bf16_host(U)
+    gc, gsf, gubits = G.unpack_act(bundle, U, M, k)
     if rows is not None:
-        gc, gsf, gu = gc[rows], gsf[rows], gu[rows]
+        gc, gsf, gubits = gc[rows], gsf[rows], gubits[rows]
     np.testing.assert_array_equal(gc, oc)
     np.testing.assert_array_equal(gsf, osf)
-    assert (L.padding_scales(G.u8(scales), M, k) == 0).all()
-    assert (gu[:, rank:] == 0).all()
+    assert L.bundle_padding_is_zero(G.u8(bundle), M, k, 128)
+    assert (gubits[:, rank:] == 0).all()
+    pad = L.lowrank_unpack(G.u8(U), (M + 127) // 128 * 128, 128)[M:]
+    assert (pad == 0).all()
     if rank:
-        assert G.excess_error(gu[:, :rank], ou) <= TOL
+        assert G.excess_error(L.bf16_bits_to_f64(gubits[:, :rank]), ou) <= TOL
 
 
 K1_CASES = [
@@ -81,15 +81,15 @@ K1_CASES = [
 def test_quantize_act_parity(case):
     m, k, n, rank = case[:4]
     xb, x, bb, p = _case(*case)
-    codes, scales, U = _run_k1(xb, m, k, rank, _weights_dev(p, rank))
-    _check_k1(x, p, rank, codes, scales, U)
+    bundle, U = _run_k1(xb, m, k, rank, _weights_dev(p, rank))
+    _check_k1(x, p, rank, bundle, U)
 
 
 def test_quantize_act_strided_rows():
     case = (100, 256, 64, 16, 10, 2, 30.0, 0, 1.0)
     xb, x, bb, p = _case(*case)
-    codes, scales, U = _run_k1(xb, 100, 256, 16, _weights_dev(p, 16), ldx=264)
-    _check_k1(x, p, 16, codes, scales, U)
+    bundle, U = _run_k1(xb, 100, 256, 16, _weights_dev(p, 16), ldx=264)
+    _check_k1(x, p, 16, bundle, U)
 
 
 def _oracle_operands(x, p, rank, rows=None):
@@ -159,9 +159,9 @@ def test_full_size_qkv_sampled():
     c = synthetic.QKV
     xb, x, bb, p = _full_case(c)
     d = _weights_dev(p, c.rank)
-    codes, scales, U = _run_k1(xb, c.m, c.k, c.rank, d)
+    bundle, U = _run_k1(xb, c.m, c.k, c.rank, d)
     rows = _sample_rows(c.m)
-    _check_k1(x, p, c.rank, codes, scales, U, rows=rows)
+    _check_k1(x, p, c.rank, bundle, U, rows=rows)
 
     oc, osf, ou = _oracle_operands(x, p, c.rank)
     Y, _ = _run_k2(oc, osf, ou, d, bb, c.m, c.n, c.k, c.rank, 0, 0)
@@ -170,8 +170,8 @@ def test_full_size_qkv_sampled():
     assert G.excess_error(G.bf16_host(Y)[rows], want) <= TOL
 
     Y2 = G.poisoned_bf16(c.m, c.n)
-    lib.svdq_linear_w4a4(codes, scales, U, d["s_a"], d["w_codes"], d["w_scales"], d["l2t"], d["s_w"],
-                         G.bf16_dev(bb), c.m, c.n, c.k, c.rank, 0, 0, Y2)
+    lib.svdq_linear_w4a4(bundle, U, d["s_a"], d["w_bundle"], d["l2t"], d["s_w"], G.bf16_dev(bb),
+                         c.m, c.n, c.k, c.rank, 0, 0, Y2)
     G.check_ok()
     assert G.excess_error(G.bf16_host(Y2)[rows], want) <= TOL   # the GPU's own K1 -> K2 chain
 
@@ -187,10 +187,10 @@ def test_full_size_mlp_pair_sampled():
     d1 = _weights_dev(p1, c1.rank)
     rows = _sample_rows(c1.m, 96, seed=1)
     # fc1 through the GPU's own chain, compared with the oracle's layer
-    codes, scales, U = _run_k1(xb, c1.m, c1.k, c1.rank, d1)
+    bundle, U = _run_k1(xb, c1.m, c1.k, c1.rank, d1)
     H = G.poisoned_bf16(c1.m, c1.n)
-    lib.svdq_linear_w4a4(codes, scales, U, d1["s_a"], d1["w_codes"], d1["w_scales"], d1["l2t"], d1["s_w"],
-                         G.bf16_dev(bb1), c1.m, c1.n, c1.k, c1.rank, lib.EPILOGUE_GELU_ERF, 0, H)
+    lib.svdq_linear_w4a4(bundle, U, d1["s_a"], d1["w_bundle"], d1["l2t"], d1["s_w"], G.bf16_dev(bb1),
+                         c1.m, c1.n, c1.k, c1.rank, lib.EPILOGUE_GELU_ERF, 0, H)
     G.check_ok()
     oc1, osf1, ou1 = _oracle_operands(x, p1, c1.rank)
     h_oracle = _want_k2(oc1, osf1, ou1, p1, bb1, lib.EPILOGUE_GELU_ERF, 0)
@@ -202,11 +202,11 @@ def test_full_size_mlp_pair_sampled():
     bb2 = synthetic.bias(c2.n, c2.seed + 100)
     p2 = svdquant.pack(formats.bf16_bits_to_float(wb2), np.max(np.abs(h), axis=0).astype(np.float32), c2.rank)
     d2 = _weights_dev(p2, c2.rank)
-    codes2, scales2, U2 = _run_k1(hb, c2.m, c2.k, c2.rank, d2)
-    _check_k1(h, p2, c2.rank, codes2, scales2, U2, rows=rows)
+    bundle2, U2 = _run_k1(hb, c2.m, c2.k, c2.rank, d2)
+    _check_k1(h, p2, c2.rank, bundle2, U2, rows=rows)
     Y = G.poisoned_bf16(c2.m, c2.n)
-    lib.svdq_linear_w4a4(codes2, scales2, U2, d2["s_a"], d2["w_codes"], d2["w_scales"], d2["l2t"], d2["s_w"],
-                         G.bf16_dev(bb2), c2.m, c2.n, c2.k, c2.rank, 0, 0, Y)
+    lib.svdq_linear_w4a4(bundle2, U2, d2["s_a"], d2["w_bundle"], d2["l2t"], d2["s_w"], G.bf16_dev(bb2),
+                         c2.m, c2.n, c2.k, c2.rank, 0, 0, Y)
     G.check_ok()
     oc2, osf2, ou2 = _oracle_operands(h, p2, c2.rank, rows)
     want = _want_k2(oc2, osf2, ou2, p2, bb2, 0, 0)

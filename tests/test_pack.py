@@ -38,13 +38,15 @@ def test_pack_matches_oracle(k, n, rank):
     s_w = nvfp4.tensor_scale(np.max(np.abs(r32)))
     assert p["s_w"][0] == s_w
     codes, sf = nvfp4.quantize_blocks(r32.T, s_w)
-    np.testing.assert_array_equal(layouts.unpack_codes(p["w_codes"], k), codes)
-    np.testing.assert_array_equal(layouts.untile_scales(p["w_scales"], n, k), sf)
-    assert (layouts.padding_scales(p["w_scales"], n, k) == 0).all()
+    gc, gsf = layouts.bundle_unpack(p["w_bundle"], n, k, 256)
+    np.testing.assert_array_equal(gc, codes)
+    np.testing.assert_array_equal(gsf, sf)
+    assert layouts.bundle_padding_is_zero(p["w_bundle"], n, k, 256)
     # the residual is W' - L1 L2 with the pack's bf16 factors
     l1 = layouts.bf16_bits_to_f64(p["l1t"]).T
-    l2 = layouts.bf16_bits_to_f64(p["l2t"])[:, :rank].T
-    assert (p["l2t"][:, rank:] == 0).all()
+    l2bits = layouts.lowrank_unpack(p["l2t"], n, 256)
+    l2 = layouts.bf16_bits_to_f64(l2bits)[:, :rank].T
+    assert (l2bits[:, rank:] == 0).all()
     np.testing.assert_allclose(r32, (o["w_prime"] - l1 @ l2).astype(F32), rtol=0, atol=1e-6)
     # L1 L2 itself is not compared with the oracle's: with a nearly flat tail
     # of the spectrum the top-r subspace is not unique (see the Eckart-Young
@@ -81,13 +83,40 @@ def test_host_quantizer_matches_oracle_bit_exactly():
     t[3, :16] = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -5, -0.25, 0, -0.0, 4, 3, 2, 1], F32)
     t[5, 16:32] = 0.0
     s_t = nvfp4.tensor_scale(np.max(np.abs(t)))
-    codes, sf = lib.svdq_quantize_host(t, s_t)
     oc, osf = nvfp4.quantize_blocks(t, s_t)
-    np.testing.assert_array_equal(layouts.unpack_codes(codes, 320), oc)
-    np.testing.assert_array_equal(layouts.untile_scales(sf, 70, 320), osf)
+    for th in (128, 256):
+        bundle = lib.svdq_quantize_host(t, s_t, th)
+        gc, gsf = layouts.bundle_unpack(bundle, 70, 320, th)
+        np.testing.assert_array_equal(gc, oc)
+        np.testing.assert_array_equal(gsf, osf)
+        assert layouts.bundle_padding_is_zero(bundle, 70, 320, th)
     oc1, osf1 = nvfp4.quantize_blocks(t[3:4], F32(1.0))
-    c1, sf1 = lib.svdq_quantize_host(t[3:4].copy(), 1.0)
-    np.testing.assert_array_equal(layouts.unpack_codes(c1, 320), oc1)
+    c1, _ = layouts.bundle_unpack(lib.svdq_quantize_host(t[3:4].copy(), 1.0), 1, 320, 128)
+    np.testing.assert_array_equal(c1, oc1)
+
+
+def test_bundle_layout_reader_round_trip():
+    """The test-side reader inverts a bundle written by hand from the header text."""
+    rng = np.random.default_rng(2)
+    rows, k, th = 130, 320, 128
+    codes = rng.integers(0, 16, (rows, k)).astype(np.uint8)
+    sf = rng.integers(0, 127, (rows, k // 16)).astype(np.uint8)
+    buf = np.zeros(((rows + th - 1) // th) * ((k + 255) // 256) * th * 144, np.uint8)
+    for m in range(rows):
+        for kk in range(0, k, 2):
+            tile = ((m // th) * ((k + 255) // 256) + kk // 256) * th * 144
+            r, byte = m % th, (kk % 256) // 2
+            buf[tile + r * 128 + (((byte // 16) ^ (r % 8)) * 16) + byte % 16] = codes[m, kk] | (codes[m, kk + 1] << 4)
+        for j16 in range(k // 16):
+            kk = j16 * 16
+            tile = ((m // th) * ((k + 255) // 256) + kk // 256) * th * 144
+            r, j = m % th, (kk % 256) // 16
+            buf[tile + th * 128 + (r // 128) * 2048 + (j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4
+                + j % 4] = sf[m, j16]
+    gc, gsf = layouts.bundle_unpack(buf, rows, k, th)
+    np.testing.assert_array_equal(gc, codes)
+    np.testing.assert_array_equal(gsf, sf)
+    np.testing.assert_array_equal(layouts.bundle_pack(codes, sf, rows, k, th), buf)
 
 
 @pytest.mark.parametrize("k,n", [(64, 16), (192, 48), (3072, 64)])

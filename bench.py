@@ -63,6 +63,33 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+# ------------------------------------------------------------------ replicas
+# The layer needs no exchange between GPUs, so N GPUs run N independent
+# replicas of the step.  The process group carries only the barriers around
+# the timed region and the max-over-ranks reduction of the timings.
+def init_replicas(world, backend, device=None, timeout_s=120):
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        kw = {"device_id": device} if backend == "nccl" else {}
+        dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s), **kw)
+
+
+def max_over_ranks(values, world, device="cpu"):
+    """Element-wise max over ranks of this rank's timings (every rank gets it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tflops(flops_per_replica_step, world, ms_per_step):
+    """Whole-job throughput: the work of all replicas over the slowest rank's step time."""
+    return flops_per_replica_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
@@ -174,9 +201,7 @@ def run_ours(args):
     rank, world, local = dist_env()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    init_replicas(world, "nccl", device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     sets = 4
     S, host, set_bytes = setup(device, sets)
@@ -236,10 +261,7 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1) / e_steps
 
     # ---- max over ranks
-    vals = torch.tensor([ms, k1, k2, k3, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms, k1, k2, k3, e2e_ms = vals.tolist()
+    ms, k1, k2, k3, e2e_ms = max_over_ranks([ms, k1, k2, k3, e2e_ms], world, device)
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -250,7 +272,7 @@ def run_ours(args):
     k2_tflops = (W4A4_FLOPS + 2 * M * RANK * N) / (k2 * 1e-3) / 1e12
     line = {
         "metric": METRIC,
-        "value": round(STEP_FLOPS * world / (ms_step * 1e-3) / 1e12, 2),
+        "value": round(aggregate_tflops(STEP_FLOPS, world, ms_step), 2),
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": args.steps,
@@ -277,7 +299,7 @@ def run_ours(args):
                              "frac_hbm": round(K3_BYTES / (k3 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
             "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how,
         },
-        "e2e": {"value": round(STEP_FLOPS * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "e2e": {"value": round(aggregate_tflops(STEP_FLOPS, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2 + AM * AK * 2, "d2h_bytes_per_step": M * N * 2 + AM * AN * 2},
         "gpu_launches": 3 * args.steps,
         "clocks": clk,

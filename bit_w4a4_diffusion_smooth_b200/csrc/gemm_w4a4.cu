@@ -3,7 +3,7 @@
 // The pages fuse the 16-bit low-rank up-projection into the 4-bit GEMM so the
 // correction branch does not eat the W4A4 gain (web page "Nunchaku Diffusers
 // 支持降低显存占用，但硬件仍决定适用范围", remio.ai, section "SVDQuant 将棘手数值移出
-// 4 位路径").  Per 128 x 256 output tile:
+// 4 位路径").  Per 256 x 256 output tile:
 //   acc  = U_tile . L2T_tile^T                 tcgen05.mma kind::f16 (bf16)
 //   acc += sum_k (qa sa)(qw sw)                tcgen05.mma kind::mxf4nvf4,
 //                                               block16 ue4m3 scales in TMEM
@@ -11,29 +11,40 @@
 // U arrives pre-divided by s_a s_w, so both branches share one fp32
 // accumulator and one scale in the epilogue.
 //
-// Structure (one CTA per SM, persistent over output tiles, 12 warps):
-//   warps 0, 3  producers: one bulk copy per stage each - the activation
-//               bundle tile (128 rows x 256 K: swizzled codes + block scales,
-//               18 KB) and the weight bundle tile (256 rows, 36 KB); at the
-//               start of a tile the U and L2T tiles of the low-rank branch
-//   warp 1      owns TMEM (512 columns), issues tcgen05.mma from one thread
-//   warp 2      moves each stage's block scales from shared memory into that
-//               stage's own TMEM columns (tcgen05.cp 32x128b.warpx4); issued
-//               from its own warp the copies overlap the MMAs, issued from
-//               the MMA thread they would serialize with them
-//   warps 4..11 epilogue: drain the 128 x 256 fp32 accumulator (each warp its
-//               32-lane quarter, 128 columns), hand TMEM back at once, then
-//               scale, add bias, GELU, round to bf16 into a 128-byte-swizzled
-//               staging tile and write it with TMA stores
-// Pipeline: 3 stages of 54 KB (the two bundle tiles, which are laid out in
-// memory exactly as the MMA reads them from shared memory); TMEM holds the
-// accumulator (256 columns) and 3 x 48 columns of block scales.
-// Every wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT, the
-// other roles see the abort flag, in-flight work is drained and TMEM freed.
+// SM pairs.  The kernel runs in clusters of two CTAs, one per SM of a TPC,
+// and every MMA is a cta_group::2 MMA of 256 x 256 x 64: CTA h of the pair
+// holds rows 128h..128h+127 of the activation tile and weight rows (output
+// columns) 128h..128h+127 of the weight tile, and its TMEM receives its own
+// 128 rows of the accumulator.  Each SM therefore loads 38 KB per k-stage
+// (its half of A and of B, plus the full 256-column block-scale slice that
+// both TMEMs need) instead of the 54 KB a one-SM 128 x 256 tile needs for the
+// same MMA time; the per-SM operand intake of the L2 fabric is what limits a
+// one-SM tile.
+//
+// Roles (one CTA per SM, persistent over pair tiles, 12 warps):
+//   warp 0      producer in both CTAs: per stage three TMA copies into its
+//               own shared memory (A half with its scales, B half, B scales),
+//               all completing on the even CTA's `full` barrier
+//   warp 1      owns TMEM (pair allocation); in the even CTA it issues the
+//               MMAs from one thread and commits each stage to both CTAs'
+//               `empty` barriers
+//   warp 2      even CTA: moves each stage's block scales from both CTAs'
+//               shared memory into their TMEM (tcgen05.cp, cta_group::2);
+//               from its own warp the copies overlap the MMAs
+//   warps 4..11 epilogue in both CTAs: drain the CTA's 128 x 256 fp32
+//               accumulator, hand TMEM back (to the even CTA's barrier),
+//               then scale, add bias, GELU, round to bf16 into a
+//               128-byte-swizzled staging tile and write it with TMA stores
+// Pipeline: 5 stages of 38 KB per CTA; TMEM holds the accumulator (256
+// columns) and 5 x 48 columns of block scales.
+// Every wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT and
+// raises the abort flag of both CTAs; in-flight work is drained, the pair
+// meets at a cluster barrier and frees TMEM.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 #include <string>
 
 #include "device_common.cuh"
@@ -42,15 +53,18 @@
 namespace svdq {
 namespace {
 
-constexpr int BM = 128, BN = 256;
-constexpr int STAGES = 3;
-constexpr int A_TILE = BM * 144;              // activation bundle tile: codes 16 KB + scales 2 KB
-constexpr int B_TILE = BN * 144;              // weight bundle tile: codes 32 KB + scales 4 KB
+constexpr int BM = 128;                       // rows per CTA (256 per pair)
+constexpr int BN = 256;                       // output columns per pair tile
+constexpr int STAGES = 5;
+constexpr int ROW = 2048;                     // bytes per row of the bundle tensor maps
+constexpr int A_BYTES = BM * 144;             // activation tile: codes 16 KB + scales 2 KB
 constexpr int SFA_OFF = BM * 128;
-constexpr int B_OFF = A_TILE;                 // 18432, a multiple of 1024
-constexpr int SFB_OFF = B_OFF + BN * 128;
-constexpr int STAGE_BYTES = A_TILE + B_TILE;  // 55296
-constexpr int U_TILE = BM * 128, L2_TILE = BN * 128;
+constexpr int B_OFF = A_BYTES;                // 18432, a multiple of 1024
+constexpr int B_BYTES = 128 * 128;            // this CTA's 128 weight rows of codes
+constexpr int SFB_OFF = B_OFF + B_BYTES;      // scales of all 256 weight rows
+constexpr int SFB_BYTES = 256 * 16;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFB_BYTES;  // 38912
+constexpr int LR_BYTES = 128 * 128;           // U (this CTA's rows) and L2T (its columns), 16 KB each
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_TILE_BYTES = 32 * 128;      // 32 rows x 64 bf16, 128-byte swizzle
 constexpr int EPI_OFF = STAGES * STAGE_BYTES;
@@ -59,25 +73,32 @@ constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
 constexpr int THREADS = (4 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 256;              // stage s: SFA at +48s (+4 kb), SFB at +48s+16 (+8 kb, +4 per row block)
+static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "MMA operand tiles start on 1024-byte boundaries");
+static_assert(A_BYTES % ROW == 0 && B_BYTES % ROW == 0 && SFB_BYTES % ROW == 0 && LR_BYTES % ROW == 0,
+              "copies are whole tensor-map rows");
+static_assert(SF_COL + 48 * STAGES <= TMEM_COLS, "scale columns fit in TMEM");
 
 // Instruction descriptors (tcgen05 instruction-descriptor bit fields):
 // [4,6) accumulator format (1 = f32), [7,10) A format, [10,13) B format,
-// [17,23) N >> 3, [24,29) M >> 4; block-scaled: [23] scale format
-// (0 = ue4m3), [29,31) / [4,6) scale-factor ids (0), A/B K-major (bits 15/16 = 0).
-constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
-constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((BM >> 4) << 24);
+// [17,23) N >> 3, [24,29) M >> 4 (M = 256: the pair); block-scaled: [23]
+// scale format (0 = ue4m3), scale-factor ids 0; A/B K-major (bits 15/16 = 0).
+constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((256 >> 4) << 24);
+constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((256 >> 4) << 24);
 
 __device__ __forceinline__ uint32_t sfa_col(int s, int kb) { return SF_COL + 48 * s + 4 * kb; }
 __device__ __forceinline__ uint32_t sfb_col(int s, int kb) { return SF_COL + 48 * s + 16 + 8 * kb; }
 
 struct Params {
-  int M, N, K, rank, epilogue, gelu_col_begin;
-  int num_m_blk, num_tiles, k_stages, lr_stages, kb_total;
-  const uint8_t *a_bundle, *w_bundle, *u, *l2t;
+  int M, N, rank, epilogue, gelu_col_begin;
+  int num_m2, num_tiles, k_stages, lr_stages, kb_total;
   const float *s_a, *s_w;
   const uint16_t *bias;
   unsigned int *status;
   unsigned long long limit_ns;
+};
+
+struct Maps {
+  CUtensorMap a, b, sfb, u, l2, y;
 };
 
 __device__ __forceinline__ float gelu_erf(float y) { return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f)); }
@@ -85,93 +106,109 @@ __device__ __forceinline__ float gelu_tanh(float y) {
   return 0.5f * y * (1.0f + tanhf(0.79788456080286536f * (y + 0.044715f * y * y * y)));
 }
 
-__device__ __forceinline__ void abort_all(volatile int *abort_flag, unsigned int *status) {
+// Raises the abort flag of this CTA and of its partner, records the timeout.
+__device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t peer_abort, unsigned int *status) {
   *abort_flag = 1;
+  dev::st_cluster_u32(peer_abort, 1u);
   dev::report(status, SVDQ_ERR_TIMEOUT);
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    gemm_w4a4_kernel(const __grid_constant__ CUtensorMap tm_y, Params p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    gemm_w4a4_kernel(const __grid_constant__ Maps maps, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);
-  uint64_t *sf_full = full + STAGES;
-  uint64_t *empty = sf_full + STAGES;
-  uint64_t *tmem_full = empty + STAGES;
-  uint64_t *tmem_empty = tmem_full + 1;
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);  // even CTA: both CTAs' bytes
+  uint64_t *sf_full = full + STAGES;                               // even CTA: scales in TMEM
+  uint64_t *empty = sf_full + STAGES;                              // both CTAs: stage free again
+  uint64_t *tmem_full = empty + STAGES;                            // both CTAs: accumulator ready
+  uint64_t *tmem_empty = tmem_full + 1;                            // even CTA: both CTAs drained it
   uint64_t *drain_mma = tmem_empty + 1;
   uint64_t *drain_cp = drain_mma + 1;
   uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(drain_cp + 1);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t h = dev::cluster_ctarank();         // 0: even CTA (issues the MMAs), 1: odd
+  const int pair = static_cast<int>(dev::cluster_id_x());
+  const int num_pairs = static_cast<int>(dev::num_clusters_x());
   const int stages_per_tile = p.lr_stages + p.k_stages;
+  const uint32_t peer_abort = dev::mapa(dev::smem_u32(const_cast<int *>(abort_flag)), h ^ 1u);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      dev::mbar_init(&full[s], 2);            // one arrival per producer warp
+      dev::mbar_init(&full[s], 1);            // the even CTA's producer arrival (+ the bytes of both CTAs)
       dev::mbar_init(&sf_full[s], 1);
       dev::mbar_init(&empty[s], 1);
     }
     dev::mbar_init(tmem_full, 1);
-    dev::mbar_init(tmem_empty, EPI_WARPS);
+    dev::mbar_init(tmem_empty, 2 * EPI_WARPS);
     dev::mbar_init(drain_mma, 1);
     dev::mbar_init(drain_cp, 1);
     *abort_flag = 0;
     dev::fence_mbar_init();
   }
   if (warp == 1) {
-    dev::tmem_alloc(tmem_base_slot, TMEM_COLS);
-    dev::tmem_relinquish();
+    dev::tmem_alloc_pair(tmem_base_slot, TMEM_COLS);
+    dev::tmem_relinquish_pair();
   }
   dev::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  dev::cluster_sync();                        // both CTAs' barriers exist before anyone arrives remotely
   dev::tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
 
-  if (warp == 0 || warp == 3) {
-    // ------------------------------------------------------------ producers (0: activations, 3: weights)
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
-      const bool act = warp == 0;
+      dev::prefetch_tmap(&maps.a);
+      dev::prefetch_tmap(&maps.b);
+      dev::prefetch_tmap(&maps.sfb);
+      if (p.lr_stages) {
+        dev::prefetch_tmap(&maps.u);
+        dev::prefetch_tmap(&maps.l2);
+      }
       int it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int m_blk = tile % p.num_m_blk, n_blk = tile / p.num_m_blk;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
+        const int m_blk = 2 * (tile % p.num_m2) + static_cast<int>(h);  // this CTA's 128-row block
+        const int n_blk = tile / p.num_m2;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
-          if (!dev::mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
+          if (!dev::mbar_wait_cluster(&empty[s], ((it / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
             ok = false;
             break;
           }
-          uint8_t *dst = smem + s * STAGE_BYTES + (act ? 0 : B_OFF);
-          const uint8_t *src;
-          uint32_t bytes;
+          const uint32_t bar = dev::mapa(dev::smem_u32(&full[s]), 0);
+          uint8_t *dst = smem + s * STAGE_BYTES;
           if (st < p.lr_stages) {
-            src = act ? p.u + static_cast<size_t>(m_blk) * U_TILE : p.l2t + static_cast<size_t>(n_blk) * L2_TILE;
-            bytes = act ? U_TILE : L2_TILE;
+            if (h == 0) dev::mbar_arrive_expect_tx(&full[s], 2u * 2u * LR_BYTES);
+            dev::tma_load_2d_pair(dst, &maps.u, bar, 0, m_blk * (LR_BYTES / ROW));
+            dev::tma_load_2d_pair(dst + B_OFF, &maps.l2, bar, 0, (2 * n_blk + static_cast<int>(h)) * (LR_BYTES / ROW));
           } else {
             const int ks = st - p.lr_stages;
-            src = act ? p.a_bundle + (static_cast<size_t>(m_blk) * p.k_stages + ks) * A_TILE
-                      : p.w_bundle + (static_cast<size_t>(n_blk) * p.k_stages + ks) * B_TILE;
-            bytes = act ? A_TILE : B_TILE;
+            const int wrow = (n_blk * p.k_stages + ks) * ((2 * B_BYTES + SFB_BYTES) / ROW);
+            if (h == 0) dev::mbar_arrive_expect_tx(&full[s], 2u * STAGE_BYTES);
+            dev::tma_load_2d_pair(dst, &maps.a, bar, 0, (m_blk * p.k_stages + ks) * (A_BYTES / ROW));
+            dev::tma_load_2d_pair(dst + B_OFF, &maps.b, bar, 0, wrow + static_cast<int>(h) * (B_BYTES / ROW));
+            dev::tma_load_2d_pair(dst + SFB_OFF, &maps.sfb, bar, 0, wrow + 2 * B_BYTES / ROW);
           }
-          dev::mbar_arrive_expect_tx(&full[s], bytes);
-          dev::bulk_load(dst, src, bytes, &full[s]);
         }
       }
-      if (!ok) {
-        abort_all(abort_flag, p.status);
-        for (int j = max(0, it - STAGES); j < it; ++j)  // let issued copies land
-          dev::mbar_wait(&full[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
+      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
+      // Before the pair may leave: the even CTA waits for every stage it
+      // armed to complete (that covers the odd CTA's copies as well).
+      if (h == 0) {
+        for (int j = max(0, it - STAGES); j < it; ++j)
+          dev::mbar_wait_cluster(&full[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (h == 0 && lane == 0) {
       int it = 0, tcount = 0;
       bool ok = true, issued_any = false;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
-        if (!dev::mbar_wait(tmem_empty, (tcount & 1) ^ 1, p.limit_ns, abort_flag)) {
+      for (int tile = pair; tile < p.num_tiles && ok; tile += num_pairs, ++tcount) {
+        if (!dev::mbar_wait_cluster(tmem_empty, (tcount & 1) ^ 1, p.limit_ns, abort_flag)) {
           ok = false;
           break;
         }
@@ -181,7 +218,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!dev::mbar_wait(&sf_full[s], ph, p.limit_ns, abort_flag) ||
-              !dev::mbar_wait(&full[s], ph, p.limit_ns, abort_flag)) {
+              !dev::mbar_wait_cluster(&full[s], ph, p.limit_ns, abort_flag)) {
             ok = false;
             break;
           }
@@ -190,41 +227,41 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sb = sa + B_OFF;
           if (st < p.lr_stages) {
             for (int j = 0; j < p.rank / 16; ++j) {  // K = 16 bf16 = 32 bytes per MMA
-              dev::umma_bf16(tmem, dev::desc_sw128(sa + 32 * j), dev::desc_sw128(sb + 32 * j), IDESC_BF16,
-                             accumulate);
+              dev::umma_bf16_pair(tmem, dev::desc_sw128(sa + 32 * j), dev::desc_sw128(sb + 32 * j), IDESC_BF16,
+                                  accumulate);
               accumulate = 1;
             }
           } else {
             const int nkb = min(4, p.kb_total - 4 * (st - p.lr_stages));
             for (int kb = 0; kb < nkb; ++kb) {  // K = 64 e2m1 = 32 bytes per MMA
-              dev::umma_nvfp4(tmem, dev::desc_sw128(sa + 32 * kb), dev::desc_sw128(sb + 32 * kb), IDESC_NVFP4,
-                              tmem + sfa_col(s, kb), tmem + sfb_col(s, kb), accumulate);
+              dev::umma_nvfp4_pair(tmem, dev::desc_sw128(sa + 32 * kb), dev::desc_sw128(sb + 32 * kb), IDESC_NVFP4,
+                                   tmem + sfa_col(s, kb), tmem + sfb_col(s, kb), accumulate);
               accumulate = 1;
             }
           }
           issued_any = true;
-          dev::tc_commit(&empty[s]);  // stage s (shared memory and TMEM scales) free once these MMAs finish
+          dev::tc_commit_pair_mc(&empty[s], 0x3);  // both CTAs' stage s free once these MMAs finish
         }
         if (!ok) break;
-        dev::tc_commit(tmem_full);    // accumulator ready for the epilogue
+        dev::tc_commit_pair_mc(tmem_full, 0x3);    // both halves of the accumulator ready
       }
-      if (!ok) abort_all(abort_flag, p.status);
-      if (issued_any) {  // the tensor core must be idle before TMEM is freed
-        dev::tc_commit(drain_mma);
+      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
+      if (issued_any) {  // the tensor cores must be idle before TMEM is freed
+        dev::tc_commit_pair(drain_mma);
         dev::mbar_wait(drain_mma, 0, p.limit_ns, nullptr);
       }
     }
   } else if (warp == 2) {
-    // ------------------------------------------------------------ scale-factor copies
-    if (lane == 0) {
+    // ------------------------------------------------------------ scale-factor copies (even CTA)
+    if (h == 0 && lane == 0) {
       int it = 0;
       bool ok = true, issued_any = false;
-      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-        const int n_blk = tile / p.num_m_blk;
+      for (int tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
+        const int n_blk = tile / p.num_m2;
         const bool b1_ok = (n_blk * 2 + 1) * 128 < p.N;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
-          if (!dev::mbar_wait(&full[s], (it / STAGES) & 1, p.limit_ns, abort_flag)) {
+          if (!dev::mbar_wait_cluster(&full[s], (it / STAGES) & 1, p.limit_ns, abort_flag)) {
             ok = false;
             break;
           }
@@ -233,33 +270,35 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t ssfa = dev::smem_u32(smem + s * STAGE_BYTES + SFA_OFF);
             const uint32_t ssfb = dev::smem_u32(smem + s * STAGE_BYTES + SFB_OFF);
             for (int kb = 0; kb < nkb; ++kb) {
-              dev::tmem_cp_32x128b_x4(tmem + sfa_col(s, kb), dev::desc_sf(ssfa + 512 * kb));
-              dev::tmem_cp_32x128b_x4(tmem + sfb_col(s, kb), dev::desc_sf(ssfb + 512 * kb));
-              if (b1_ok) dev::tmem_cp_32x128b_x4(tmem + sfb_col(s, kb) + 4, dev::desc_sf(ssfb + 2048 + 512 * kb));
+              dev::tmem_cp_32x128b_x4_pair(tmem + sfa_col(s, kb), dev::desc_sf(ssfa + 512 * kb));
+              dev::tmem_cp_32x128b_x4_pair(tmem + sfb_col(s, kb), dev::desc_sf(ssfb + 512 * kb));
+              if (b1_ok) dev::tmem_cp_32x128b_x4_pair(tmem + sfb_col(s, kb) + 4, dev::desc_sf(ssfb + 2048 + 512 * kb));
             }
             issued_any = true;
           }
-          dev::tc_commit(&sf_full[s]);  // arrives once this stage's copies have landed
+          dev::tc_commit_pair(&sf_full[s]);  // arrives once this stage's copies have landed
         }
       }
-      if (!ok) abort_all(abort_flag, p.status);
+      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
       if (issued_any) {
-        dev::tc_commit(drain_cp);
+        dev::tc_commit_pair(drain_cp);
         dev::mbar_wait(drain_cp, 0, p.limit_ns, nullptr);
       }
     }
-  } else {
-    // ------------------------------------------------------------ epilogue
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int e = warp - 4;
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int half = e >> 2;                // which 128 of the 256 columns
     uint8_t *stage_out = smem + EPI_OFF + e * EPI_TILE_BYTES;
+    const uint32_t tmem_empty_even = dev::mapa(dev::smem_u32(tmem_empty), 0);
     const float alpha = __fmul_rn(__ldg(p.s_a), __ldg(p.s_w));
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      const int m_blk = tile % p.num_m_blk, n_blk = tile / p.num_m_blk;
-      if (!dev::mbar_wait(tmem_full, tcount & 1, p.limit_ns, abort_flag)) {
-        abort_all(abort_flag, p.status);
+    for (int tile = pair; tile < p.num_tiles; tile += num_pairs, ++tcount) {
+      const int m_blk = 2 * (tile % p.num_m2) + static_cast<int>(h);
+      const int n_blk = tile / p.num_m2;
+      if (!dev::mbar_wait_cluster(tmem_full, tcount & 1, p.limit_ns, abort_flag)) {
+        abort_pair(abort_flag, peer_abort, p.status);
         break;
       }
       dev::tc_fence_after();
@@ -270,7 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       dev::tmem_wait_ld();
       dev::tc_fence_before();
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(tmem_empty);  // the MMA warp may start the next tile
+      if (lane == 0) dev::mbar_arrive_cluster(tmem_empty_even);  // the MMA thread may start the next tile
 
       const int row0 = m_blk * BM + 32 * q;
       const int col0 = n_blk * BN + half * 128;
@@ -310,8 +349,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (act1) y1 = gelu_tanh(y1);
               }
             }
-            __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-            out[j] = *reinterpret_cast<uint32_t *>(&h);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
+            out[j] = *reinterpret_cast<uint32_t *>(&hv);
           }
           // row `lane` of the 32 x 64 staging tile, 16-byte chunk g, 128-byte swizzle
           *reinterpret_cast<uint4 *>(stage_out + lane * 128 + ((g ^ (lane & 7)) << 4)) =
@@ -320,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         dev::fence_proxy_async();  // make the generic writes visible to the TMA store
         __syncwarp();
         if (lane == 0 && row0 < p.M && col0 + 64 * c2 < p.N) {  // the TMA clips the ragged edges
-          dev::tma_store_2d(&tm_y, stage_out, col0 + 64 * c2, row0);
+          dev::tma_store_2d(&maps.y, stage_out, col0 + 64 * c2, row0);
           dev::bulk_commit_group();
         }
       }
@@ -329,11 +368,39 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   dev::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  dev::cluster_sync();                        // no MMA or copy of the pair is still running
   if (warp == 1) {
     dev::tc_fence_after();
-    dev::tmem_dealloc(tmem, TMEM_COLS);
+    dev::tmem_dealloc_pair(tmem, TMEM_COLS);
   }
+}
+
+// Per device, once: the shared-memory opt-in of the kernel and the number of
+// SM pairs that can hold one CTA each at that size.
+int prepare_device(int sm_count, int *pairs_out) {
+  static std::mutex mu;
+  static int cached[64] = {0};
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64)
+    return fail(SVDQ_ERR_CUDA, "svdq_linear_w4a4: no current device");
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev_id] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4: ") + cudaGetErrorString(e));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sm_count & ~1), 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = sm_count / 2;
+    }
+    cached[dev_id] = n;
+  }
+  *pairs_out = cached[dev_id];
+  return SVDQ_OK;
 }
 
 }  // namespace
@@ -363,35 +430,52 @@ extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const fl
   Params p;
   p.M = M;
   p.N = N;
-  p.K = K;
   p.rank = rank;
   p.epilogue = epilogue;
   p.gelu_col_begin = gelu_col_begin;
-  p.num_m_blk = (M + BM - 1) / BM;
+  p.num_m2 = (M + 2 * BM - 1) / (2 * BM);
   const int num_n_blk = (N + BN - 1) / BN;
-  p.num_tiles = p.num_m_blk * num_n_blk;
+  p.num_tiles = p.num_m2 * num_n_blk;
   p.kb_total = K / 64;
   p.k_stages = bundle_ks(K);
   p.lr_stages = rank > 0 ? 1 : 0;
-  p.a_bundle = a_bundle;
-  p.w_bundle = w_bundle;
-  p.u = static_cast<const uint8_t *>(U);
-  p.l2t = static_cast<const uint8_t *>(l2t);
   p.s_a = s_a;
   p.s_w = s_w;
   p.bias = static_cast<const uint16_t *>(bias);
   p.status = st->status_word;
   p.limit_ns = kWaitLimitNs;
 
-  CUtensorMap ty;
-  int rc = encode_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
-                          static_cast<uint64_t>(ldy) * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  // The bundles are read as rows of 2 KB (256 x 8-byte elements); a copy is
+  // a box of whole rows.  Rows past the end of a buffer (the odd half of a
+  // pair tile whose rows lie beyond M) read as zeros.
+  Maps maps;
+  const auto u64 = CU_TENSOR_MAP_DATA_TYPE_UINT64;
+  const auto none = CU_TENSOR_MAP_SWIZZLE_NONE;
+  const uint64_t a_rows = bundle_bytes(M, K, 128) / ROW, w_rows = bundle_bytes(N, K, 256) / ROW;
+  int rc = encode_tmap_2d(&maps.a, u64, a_bundle, ROW / 8, a_rows, ROW, ROW / 8, A_BYTES / ROW, none);
+  if (rc == SVDQ_OK) rc = encode_tmap_2d(&maps.b, u64, w_bundle, ROW / 8, w_rows, ROW, ROW / 8, B_BYTES / ROW, none);
+  if (rc == SVDQ_OK)
+    rc = encode_tmap_2d(&maps.sfb, u64, w_bundle, ROW / 8, w_rows, ROW, ROW / 8, SFB_BYTES / ROW, none);
+  if (rc == SVDQ_OK && rank > 0) {
+    rc = encode_tmap_2d(&maps.u, u64, U, ROW / 8, lowrank_bytes(M, 128) / ROW, ROW, ROW / 8, LR_BYTES / ROW, none);
+    if (rc == SVDQ_OK)
+      rc = encode_tmap_2d(&maps.l2, u64, l2t, ROW / 8, lowrank_bytes(N, 256) / ROW, ROW, ROW / 8, LR_BYTES / ROW,
+                          none);
+  } else {
+    maps.u = maps.a;  // unused without the low-rank stage
+    maps.l2 = maps.a;
+  }
+  if (rc == SVDQ_OK)
+    rc = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(N),
+                        static_cast<uint64_t>(M), static_cast<uint64_t>(ldy) * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != SVDQ_OK) return rc;
-  cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4: ") + cudaGetErrorString(e));
-  const int grid = std::min(p.num_tiles, st->sm_count);
-  gemm_w4a4_kernel<<<grid, THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(ty, p);
-  e = cudaGetLastError();
+
+  int resident = 0;
+  rc = prepare_device(st->sm_count, &resident);
+  if (rc != SVDQ_OK) return rc;
+  const int pairs = std::min(p.num_tiles, resident);
+  gemm_w4a4_kernel<<<2 * pairs, THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(maps, p);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4 launch: ") + cudaGetErrorString(e));
   return ok();
 }

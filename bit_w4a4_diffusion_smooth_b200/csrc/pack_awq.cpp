@@ -41,18 +41,26 @@ double bf16_value(uint16_t b) {
 }
 
 // Position of weight (output column n, input k) in the packed qweight array:
-// the fragment order of the W4A16 kernel.  Columns come in blocks of 16 and K
-// in groups of 64; each (block, group) holds 32 lanes x 4 words, word j of a
-// lane covering k16-step j of the group.  Lane = 4 g + t and the 8 nibbles of
-// a word hold, with c = column within the block and kq = k within the step:
+// the fragment order of the W4A16 kernel.  Columns come in quads of 64 (four
+// blocks of 16) and K in groups of 64; the quads follow each other, and
+// inside a quad the groups, so that the four blocks of one group are 2 KB of
+// contiguous memory.  Each (quad, group, block) holds 32 lanes x 4 words,
+// word j of a lane covering k16-step j of the group.  Lane = 4 g + t and the
+// 8 nibbles of a word hold, with c = column within the block and kq = k
+// within the step:
 //   nibble 0 / 4: c = g,     kq = 2t / 2t+1
 //   nibble 1 / 5: c = g + 8, kq = 2t / 2t+1
 //   nibble 2 / 6: c = g,     kq = 2t+8 / 2t+9
 //   nibble 3 / 7: c = g + 8, kq = 2t+8 / 2t+9
 size_t awq_word_index(int n, int k, int G) {
-  const int nb = n / 16, c = n % 16, grp = k / 64, j = (k % 64) / 16, kq = k % 16;
+  const int quad = n / 64, blk = (n / 16) % 4, c = n % 16, grp = k / 64, j = (k % 64) / 16, kq = k % 16;
   const int lane = (c % 8) * 4 + (kq % 8) / 2;
-  return ((static_cast<size_t>(nb) * G + grp) * 32 + lane) * 4 + j;
+  return (((static_cast<size_t>(quad) * G + grp) * 4 + blk) * 32 + lane) * 4 + j;
+}
+// Position of the scale / zero point of (output column n, group g): the 64
+// values of one (quad, group) are contiguous.
+size_t awq_group_index(int n, int g, int G) {
+  return (static_cast<size_t>(n / 64) * G + g) * 64 + n % 64;
 }
 int awq_nibble_index(int n, int k) {
   const int c = n % 16, kq = k % 16;
@@ -68,8 +76,8 @@ extern "C" int awq_pack_weights(const uint16_t *W, int K, int N, const float *aw
   if (!W || !awq_scale || !qweight || !scales || !zeros || !inv_awq)
     return fail(SVDQ_ERR_INVALID_ARG, "awq_pack_weights: null pointer");
   if (group != 64) return fail(SVDQ_ERR_SHAPE, "awq_pack_weights: group must be 64");
-  if (K < group || K % group || N < 16 || N % 16)
-    return fail(SVDQ_ERR_SHAPE, "awq_pack_weights: need K % 64 == 0 and N % 16 == 0");
+  if (K < group || K % group || N < 64 || N % 64)
+    return fail(SVDQ_ERR_SHAPE, "awq_pack_weights: need K % 64 == 0 and N % 64 == 0");
   for (int k = 0; k < K; ++k)
     if (!(awq_scale[k] > 0.0f) || !std::isfinite(awq_scale[k]))
       return fail(SVDQ_ERR_INVALID_ARG, "awq_pack_weights: AWQ scales must be finite and > 0");
@@ -92,8 +100,8 @@ extern "C" int awq_pack_weights(const uint16_t *W, int K, int N, const float *aw
       } else {
         z = std::min(15.0, std::max(0.0, std::nearbyint(-lo / s)));
       }
-      scales[static_cast<size_t>(n) * G + g] = bf16_bits_of_exact(s);
-      zeros[static_cast<size_t>(n) * G + g] = bf16_bits_of_exact(z);
+      scales[awq_group_index(n, g, G)] = bf16_bits_of_exact(s);
+      zeros[awq_group_index(n, g, G)] = bf16_bits_of_exact(z);
       for (int i = 0; i < group; ++i) {
         int k = g * group + i;
         double q = std::min(15.0, std::max(0.0, std::nearbyint(wa[i] / s) + z));

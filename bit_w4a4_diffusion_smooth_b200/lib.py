@@ -205,12 +205,13 @@ def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, 
 
 
 def awq_pack_weights(W_bits, awq_scale, group=64):
-    """Host AWQ pack: returns qweight (u32, fragment order), scales, zeros (u16 [N, K/g]), inv_awq."""
+    """Host AWQ pack: returns qweight (u32, fragment order), scales, zeros (u16 [N/64, K/g, 64]), inv_awq."""
     W_bits = np.ascontiguousarray(W_bits, dtype=np.uint16)
     awq_scale = np.ascontiguousarray(awq_scale, dtype=np.float32)
     K, N = W_bits.shape
-    out = dict(qweight=np.zeros(N * K // 8, np.uint32), scales=np.zeros((N, K // group), np.uint16),
-               zeros=np.zeros((N, K // group), np.uint16), inv_awq=np.zeros(K, np.float32))
+    gshape = (N // 64, K // group, 64) if N % 64 == 0 and K % group == 0 else (N, max(K // group, 1))
+    out = dict(qweight=np.zeros(N * K // 8, np.uint32), scales=np.zeros(gshape, np.uint16),
+               zeros=np.zeros(gshape, np.uint16), inv_awq=np.zeros(K, np.float32))
     _check("awq_pack_weights", load().awq_pack_weights(
         _hptr(W_bits, np.uint16, "W"), K, N, _hptr(awq_scale, np.float32, "awq_scale"), group,
         _hptr(out["qweight"], np.uint32, "qweight"), _hptr(out["scales"], np.uint16, "scales"),

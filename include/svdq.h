@@ -52,13 +52,16 @@
  *           with the 128-byte swizzle: element (m, j) at (m/TH)*TH*128 +
  *           (m%TH)*128 + (((j/8) ^ (m%8)) * 16) + (j%8)*2; columns >= rank are 0.
  *   AWQ     qweight: N*K/8 uint32 words in the fragment order of the W4A16
- *           kernel's tensor-core tiles.  Columns go in blocks of 16 and K in
- *           groups of 64; block b, group G owns words [(b*(K/64)+G)*128, +128):
+ *           kernel's tensor-core tiles.  Columns go in quads of 64 = four
+ *           blocks of 16, K in groups of 64; quad Q, group G, block b owns
+ *           words [((Q*(K/64)+G)*4+b)*128, +128) - the four blocks of one
+ *           group of one quad are 2 KB of contiguous memory:
  *           32 lanes x 4 words, word j of lane 4g+t covering k = 64G+16j+kq.
  *           Its nibbles (bits 4i..4i+3) hold, for column c of the block:
  *             i = 0 / 4: c = g,   kq = 2t / 2t+1;   i = 1 / 5: c = g+8, kq = 2t / 2t+1
  *             i = 2 / 6: c = g,   kq = 2t+8/2t+9;   i = 3 / 7: c = g+8, kq = 2t+8/2t+9
- *           scales, zeros [N][K/group] bf16 (zeros are integers 0..15).
+ *           scales, zeros: N*K/64 bf16 each (zeros are integers 0..15), the
+ *           value of column n and group G at (((n/64)*(K/64)+G)*64 + n%64).
  */
 #ifndef SVDQ_B200_H
 #define SVDQ_B200_H
@@ -206,19 +209,19 @@ int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const float *s_a,
  *   z = clamp(rne(-lo / s), 0, 15), q = clamp(rne(W_a / s) + z, 0, 15);
  *   an all-zero group takes s = 1, z = 0.  inv_awq[k] = f32(1 / awq_scale[k]).
  * Args: W [K][N] bf16 host; awq_scale [K] f32 (> 0); group 64 (K % group == 0);
- * N % 16 == 0; outputs qweight (N*K/8 u32, fragment order above),
- * scales/zeros [N][K/group] bf16, inv_awq [K].
+ * N % 64 == 0; outputs qweight (N*K/8 u32, fragment order above),
+ * scales/zeros (N*K/group bf16 each, layout above), inv_awq [K].
  */
 int awq_pack_weights(const uint16_t *W, int K, int N, const float *awq_scale, int group,
                      uint32_t *qweight, uint16_t *scales, uint16_t *zeros, float *inv_awq);
 
 /*
  * AWQ W4A16 projection for small row counts (the modulation / adaLN layers):
- *   Y[m][n] = bf16( sum_g s[n][g] * sum_{k in g} f32(x[m][k] inv_awq[k]) (q - z[n][g]) + bias[n] )
+ *   Y[m][n] = bf16( sum_g s(n,g) * sum_{k in g} f32(x[m][k] inv_awq[k]) (q - z(n,g)) + bias[n] )
  * in fp32.  X [M][ldx] bf16; inv_awq [K] f32 or NULL (= 1); bias [N] or NULL.
  * The products run on tensor cores with X^ split into bf16 hi + lo parts
  * (relative error of the split ~2^-17).
- * Rules: 1 <= M <= 16, group == 64, K % 64 == 0, N % 16 == 0, ldx >= K,
+ * Rules: 1 <= M <= 16, group == 64, K % 64 == 0, N % 64 == 0, ldx >= K,
  * ldy >= N, ldx % 8 == 0, ldy % 8 == 0.
  */
 int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq,

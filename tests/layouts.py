@@ -93,23 +93,37 @@ def lowrank_pack(bits, th):
     return buf
 
 
-def awq_unpack(qweight, K, N):
-    """Fragment-order words -> q [K, N] (see the AWQ layout in svdq.h)."""
-    nb_n, g_n = N // 16, K // 64
-    w = np.asarray(qweight, dtype=np.uint32).reshape(nb_n, g_n, 32, 4)
-    q = np.empty((K, N), dtype=np.uint8)
-    lane = np.arange(32)
+def _awq_positions(K, N):
+    """(k index, n index) of every nibble of the qweight array, by word and nibble, written
+    from the layout in svdq.h: word (((Q*G + grp)*4 + b)*32 + lane)*4 + j, lane = 4g + t."""
+    G = K // 64
+    shape = (N // 64, G, 4, 32, 4)            # quad, group, block, lane, word j
+    Q, grp, b, lane, j = np.indices(shape)
     g, t = lane // 4, lane % 4
+    ks, ns = [], []
     for i in range(8):
-        nib = ((w >> np.uint32(4 * i)) & np.uint32(15)).astype(np.uint8)
         reg, odd = i % 4, i // 4
         c = g + 8 * (reg % 2)
         kq = 2 * t + odd + 8 * (reg // 2)
-        k_idx = (np.arange(g_n)[None, :, None, None] * 64 + np.arange(4)[None, None, None, :] * 16
-                 + kq[None, None, :, None])
-        n_idx = np.arange(nb_n)[:, None, None, None] * 16 + c[None, None, :, None]
-        q[np.broadcast_to(k_idx, nib.shape), np.broadcast_to(n_idx, nib.shape)] = nib
+        ks.append(grp * 64 + j * 16 + kq)
+        ns.append(Q * 64 + b * 16 + c)
+    return ks, ns
+
+
+def awq_unpack(qweight, K, N):
+    """Fragment-order words -> q [K, N] (see the AWQ layout in svdq.h)."""
+    w = np.asarray(qweight, dtype=np.uint32).reshape(N // 64, K // 64, 4, 32, 4)
+    q = np.empty((K, N), dtype=np.uint8)
+    ks, ns = _awq_positions(K, N)
+    for i in range(8):
+        q[ks[i], ns[i]] = ((w >> np.uint32(4 * i)) & np.uint32(15)).astype(np.uint8)
     return q
+
+
+def awq_group_unpack(vals, K, N):
+    """Per-group parameters (scales or zeros) in the library layout -> [K/64, N]."""
+    v = np.asarray(vals).reshape(N // 64, K // 64, 64)
+    return v.transpose(1, 0, 2).reshape(K // 64, N)
 
 
 def bf16_bits_to_f64(bits):
@@ -124,20 +138,18 @@ def awq_pack(q):
     """q [K, N] (0..15) -> fragment-order words (the inverse of awq_unpack)."""
     q = np.asarray(q, dtype=np.uint8)
     K, N = q.shape
-    nb_n, g_n = N // 16, K // 64
-    w = np.zeros((nb_n, g_n, 32, 4), dtype=np.uint32)
-    lane = np.arange(32)
-    g, t = lane // 4, lane % 4
+    w = np.zeros((N // 64, K // 64, 4, 32, 4), dtype=np.uint32)
+    ks, ns = _awq_positions(K, N)
     for i in range(8):
-        reg, odd = i % 4, i // 4
-        c = g + 8 * (reg % 2)
-        kq = 2 * t + odd + 8 * (reg // 2)
-        k_idx = (np.arange(g_n)[None, :, None, None] * 64 + np.arange(4)[None, None, None, :] * 16
-                 + kq[None, None, :, None])
-        n_idx = np.arange(nb_n)[:, None, None, None] * 16 + c[None, None, :, None]
-        nib = q[np.broadcast_to(k_idx, w.shape), np.broadcast_to(n_idx, w.shape)].astype(np.uint32)
-        w |= nib << np.uint32(4 * i)
+        w |= q[ks[i], ns[i]].astype(np.uint32) << np.uint32(4 * i)
     return w.reshape(-1)
+
+
+def awq_group_pack(vals):
+    """[K/64, N] per-group parameters -> the library layout ((n/64)*G + g)*64 + n%64 (flattened)."""
+    v = np.asarray(vals)
+    g_n, N = v.shape
+    return np.ascontiguousarray(v.reshape(g_n, N // 64, 64).transpose(1, 0, 2)).reshape(-1)
 
 
 def bf16_bits(values):

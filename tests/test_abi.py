@@ -81,6 +81,6 @@ def test_pack_argument_checks():
     with pytest.raises(lib.SvdqError):
         lib.svdq_pack_weights(w, np.ones(100, np.float32), 16)
     with pytest.raises(lib.SvdqError):
-        lib.awq_pack_weights(np.zeros((64, 24), np.uint16), np.ones(64, np.float32))
+        lib.awq_pack_weights(np.zeros((64, 48), np.uint16), np.ones(64, np.float32))
     with pytest.raises(lib.SvdqError):
-        lib.awq_pack_weights(np.zeros((64, 32), np.uint16), np.zeros(64, np.float32))
+        lib.awq_pack_weights(np.zeros((64, 64), np.uint16), np.zeros(64, np.float32))

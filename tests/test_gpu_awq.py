@@ -28,7 +28,7 @@ def _run(m, k, n, seed, with_bias=True, use_inv=True):
     p = oawq.pack(formats.bf16_bits_to_float(wb), a)
     Y = G.poisoned_bf16(m, n)
     lib.awq_linear_w4a16(G.bf16_dev(xb), G.dev(p["inv_a"]) if use_inv else None, G.dev(L.awq_pack(p["q"])),
-                         G.bf16_dev(L.bf16_bits(p["s"].T)), G.bf16_dev(L.bf16_bits(p["z"].T)),
+                         G.bf16_dev(L.bf16_bits(L.awq_group_pack(p["s"]))), G.bf16_dev(L.bf16_bits(L.awq_group_pack(p["z"]))),
                          G.bf16_dev(bb) if with_bias else None, n, Y)
     G.check_ok()
     x = formats.bf16_bits_to_float(xb)
@@ -36,8 +36,13 @@ def _run(m, k, n, seed, with_bias=True, use_inv=True):
     return G.excess_error(G.bf16_host(Y), want)
 
 
-@pytest.mark.parametrize("m,k,n", [(1, 64, 16), (2, 192, 48), (5, 1024, 320), (8, 512, 64), (9, 256, 96),
-                                   (16, 3072, 512), (3, 4096, 112)])
+@pytest.mark.parametrize("m,k,n", [
+    # ring kernel (M <= 8): one stage per quad, partial last stage, several stages per quad,
+    # groups past K, more 64-column quads than SMs, 2-3 ring stages when X^ is large
+    (1, 64, 64), (2, 192, 128), (5, 1024, 320), (8, 512, 64), (2, 2048, 128), (4, 4096, 192),
+    (2, 6144, 64), (7, 1600, 256), (8, 1024, 12800), (8, 12288, 128),
+    # direct kernel (M > 8)
+    (9, 256, 192), (16, 3072, 512), (12, 4096, 128)])
 def test_awq_parity(m, k, n):
     assert _run(m, k, n, seed=m + k + n) <= 1e-2
 

@@ -119,27 +119,44 @@ def test_bundle_layout_reader_round_trip():
     np.testing.assert_array_equal(layouts.bundle_pack(codes, sf, rows, k, th), buf)
 
 
-@pytest.mark.parametrize("k,n", [(64, 16), (192, 48), (3072, 64)])
+@pytest.mark.parametrize("k,n", [(64, 64), (192, 128), (3072, 64)])
 def test_awq_pack_matches_oracle(k, n):
     wb, _ = synthetic.weight(k, n, 11, 0.02)
     a = synthetic.awq_scales(k, 11)
     p = lib.awq_pack_weights(wb, a)
     o = oawq.pack(formats.bf16_bits_to_float(wb), a)
     np.testing.assert_array_equal(layouts.awq_unpack(p["qweight"], k, n), o["q"])
-    np.testing.assert_array_equal(layouts.bf16_bits_to_f64(p["scales"]).T, o["s"])
-    np.testing.assert_array_equal(layouts.bf16_bits_to_f64(p["zeros"]).T, o["z"])
+    np.testing.assert_array_equal(layouts.awq_group_unpack(layouts.bf16_bits_to_f64(p["scales"]), k, n), o["s"])
+    np.testing.assert_array_equal(layouts.awq_group_unpack(layouts.bf16_bits_to_f64(p["zeros"]), k, n), o["z"])
     np.testing.assert_array_equal(p["inv_awq"], o["inv_a"])
 
 
 def test_awq_layout_reader_round_trip():
     """The test-side reader inverts a layout written by hand from the header text."""
-    k, n = 64, 16
+    k, n = 128, 128
+    G = k // 64
     q = np.random.default_rng(1).integers(0, 16, (k, n)).astype(np.uint8)
     words = np.zeros(n * k // 8, np.uint32)
     for kk in range(k):
         for c in range(n):
-            j, kq = (kk % 64) // 16, kk % 16
-            lane = (c % 8) * 4 + (kq % 8) // 2
-            i = (c // 8) + 2 * (kq // 8) + 4 * (kq % 2)
-            words[((c // 16) * 1 + kk // 64) * 128 + lane * 4 + j] |= np.uint32(q[kk, c]) << np.uint32(4 * i)
+            quad, blk, cc = c // 64, (c // 16) % 4, c % 16
+            grp, j, kq = kk // 64, (kk % 64) // 16, kk % 16
+            lane = (cc % 8) * 4 + (kq % 8) // 2
+            i = (cc // 8) + 2 * (kq // 8) + 4 * (kq % 2)
+            words[(((quad * G + grp) * 4 + blk) * 32 + lane) * 4 + j] |= np.uint32(q[kk, c]) << np.uint32(4 * i)
     np.testing.assert_array_equal(layouts.awq_unpack(words, k, n), q)
+    np.testing.assert_array_equal(layouts.awq_pack(q), words)
+
+
+def test_awq_group_layout_from_header_text():
+    """Scale / zero position of (column n, group g) = ((n/64)*G + g)*64 + n%64, written by
+    hand; the test-side reader and writer agree with it."""
+    k, n = 192, 128
+    g_n = k // 64
+    v = np.random.default_rng(2).integers(0, 1000, (g_n, n))
+    flat = np.zeros(g_n * n, np.int64)
+    for g in range(g_n):
+        for c in range(n):
+            flat[((c // 64) * g_n + g) * 64 + c % 64] = v[g, c]
+    np.testing.assert_array_equal(layouts.awq_group_unpack(flat, k, n), v)
+    np.testing.assert_array_equal(layouts.awq_group_pack(v), flat)

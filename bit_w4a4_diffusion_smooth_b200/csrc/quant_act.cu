@@ -9,21 +9,26 @@
 //   * U = (bf16(X^) . L1) / (s_a s_w), the low-rank activations the GEMM adds,
 //     written as 128-row swizzled tiles.
 //
-// Design (memory bound: X is read once, ~0.3 B written per byte read):
+// Design (X is read once, ~0.3 B written per byte read):
 //   * one CTA per 32 rows, 16 compute warps + 1 TMA warp; a 4-stage ring of
 //     [32 rows x 256 cols] bf16 tiles of X, [rank x 256] tiles of L1^T and
 //     256-float slices of inv_lambda, loaded by TMA / bulk copies; X and L1^T
 //     land with the 128-byte swizzle (conflict-free for the row-wise pass and
 //     for ldmatrix);
-//   * quantize pass: each warp owns 2 rows, each lane 8 consecutive elements
-//     (two lanes per 16-block, one shuffle for the block max); codes go out
-//     as one 128-byte row segment per warp and row, four block scales per
-//     32-bit store; X^ is written back in place as bf16;
-//   * down-projection pass: warp w multiplies k16-slice w of the tile with
-//     mma.sync (bf16 in, fp32 accumulate); partial sums are added across the
-//     warps once at the end;
-//   * every wait is bounded (mbarrier try_wait + %globaltimer); a wait that
-//     runs out records SVDQ_ERR_TIMEOUT and the block leaves cleanly.
+//   * quantize pass: each lane owns one 16-element block of one row: two
+//     16-byte loads, the block maximum in registers, one f32 division for the
+//     block scale, and 1/scale from a per-CTA table of all 128 scale codes
+//     (the tensor scale is fixed per call, so f32(1 / f32(e4m3 * s_a)) has
+//     only 128 possible values); the block's 8 code bytes go out as one
+//     8-byte store, four lanes' scale bytes as one 32-bit store, and X^ is
+//     written back in place as bf16;
+//   * down-projection pass: each warp owns one 16 x 8 tile of U and a share
+//     of the stage's 16 k16-slices (mma.sync, bf16 in, fp32 accumulate); at
+//     most 4 partial sums per output are added at the end;
+//   * the compute warps meet at named barriers; every mbarrier wait is
+//     bounded (try_wait + %globaltimer) and decided warp-uniformly - a warp
+//     whose wait runs out records SVDQ_ERR_TIMEOUT, skips its work and keeps
+//     meeting the others at the barriers, so the block always finishes.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -61,7 +66,7 @@ __host__ __device__ constexpr int stage_bytes() {
 }
 template <int RANK>
 __host__ __device__ constexpr int smem_bytes() {
-  return 1024 + STAGES * stage_bytes<RANK>() + 256;
+  return 1024 + STAGES * stage_bytes<RANK>() + 128 * 4 + 256;
 }
 
 // Byte offset of the 16-byte chunk holding column c (0..63, multiple of 8) of
@@ -70,26 +75,47 @@ __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return static_cast<uint32_t>(r * 128 + ((((c >> 3) ^ r) & 7) << 4));
 }
 
-__device__ __forceinline__ void fail_wait(volatile int *abort_flag, unsigned int *status) {
-  *abort_flag = 1;
-  dev::report(status, SVDQ_ERR_TIMEOUT);
+// x^ = f32(x * inv) for the 8 bf16 of `w`, into out[0..7].
+__device__ __forceinline__ void smooth8(const uint4 &w, const float4 &i0, const float4 &i1, float (&out)[8]) {
+  out[0] = __fmul_rn(__uint_as_float(w.x << 16), i0.x);
+  out[1] = __fmul_rn(__uint_as_float(w.x & 0xFFFF0000u), i0.y);
+  out[2] = __fmul_rn(__uint_as_float(w.y << 16), i0.z);
+  out[3] = __fmul_rn(__uint_as_float(w.y & 0xFFFF0000u), i0.w);
+  out[4] = __fmul_rn(__uint_as_float(w.z << 16), i1.x);
+  out[5] = __fmul_rn(__uint_as_float(w.z & 0xFFFF0000u), i1.y);
+  out[6] = __fmul_rn(__uint_as_float(w.w << 16), i1.z);
+  out[7] = __fmul_rn(__uint_as_float(w.w & 0xFFFF0000u), i1.w);
 }
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Warps of the down-projection: (16-row half mt, 8-column tile nt) pairs, the
+// k16-slices of a stage split KSPLIT ways between warps with the same pair.
+template <int RANK>
+struct LrSplit {
+  static constexpr int NT8 = RANK > 0 ? RANK / 8 : 1;
+  static constexpr int P = 2 * NT8;
+  static constexpr int PP = P <= 4 ? 4 : P <= 8 ? 8 : 16;   // pairs rounded up to a power of 2
+  static constexpr int KSPLIT = CWARPS / PP;                 // 4, 2 or 1
+  static constexpr int SLICES = 16 / KSPLIT;                 // k16-slices per warp and stage
+};
 
 template <int RANK>
 __global__ void __launch_bounds__(THREADS, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1, Params p) {
-  constexpr int NP = RANK / 16;           // pairs of 8-wide MMA column tiles
+  using LS = LrSplit<RANK>;
   constexpr int L1_BOX = RANK * 128;
   constexpr int STAGE = stage_bytes<RANK>();
   constexpr int INV_OFF = X_STAGE + 4 * L1_BOX;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE);
+  float *rinv_tab = reinterpret_cast<float *>(smem + STAGES * STAGE);   // [128]
+  uint64_t *full = reinterpret_cast<uint64_t *>(rinv_tab + 128);
   uint64_t *empty = full + STAGES;
-  uint64_t *ready = empty + STAGES;       // X^ written back, per stage
-  uint64_t *sync = ready + STAGES;        // two end-of-loop syncs
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(sync + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
@@ -98,11 +124,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       dev::mbar_init(&full[s], 1);
       dev::mbar_init(&empty[s], CWARPS);
-      dev::mbar_init(&ready[s], CWARPS);
     }
-    dev::mbar_init(sync, CWARPS);
     *abort_flag = 0;
     dev::fence_mbar_init();
+  }
+  const float s_a = __ldg(p.s_a);
+  if (threadIdx.x < 128) {
+    // 1 / (scale of code c): the same two f32 roundings as the quantizer
+    // definition, f32(e4m3(c) * s_a) then f32(1 / that)
+    const uint32_t c = threadIdx.x;
+    const float scale = c < 127u ? __fmul_rn(dev::e4m3_value(c), s_a) : 0.0f;
+    rinv_tab[c] = scale == 0.0f ? 0.0f : __frcp_rn(scale);
   }
   __syncthreads();
 
@@ -115,7 +147,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int c = 0; c < p.KS; ++c) {
         const int s = c % STAGES;
         if (!dev::mbar_wait(&empty[s], ((c / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
-          fail_wait(abort_flag, p.status);
+          *abort_flag = 1;
+          dev::report(p.status, SVDQ_ERR_TIMEOUT);
           break;
         }
         const int nbox = min(4, (p.K - c * KC) / 64);
@@ -128,130 +161,106 @@ __global__ void __launch_bounds__(THREADS, 1)
         dev::bulk_load(st + INV_OFF, p.inv_lambda + c * KC, static_cast<uint32_t>(nbox * 256), &full[s]);
         ++issued;
       }
-      if (*abort_flag) {
-        // Let copies already in flight land before the block exits.
-        for (int c = max(0, issued - STAGES); c < issued; ++c)
-          dev::mbar_wait(&full[c % STAGES], (c / STAGES) & 1, p.limit_ns, nullptr);
-      }
+      // every issued copy lands before the block leaves
+      for (int c = max(0, issued - STAGES); c < issued; ++c)
+        dev::mbar_wait(&full[c % STAGES], (c / STAGES) & 1, p.limit_ns, nullptr);
     }
     return;
   }
 
   // -------------------------------------------------------------- compute warps
-  float acc[2][2 * NP + 1][4];
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int b = 0; b < 2 * NP + 1; ++b)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.0f;
-
-  const float s_a = __ldg(p.s_a);
-  const float d6 = __fmul_rn(6.0f, s_a);
+  // quantize pass: lane -> (row r, 16-block jb of box b)
+  const int b = warp >> 2;                        // 64-column box of the stage
+  const int r = (warp & 3) * 8 + (lane & 7);      // row within the CTA's 32
+  const int jb = lane >> 3;                       // block within the box
+  const int rt = m0 % 128 + r;                    // row inside the 128-row bundle tile
   const int m_blk = m0 / 128;
-  const int r_base = m0 % 128;            // row of this CTA's first row inside its 128-row tile
+  const float d6 = __fmul_rn(6.0f, s_a);
+  // down-projection pass: this warp's 16 x 8 tile of U and its k16-slices
+  const int pi = warp % LS::PP, kq = warp / LS::PP;
+  const int mt = pi & 1, nt = pi >> 1;
+  const bool lr_active = RANK > 0 && nt < LS::NT8;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  bool failed = false;
 
   for (int c = 0; c < p.KS; ++c) {
     const int s = c % STAGES;
     const uint32_t ph = (c / STAGES) & 1;
-    if (!dev::mbar_wait(&full[s], ph, p.limit_ns, abort_flag)) {
-      fail_wait(abort_flag, p.status);
-      return;
+    if (!failed && !dev::mbar_wait_warp(&full[s], ph, p.limit_ns, abort_flag)) {
+      *abort_flag = 1;
+      dev::report(p.status, SVDQ_ERR_TIMEOUT);
+      failed = true;
     }
     const int nbox = min(4, (p.K - c * KC) / 64);
     uint8_t *st = smem + s * STAGE;
-    const int box = lane >> 3;
-    const bool col_ok = box < nbox;       // columns past K quantize as zeros
-    uint8_t *tile = p.bundle + (static_cast<size_t>(m_blk) * p.KS + c) * bundle_tile_bytes(128);
-
-    float inv[8];
-    if (col_ok) {
-      const float4 i0 = *reinterpret_cast<const float4 *>(st + INV_OFF + 32 * lane);
-      const float4 i1 = *reinterpret_cast<const float4 *>(st + INV_OFF + 32 * lane + 16);
-      inv[0] = i0.x; inv[1] = i0.y; inv[2] = i0.z; inv[3] = i0.w;
-      inv[4] = i1.x; inv[5] = i1.y; inv[6] = i1.z; inv[7] = i1.w;
-    } else {
+    if (!failed) {
+      const bool col_ok = b < nbox;                 // columns past K quantize as zeros
+      uint8_t *chunk0 = st + b * X_BOX + sw_off(r, 16 * jb);
+      uint8_t *chunk1 = st + b * X_BOX + sw_off(r, 16 * jb + 8);
+      float xh[16];
+      if (col_ok) {
+        const float4 *iv = reinterpret_cast<const float4 *>(st + INV_OFF + (b * 64 + 16 * jb) * 4);
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(chunk0);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(chunk1);
+        float lo[8], hi[8];
+        smooth8(w0, iv[0], iv[1], lo);
+        smooth8(w1, iv[2], iv[3], hi);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) inv[i] = 0.0f;
-    }
-
-    // ---- quantize pass: rows 2*warp, 2*warp+1
+        for (int i = 0; i < 8; ++i) {
+          xh[i] = lo[i];
+          xh[8 + i] = hi[i];
+        }
+      } else {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int r = warp * 2 + i;
-      const int rt = r_base + r;          // row inside the 128-row bundle tile
-      uint8_t *chunk = st + box * X_BOX + sw_off(r, (8 * lane) & 63);
-      uint4 raw = make_uint4(0, 0, 0, 0);
-      if (col_ok) raw = *reinterpret_cast<const uint4 *>(chunk);
-      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-      float xh[8];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        xh[2 * j] = __fmul_rn(__uint_as_float(w[j] << 16), inv[2 * j]);
-        xh[2 * j + 1] = __fmul_rn(__uint_as_float(w[j] & 0xFFFF0000u), inv[2 * j + 1]);
+        for (int i = 0; i < 16; ++i) xh[i] = 0.0f;
       }
       float amax = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(xh[j]));
-      amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xh[i]));
       const uint32_t sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
-      const float scale = __fmul_rn(dev::e4m3_value(sb), s_a);
-      const float rinv = scale == 0.0f ? 0.0f : __frcp_rn(scale);
-      uint32_t packed = 0;
+      const float rinv = rinv_tab[sb];
+      uint32_t q[2] = {0u, 0u};
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        packed |= dev::cvt_e2m1x2(__fmul_rn(xh[2 * j], rinv), __fmul_rn(xh[2 * j + 1], rinv)) << (8 * j);
-      // this lane's 4 code bytes: byte 4*lane of the row, 128-byte swizzle
-      *reinterpret_cast<uint32_t *>(tile + rt * 128 + ((((lane >> 2) ^ rt) & 7) << 4) + (lane & 3) * 4) = packed;
-      // four consecutive block scales (lanes 8q, 8q+2, 8q+4, 8q+6) -> one word of atom q
-      const int base = lane & ~7;
-      const uint32_t word = __shfl_sync(0xFFFFFFFFu, sb, base) | (__shfl_sync(0xFFFFFFFFu, sb, base + 2) << 8) |
-                            (__shfl_sync(0xFFFFFFFFu, sb, base + 4) << 16) |
-                            (__shfl_sync(0xFFFFFFFFu, sb, base + 6) << 24);
-      if ((lane & 7) == 0)
-        *reinterpret_cast<uint32_t *>(tile + 128 * 128 + box * 512 + (rt & 31) * 16 + ((rt >> 5) & 3) * 4) = word;
+      for (int i = 0; i < 8; ++i)
+        q[i >> 2] |= dev::cvt_e2m1x2(__fmul_rn(xh[2 * i], rinv), __fmul_rn(xh[2 * i + 1], rinv)) << (8 * (i & 3));
+      // the block's 8 code bytes: byte 8 (4 b + jb) of the row, 128-byte swizzle
+      uint8_t *tile = p.bundle + (static_cast<size_t>(m_blk) * p.KS + c) * bundle_tile_bytes(128);
+      const int j = 4 * b + jb;
+      *reinterpret_cast<uint2 *>(tile + rt * 128 + ((((j >> 1) ^ rt) & 7) << 4) + 8 * (j & 1)) = make_uint2(q[0], q[1]);
+      // the 4 block scales of this row in box b -> one word of atom b
+      const uint32_t word = __shfl_sync(0xFFFFFFFFu, sb, lane & 7) | (__shfl_sync(0xFFFFFFFFu, sb, (lane & 7) + 8) << 8) |
+                            (__shfl_sync(0xFFFFFFFFu, sb, (lane & 7) + 16) << 16) |
+                            (__shfl_sync(0xFFFFFFFFu, sb, (lane & 7) + 24) << 24);
+      if (jb == 0)
+        *reinterpret_cast<uint32_t *>(tile + 128 * 128 + b * 512 + (rt & 31) * 16 + ((rt >> 5) & 3) * 4) = word;
       if (RANK > 0 && col_ok) {
-        uint4 o;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(xh[0], xh[1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(xh[2], xh[3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(xh[4], xh[5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(xh[6], xh[7]);
-        o.x = *reinterpret_cast<uint32_t *>(&h0);
-        o.y = *reinterpret_cast<uint32_t *>(&h1);
-        o.z = *reinterpret_cast<uint32_t *>(&h2);
-        o.w = *reinterpret_cast<uint32_t *>(&h3);
-        *reinterpret_cast<uint4 *>(chunk) = o;
+        *reinterpret_cast<uint4 *>(chunk0) =
+            make_uint4(bf16x2(xh[0], xh[1]), bf16x2(xh[2], xh[3]), bf16x2(xh[4], xh[5]), bf16x2(xh[6], xh[7]));
+        *reinterpret_cast<uint4 *>(chunk1) = make_uint4(bf16x2(xh[8], xh[9]), bf16x2(xh[10], xh[11]),
+                                                       bf16x2(xh[12], xh[13]), bf16x2(xh[14], xh[15]));
       }
     }
 
-    // ---- down-projection pass: warp w takes columns [16w, 16w+16) of the tile
     if (RANK > 0) {
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&ready[s]);
-      if (!dev::mbar_wait(&ready[s], ph, p.limit_ns, abort_flag)) {
-        fail_wait(abort_flag, p.status);
-        return;
-      }
-      const int kbox = warp >> 2;
-      if (kbox < nbox) {
-        const uint32_t xbase = dev::smem_u32(st + kbox * X_BOX);
-        const uint32_t lbase = dev::smem_u32(st + X_STAGE + kbox * L1_BOX);
-        const int kc = (warp & 3) * 16;
-        uint32_t a[2][4];
+      dev::named_barrier(1, CWARPS * 32);           // every warp's bf16(X^) is in place
+      if (!failed && lr_active) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          const int r = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          dev::ldmatrix_x4(xbase + sw_off(r, kc + (lane >> 4) * 8), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-        }
-#pragma unroll
-        for (int np = 0; np < NP; ++np) {
-          const int n = np * 16 + (lane & 7) + (lane >> 4) * 8;
-          uint32_t b0, b1, b2, b3;
-          dev::ldmatrix_x4(lbase + sw_off(n, kc + ((lane >> 3) & 1) * 8), b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            dev::mma_bf16_16816(acc[mt][2 * np], a[mt], b0, b1);
-            dev::mma_bf16_16816(acc[mt][2 * np + 1], a[mt], b2, b3);
+        for (int i = 0; i < LS::SLICES; i += 2) {    // two k16-slices (of one box) per step
+          const int slice = kq * LS::SLICES + i;
+          const int sbx = slice >> 2;
+          if (sbx < nbox) {
+            const int kc = (slice & 3) * 16;
+            const uint32_t xbase = dev::smem_u32(st + sbx * X_BOX);
+            const uint32_t lbase = dev::smem_u32(st + X_STAGE + sbx * L1_BOX);
+            uint32_t a0[4], a1[4], bq[4];
+            const int ar = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            dev::ldmatrix_x4(xbase + sw_off(ar, kc + (lane >> 4) * 8), a0[0], a0[1], a0[2], a0[3]);
+            dev::ldmatrix_x4(xbase + sw_off(ar, kc + 16 + (lane >> 4) * 8), a1[0], a1[1], a1[2], a1[3]);
+            // B: rows 8 nt .. +7 of L1^T; lanes 0-15 slice i (k 0-7, 8-15), lanes 16-31 slice i + 1
+            dev::ldmatrix_x4(lbase + sw_off(nt * 8 + (lane & 7), kc + ((lane >> 3) & 3) * 8), bq[0], bq[1], bq[2],
+                             bq[3]);
+            dev::mma_bf16_16816(acc, a0, bq[0], bq[1]);
+            dev::mma_bf16_16816(acc, a1, bq[2], bq[3]);
           }
         }
       }
@@ -259,59 +268,42 @@ __global__ void __launch_bounds__(THREADS, 1)
       dev::fence_proxy_async();
     }
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(&empty[s]);
+    if (lane == 0 && !failed) dev::mbar_arrive(&empty[s]);
   }
 
   // ---- U = (sum of the warps' partial products) / (s_a s_w), bf16, 128-row tiles
   const int tid = threadIdx.x;  // 0..511
   if (RANK > 0) {
-    // every warp is done with the stage buffers -> reuse them for partials
-    __syncwarp();
-    if (lane == 0) dev::mbar_arrive(sync);
-    if (!dev::mbar_wait(sync, 0, p.limit_ns, abort_flag)) {
-      fail_wait(abort_flag, p.status);
-      return;
+    dev::named_barrier(1, CWARPS * 32);            // the stage buffers are free: reuse for the partials
+    float *red = reinterpret_cast<float *>(smem);  // [KSPLIT][BM][RANK]
+    if (lr_active) {
+      const int g = lane >> 2, t = lane & 3;
+      float *base = red + kq * BM * RANK;
+      const int row = mt * 16 + g, col = nt * 8 + 2 * t;
+      base[row * RANK + col] = acc[0];
+      base[row * RANK + col + 1] = acc[1];
+      base[(row + 8) * RANK + col] = acc[2];
+      base[(row + 8) * RANK + col + 1] = acc[3];
     }
-    float *red = reinterpret_cast<float *>(smem);  // [CWARPS][BM][RANK]
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 2 * NP; ++nt) {
-        const int r = mt * 16 + g, n = nt * 8 + 2 * t;
-        float *base = red + (warp * BM) * RANK;
-        base[r * RANK + n] = acc[mt][nt][0];
-        base[r * RANK + n + 1] = acc[mt][nt][1];
-        base[(r + 8) * RANK + n] = acc[mt][nt][2];
-        base[(r + 8) * RANK + n + 1] = acc[mt][nt][3];
-      }
-    __syncwarp();
-    if (lane == 0) dev::mbar_arrive(sync);
-    if (!dev::mbar_wait(sync, 1, p.limit_ns, abort_flag)) {
-      fail_wait(abort_flag, p.status);
-      return;
-    }
+    dev::named_barrier(1, CWARPS * 32);
   }
   const float alpha = __fmul_rn(s_a, __ldg(p.s_w));
   for (int idx = tid; idx < BM * (SVDQ_LR_STRIDE / 8); idx += CWARPS * 32) {
-    const int r = idx >> 3, cc = idx & 7;   // row, 8-column chunk
-    const int m = m0 + r;
+    const int rr = idx >> 3, cc = idx & 7;   // row, 8-column chunk
+    const int m = m0 + rr;
     uint32_t o[4] = {0, 0, 0, 0};
-    if (RANK > 0 && 8 * cc < RANK) {
+    if (RANK > 0 && 8 * cc < RANK && !failed) {
       const float *red = reinterpret_cast<const float *>(smem);
       float v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int jj = 0; jj < 8; ++jj) {
         float sum = 0.0f;
 #pragma unroll
-        for (int w = 0; w < CWARPS; ++w) sum += red[(w * BM + r) * RANK + 8 * cc + j];
-        v[j] = __fdiv_rn(sum, alpha);
+        for (int w = 0; w < LS::KSPLIT; ++w) sum += red[(w * BM + rr) * RANK + 8 * cc + jj];
+        v[jj] = __fdiv_rn(sum, alpha);
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-        o[j] = *reinterpret_cast<uint32_t *>(&h);
-      }
+      for (int jj = 0; jj < 4; ++jj) o[jj] = bf16x2(v[2 * jj], v[2 * jj + 1]);
     }
     *reinterpret_cast<uint4 *>(p.U + lowrank_offset(m, 8 * cc, 128)) = make_uint4(o[0], o[1], o[2], o[3]);
   }

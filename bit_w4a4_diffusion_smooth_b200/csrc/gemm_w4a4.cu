@@ -36,7 +36,14 @@
 //               then scale, add bias, GELU, round to bf16 into a
 //               128-byte-swizzled staging tile and write it with TMA stores
 // Pipeline: 5 stages of 38 KB per CTA; TMEM holds the accumulator (256
-// columns) and 5 x 48 columns of block scales.
+// columns) and 5 x 48 columns of block scales.  A pair walks a contiguous
+// run of tiles, n fastest (one row block's A tiles stay hot in L2 while its
+// output columns are swept).
+// Measured limit: every tcgen05.cp of block scales (512 bytes, 128 rows x
+// one k-block) takes ~115 cycles of the SM's copy engine whatever its size,
+// and a k-stage needs 12 of them (A: 1, B: 2 per k-block) against 4 MMAs of
+// ~128 cycles, so a stage costs ~1.4k cycles; the copies overlap the MMAs of
+// other stages, but not enough to hide.
 // Every wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT and
 // raises the abort flag of both CTAs; in-flight work is drained, the pair
 // meets at a cluster barrier and frees TMEM.
@@ -90,7 +97,7 @@ __device__ __forceinline__ uint32_t sfb_col(int s, int kb) { return SF_COL + 48 
 
 struct Params {
   int M, N, rank, epilogue, gelu_col_begin;
-  int num_m2, num_tiles, k_stages, lr_stages, kb_total;
+  int num_m2, num_n, num_tiles, k_stages, lr_stages, kb_total;
   const float *s_a, *s_w;
   const uint16_t *bias;
   unsigned int *status;
@@ -131,6 +138,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t h = dev::cluster_ctarank();         // 0: even CTA (issues the MMAs), 1: odd
   const int pair = static_cast<int>(dev::cluster_id_x());
   const int num_pairs = static_cast<int>(dev::num_clusters_x());
+  // this pair's tiles: a contiguous run of tile ids, n fastest
+  const int t_begin = static_cast<int>((static_cast<long long>(pair) * p.num_tiles) / num_pairs);
+  const int t_end = static_cast<int>((static_cast<long long>(pair + 1) * p.num_tiles) / num_pairs);
   const int stages_per_tile = p.lr_stages + p.k_stages;
   const uint32_t peer_abort = dev::mapa(dev::smem_u32(const_cast<int *>(abort_flag)), h ^ 1u);
 
@@ -169,9 +179,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       }
       int it = 0;
       bool ok = true;
-      for (int tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
-        const int m_blk = 2 * (tile % p.num_m2) + static_cast<int>(h);  // this CTA's 128-row block
-        const int n_blk = tile / p.num_m2;
+      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        const int m_blk = 2 * (tile / p.num_n) + static_cast<int>(h);  // this CTA's 128-row block
+        const int n_blk = tile % p.num_n;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
           if (!dev::mbar_wait_cluster(&empty[s], ((it / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
@@ -207,7 +217,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (h == 0 && lane == 0) {
       int it = 0, tcount = 0;
       bool ok = true, issued_any = false;
-      for (int tile = pair; tile < p.num_tiles && ok; tile += num_pairs, ++tcount) {
+      for (int tile = t_begin; tile < t_end && ok; ++tile, ++tcount) {
         if (!dev::mbar_wait_cluster(tmem_empty, (tcount & 1) ^ 1, p.limit_ns, abort_flag)) {
           ok = false;
           break;
@@ -256,8 +266,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (h == 0 && lane == 0) {
       int it = 0;
       bool ok = true, issued_any = false;
-      for (int tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
-        const int n_blk = tile / p.num_m2;
+      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        const int n_blk = tile % p.num_n;
         const bool b1_ok = (n_blk * 2 + 1) * 128 < p.N;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
@@ -294,9 +304,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const uint32_t tmem_empty_even = dev::mapa(dev::smem_u32(tmem_empty), 0);
     const float alpha = __fmul_rn(__ldg(p.s_a), __ldg(p.s_w));
     int tcount = 0;
-    for (int tile = pair; tile < p.num_tiles; tile += num_pairs, ++tcount) {
-      const int m_blk = 2 * (tile % p.num_m2) + static_cast<int>(h);
-      const int n_blk = tile / p.num_m2;
+    for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
+      const int m_blk = 2 * (tile / p.num_n) + static_cast<int>(h);
+      const int n_blk = tile % p.num_n;
       if (!dev::mbar_wait_cluster(tmem_full, tcount & 1, p.limit_ns, abort_flag)) {
         abort_pair(abort_flag, peer_abort, p.status);
         break;
@@ -434,8 +444,8 @@ extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const fl
   p.epilogue = epilogue;
   p.gelu_col_begin = gelu_col_begin;
   p.num_m2 = (M + 2 * BM - 1) / (2 * BM);
-  const int num_n_blk = (N + BN - 1) / BN;
-  p.num_tiles = p.num_m2 * num_n_blk;
+  p.num_n = (N + BN - 1) / BN;
+  p.num_tiles = p.num_m2 * p.num_n;
   p.kb_total = K / 64;
   p.k_stages = bundle_ks(K);
   p.lr_stages = rank > 0 ? 1 : 0;

@@ -48,6 +48,9 @@ K2_BYTES = (M * K // 2 + M * K // 16 + M * RANK * 2     # activation codes, scal
             + N * 2 + M * N * 2)                        # bias, Y
 K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
             + AM * AK * 2 + AK * 4 + AN * 2 + AM * AN * 2)
+# DRAM bytes of one K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu capture
+# summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; set to None whenever K2 changes.
+K2_TRAFFIC_BYTES = 26_900_224 + 36_975_360
 
 
 def peaks():
@@ -288,7 +291,8 @@ def run_ours(args):
                    "flops_per_step": STEP_FLOPS},
         "roofline": {"bound": "tensor", "kernel": "svdq_linear_w4a4 (K2)",
                      "achieved": round(k2_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(k2_tflops / fp4_peak, 4), "traffic": None,
+                     "frac": round(k2_tflops / fp4_peak, 4), "traffic": K2_TRAFFIC_BYTES,
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{how} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16)"},
         "kernels": {
             "K1_quantize_act": {"us": round(k1 * 1e3, 2), "GB/s": round(K1_BYTES / (k1 * 1e-3) / 1e9, 1),

@@ -49,8 +49,9 @@ K2_BYTES = (M * K // 2 + M * K // 16 + M * RANK * 2     # activation codes, scal
 K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
             + AM * AK * 2 + AK * 4 + AN * 2 + AM * AN * 2)
 # DRAM bytes of one K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu capture
-# summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; set to None whenever K2 changes.
-K2_TRAFFIC_BYTES = 26_900_224 + 36_975_360
+# summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; None until that capture matches the
+# current K2 again.
+K2_TRAFFIC_BYTES = None
 
 
 def peaks():

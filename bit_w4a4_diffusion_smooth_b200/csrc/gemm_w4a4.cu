@@ -166,6 +166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   dev::cluster_sync();                        // both CTAs' barriers exist before anyone arrives remotely
   dev::tc_fence_after();
   const uint32_t tmem = *tmem_base_slot;
+  dev::grid_dependency_wait();                // the operands written by the previous kernel are visible
+  dev::grid_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -484,8 +486,9 @@ extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const fl
   rc = prepare_device(st->sm_count, &resident);
   if (rc != SVDQ_OK) return rc;
   const int pairs = std::min(p.num_tiles, resident);
-  gemm_w4a4_kernel<<<2 * pairs, THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(maps, p);
-  cudaError_t e = cudaGetLastError();
+  DependentLaunch dl(dim3(2 * pairs), dim3(THREADS), SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel, maps, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4 launch: ") + cudaGetErrorString(e));
   return ok();
 }

@@ -106,6 +106,8 @@ __global__ void __launch_bounds__(D_THREADS, 1) awq_gemv_kernel(Params p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t = lane & 3;
   const int quad = blockIdx.x;
+  dev::grid_dependency_wait();
+  dev::grid_launch_dependents();
 
   float tot[4][NT][4];
 #pragma unroll
@@ -221,8 +223,9 @@ int launch_direct(const Params &p, cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(awq_gemv_kernel<NT, GPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16: ") + cudaGetErrorString(e));
-  awq_gemv_kernel<NT, GPW><<<p.N / 64, D_THREADS, smem, stream>>>(p);
-  e = cudaGetLastError();
+  DependentLaunch dl(dim3(p.N / 64), dim3(D_THREADS), smem, stream);
+  e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT, GPW>, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16 launch: ") + cudaGetErrorString(e));
   return ok();
 }

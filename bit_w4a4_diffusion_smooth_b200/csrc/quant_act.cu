@@ -128,6 +128,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort_flag = 0;
     dev::fence_mbar_init();
   }
+  dev::grid_dependency_wait();
+  dev::grid_launch_dependents();
   const float s_a = __ldg(p.s_a);
   if (threadIdx.x < 128) {
     // 1 / (scale of code c): the same two f32 roundings as the quantizer
@@ -314,8 +316,9 @@ int launch(const CUtensorMap &tx, const CUtensorMap &tl, const Params &p, int gr
   const int smem = smem_bytes<RANK>();
   cudaError_t e = cudaFuncSetAttribute(quant_act_kernel<RANK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_quantize_act: ") + cudaGetErrorString(e));
-  quant_act_kernel<RANK><<<grid, THREADS, smem, stream>>>(tx, tl, p);
-  e = cudaGetLastError();
+  DependentLaunch dl(dim3(grid), dim3(THREADS), smem, stream);
+  e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK>, tx, tl, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_quantize_act launch: ") + cudaGetErrorString(e));
   return ok();
 }

@@ -6,6 +6,7 @@
 #include <string>
 
 #include <cuda.h>
+#include <cuda_runtime.h>
 
 #include "../../include/svdq.h"
 
@@ -87,6 +88,27 @@ struct DeviceState {
 // State of the current device, or nullptr (after recording an error) if the
 // current device was not initialized.
 DeviceState *current_device_state();
+
+#ifdef __CUDACC__
+// Launch configuration for the hot-path kernels: programmatic stream
+// serialization lets a kernel start while its predecessor finishes (each
+// kernel waits for its predecessors before touching global memory).
+struct DependentLaunch {
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg;
+  DependentLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t stream) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
+#endif
 
 // Bounded-wait limit handed to every kernel, in nanoseconds.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;

@@ -13,6 +13,10 @@ step reads what the previous one left in L2.  Multi-GPU runs are independent
 replicas (the layer needs no exchange between GPUs): weak scaling.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                       [--workload qkv|dit-step]
+
+--workload dit-step times every projection linear of one denoising step of a
+12B-class DiT (228 W4A4 layers + 76 AWQ projections) as one CUDA graph.
 """
 import argparse
 import json
@@ -396,6 +400,171 @@ def run_reference(args):
     }))
 
 
+# ------------------------------------------------------------------ one DiT denoising step
+DIT_METRIC = "DiT step: every projection linear (SVDQ W4A4 + AWQ W4A16), FLOP-weighted TFLOPS"
+
+
+def dit_step_plan():
+    """Layers of one step in execution order: (kind, name, m, k, n, gelu_col_begin or None)."""
+    from bit_w4a4_diffusion_smooth_b200 import synthetic
+    d = synthetic.DitStep()
+    by_name = {name: (m, k, n, gelu, gbeg) for name, m, k, n, gelu, gbeg, _ in d.layers}
+    plan = []
+    for _ in range(d.dual_blocks):
+        for stream in ("img", "txt"):
+            plan.append(("awq", f"dual.{stream}.adaln", 2, d.hidden, 6 * d.hidden, None))
+        for stream in ("img", "txt"):
+            for name in ("qkv", "out", "fc1", "fc2"):
+                m, k, n, gelu, gbeg = by_name[f"dual.{stream}.{name}"]
+                plan.append(("w4a4", f"dual.{stream}.{name}", m, k, n, gbeg if gelu else None))
+    for _ in range(d.single_blocks):
+        plan.append(("awq", "single.adaln", 2, d.hidden, 3 * d.hidden, None))
+        for name in ("single.qkv_mlp", "single.out"):
+            m, k, n, gelu, gbeg = by_name[name]
+            plan.append(("w4a4", name, m, k, n, gbeg if gelu else None))
+    return d, plan
+
+
+def run_dit_step(args):
+    """Every projection linear of one denoising step of a 12B-class DiT (19 dual-stream and 38
+    single-stream blocks: 228 SVDQ W4A4 layers, each K1 + K2, and 76 AWQ W4A16 projections),
+    on distinct random-valid packed weights, replayed as one CUDA graph.  fc2 reads fc1's
+    output; the other layers read synthetic activations from rotating pools."""
+    import torch
+
+    from bit_w4a4_diffusion_smooth_b200 import lib
+
+    rank, world, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_replicas(world, "nccl", device)
+    lib.svdq_init(device.index)
+    d, plan = dit_step_plan()
+    r = d.rank
+    gen = torch.Generator(device=device)
+    gen.manual_seed(d.seed)
+
+    def rand_bundle(nbytes):
+        # valid NVFP4 bytes: e2m1 codes 0..7 in both nibbles, e4m3 scales <= 240 (no NaN)
+        return torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device=device, generator=gen) & 0x77
+
+    def rand_bf16(*shape, std=1.0):
+        return (torch.randn(*shape, device=device, generator=gen) * std).to(torch.bfloat16)
+
+    one = torch.ones(1, device=device)
+    s_w = torch.full((1,), 1e-3, device=device)
+    pools, act, layers = {}, {}, []
+    for kind, name, m, k, n, gbeg in plan:
+        if kind == "awq":
+            g_n = k // 64
+            layers.append(dict(kind=kind, m=m, k=k, n=n,
+                               X=rand_bf16(m, k), inv=torch.ones(k, device=device),
+                               qw=torch.randint(0, 2 ** 31, (k // 8 * n,), dtype=torch.int32, device=device,
+                                                generator=gen),
+                               sc=(torch.rand(g_n * n, device=device, generator=gen) * 1e-3).to(torch.bfloat16),
+                               z=torch.randint(0, 16, (g_n * n,), device=device, generator=gen).to(torch.bfloat16),
+                               b=rand_bf16(n, std=0.01), Y=torch.empty(m, n, dtype=torch.bfloat16, device=device)))
+            continue
+        ws = lib.svdq_weight_sizes(k, n, r)
+        if (m, k) not in act:
+            sz = lib.svdq_act_sizes(m, k)
+            act[(m, k)] = (torch.empty(sz["a_bundle"], dtype=torch.uint8, device=device),
+                           torch.empty(sz["u"], dtype=torch.uint8, device=device))
+        if (m, k) not in pools:  # 6 rotating inputs per shape: more than L2 holds for the big ones
+            pools[(m, k)] = [rand_bf16(m, k) for _ in range(6)]
+        layers.append(dict(kind=kind, name=name, m=m, k=k, n=n, gbeg=gbeg,
+                           inv=torch.ones(k, device=device), l1t=rand_bf16(r, k, std=0.02),
+                           l2t=rand_bundle(ws["l2t"]) & 0x3F, w=rand_bundle(ws["w_bundle"]),
+                           b=rand_bf16(n, std=0.01), Y=torch.empty(m, n, dtype=torch.bfloat16, device=device)))
+    use = {}
+    prev_fc1 = {}
+    for L in layers:  # inputs: fc2 takes its stream's fc1 output, the rest a pool buffer
+        if L["kind"] != "w4a4":
+            continue
+        if L["name"].endswith(".fc2"):
+            L["X"] = prev_fc1[L["name"].rsplit(".", 1)[0]]
+        else:
+            key = (L["m"], L["k"])
+            i = use.get(key, 0)
+            use[key] = i + 1
+            L["X"] = pools[key][i % 6]
+        if L["name"].endswith(".fc1"):
+            prev_fc1[L["name"].rsplit(".", 1)[0]] = L["Y"]
+
+    def step():
+        for L in layers:
+            if L["kind"] == "awq":
+                lib.awq_linear_w4a16(L["X"], L["inv"], L["qw"], L["sc"], L["z"], L["b"], L["n"], L["Y"])
+                continue
+            ab, U = act[(L["m"], L["k"])]
+            lib.svdq_quantize_act(L["X"], L["inv"], L["l1t"], r, one, s_w, ab, U)
+            epi = lib.EPILOGUE_GELU_ERF if L["gbeg"] is not None else lib.EPILOGUE_NONE
+            lib.svdq_linear_w4a4(ab, U, one, L["w"], L["l2t"], s_w, L["b"], L["m"], L["n"], L["k"], r, epi,
+                                 L["gbeg"] or 0, L["Y"])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    rc = lib.svdq_check_status()
+    if rc != lib.OK:
+        raise RuntimeError(f"device status after warm-up: {lib.status_name(rc)}")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    graph.replay()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    t1.record()
+    barrier()
+    clk = clocks.stop()
+    rc = lib.svdq_check_status()
+    if rc != lib.OK:
+        raise RuntimeError(f"device status after timing: {lib.status_name(rc)}")
+    (ms,) = max_over_ranks([t0.elapsed_time(t1) / args.steps], world, device)
+    del graph
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    w4a4 = sum(2 * L["m"] * L["k"] * L["n"] for L in layers if L["kind"] == "w4a4")
+    lowrank = sum(2 * L["m"] * r * (L["k"] + L["n"]) for L in layers if L["kind"] == "w4a4")
+    awq = sum(2 * L["m"] * L["k"] * L["n"] for L in layers if L["kind"] == "awq")
+    flops = w4a4 + lowrank + awq
+    n_w4a4 = sum(1 for L in layers if L["kind"] == "w4a4")
+    n_awq = len(layers) - n_w4a4
+    print(json.dumps({
+        "metric": DIT_METRIC, "value": round(aggregate_tflops(flops, world, ms), 2), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 x e4m3-scaled, fp32 accumulate); bf16 low-rank; int4 x bf16",
+        "data": "synthetic (random-valid packed weights per layer; seeded activations)",
+        "config": {"workload": "all projection linears of one denoising step of a 12B-class DiT: 19 dual-stream "
+                               "blocks (img 4096 / txt 512 tokens: QKV 3072->9216, out 3072->3072, "
+                               "fc1 3072->12288 +GELU, fc2 12288->3072) + 38 single-stream blocks (4608 tokens: "
+                               "3072->21504 with GELU on the last 12288 columns, 15360->3072), rank 32; "
+                               "adaLN AWQ 2x3072->18432 (x38) and 2x3072->9216 (x38)",
+                   "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step",
+                   "layers": {"w4a4": n_w4a4, "awq": n_awq}, "flops_per_step": flops},
+        "gpu_launches": args.steps * (2 * n_w4a4 + n_awq),
+        "clocks": clk,
+    }))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -403,11 +572,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=("qkv", "dit-step"), default="qkv",
+                    help="qkv: the QKV layer + AWQ projection (default); dit-step: one whole DiT step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "dit-step":
+        run_dit_step(args)
     else:
         run_ours(args)
 

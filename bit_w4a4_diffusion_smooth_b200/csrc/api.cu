@@ -181,6 +181,28 @@ extern "C" int svdq_debug_wait_timeout(uint64_t limit_ns, svdq_stream_t stream) 
   return ok();
 }
 
+namespace svdq {
+namespace {
+__global__ void gelu_probe_kernel(const float *in, int n, int kind, float *out) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = kind == SVDQ_EPILOGUE_GELU_TANH ? dev::gelu_tanh(in[i]) : dev::gelu_erf(in[i]);
+}
+}  // namespace
+}  // namespace svdq
+
+extern "C" int svdq_debug_gelu(const float *in, int n, int kind, float *out, svdq_stream_t stream) {
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  if (!in || !out) return fail(SVDQ_ERR_INVALID_ARG, "svdq_debug_gelu: null pointer");
+  if (kind != SVDQ_EPILOGUE_GELU_ERF && kind != SVDQ_EPILOGUE_GELU_TANH)
+    return fail(SVDQ_ERR_INVALID_ARG, "svdq_debug_gelu: kind must be a GELU epilogue");
+  if (n < 1) return fail(SVDQ_ERR_SHAPE, "svdq_debug_gelu: n must be >= 1");
+  gelu_probe_kernel<<<(n + 255) / 256, 256, 0, stream>>>(in, n, kind, out);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return ok();
+}
+
 extern "C" int svdq_debug_convert(const float *in, int n, uint8_t *e2m1_out, uint8_t *e4m3_out,
                                   svdq_stream_t stream) {
   DeviceState *st = current_device_state();

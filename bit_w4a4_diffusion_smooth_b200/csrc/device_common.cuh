@@ -374,6 +374,30 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// ---------------------------------------------------------------- GELU
+// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
+// 7.1.26: for x >= 0, erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5)
+// exp(-x^2) with t = 1 / (1 + p x), |error| <= 1.5e-7; odd in x.  Evaluated
+// with the fast exp and division (a few 1e-7 more), it is far below the bf16
+// rounding of the GEMM output it feeds, at a third of the instructions of a
+// correctly rounded erf - the GELU epilogue runs once per output element.
+__device__ __forceinline__ float erf_as7126(float x) {
+  const float ax = fabsf(x);
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  return copysignf(1.0f - poly * __expf(-ax * ax), x);
+}
+// GELU, erf form: y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)).
+__device__ __forceinline__ float gelu_erf(float y) { return 0.5f * y * (1.0f + erf_as7126(y * 0.70710678118654752f)); }
+// GELU, tanh form: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))).
+__device__ __forceinline__ float gelu_tanh(float y) {
+  return 0.5f * y * (1.0f + tanhf(0.79788456080286536f * (y + 0.044715f * y * y * y)));
+}
+
 // ---------------------------------------------------------------- conversions
 // Packs e2m1(hi) into bits 4..7 and e2m1(lo) into bits 0..3 (RNE, satfinite).
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {

@@ -108,10 +108,6 @@ struct Maps {
   CUtensorMap a, b, sfb, u, l2, y;
 };
 
-__device__ __forceinline__ float gelu_erf(float y) { return 0.5f * y * (1.0f + erff(y * 0.70710678118654752f)); }
-__device__ __forceinline__ float gelu_tanh(float y) {
-  return 0.5f * y * (1.0f + tanhf(0.79788456080286536f * (y + 0.044715f * y * y * y)));
-}
 
 // Raises the abort flag of this CTA and of its partner, records the timeout.
 __device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t peer_abort, unsigned int *status) {
@@ -120,6 +116,11 @@ __device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t pe
   dev::report(status, SVDQ_ERR_TIMEOUT);
 }
 
+// EPI: the epilogue (SVDQ_EPILOGUE_*), a template parameter so that each
+// instantiation holds only its own, fully unrolled epilogue: with both GELU
+// forms behind runtime branches the kernel's code outgrew the instruction
+// cache and every role stalled on instruction fetch.
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_w4a4_kernel(const __grid_constant__ Maps maps, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -351,14 +352,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           for (int j = 0; j < 4; ++j) {
             float y0 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * (g & 3) + 2 * j]), b[2 * j]);
             float y1 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * (g & 3) + 2 * j + 1]), b[2 * j + 1]);
-            if (p.epilogue != SVDQ_EPILOGUE_NONE) {
+            if constexpr (EPI != SVDQ_EPILOGUE_NONE) {
               const bool act0 = col + 2 * j >= p.gelu_col_begin, act1 = col + 2 * j + 1 >= p.gelu_col_begin;
-              if (p.epilogue == SVDQ_EPILOGUE_GELU_ERF) {
-                if (act0) y0 = gelu_erf(y0);
-                if (act1) y1 = gelu_erf(y1);
+              if constexpr (EPI == SVDQ_EPILOGUE_GELU_ERF) {
+                if (act0) y0 = dev::gelu_erf(y0);
+                if (act1) y1 = dev::gelu_erf(y1);
               } else {
-                if (act0) y0 = gelu_tanh(y0);
-                if (act1) y1 = gelu_tanh(y1);
+                if (act0) y0 = dev::gelu_tanh(y0);
+                if (act1) y1 = dev::gelu_tanh(y1);
               }
             }
             __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
@@ -398,14 +399,21 @@ int prepare_device(int sm_count, int *pairs_out) {
     return fail(SVDQ_ERR_CUDA, "svdq_linear_w4a4: no current device");
   std::lock_guard<std::mutex> lock(mu);
   if (cached[dev_id] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4: ") + cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(sm_count & ~1), 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = sm_count / 2;
     }
@@ -487,7 +495,11 @@ extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const fl
   if (rc != SVDQ_OK) return rc;
   const int pairs = std::min(p.num_tiles, resident);
   DependentLaunch dl(dim3(2 * pairs), dim3(THREADS), SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
-  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel, maps, p);
+  cudaError_t e = epilogue == SVDQ_EPILOGUE_GELU_ERF
+                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF>, maps, p)
+                  : epilogue == SVDQ_EPILOGUE_GELU_TANH
+                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH>, maps, p)
+                      : cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE>, maps, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4 launch: ") + cudaGetErrorString(e));
   return ok();

@@ -48,6 +48,7 @@ _SIGNATURES = {
     "svdq_check_status": (_I, [_P]),
     "svdq_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "svdq_debug_convert": (_I, [_P, _I, _P, _P, _P]),
+    "svdq_debug_gelu": (_I, [_P, _I, _I, _P, _P]),
 }
 EXPORTS = tuple(_SIGNATURES)
 
@@ -245,3 +246,10 @@ def svdq_debug_convert(x, e2m1_out, e4m3_out, stream=None):
     _check("svdq_debug_convert", load().svdq_debug_convert(
         _dptr(x, "x", torch.float32), x.numel(), _dptr(e2m1_out, "e2m1_out", torch.uint8),
         _dptr(e4m3_out, "e4m3_out", torch.uint8), _stream(stream)))
+
+
+def svdq_debug_gelu(x, kind, out, stream=None):
+    """out = GELU(x) through the epilogue's device function (x, out: float32 CUDA)."""
+    import torch
+    _check("svdq_debug_gelu", load().svdq_debug_gelu(
+        _dptr(x, "x", torch.float32), x.numel(), int(kind), _dptr(out, "out", torch.float32), _stream(stream)))

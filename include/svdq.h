@@ -254,6 +254,14 @@ int svdq_debug_wait_timeout(uint64_t limit_ns, svdq_stream_t stream);
 int svdq_debug_convert(const float *in, int n, uint8_t *e2m1_out, uint8_t *e4m3_out,
                        svdq_stream_t stream);
 
+/*
+ * GELU probe (device buffers): out[i] = GELU(in[i]) for i < n through the
+ * device function the W4A4 epilogue applies, kind = SVDQ_EPILOGUE_GELU_ERF
+ * (erf form, erf by Abramowitz & Stegun 7.1.26) or SVDQ_EPILOGUE_GELU_TANH.
+ * Lets the tests bound that function's error against the definition.
+ */
+int svdq_debug_gelu(const float *in, int n, int kind, float *out, svdq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -85,3 +85,36 @@ def test_init_rejects_missing_device():
     with pytest.raises(lib.SvdqError) as e:
         lib.svdq_init(torch.cuda.device_count() + 3)
     assert e.value.status == lib.ERR_INVALID_ARG
+
+
+def _gelu_probe(x, kind):
+    xs = torch.from_numpy(x).to(G.DEV)
+    out = torch.empty_like(xs)
+    lib.svdq_debug_gelu(xs, kind, out)
+    G.check_ok()
+    return out.cpu().numpy().astype(np.float64)
+
+
+def test_gelu_erf_matches_definition():
+    """The epilogue's erf-form GELU (erf by Abramowitz & Stegun 7.1.26, |error| <= 1.5e-7, through
+    fast exp / division) against 0.5 x (1 + erf(x / sqrt 2)) in float64: absolute error within
+    1e-6 |x| + 1e-30 over [-12, 12], far below the bf16 rounding of the output it feeds."""
+    from scipy.special import erf
+    rng = np.random.default_rng(3)
+    x = np.concatenate([np.linspace(-12, 12, 200001), rng.normal(0, 3, 100000),
+                        [0.0, -0.0, 1e-30, -1e-30, 1e-6, -1e-6, 30.0, -30.0]]).astype(np.float32)
+    got = _gelu_probe(x, lib.EPILOGUE_GELU_ERF)
+    xd = x.astype(np.float64)
+    want = 0.5 * xd * (1.0 + erf(xd / np.sqrt(2.0)))
+    err = np.abs(got - want)
+    assert np.all(err <= 1e-6 * np.abs(xd) + 1e-30), float(np.max(err / (np.abs(xd) + 1e-30)))
+    assert got[x == 30.0][0] == 30.0 and got[x == -30.0][0] == 0.0
+
+
+def test_gelu_tanh_matches_definition():
+    rng = np.random.default_rng(4)
+    x = np.concatenate([np.linspace(-12, 12, 100001), rng.normal(0, 3, 50000)]).astype(np.float32)
+    got = _gelu_probe(x, lib.EPILOGUE_GELU_TANH)
+    xd = x.astype(np.float64)
+    want = 0.5 * xd * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (xd + 0.044715 * xd ** 3)))
+    assert np.all(np.abs(got - want) <= 2e-6 * np.abs(xd) + 1e-30)

@@ -55,7 +55,7 @@ K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
 # DRAM bytes of one K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu capture
 # summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; None until that capture matches the
 # current K2 again.
-K2_TRAFFIC_BYTES = None
+K2_TRAFFIC_BYTES = 26_721_024 + 34_769_152
 
 
 def peaks():
@@ -451,7 +451,7 @@ def run_dit_step(args):
     def rand_bf16(*shape, std=1.0):
         return (torch.randn(*shape, device=device, generator=gen) * std).to(torch.bfloat16)
 
-    one = torch.ones(1, device=device)
+    one_t = torch.ones(1, device=device)
     s_w = torch.full((1,), 1e-3, device=device)
     pools, act, layers = {}, {}, []
     for kind, name, m, k, n, gbeg in plan:
@@ -497,9 +497,9 @@ def run_dit_step(args):
                 lib.awq_linear_w4a16(L["X"], L["inv"], L["qw"], L["sc"], L["z"], L["b"], L["n"], L["Y"])
                 continue
             ab, U = act[(L["m"], L["k"])]
-            lib.svdq_quantize_act(L["X"], L["inv"], L["l1t"], r, one, s_w, ab, U)
+            lib.svdq_quantize_act(L["X"], L["inv"], L["l1t"], r, one_t, s_w, ab, U)
             epi = lib.EPILOGUE_GELU_ERF if L["gbeg"] is not None else lib.EPILOGUE_NONE
-            lib.svdq_linear_w4a4(ab, U, one, L["w"], L["l2t"], s_w, L["b"], L["m"], L["n"], L["k"], r, epi,
+            lib.svdq_linear_w4a4(ab, U, one_t, L["w"], L["l2t"], s_w, L["b"], L["m"], L["n"], L["k"], r, epi,
                                  L["gbeg"] or 0, L["Y"])
 
     for _ in range(args.warmup):
@@ -536,6 +536,37 @@ def run_dit_step(args):
         raise RuntimeError(f"device status after timing: {lib.status_name(rc)}")
     (ms,) = max_over_ranks([t0.elapsed_time(t1) / args.steps], world, device)
     del graph
+
+    # per layer type: one instance's K1 + K2 (or K3) replayed back to back, times the count
+    per_type = {}
+    for L in layers:
+        key = (L["kind"], L.get("name", "adaln"), L["m"], L["k"], L["n"])
+        per_type.setdefault(key, [L, 0])[1] += 1
+    breakdown = []
+    for (kind, name, m, k, n), (L, cnt) in per_type.items():
+        def one(L=L):
+            if L["kind"] == "awq":
+                lib.awq_linear_w4a16(L["X"], L["inv"], L["qw"], L["sc"], L["z"], L["b"], L["n"], L["Y"])
+                return
+            ab, U = act[(L["m"], L["k"])]
+            lib.svdq_quantize_act(L["X"], L["inv"], L["l1t"], r, one_t, s_w, ab, U)
+            epi = lib.EPILOGUE_GELU_ERF if L["gbeg"] is not None else lib.EPILOGUE_NONE
+            lib.svdq_linear_w4a4(ab, U, one_t, L["w"], L["l2t"], s_w, L["b"], L["m"], L["n"], L["k"], r, epi,
+                                 L["gbeg"] or 0, L["Y"])
+        for _ in range(3):
+            one()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            one()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / 10 * 1e3
+        fl = 2 * m * k * n + (2 * m * r * (k + n) if kind == "w4a4" else 0)
+        breakdown.append({"layer": name if kind == "w4a4" else f"{name} (AWQ)", "m": m, "k": k, "n": n,
+                          "count": cnt, "us_each": round(us, 2), "TFLOP/s": round(fl / (us * 1e-6) / 1e12, 1),
+                          "ms_per_step": round(us * cnt / 1e3, 3)})
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -560,6 +591,7 @@ def run_dit_step(args):
                                "adaLN AWQ 2x3072->18432 (x38) and 2x3072->9216 (x38)",
                    "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step",
                    "layers": {"w4a4": n_w4a4, "awq": n_awq}, "flops_per_step": flops},
+        "breakdown": breakdown,
         "gpu_launches": args.steps * (2 * n_w4a4 + n_awq),
         "clocks": clk,
     }))

@@ -82,6 +82,21 @@ int encode_tmap_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base
   return SVDQ_OK;
 }
 
+int encode_tmap_3d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, const uint64_t (&dims)[3],
+                   const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  cuuint64_t st[2] = {strides[0], strides[1]};
+  cuuint32_t bx[3] = {box[0], box[1], box[2]};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(out, dtype, 3, const_cast<void *>(base), d, st, bx, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (code " + std::to_string(static_cast<int>(r)) + ")");
+  return SVDQ_OK;
+}
+
 namespace {
 __global__ void wait_timeout_kernel(unsigned long long limit_ns, unsigned int *status) {
   __shared__ uint64_t bar;

@@ -10,25 +10,29 @@
 //     written as 128-row swizzled tiles.
 //
 // Design (X is read once, ~0.3 B written per byte read):
-//   * one CTA per 32 rows, 16 compute warps + 1 TMA warp; a 4-stage ring of
-//     [32 rows x 256 cols] bf16 tiles of X, [rank x 256] tiles of L1^T and
-//     256-float slices of inv_lambda, loaded by TMA / bulk copies; X and L1^T
-//     land with the 128-byte swizzle (conflict-free for the row-wise pass and
-//     for ldmatrix);
-//   * quantize pass: each lane owns one 16-element block of one row: two
-//     16-byte loads, the block maximum in registers, one f32 division for the
-//     block scale, and 1/scale from a per-CTA table of all 128 scale codes
-//     (the tensor scale is fixed per call, so f32(1 / f32(e4m3 * s_a)) has
-//     only 128 possible values); the block's 8 code bytes go out as one
-//     8-byte store, four lanes' scale bytes as one 32-bit store, and X^ is
-//     written back in place as bf16;
-//   * down-projection pass: each warp owns one 16 x 8 tile of U and a share
-//     of the stage's 16 k16-slices (mma.sync, bf16 in, fp32 accumulate); at
-//     most 4 partial sums per output are added at the end;
-//   * the compute warps meet at named barriers; every mbarrier wait is
-//     bounded (try_wait + %globaltimer) and decided warp-uniformly - a warp
-//     whose wait runs out records SVDQ_ERR_TIMEOUT, skips its work and keeps
-//     meeting the others at the barriers, so the block always finishes.
+//   * one CTA per 32 rows, 16 compute warps + 1 TMA warp; a ring of stages,
+//     each a [32 rows x 256 cols] bf16 tile of X, an [r x 256] tile of L1^T
+//     (one 3-D TMA copy each, as four 64-column boxes with the 128-byte
+//     swizzle) and the stage's 256-float slice of inv_lambda (a bulk copy);
+//   * compute warp w owns the 16-column slice w of every stage for all 32
+//     rows.  It loads the slice once, with ldmatrix, straight into the
+//     m16n8k16 A-fragment layout: lane (g, t) holds columns 2t, 2t+1, 2t+8,
+//     2t+9 of rows g + 8q, q = 0..3, i.e. a quarter of four 16-element blocks;
+//   * from those registers: x^ = x * inv_lambda, the bf16 A fragments of the
+//     down-projection (mma.sync into r/2 independent accumulators per lane),
+//     and the block maxima, reduced over the 4 lanes of a row group by a
+//     butterfly that leaves each lane owning one whole block.  That lane
+//     takes the f32 division for the block scale and looks 1/scale up in a
+//     per-CTA table of all 128 scale codes (the tensor scale is fixed per
+//     call, so f32(1 / f32(e4m3 * s_a)) has only 128 values); the four
+//     1/scale values come back by shuffles, every lane converts its 16
+//     elements, and a second butterfly gathers each block's 8 code bytes in
+//     its owner lane for one 8-byte store (plus one scale byte);
+//   * warps never meet inside the loop: each waits for its stage with a
+//     bounded mbarrier wait (decided warp-uniformly; a warp whose wait runs
+//     out records SVDQ_ERR_TIMEOUT and leaves the loop) and releases it with
+//     one arrive.  At the end the 16 per-slice partial U tiles are added in
+//     shared memory and written as 128-row swizzled tiles.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -43,12 +47,13 @@ namespace {
 
 constexpr int BM = 32;             // rows per CTA
 constexpr int KC = kStageK;        // columns per stage (one bundle k-stage)
-constexpr int STAGES = 4;
-constexpr int CWARPS = 16;         // compute warps
-constexpr int THREADS = (CWARPS + 1) * 32;
+constexpr int CWARPS = 16;         // compute warps: one 16-column slice each
+constexpr int THREADS = (CWARPS + 2) * 32;   // + TMA warp + store warp
 constexpr int X_BOX = BM * 128;    // one [32 x 64] bf16 box, 128-byte rows
 constexpr int X_STAGE = 4 * X_BOX;
 constexpr int INV_BYTES = KC * 4;
+constexpr int OUT_BYTES = 6144;   // inv_lambda slice (1 KB), code rows (4 KB), scale words (512 B), padded
+constexpr int RING_BYTES = 224 * 1024;
 
 struct Params {
   int M, K, KS;
@@ -62,60 +67,57 @@ struct Params {
 
 template <int RANK>
 __host__ __device__ constexpr int stage_bytes() {
-  return X_STAGE + 4 * RANK * 128 + INV_BYTES;
+  return X_STAGE + 4 * RANK * 128 + OUT_BYTES;
+}
+template <int RANK>
+__host__ __device__ constexpr int num_stages() {
+  return RING_BYTES / stage_bytes<RANK>() < 8 ? RING_BYTES / stage_bytes<RANK>() : 8;
 }
 template <int RANK>
 __host__ __device__ constexpr int smem_bytes() {
-  return 1024 + STAGES * stage_bytes<RANK>() + 128 * 4 + 256;
+  return 1024 + num_stages<RANK>() * stage_bytes<RANK>() + 128 * 4 + 512;
 }
+// the per-slice partial U tiles reuse the ring at the end
+static_assert(CWARPS * BM * (64 + 4) * 4 <= num_stages<64>() * stage_bytes<64>(), "partials must fit the ring");
 
 // Byte offset of the 16-byte chunk holding column c (0..63, multiple of 8) of
 // row r inside a 128-byte-swizzled box of 128-byte rows.
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return static_cast<uint32_t>(r * 128 + ((((c >> 3) ^ r) & 7) << 4));
 }
-
-// x^ = f32(x * inv) for the 8 bf16 of `w`, into out[0..7].
-__device__ __forceinline__ void smooth8(const uint4 &w, const float4 &i0, const float4 &i1, float (&out)[8]) {
-  out[0] = __fmul_rn(__uint_as_float(w.x << 16), i0.x);
-  out[1] = __fmul_rn(__uint_as_float(w.x & 0xFFFF0000u), i0.y);
-  out[2] = __fmul_rn(__uint_as_float(w.y << 16), i0.z);
-  out[3] = __fmul_rn(__uint_as_float(w.y & 0xFFFF0000u), i0.w);
-  out[4] = __fmul_rn(__uint_as_float(w.z << 16), i1.x);
-  out[5] = __fmul_rn(__uint_as_float(w.z & 0xFFFF0000u), i1.y);
-  out[6] = __fmul_rn(__uint_as_float(w.w << 16), i1.z);
-  out[7] = __fmul_rn(__uint_as_float(w.w & 0xFFFF0000u), i1.w);
-}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
 }
-
-// Warps of the down-projection: (16-row half mt, 8-column tile nt) pairs, the
-// k16-slices of a stage split KSPLIT ways between warps with the same pair.
-template <int RANK>
-struct LrSplit {
-  static constexpr int NT8 = RANK > 0 ? RANK / 8 : 1;
-  static constexpr int P = 2 * NT8;
-  static constexpr int PP = P <= 4 ? 4 : P <= 8 ? 8 : 16;   // pairs rounded up to a power of 2
-  static constexpr int KSPLIT = CWARPS / PP;                 // 4, 2 or 1
-  static constexpr int SLICES = 16 / KSPLIT;                 // k16-slices per warp and stage
-};
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
+  return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
+}
 
 template <int RANK>
 __global__ void __launch_bounds__(THREADS, 1)
     quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1, Params p) {
-  using LS = LrSplit<RANK>;
+  constexpr int STAGES = num_stages<RANK>();
   constexpr int L1_BOX = RANK * 128;
   constexpr int STAGE = stage_bytes<RANK>();
   constexpr int INV_OFF = X_STAGE + 4 * L1_BOX;
+  constexpr int CODE_OFF = INV_OFF + INV_BYTES;    // [32 rows x 128 B] code rows, bundle swizzle
+  constexpr int SC_OFF = CODE_OFF + BM * 128;      // [4 boxes][32 rows] scale words
+  constexpr int NT = RANK / 8;     // 8-column tiles of U
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *rinv_tab = reinterpret_cast<float *>(smem + STAGES * STAGE);   // [128]
   uint64_t *full = reinterpret_cast<uint64_t *>(rinv_tab + 128);
-  uint64_t *empty = full + STAGES;
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + STAGES);
+  uint64_t *empty = full + STAGES;   // the store warp has written the stage out
+  uint64_t *done = empty + STAGES;   // the compute warps have staged the stage's codes and scales
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(done + STAGES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
@@ -123,7 +125,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       dev::mbar_init(&full[s], 1);
-      dev::mbar_init(&empty[s], CWARPS);
+      dev::mbar_init(&empty[s], 1);
+      dev::mbar_init(&done[s], CWARPS);
     }
     *abort_flag = 0;
     dev::fence_mbar_init();
@@ -154,12 +157,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const int nbox = min(4, (p.K - c * KC) / 64);
-        dev::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox * (X_BOX + L1_BOX + 256)));
+        // the 3-D boxes always land whole (columns past K as zeros)
+        dev::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(X_STAGE + 4 * L1_BOX + nbox * 256));
         uint8_t *st = smem + s * STAGE;
-        for (int b = 0; b < nbox; ++b) {
-          dev::tma_load_2d(st + b * X_BOX, &tm_x, &full[s], c * KC + b * 64, m0);
-          if (RANK > 0) dev::tma_load_2d(st + X_STAGE + b * L1_BOX, &tm_l1, &full[s], c * KC + b * 64, 0);
-        }
+        dev::tma_load_3d(st, &tm_x, &full[s], 0, m0, 4 * c);
+        if (RANK > 0) dev::tma_load_3d(st + X_STAGE, &tm_l1, &full[s], 0, 0, 4 * c);
         dev::bulk_load(st + INV_OFF, p.inv_lambda + c * KC, static_cast<uint32_t>(nbox * 256), &full[s]);
         ++issued;
       }
@@ -170,144 +172,203 @@ __global__ void __launch_bounds__(THREADS, 1)
     return;
   }
 
-  // -------------------------------------------------------------- compute warps
-  // quantize pass: lane -> (row r, 16-block jb of box b)
-  const int b = warp >> 2;                        // 64-column box of the stage
-  const int r = (warp & 3) * 8 + (lane & 7);      // row within the CTA's 32
-  const int jb = lane >> 3;                       // block within the box
-  const int rt = m0 % 128 + r;                    // row inside the 128-row bundle tile
   const int m_blk = m0 / 128;
+  if (warp == CWARPS + 1) {
+    // ---------------------------------------------------------- store warp
+    // copies each stage's staged code rows (4 KB, contiguous in the bundle
+    // tile) and scale words out with full-line stores, then frees the stage
+    const uint32_t qd = static_cast<uint32_t>((m0 % 128) >> 5);
+    for (int c = 0; c < p.KS; ++c) {
+      const int s = c % STAGES;
+      if (!dev::mbar_wait_warp(&done[s], (c / STAGES) & 1, p.limit_ns, abort_flag)) {
+        *abort_flag = 1;
+        dev::report(p.status, SVDQ_ERR_TIMEOUT);
+        break;
+      }
+      const uint8_t *st = smem + s * STAGE;
+      uint8_t *tile = p.bundle + (static_cast<size_t>(m_blk) * p.KS + c) * bundle_tile_bytes(128);
+      uint4 v[8];
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = *reinterpret_cast<const uint4 *>(st + CODE_OFF + (i * 32 + lane) * 16);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) w[b] = *reinterpret_cast<const uint32_t *>(st + SC_OFF + (b * 32 + lane) * 4);
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&empty[s]);
+      uint8_t *rows = tile + (m0 % 128) * 128;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4 *>(rows + (i * 32 + lane) * 16) = v[i];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        *reinterpret_cast<uint32_t *>(tile + 128 * 128 + b * 512 + lane * 16 + qd * 4) = w[b];
+    }
+    if (RANK > 0) dev::named_barrier(1, (CWARPS + 1) * 32);   // the ring may now hold the partials
+    return;
+  }
+
+  // -------------------------------------------------------------- compute warps
+  const int g = lane >> 2, t = lane & 3;
+  const int bx = warp >> 2;                     // 64-column box of this warp's slice
+  const int kc = (warp & 3) * 16;               // slice offset inside the box
+  const bool o1 = (t & 1) != 0, o2 = (t & 2) != 0;
+  // the block this lane owns after the butterflies: rows g + 8 q, q = 2 o1 + o2
+  const int row_own = 8 * (2 * (t & 1) + ((t >> 1) & 1)) + g;
+  // staged like the bundle tile: code chunk (warp >> 1) of the row, 128-byte swizzle on the row
+  // inside the 128-row tile (m0 is a multiple of 32, so that row and row_own agree mod 8)
+  const uint32_t code_off =
+      static_cast<uint32_t>(CODE_OFF + row_own * 128 + ((((warp >> 1) ^ row_own) & 7) << 4) + 8 * (warp & 1));
+  const uint32_t scale_off = static_cast<uint32_t>(SC_OFF + (bx * 32 + row_own) * 4 + (warp & 3));
   const float d6 = __fmul_rn(6.0f, s_a);
-  // down-projection pass: this warp's 16 x 8 tile of U and its k16-slices
-  const int pi = warp % LS::PP, kq = warp / LS::PP;
-  const int mt = pi & 1, nt = pi >> 1;
-  const bool lr_active = RANK > 0 && nt < LS::NT8;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // ldmatrix lane addresses: A rows (per 16-row half), B rows of L1^T (per pair of 8-column tiles)
+  const uint32_t a_off0 = sw_off((lane & 7) + ((lane >> 3) & 1) * 8, kc + (lane >> 4) * 8);
+  const uint32_t a_off1 = sw_off(16 + (lane & 7) + ((lane >> 3) & 1) * 8, kc + (lane >> 4) * 8);
+  const int lsrc = lane & ~3;
+  // prmt selectors of the code-byte gather (they depend on the lane's parity bits)
+  const uint32_t sel_a = o1 ? 0x1504u : 0x5140u, sel_b = o1 ? 0x3726u : 0x7362u;
+  const uint32_t sel_w0 = o2 ? 0x1054u : 0x5410u, sel_w1 = o2 ? 0x3276u : 0x7632u;
+
+  float acc[2][NT > 0 ? NT : 1][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int n = 0; n < (NT > 0 ? NT : 1); ++n)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[mt][n][i] = 0.0f;
   bool failed = false;
 
   for (int c = 0; c < p.KS; ++c) {
     const int s = c % STAGES;
-    const uint32_t ph = (c / STAGES) & 1;
-    if (!failed && !dev::mbar_wait_warp(&full[s], ph, p.limit_ns, abort_flag)) {
+    if (!dev::mbar_wait_warp(&full[s], (c / STAGES) & 1, p.limit_ns, abort_flag)) {
       *abort_flag = 1;
       dev::report(p.status, SVDQ_ERR_TIMEOUT);
       failed = true;
+      break;
     }
     const int nbox = min(4, (p.K - c * KC) / 64);
     uint8_t *st = smem + s * STAGE;
-    if (!failed) {
-      const bool col_ok = b < nbox;                 // columns past K quantize as zeros
-      uint8_t *chunk0 = st + b * X_BOX + sw_off(r, 16 * jb);
-      uint8_t *chunk1 = st + b * X_BOX + sw_off(r, 16 * jb + 8);
-      float xh[16];
-      if (col_ok) {
-        const float4 *iv = reinterpret_cast<const float4 *>(st + INV_OFF + (b * 64 + 16 * jb) * 4);
-        const uint4 w0 = *reinterpret_cast<const uint4 *>(chunk0);
-        const uint4 w1 = *reinterpret_cast<const uint4 *>(chunk1);
-        float lo[8], hi[8];
-        smooth8(w0, iv[0], iv[1], lo);
-        smooth8(w1, iv[2], iv[3], hi);
+    // x^ of the lane's 16 elements: xs[q][0..3] = row g + 8q, columns 2t, 2t+1, 2t+8, 2t+9
+    float xs[4][4];
+    if (bx < nbox) {
+      const uint32_t xbase = dev::smem_u32(st + bx * X_BOX);
+      uint32_t a0[4], a1[4];
+      dev::ldmatrix_x4(xbase + a_off0, a0[0], a0[1], a0[2], a0[3]);
+      dev::ldmatrix_x4(xbase + a_off1, a1[0], a1[1], a1[2], a1[3]);
+      const float *iv = reinterpret_cast<const float *>(st + INV_OFF) + bx * 64 + kc + 2 * t;
+      const float2 i0 = *reinterpret_cast<const float2 *>(iv);
+      const float2 i1 = *reinterpret_cast<const float2 *>(iv + 8);
+      // fragment register h of half mt: rows g (h even) / g + 8 (h odd), columns 2t.. (h < 2) / 2t+8.. (h >= 2)
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          xh[i] = lo[i];
-          xh[8 + i] = hi[i];
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = (q >> 1) ? a1[q & 1] : a0[q & 1];
+        const uint32_t hi = (q >> 1) ? a1[2 + (q & 1)] : a0[2 + (q & 1)];
+        xs[q][0] = __fmul_rn(bf16_lo(lo), i0.x);
+        xs[q][1] = __fmul_rn(bf16_hi(lo), i0.y);
+        xs[q][2] = __fmul_rn(bf16_lo(hi), i1.x);
+        xs[q][3] = __fmul_rn(bf16_hi(hi), i1.y);
+      }
+      if (RANK > 0) {
+        // down-projection of this slice: A = bf16(x^), B = L1^T rows (ldmatrix of 2 tiles x 2 k-halves)
+        uint32_t af[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          af[mt][0] = bf16x2(xs[2 * mt][0], xs[2 * mt][1]);
+          af[mt][1] = bf16x2(xs[2 * mt + 1][0], xs[2 * mt + 1][1]);
+          af[mt][2] = bf16x2(xs[2 * mt][2], xs[2 * mt][3]);
+          af[mt][3] = bf16x2(xs[2 * mt + 1][2], xs[2 * mt + 1][3]);
         }
-      } else {
+        const uint32_t lbase = dev::smem_u32(st + X_STAGE + bx * L1_BOX);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) xh[i] = 0.0f;
-      }
-      float amax = 0.0f;
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t b[4];
+          dev::ldmatrix_x4(lbase + sw_off(np * 16 + (lane >> 4) * 8 + (lane & 7), kc + ((lane >> 3) & 1) * 8), b[0],
+                           b[1], b[2], b[3]);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(xh[i]));
-      const uint32_t sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
-      const float rinv = rinv_tab[sb];
-      uint32_t q[2] = {0u, 0u};
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        q[i >> 2] |= dev::cvt_e2m1x2(__fmul_rn(xh[2 * i], rinv), __fmul_rn(xh[2 * i + 1], rinv)) << (8 * (i & 3));
-      // the block's 8 code bytes: byte 8 (4 b + jb) of the row, 128-byte swizzle
-      uint8_t *tile = p.bundle + (static_cast<size_t>(m_blk) * p.KS + c) * bundle_tile_bytes(128);
-      const int j = 4 * b + jb;
-      *reinterpret_cast<uint2 *>(tile + rt * 128 + ((((j >> 1) ^ rt) & 7) << 4) + 8 * (j & 1)) = make_uint2(q[0], q[1]);
-      // the 4 block scales of this row in box b -> one word of atom b
-      const uint32_t word = __shfl_sync(0xFFFFFFFFu, sb, lane & 7) | (__shfl_sync(0xFFFFFFFFu, sb, (lane & 7) + 8) << 8) |
-                            (__shfl_sync(0xFFFFFFFFu, sb, (lane & 7) + 16) << 16) |
-                            (__shfl_sync(0xFFFFFFFFu, sb, (lane & 7) + 24) << 24);
-      if (jb == 0)
-        *reinterpret_cast<uint32_t *>(tile + 128 * 128 + b * 512 + (rt & 31) * 16 + ((rt >> 5) & 3) * 4) = word;
-      if (RANK > 0 && col_ok) {
-        *reinterpret_cast<uint4 *>(chunk0) =
-            make_uint4(bf16x2(xh[0], xh[1]), bf16x2(xh[2], xh[3]), bf16x2(xh[4], xh[5]), bf16x2(xh[6], xh[7]));
-        *reinterpret_cast<uint4 *>(chunk1) = make_uint4(bf16x2(xh[8], xh[9]), bf16x2(xh[10], xh[11]),
-                                                       bf16x2(xh[12], xh[13]), bf16x2(xh[14], xh[15]));
-      }
-    }
-
-    if (RANK > 0) {
-      dev::named_barrier(1, CWARPS * 32);           // every warp's bf16(X^) is in place
-      if (!failed && lr_active) {
-#pragma unroll
-        for (int i = 0; i < LS::SLICES; i += 2) {    // two k16-slices (of one box) per step
-          const int slice = kq * LS::SLICES + i;
-          const int sbx = slice >> 2;
-          if (sbx < nbox) {
-            const int kc = (slice & 3) * 16;
-            const uint32_t xbase = dev::smem_u32(st + sbx * X_BOX);
-            const uint32_t lbase = dev::smem_u32(st + X_STAGE + sbx * L1_BOX);
-            uint32_t a0[4], a1[4], bq[4];
-            const int ar = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            dev::ldmatrix_x4(xbase + sw_off(ar, kc + (lane >> 4) * 8), a0[0], a0[1], a0[2], a0[3]);
-            dev::ldmatrix_x4(xbase + sw_off(ar, kc + 16 + (lane >> 4) * 8), a1[0], a1[1], a1[2], a1[3]);
-            // B: rows 8 nt .. +7 of L1^T; lanes 0-15 slice i (k 0-7, 8-15), lanes 16-31 slice i + 1
-            dev::ldmatrix_x4(lbase + sw_off(nt * 8 + (lane & 7), kc + ((lane >> 3) & 3) * 8), bq[0], bq[1], bq[2],
-                             bq[3]);
-            dev::mma_bf16_16816(acc, a0, bq[0], bq[1]);
-            dev::mma_bf16_16816(acc, a1, bq[2], bq[3]);
+          for (int mt = 0; mt < 2; ++mt) {
+            dev::mma_bf16_16816(acc[mt][2 * np], af[mt], b[0], b[1]);
+            dev::mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b[2], b[3]);
           }
         }
       }
-      // the next TMA load into this stage must come after our generic writes
-      dev::fence_proxy_async();
+    } else {
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xs[q][i] = 0.0f;   // columns past K quantize as zeros
     }
+
+    // block maxima: lane partials, then a butterfly over the row group's 4 lanes
+    const float m0q = absmax4(xs[0][0], xs[0][1], xs[0][2], xs[0][3]);
+    const float m1q = absmax4(xs[1][0], xs[1][1], xs[1][2], xs[1][3]);
+    const float m2q = absmax4(xs[2][0], xs[2][1], xs[2][2], xs[2][3]);
+    const float m3q = absmax4(xs[3][0], xs[3][1], xs[3][2], xs[3][3]);
+    float ka = o1 ? m2q : m0q, kb = o1 ? m3q : m1q;       // keep blocks {2 o1, 2 o1 + 1}
+    ka = fmaxf(ka, __shfl_xor_sync(0xFFFFFFFFu, o1 ? m0q : m2q, 1));
+    kb = fmaxf(kb, __shfl_xor_sync(0xFFFFFFFFu, o1 ? m1q : m3q, 1));
+    const float amax = fmaxf(o2 ? kb : ka, __shfl_xor_sync(0xFFFFFFFFu, o2 ? ka : kb, 2));   // block 2 o1 + o2
+    const uint32_t sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
+    const float rown = rinv_tab[sb];
+    // 1/scale of blocks 0..3 from their owners (lanes t = 0, 2, 1, 3)
+    float rq[4];
+    rq[0] = __shfl_sync(0xFFFFFFFFu, rown, lsrc);
+    rq[1] = __shfl_sync(0xFFFFFFFFu, rown, lsrc + 2);
+    rq[2] = __shfl_sync(0xFFFFFFFFu, rown, lsrc + 1);
+    rq[3] = __shfl_sync(0xFFFFFFFFu, rown, lsrc + 3);
+    // code bytes t (columns 2t, 2t+1) and t + 4 (columns 2t+8, 2t+9) of each block
+    uint32_t cq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      cq[q] = dev::cvt_e2m1x2(__fmul_rn(xs[q][0], rq[q]), __fmul_rn(xs[q][1], rq[q])) |
+              (dev::cvt_e2m1x2(__fmul_rn(xs[q][2], rq[q]), __fmul_rn(xs[q][3], rq[q])) << 8);
+    // gather: after the xor-1 step a lane holds bytes {e, e+1, e+4, e+5} (e = t & 2) of its
+    // two kept blocks, after the xor-2 step all 8 bytes of the block it owns
+    const uint32_t keep = o1 ? (cq[2] | (cq[3] << 16)) : (cq[0] | (cq[1] << 16));
+    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, o1 ? (cq[0] | (cq[1] << 16)) : (cq[2] | (cq[3] << 16)), 1);
+    const uint32_t da = prmt(keep, recv, sel_a), db = prmt(keep, recv, sel_b);
+    const uint32_t mine = o2 ? db : da;
+    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, o2 ? da : db, 2);
+    *reinterpret_cast<uint2 *>(st + code_off) = make_uint2(prmt(mine, other, sel_w0), prmt(mine, other, sel_w1));
+    st[scale_off] = static_cast<uint8_t>(sb);
     __syncwarp();
-    if (lane == 0 && !failed) dev::mbar_arrive(&empty[s]);
+    if (lane == 0) dev::mbar_arrive(&done[s]);
   }
 
-  // ---- U = (sum of the warps' partial products) / (s_a s_w), bf16, 128-row tiles
+  // ---- U = (sum of the 16 slices' partial products) / (s_a s_w), bf16, 128-row tiles
   const int tid = threadIdx.x;  // 0..511
+  constexpr int RS = RANK + 4;   // padded row of a partial tile
   if (RANK > 0) {
-    dev::named_barrier(1, CWARPS * 32);            // the stage buffers are free: reuse for the partials
-    float *red = reinterpret_cast<float *>(smem);  // [KSPLIT][BM][RANK]
-    if (lr_active) {
-      const int g = lane >> 2, t = lane & 3;
-      float *base = red + kq * BM * RANK;
-      const int row = mt * 16 + g, col = nt * 8 + 2 * t;
-      base[row * RANK + col] = acc[0];
-      base[row * RANK + col + 1] = acc[1];
-      base[(row + 8) * RANK + col] = acc[2];
-      base[(row + 8) * RANK + col + 1] = acc[3];
+    dev::named_barrier(1, (CWARPS + 1) * 32);      // the ring is no longer read (store warp included)
+    float *red = reinterpret_cast<float *>(smem) + warp * BM * RS;   // [CWARPS][BM][RS]
+    if (!failed) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int n = 0; n < (NT > 0 ? NT : 1); ++n) {
+          const int row = mt * 16 + g, col = n * 8 + 2 * t;
+          *reinterpret_cast<float2 *>(red + row * RS + col) = make_float2(acc[mt][n][0], acc[mt][n][1]);
+          *reinterpret_cast<float2 *>(red + (row + 8) * RS + col) = make_float2(acc[mt][n][2], acc[mt][n][3]);
+        }
     }
-    dev::named_barrier(1, CWARPS * 32);
+    dev::named_barrier(2, CWARPS * 32);
   }
+  // a wait that ran out anywhere leaves U zero (the status word carries the error)
+  const bool any_failed = RANK > 0 && *abort_flag != 0;
   const float alpha = __fmul_rn(s_a, __ldg(p.s_w));
-  for (int idx = tid; idx < BM * (SVDQ_LR_STRIDE / 8); idx += CWARPS * 32) {
-    const int rr = idx >> 3, cc = idx & 7;   // row, 8-column chunk
-    const int m = m0 + rr;
-    uint32_t o[4] = {0, 0, 0, 0};
-    if (RANK > 0 && 8 * cc < RANK && !failed) {
-      const float *red = reinterpret_cast<const float *>(smem);
-      float v[8];
+  // every thread: column pairs (2 cp, 2 cp + 1) of the CTA's rows, the 16 partials added in order
+  for (int idx = tid; idx < BM * (SVDQ_LR_STRIDE / 2); idx += CWARPS * 32) {
+    const int rr = idx / (SVDQ_LR_STRIDE / 2), cp = idx % (SVDQ_LR_STRIDE / 2);
+    uint32_t o = 0;
+    if (RANK > 0 && 2 * cp < RANK && !any_failed) {
+      const float *red = reinterpret_cast<const float *>(smem) + rr * RS + 2 * cp;
+      float2 sum = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        float sum = 0.0f;
-#pragma unroll
-        for (int w = 0; w < LS::KSPLIT; ++w) sum += red[(w * BM + rr) * RANK + 8 * cc + jj];
-        v[jj] = __fdiv_rn(sum, alpha);
+      for (int w = 0; w < CWARPS; ++w) {
+        const float2 v = *reinterpret_cast<const float2 *>(red + w * BM * RS);
+        sum.x += v.x;
+        sum.y += v.y;
       }
-#pragma unroll
-      for (int jj = 0; jj < 4; ++jj) o[jj] = bf16x2(v[2 * jj], v[2 * jj + 1]);
+      o = bf16x2(__fdiv_rn(sum.x, alpha), __fdiv_rn(sum.y, alpha));
     }
-    *reinterpret_cast<uint4 *>(p.U + lowrank_offset(m, 8 * cc, 128)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint32_t *>(p.U + lowrank_offset(m0 + rr, 2 * cp, 128)) = o;
   }
 }
 
@@ -355,13 +416,15 @@ extern "C" int svdq_quantize_act(const void *X, int M, int K, int ldx, const flo
   p.status = st->status_word;
   p.limit_ns = kWaitLimitNs;
 
+  // X as [K/64 boxes][M rows][64 columns] and L1^T as [K/64][rank][64]: one copy per stage each
   CUtensorMap tx, tl;
-  int rc = encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K), static_cast<uint64_t>(M),
-                          static_cast<uint64_t>(ldx) * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  const uint64_t kb = static_cast<uint64_t>(K / 64);
+  int rc = encode_tmap_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, {64, static_cast<uint64_t>(M), kb},
+                          {static_cast<uint64_t>(ldx) * 2, 128}, {64, BM, 4}, CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc != SVDQ_OK) return rc;
   if (rank > 0) {
-    rc = encode_tmap_2d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l1t, static_cast<uint64_t>(K),
-                        static_cast<uint64_t>(rank), static_cast<uint64_t>(K) * 2, 64, static_cast<uint32_t>(rank),
+    rc = encode_tmap_3d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l1t, {64, static_cast<uint64_t>(rank), kb},
+                        {static_cast<uint64_t>(K) * 2, 128}, {64, static_cast<uint32_t>(rank), 4},
                         CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc != SVDQ_OK) return rc;
   } else {

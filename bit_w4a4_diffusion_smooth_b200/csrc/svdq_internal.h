@@ -122,4 +122,10 @@ int encode_tmap_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base
                    uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                    CUtensorMapSwizzle swizzle);
 
+// Encodes a 3-D TMA descriptor (tiled, zero fill out of bounds): dims[0] is
+// contiguous, strides[0] / strides[1] are the byte strides of dims 1 and 2
+// (any order, multiples of 16).
+int encode_tmap_3d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, const uint64_t (&dims)[3],
+                   const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
+
 }  // namespace svdq

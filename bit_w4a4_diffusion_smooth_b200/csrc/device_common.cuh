@@ -236,6 +236,13 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (static_cast<uint64_t>(128 >> 4) << 32) |
          (static_cast<uint64_t>(1) << 46);
 }
+// Descriptor for a tcgen05.cp source of 128 rows x 32 bytes, no swizzle,
+// stored as two 2 KB halves (bytes 0-15 of every row, then bytes 16-31):
+// 8-row core matrices 128 bytes apart, the two halves 2048 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf_2x(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFF) | (static_cast<uint64_t>(2048 >> 4) << 16) |
+         (static_cast<uint64_t>(128 >> 4) << 32) | (static_cast<uint64_t>(1) << 46);
+}
 
 // ---------------------------------------------------------------- clusters and SM pairs
 // A kernel that issues tcgen05 operations with .cta_group::2 runs in clusters
@@ -363,6 +370,11 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
 // 512 bytes at the same shared-memory offset of its own CTA.
 __device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+// Each CTA of the pair: 128 rows x 32 bytes of its shared memory -> TMEM
+// lanes 0..127, 8 columns from taddr.
+__device__ __forceinline__ void tmem_cp_128x256b_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // ---------------------------------------------------------------- warp MMA

@@ -34,16 +34,18 @@
 //   warps 4..11 epilogue in both CTAs: drain the CTA's 128 x 256 fp32
 //               accumulator, hand TMEM back (to the even CTA's barrier),
 //               then scale, add bias, GELU, round to bf16 into a
-//               128-byte-swizzled staging tile and write it with TMA stores
-// Pipeline: 5 stages of 38 KB per CTA; TMEM holds the accumulator (256
-// columns) and 5 x 48 columns of block scales.  A pair walks a contiguous
+//               64-byte-swizzled 32 x 32 staging tile and write it with TMA
+//               stores
+// Pipeline: 4 stages of 50 KB per CTA; TMEM holds the accumulator (256
+// columns) and 4 x 48 columns of block scales.  A pair walks a contiguous
 // run of tiles, n fastest (one row block's A tiles stay hot in L2 while its
 // output columns are swept).
-// Measured limit: every tcgen05.cp of block scales (512 bytes, 128 rows x
-// one k-block) takes ~115 cycles of the SM's copy engine whatever its size,
-// and a k-stage needs 12 of them (A: 1, B: 2 per k-block) against 4 MMAs of
-// ~128 cycles, so a stage costs ~1.4k cycles; the copies overlap the MMAs of
-// other stages, but not enough to hide.
+// Measured limit: every tcgen05.cp of block scales takes ~115 cycles of the
+// SM's copy engine whatever its size (a 512-byte 32x128b.warpx4 atom or a
+// 4 KB 128x256b block alike).  The weight bundle therefore stores each B-scale
+// atom four times over, the image of its warpx4 copy, so one 128x256b copy
+// moves a k-block's scales for all 256 weight rows: a k-stage needs 8 copies
+// (A: 1, B: 1 per k-block) instead of 12, against 4 MMAs of ~128 cycles.
 // Every wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT and
 // raises the abort flag of both CTAs; in-flight work is drained, the pair
 // meets at a cluster barrier and frees TMEM.
@@ -62,18 +64,20 @@ namespace {
 
 constexpr int BM = 128;                       // rows per CTA (256 per pair)
 constexpr int BN = 256;                       // output columns per pair tile
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int ROW = 2048;                     // bytes per row of the bundle tensor maps
 constexpr int A_BYTES = BM * 144;             // activation tile: codes 16 KB + scales 2 KB
 constexpr int SFA_OFF = BM * 128;
+constexpr int A_CODE_BYTES = BM * 128;
+constexpr int SFA_BYTES = BM * 16;
 constexpr int B_OFF = A_BYTES;                // 18432, a multiple of 1024
 constexpr int B_BYTES = 128 * 128;            // this CTA's 128 weight rows of codes
-constexpr int SFB_OFF = B_OFF + B_BYTES;      // scales of all 256 weight rows
-constexpr int SFB_BYTES = 256 * 16;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFB_BYTES;  // 38912
+constexpr int SFB_OFF = B_OFF + B_BYTES;      // scales of all 256 weight rows, each atom 4 times
+constexpr int SFB_BYTES = 4 * 4096;           // per k-block: [rows 0-127: 4 x 512 B][rows 128-255: 4 x 512 B]
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFB_BYTES;  // 51200
 constexpr int LR_BYTES = 128 * 128;           // U (this CTA's rows) and L2T (its columns), 16 KB each
 constexpr int EPI_WARPS = 8;
-constexpr int EPI_TILE_BYTES = 32 * 128;      // 32 rows x 64 bf16, 128-byte swizzle
+constexpr int EPI_TILE_BYTES = 32 * 64;       // 32 rows x 32 bf16, 64-byte swizzle
 constexpr int EPI_OFF = STAGES * STAGE_BYTES;
 constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * EPI_TILE_BYTES;
 constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
@@ -81,7 +85,8 @@ constexpr int THREADS = (4 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL = 256;              // stage s: SFA at +48s (+4 kb), SFB at +48s+16 (+8 kb, +4 per row block)
 static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "MMA operand tiles start on 1024-byte boundaries");
-static_assert(A_BYTES % ROW == 0 && B_BYTES % ROW == 0 && SFB_BYTES % ROW == 0 && LR_BYTES % ROW == 0,
+static_assert(A_CODE_BYTES % ROW == 0 && SFA_BYTES % ROW == 0 && B_BYTES % ROW == 0 && SFB_BYTES % ROW == 0 &&
+                  LR_BYTES % ROW == 0,
               "copies are whole tensor-map rows");
 static_assert(SF_COL + 48 * STAGES <= TMEM_COLS, "scale columns fit in TMEM");
 
@@ -105,7 +110,7 @@ struct Params {
 };
 
 struct Maps {
-  CUtensorMap a, b, sfb, u, l2, y;
+  CUtensorMap a, sfa, b, sfb, u, l2, y;
 };
 
 
@@ -132,7 +137,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   uint64_t *tmem_empty = tmem_full + 1;                            // even CTA: both CTAs drained it
   uint64_t *drain_mma = tmem_empty + 1;
   uint64_t *drain_cp = drain_mma + 1;
-  uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(drain_cp + 1);
+  uint64_t *sf_loaded = drain_cp + 1;                              // even CTA: both CTAs' scale bytes
+  uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(sf_loaded + STAGES);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -150,6 +156,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       dev::mbar_init(&full[s], 1);            // the even CTA's producer arrival (+ the bytes of both CTAs)
       dev::mbar_init(&sf_full[s], 1);
       dev::mbar_init(&empty[s], 1);
+      dev::mbar_init(&sf_loaded[s], 1);
     }
     dev::mbar_init(tmem_full, 1);
     dev::mbar_init(tmem_empty, 2 * EPI_WARPS);
@@ -194,16 +201,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           const uint32_t bar = dev::mapa(dev::smem_u32(&full[s]), 0);
           uint8_t *dst = smem + s * STAGE_BYTES;
           if (st < p.lr_stages) {
-            if (h == 0) dev::mbar_arrive_expect_tx(&full[s], 2u * 2u * LR_BYTES);
+            if (h == 0) {
+              dev::mbar_arrive(&sf_loaded[s]);    // no scales in the low-rank stage
+              dev::mbar_arrive_expect_tx(&full[s], 2u * 2u * LR_BYTES);
+            }
             dev::tma_load_2d_pair(dst, &maps.u, bar, 0, m_blk * (LR_BYTES / ROW));
             dev::tma_load_2d_pair(dst + B_OFF, &maps.l2, bar, 0, (2 * n_blk + static_cast<int>(h)) * (LR_BYTES / ROW));
           } else {
             const int ks = st - p.lr_stages;
             const int wrow = (n_blk * p.k_stages + ks) * ((2 * B_BYTES + SFB_BYTES) / ROW);
-            if (h == 0) dev::mbar_arrive_expect_tx(&full[s], 2u * STAGE_BYTES);
-            dev::tma_load_2d_pair(dst, &maps.a, bar, 0, (m_blk * p.k_stages + ks) * (A_BYTES / ROW));
+            const int arow = (m_blk * p.k_stages + ks) * (A_BYTES / ROW);
+            const uint32_t sbar = dev::mapa(dev::smem_u32(&sf_loaded[s]), 0);
+            if (h == 0) {
+              dev::mbar_arrive_expect_tx(&sf_loaded[s], 2u * (SFA_BYTES + SFB_BYTES));
+              dev::mbar_arrive_expect_tx(&full[s], 2u * (A_CODE_BYTES + B_BYTES));
+            }
+            // the scales first, on their own barrier: their copies into TMEM
+            // then overlap the transfer of the codes
+            dev::tma_load_2d_pair(dst + SFA_OFF, &maps.sfa, sbar, 0, arow + SFA_OFF / ROW);
+            dev::tma_load_2d_pair(dst + SFB_OFF, &maps.sfb, sbar, 0, wrow + 2 * B_BYTES / ROW);
+            dev::tma_load_2d_pair(dst, &maps.a, bar, 0, arow);
             dev::tma_load_2d_pair(dst + B_OFF, &maps.b, bar, 0, wrow + static_cast<int>(h) * (B_BYTES / ROW));
-            dev::tma_load_2d_pair(dst + SFB_OFF, &maps.sfb, bar, 0, wrow + 2 * B_BYTES / ROW);
           }
         }
       }
@@ -211,8 +229,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       // Before the pair may leave: the even CTA waits for every stage it
       // armed to complete (that covers the odd CTA's copies as well).
       if (h == 0) {
-        for (int j = max(0, it - STAGES); j < it; ++j)
+        for (int j = max(0, it - STAGES); j < it; ++j) {
           dev::mbar_wait_cluster(&full[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
+          dev::mbar_wait_cluster(&sf_loaded[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
+        }
       }
     }
   } else if (warp == 1) {
@@ -270,11 +290,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int it = 0;
       bool ok = true, issued_any = false;
       for (int tile = t_begin; tile < t_end && ok; ++tile) {
-        const int n_blk = tile % p.num_n;
-        const bool b1_ok = (n_blk * 2 + 1) * 128 < p.N;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
-          if (!dev::mbar_wait_cluster(&full[s], (it / STAGES) & 1, p.limit_ns, abort_flag)) {
+          if (!dev::mbar_wait_cluster(&sf_loaded[s], (it / STAGES) & 1, p.limit_ns, abort_flag)) {
             ok = false;
             break;
           }
@@ -284,8 +302,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const uint32_t ssfb = dev::smem_u32(smem + s * STAGE_BYTES + SFB_OFF);
             for (int kb = 0; kb < nkb; ++kb) {
               dev::tmem_cp_32x128b_x4_pair(tmem + sfa_col(s, kb), dev::desc_sf(ssfa + 512 * kb));
-              dev::tmem_cp_32x128b_x4_pair(tmem + sfb_col(s, kb), dev::desc_sf(ssfb + 512 * kb));
-              if (b1_ok) dev::tmem_cp_32x128b_x4_pair(tmem + sfb_col(s, kb) + 4, dev::desc_sf(ssfb + 2048 + 512 * kb));
+              // both 128-row halves of the B scales in one copy: the four replicas of an
+              // atom fill the four lane quarters as one warpx4 copy of it would
+              dev::tmem_cp_128x256b_pair(tmem + sfb_col(s, kb), dev::desc_sf_2x(ssfb + 4096 * kb));
             }
             issued_any = true;
           }
@@ -327,13 +346,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       const int row0 = m_blk * BM + 32 * q;
       const int col0 = n_blk * BN + half * 128;
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {        // two 64-column chunks
+      for (int c = 0; c < 4; ++c) {           // four 32-column chunks
         if (lane == 0) dev::bulk_wait_group_read<0>();  // staging tile free again
         __syncwarp();
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {         // 8 columns (16 bytes) at a time
-          const int c = 2 * c2 + (g >> 2);
-          const int col = col0 + 64 * c2 + 8 * g;
+        for (int g = 0; g < 4; ++g) {         // 8 columns (16 bytes) at a time
+          const int col = col0 + 32 * c + 8 * g;
           float b[8];
           if (p.bias && col + 8 <= p.N) {
             const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
@@ -350,8 +368,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           uint32_t out[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            float y0 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * (g & 3) + 2 * j]), b[2 * j]);
-            float y1 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * (g & 3) + 2 * j + 1]), b[2 * j + 1]);
+            float y0 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j]), b[2 * j]);
+            float y1 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j + 1]), b[2 * j + 1]);
             if constexpr (EPI != SVDQ_EPILOGUE_NONE) {
               const bool act0 = col + 2 * j >= p.gelu_col_begin, act1 = col + 2 * j + 1 >= p.gelu_col_begin;
               if constexpr (EPI == SVDQ_EPILOGUE_GELU_ERF) {
@@ -365,14 +383,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
             out[j] = *reinterpret_cast<uint32_t *>(&hv);
           }
-          // row `lane` of the 32 x 64 staging tile, 16-byte chunk g, 128-byte swizzle
-          *reinterpret_cast<uint4 *>(stage_out + lane * 128 + ((g ^ (lane & 7)) << 4)) =
+          // row `lane` of the 32 x 32 staging tile, 16-byte chunk g, 64-byte swizzle
+          *reinterpret_cast<uint4 *>(stage_out + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) =
               make_uint4(out[0], out[1], out[2], out[3]);
         }
         dev::fence_proxy_async();  // make the generic writes visible to the TMA store
         __syncwarp();
-        if (lane == 0 && row0 < p.M && col0 + 64 * c2 < p.N) {  // the TMA clips the ragged edges
-          dev::tma_store_2d(&maps.y, stage_out, col0 + 64 * c2, row0);
+        if (lane == 0 && row0 < p.M && col0 + 32 * c < p.N) {  // the TMA clips the ragged edges
+          dev::tma_store_2d(&maps.y, stage_out, col0 + 32 * c, row0);
           dev::bulk_commit_group();
         }
       }
@@ -472,7 +490,8 @@ extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const fl
   const auto u64 = CU_TENSOR_MAP_DATA_TYPE_UINT64;
   const auto none = CU_TENSOR_MAP_SWIZZLE_NONE;
   const uint64_t a_rows = bundle_bytes(M, K, 128) / ROW, w_rows = bundle_bytes(N, K, 256) / ROW;
-  int rc = encode_tmap_2d(&maps.a, u64, a_bundle, ROW / 8, a_rows, ROW, ROW / 8, A_BYTES / ROW, none);
+  int rc = encode_tmap_2d(&maps.a, u64, a_bundle, ROW / 8, a_rows, ROW, ROW / 8, A_CODE_BYTES / ROW, none);
+  if (rc == SVDQ_OK) rc = encode_tmap_2d(&maps.sfa, u64, a_bundle, ROW / 8, a_rows, ROW, ROW / 8, SFA_BYTES / ROW, none);
   if (rc == SVDQ_OK) rc = encode_tmap_2d(&maps.b, u64, w_bundle, ROW / 8, w_rows, ROW, ROW / 8, B_BYTES / ROW, none);
   if (rc == SVDQ_OK)
     rc = encode_tmap_2d(&maps.sfb, u64, w_bundle, ROW / 8, w_rows, ROW, ROW / 8, SFB_BYTES / ROW, none);
@@ -487,7 +506,7 @@ extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const fl
   }
   if (rc == SVDQ_OK)
     rc = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(N),
-                        static_cast<uint64_t>(M), static_cast<uint64_t>(ldy) * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+                        static_cast<uint64_t>(M), static_cast<uint64_t>(ldy) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   if (rc != SVDQ_OK) return rc;
 
   int resident = 0;

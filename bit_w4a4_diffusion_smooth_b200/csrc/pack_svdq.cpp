@@ -295,7 +295,7 @@ static void quantize_rows_f32(const float *T, int rows, int K, float s_t, int th
           uint8_t hi = e2m1_code(t[k + 1] * inv);
           bundle[bundle_code_offset(m, k, K, th)] = static_cast<uint8_t>(lo | (hi << 4));
         }
-        bundle[bundle_scale_offset(m, kb * 16, K, th)] = sb;
+        for (int rep = 0; rep < bundle_scale_replicas(th); ++rep) bundle[bundle_scale_offset(m, kb * 16, K, th, rep)] = sb;
       }
     }
   });

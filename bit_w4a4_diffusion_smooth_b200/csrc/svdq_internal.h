@@ -37,14 +37,21 @@ int ok();
 //     r*128 + ((c ^ (r % 8)) * 16) - the shared-memory image a tcgen05 MMA
 //     reads with a SWIZZLE_128B K-major descriptor;
 //   * then TH/128 x 4 atoms of 512 bytes of ue4m3 block scales: the scale of
-//     (row r, 16-block j of the tile) at TH*128 + (r/128)*2048 + (j/4)*512 +
-//     (r%32)*16 + ((r%128)/32)*4 + j%4 - the order in which tcgen05.cp
-//     (32x128b, warpx4) moves one atom into four TMEM columns.
+//     (row r, 16-block j of the tile) at TH*128 + (j/4)*(TH/128)*512*RP +
+//     (r/128)*512*RP + (r%32)*16 + ((r%128)/32)*4 + j%4, in each of RP
+//     replicas 512 bytes apart.  One 512-byte atom (128 rows x one k-block)
+//     is the image of a tcgen05.cp 32x128b.warpx4 copy; four replicas of it
+//     are the image of the same columns written by one 128x256b copy, and the
+//     two 128-row halves of a 256-row tile side by side fill its 8 columns.
+//     RP = 1 for 128-row tiles (activations), 4 for 256-row tiles (weights).
 // Rows past `rows` and elements past K are zero (codes and scales).
 constexpr int kStageK = 256;
 
 SVDQ_HD int bundle_ks(int K) { return (K + kStageK - 1) / kStageK; }
-SVDQ_HD size_t bundle_tile_bytes(int th) { return static_cast<size_t>(th) * 144u; }
+SVDQ_HD int bundle_scale_replicas(int th) { return th == 256 ? 4 : 1; }
+SVDQ_HD size_t bundle_tile_bytes(int th) {
+  return static_cast<size_t>(th) * 128u + static_cast<size_t>(th / 128) * 2048u * bundle_scale_replicas(th);
+}
 SVDQ_HD size_t bundle_bytes(int rows, int K, int th) {
   return static_cast<size_t>((rows + th - 1) / th) * static_cast<size_t>(bundle_ks(K)) * bundle_tile_bytes(th);
 }
@@ -58,12 +65,14 @@ SVDQ_HD size_t bundle_code_offset(int m, int k, int K, int th) {
   return bundle_tile_offset(m, k, K, th) + static_cast<size_t>(r) * 128u +
          static_cast<size_t>((((kb >> 4) ^ r) & 7) << 4) + static_cast<size_t>(kb & 15);
 }
-// Byte holding the block scale of element (m, k).
-SVDQ_HD size_t bundle_scale_offset(int m, int k, int K, int th) {
+// Byte holding the block scale of element (m, k) in replica `rep`.
+SVDQ_HD size_t bundle_scale_offset(int m, int k, int K, int th, int rep = 0) {
   const int r = m % th, j = (k % kStageK) / 16;
-  return bundle_tile_offset(m, k, K, th) + static_cast<size_t>(th) * 128u + static_cast<size_t>(r >> 7) * 2048u +
-         static_cast<size_t>(j >> 2) * 512u + static_cast<size_t>(r & 31) * 16u +
-         static_cast<size_t>((r >> 5) & 3) * 4u + static_cast<size_t>(j & 3);
+  const size_t atom = 512u * static_cast<size_t>(bundle_scale_replicas(th));
+  return bundle_tile_offset(m, k, K, th) + static_cast<size_t>(th) * 128u +
+         static_cast<size_t>(j >> 2) * static_cast<size_t>(th / 128) * atom + static_cast<size_t>(r >> 7) * atom +
+         static_cast<size_t>(rep) * 512u + static_cast<size_t>(r & 31) * 16u + static_cast<size_t>((r >> 5) & 3) * 4u +
+         static_cast<size_t>(j & 3);
 }
 
 // Low-rank operands: tiles of TH rows x 64 bf16 (TH = 128 for U, 256 for

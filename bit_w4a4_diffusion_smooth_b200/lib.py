@@ -173,7 +173,8 @@ def svdq_quantize_host(T, s_t, tile_rows=128):
     T = np.ascontiguousarray(T, dtype=np.float32)
     rows, K = T.shape
     ks = (K + 255) // 256
-    bundle = np.zeros(((rows + tile_rows - 1) // tile_rows) * ks * tile_rows * 144, np.uint8)
+    tile_bytes = tile_rows * (144 if tile_rows == 128 else 192)
+    bundle = np.zeros(((rows + tile_rows - 1) // tile_rows) * ks * tile_bytes, np.uint8)
     _check("svdq_quantize_host", load().svdq_quantize_host(
         _hptr(T, np.float32, "T"), rows, K, ctypes.c_float(float(s_t)), tile_rows,
         _hptr(bundle, np.uint8, "bundle")))

@@ -36,14 +36,18 @@
  * move them around as opaque bytes):
  *   bundle  NVFP4 operand (e2m1 codes + ue4m3 block scales), cut into tiles
  *           of TH rows x 256 K-elements (TH = 128 for activations, 256 for
- *           weights).  Tile (tr, ks) starts at (tr * ceil(K/256) + ks) * TH*144
- *           bytes and holds TH rows x 128 bytes of codes (element k of row r in
+ *           weights).  Tile (tr, ks) starts at (tr * ceil(K/256) + ks) * T
+ *           bytes, T = TH*144 for TH = 128 and TH*192 for TH = 256, and holds
+ *           TH rows x 128 bytes of codes (element k of row r in
  *           byte k/2 of the row, low nibble for even k; code = sign bit 3 |
  *           e2m1 magnitude 0..7; the 16-byte chunks of a row permuted by the
  *           128-byte swizzle: chunk c of row r at r*128 + ((c ^ (r%8)) * 16)),
- *           then TH/128 x 4 atoms of 512 bytes of block scales (scale of row r,
- *           16-block j of the tile at TH*128 + (r/128)*2048 + (j/4)*512 +
- *           (r%32)*16 + ((r%128)/32)*4 + j%4).  Rows past the matrix and
+ *           then 4 x TH/128 x RP atoms of 512 bytes of block scales (RP = 1 for
+ *           TH = 128, 4 for TH = 256): the scale of row r, 16-block j of the
+ *           tile is at TH*128 + (j/4)*(TH/128)*512*RP + (r/128)*512*RP +
+ *           q*512 + (r%32)*16 + ((r%128)/32)*4 + j%4 for every replica q < RP
+ *           (the weight scales are stored four times over: the shared-memory
+ *           image of one wide tensor-memory copy).  Rows past the matrix and
  *           elements past K are zero.  Each tile is the shared-memory image of
  *           one GEMM pipeline stage, so a stage is one contiguous copy.
  *   L1T     low-rank down-projection, transposed: [rank][K] bf16, row-major.

@@ -11,12 +11,21 @@ def _ks(K):
     return (K + 255) // 256
 
 
+def _replicas(th):
+    """Copies of each scale atom: 4 in 256-row (weight) tiles, 1 in 128-row tiles."""
+    return 4 if th == 256 else 1
+
+
+def _tile_bytes(th):
+    return th * 128 + (th // 128) * 2048 * _replicas(th)
+
+
 def bundle_size(rows, K, th):
-    return ((rows + th - 1) // th) * _ks(K) * th * 144
+    return ((rows + th - 1) // th) * _ks(K) * _tile_bytes(th)
 
 
 def _tile(m, k, K, th):
-    return ((m // th) * _ks(K) + k // 256) * th * 144
+    return ((m // th) * _ks(K) + k // 256) * _tile_bytes(th)
 
 
 def code_index(rows, K, th):
@@ -28,14 +37,22 @@ def code_index(rows, K, th):
     return _tile(m, k, K, th) + r * 128 + ((((kb >> 4) ^ r) & 7) << 4) + (kb & 15)
 
 
-def scale_index(rows, K, th):
-    """Byte offsets of the block scales of rows x K/16, in bundle order."""
+def scale_index(rows, K, th, rep=0):
+    """Byte offsets of the block scales of rows x K/16 (replica rep), in bundle order."""
     m = np.arange(rows)[:, None]
     k = np.arange(0, K, 16)[None, :]
     r = m % th
     j = (k % 256) // 16
-    return (_tile(m, k, K, th) + th * 128 + (r // 128) * 2048 + (j // 4) * 512 + (r % 32) * 16
-            + ((r % 128) // 32) * 4 + j % 4)
+    atom = 512 * _replicas(th)
+    return (_tile(m, k, K, th) + th * 128 + (j // 4) * (th // 128) * atom + (r // 128) * atom + rep * 512
+            + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4)
+
+
+def scale_replicas_agree(buf, rows, K, th):
+    """Every replica of every block scale holds the same byte."""
+    buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
+    first = buf[scale_index(rows, K, th)]
+    return all(np.array_equal(buf[scale_index(rows, K, th, q)], first) for q in range(1, _replicas(th)))
 
 
 def bundle_unpack(buf, rows, K, th):
@@ -53,7 +70,8 @@ def bundle_pack(codes, scales, rows, K, th):
     buf = np.zeros(bundle_size(rows, K, th), dtype=np.uint8)
     c = np.asarray(codes, dtype=np.uint8)
     buf[code_index(rows, K, th)] = c[:, 0::2] | (c[:, 1::2] << 4)
-    buf[scale_index(rows, K, th)] = np.asarray(scales, dtype=np.uint8)
+    for q in range(_replicas(th)):
+        buf[scale_index(rows, K, th, q)] = np.asarray(scales, dtype=np.uint8)
     return buf
 
 
@@ -61,7 +79,8 @@ def bundle_padding_is_zero(buf, rows, K, th):
     buf = np.asarray(buf, dtype=np.uint8).reshape(-1)
     used = np.zeros(buf.size, dtype=bool)
     used[code_index(rows, K, th)] = True
-    used[scale_index(rows, K, th)] = True
+    for q in range(_replicas(th)):
+        used[scale_index(rows, K, th, q)] = True
     return not buf[~used].any()
 
 

@@ -36,7 +36,7 @@ def test_status_strings():
 
 def test_sizes():
     s = lib.svdq_weight_sizes(3072, 9216, 32)
-    assert s["w_bundle"] == 9216 * 1536 + 9216 * 192       # codes + scales, 256-row tiles fit exactly
+    assert s["w_bundle"] == 9216 * 1536 + 9216 * 192 * 4   # codes + 4 copies of the scales, 256-row tiles fit exactly
     assert s["l1t"] == 32 * 3072 * 2 and s["l2t"] == 9216 * 64 * 2
     a = lib.svdq_act_sizes(200, 320)
     assert a["a_bundle"] == 2 * 2 * 128 * 144                # rows padded to 256, K to 512

@@ -39,6 +39,7 @@ def test_pack_matches_oracle(k, n, rank):
     assert p["s_w"][0] == s_w
     codes, sf = nvfp4.quantize_blocks(r32.T, s_w)
     gc, gsf = layouts.bundle_unpack(p["w_bundle"], n, k, 256)
+    assert layouts.scale_replicas_agree(p["w_bundle"], n, k, 256)
     np.testing.assert_array_equal(gc, codes)
     np.testing.assert_array_equal(gsf, sf)
     assert layouts.bundle_padding_is_zero(p["w_bundle"], n, k, 256)
@@ -95,24 +96,27 @@ def test_host_quantizer_matches_oracle_bit_exactly():
     np.testing.assert_array_equal(c1, oc1)
 
 
-def test_bundle_layout_reader_round_trip():
+@pytest.mark.parametrize("rows,k,th", [(130, 320, 128), (300, 576, 256)])
+def test_bundle_layout_reader_round_trip(rows, k, th):
     """The test-side reader inverts a bundle written by hand from the header text."""
     rng = np.random.default_rng(2)
-    rows, k, th = 130, 320, 128
     codes = rng.integers(0, 16, (rows, k)).astype(np.uint8)
     sf = rng.integers(0, 127, (rows, k // 16)).astype(np.uint8)
-    buf = np.zeros(((rows + th - 1) // th) * ((k + 255) // 256) * th * 144, np.uint8)
+    tile_bytes = th * 144 if th == 128 else th * 192
+    rp = 1 if th == 128 else 4
+    buf = np.zeros(((rows + th - 1) // th) * ((k + 255) // 256) * tile_bytes, np.uint8)
     for m in range(rows):
         for kk in range(0, k, 2):
-            tile = ((m // th) * ((k + 255) // 256) + kk // 256) * th * 144
+            tile = ((m // th) * ((k + 255) // 256) + kk // 256) * tile_bytes
             r, byte = m % th, (kk % 256) // 2
             buf[tile + r * 128 + (((byte // 16) ^ (r % 8)) * 16) + byte % 16] = codes[m, kk] | (codes[m, kk + 1] << 4)
         for j16 in range(k // 16):
             kk = j16 * 16
-            tile = ((m // th) * ((k + 255) // 256) + kk // 256) * th * 144
+            tile = ((m // th) * ((k + 255) // 256) + kk // 256) * tile_bytes
             r, j = m % th, (kk % 256) // 16
-            buf[tile + th * 128 + (r // 128) * 2048 + (j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4
-                + j % 4] = sf[m, j16]
+            for q in range(rp):
+                buf[tile + th * 128 + (j // 4) * (th // 128) * 512 * rp + (r // 128) * 512 * rp + q * 512
+                    + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4] = sf[m, j16]
     gc, gsf = layouts.bundle_unpack(buf, rows, k, th)
     np.testing.assert_array_equal(gc, codes)
     np.testing.assert_array_equal(gsf, sf)

@@ -371,14 +371,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             float y0 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j]), b[2 * j]);
             float y1 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j + 1]), b[2 * j + 1]);
             if constexpr (EPI != SVDQ_EPILOGUE_NONE) {
+              // computed for every column and selected: straight-line code lets the
+              // independent GELU chains of a chunk interleave (a branch per element
+              // serialised them)
               const bool act0 = col + 2 * j >= p.gelu_col_begin, act1 = col + 2 * j + 1 >= p.gelu_col_begin;
+              float g0, g1;
               if constexpr (EPI == SVDQ_EPILOGUE_GELU_ERF) {
-                if (act0) y0 = dev::gelu_erf(y0);
-                if (act1) y1 = dev::gelu_erf(y1);
+                g0 = dev::gelu_erf(y0);
+                g1 = dev::gelu_erf(y1);
               } else {
-                if (act0) y0 = dev::gelu_tanh(y0);
-                if (act1) y1 = dev::gelu_tanh(y1);
+                g0 = dev::gelu_tanh(y0);
+                g1 = dev::gelu_tanh(y1);
               }
+              y0 = act0 ? g0 : y0;
+              y1 = act1 ? g1 : y1;
             }
             __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
             out[j] = *reinterpret_cast<uint32_t *>(&hv);

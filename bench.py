@@ -55,7 +55,7 @@ K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
 # DRAM bytes of one K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu capture
 # summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; None until that capture matches the
 # current K2 again.
-K2_TRAFFIC_BYTES = 26_721_024 + 34_769_152
+K2_TRAFFIC_BYTES = 33_172_992 + 46_266_880
 
 
 def peaks():
@@ -117,7 +117,18 @@ class ClockSampler:
                  "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.3)
+            return
+        # nvidia-smi needs a moment before its first sample: start timing only once it samples
+        t_end = time.time() + 5.0
+        while time.time() < t_end:
+            self.out.flush()
+            try:
+                if os.path.getsize(self.out.name) > 0:
+                    break
+            except OSError:
+                break
+            time.sleep(0.05)
+        time.sleep(0.1)
 
     def stop(self):
         if self.proc is None:
@@ -600,13 +611,17 @@ def run_dit_step(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 3000 for the layer step, about 0.4 s timed, so that the clock "
+                         "sampler sees the timed region; 200 for --workload dit-step and --impl reference)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=("qkv", "dit-step"), default="qkv",
                     help="qkv: the QKV layer + AWQ projection (default); dit-step: one whole DiT step")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 3000 if (args.impl == "ours" and args.workload == "qkv") else 200
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":

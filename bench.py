@@ -56,6 +56,8 @@ K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
 # summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; None until that capture matches the
 # current K2 again.
 K2_TRAFFIC_BYTES = 33_172_992 + 46_266_880
+# Steps of the timed region that carry per-kernel CUDA events (1 in EV_EVERY).
+EV_EVERY = 16
 
 
 def peaks():
@@ -239,8 +241,9 @@ def run_ours(args):
     if rc != lib.OK:
         raise RuntimeError(f"device status after warm-up: {lib.status_name(rc)}")
 
-    # ---- device-timed region: K steps, per-kernel events
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # ---- device-timed region: K steps; per-kernel events on every EV_EVERY-th step only, since an
+    # event between two kernels keeps the next one from launching early (dependent launches)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(0, args.steps, EV_EVERY)]
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
@@ -248,34 +251,56 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for i in range(args.steps):
-        step(S, i, evs[i])
+        step(S, i, evs[i // EV_EVERY] if i % EV_EVERY == 0 else None)
     t1.record()
     barrier()
     clk = clocks.stop()
     ms = t0.elapsed_time(t1)
-    k1 = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    k2 = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    k3 = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    k1 = sum(e[0].elapsed_time(e[1]) for e in evs) / len(evs)
+    k2 = sum(e[1].elapsed_time(e[2]) for e in evs) / len(evs)
+    k3 = sum(e[2].elapsed_time(e[3]) for e in evs) / len(evs)
     rc = lib.svdq_check_status()
     if rc != lib.OK:
         raise RuntimeError(f"device status after timing: {lib.status_name(rc)}")
 
-    # ---- end to end through the public API, host buffers in and out
-    yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
-    ayh = torch.empty((AM, AN), dtype=torch.bfloat16, pin_memory=True)
+    # ---- end to end through the public API, host buffers in and out.  Every step copies its
+    # inputs in from pinned host memory and its outputs back out; the uploads, the kernels and
+    # the downloads of consecutive steps run on three streams (the two DMA directions and the
+    # compute stream), ordered by events, over the rotating device buffer sets.
+    yh = [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    ayh = [torch.empty((AM, AN), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     e_steps = max(3, min(args.steps, 20))
+    main_s = torch.cuda.current_stream(device)
+    in_s, out_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(e_steps)]
+    ev_done = [torch.cuda.Event() for _ in range(e_steps)]
+    ev_out = [torch.cuda.Event() for _ in range(e_steps)]
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(main_s)
+    in_s.wait_event(e0)
+    out_s.wait_event(e0)
     for i in range(e_steps):
         s = S[i % len(S)]
-        s["X"].copy_(host["X"], non_blocking=True)
-        s["AX"].copy_(host["AX"], non_blocking=True)
+        with torch.cuda.stream(in_s):
+            if i >= len(S):
+                in_s.wait_event(ev_done[i - len(S)])    # the set's previous inputs have been consumed
+            s["X"].copy_(host["X"], non_blocking=True)
+            s["AX"].copy_(host["AX"], non_blocking=True)
+            ev_in[i].record(in_s)
+        main_s.wait_event(ev_in[i])
+        if i >= len(S):
+            main_s.wait_event(ev_out[i - len(S)])       # the set's previous outputs have been read out
         step(S, i)
-        yh.copy_(s["Y"], non_blocking=True)
-        ayh.copy_(s["AY"], non_blocking=True)
-    e1.record()
+        ev_done[i].record(main_s)
+        with torch.cuda.stream(out_s):
+            out_s.wait_event(ev_done[i])
+            yh[i % 2].copy_(s["Y"], non_blocking=True)
+            ayh[i % 2].copy_(s["AY"], non_blocking=True)
+            ev_out[i].record(out_s)
+    main_s.wait_event(ev_out[e_steps - 1])
+    e1.record(main_s)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e_steps
 
@@ -318,6 +343,7 @@ def run_ours(args):
             "K3_awq_w4a16": {"us": round(k3 * 1e3, 2), "GB/s": round(K3_BYTES / (k3 * 1e-3) / 1e9, 1),
                              "frac_hbm": round(K3_BYTES / (k3 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
             "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how,
+            "events_on": f"{len(evs)} of {args.steps} timed steps (per-kernel CUDA events)",
         },
         "e2e": {"value": round(aggregate_tflops(STEP_FLOPS, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2 + AM * AK * 2, "d2h_bytes_per_step": M * N * 2 + AM * AN * 2},

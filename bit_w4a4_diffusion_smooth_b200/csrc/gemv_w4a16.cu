@@ -18,6 +18,9 @@
 //     gives (q - z) exactly;
 //   * per group the fp32 partial is scaled by s in registers; the warps'
 //     partials are added through shared memory.
+// More than 16 rows (a batch of modulation vectors) run as blocks of 16 rows
+// on the grid's second dimension; each block is one more pass over the
+// weights, mostly from L2.
 // The weight layout (qweight) is the MMA fragment order; see svdq.h.
 #include <cuda_runtime.h>
 
@@ -47,7 +50,7 @@ __device__ __forceinline__ void a_frags(uint32_t w, uint32_t (&a)[4]) {
 }
 
 // ===========================================================================
-// Direct kernel (any M <= 16): one CTA per quad, 16 warps split K by groups.
+// Direct kernel: one CTA per quad and block of 8 NT rows, 16 warps split K by groups.
 constexpr int D_THREADS = 512;
 constexpr int D_WARPS = D_THREADS / 32;
 
@@ -106,6 +109,12 @@ __global__ void __launch_bounds__(D_THREADS, 1) awq_gemv_kernel(Params p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t = lane & 3;
   const int quad = blockIdx.x;
+  {  // this CTA's block of 8 NT rows
+    const int r0 = static_cast<int>(blockIdx.y) * 8 * NT;
+    p.X += static_cast<size_t>(r0) * p.ldx;
+    p.Y += static_cast<size_t>(r0) * p.ldy;
+    p.M = min(8 * NT, p.M - r0);
+  }
   dev::grid_dependency_wait();
   dev::grid_launch_dependents();
 
@@ -223,7 +232,7 @@ int launch_direct(const Params &p, cudaStream_t stream) {
   cudaError_t e =
       cudaFuncSetAttribute(awq_gemv_kernel<NT, GPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16: ") + cudaGetErrorString(e));
-  DependentLaunch dl(dim3(p.N / 64), dim3(D_THREADS), smem, stream);
+  DependentLaunch dl(dim3(p.N / 64, (p.M + 8 * NT - 1) / (8 * NT)), dim3(D_THREADS), smem, stream);
   e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT, GPW>, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16 launch: ") + cudaGetErrorString(e));
@@ -251,9 +260,10 @@ extern "C" int awq_linear_w4a16(const void *X, int M, int K, int ldx, const floa
                                 int ldy, svdq_stream_t stream) {
   if (!X || !qweight || !scales || !zeros || !Y) return fail(SVDQ_ERR_INVALID_ARG, "awq_linear_w4a16: null pointer");
   if (group != 64) return fail(SVDQ_ERR_SHAPE, "awq_linear_w4a16: group must be 64");
-  if (M < 1 || M > 16 || K < 64 || K % 64 || N < 64 || N % 64 || ldx < K || ldx % 8 || ldy < N || ldy % 8)
-    return fail(SVDQ_ERR_SHAPE,
-                "awq_linear_w4a16: need 1 <= M <= 16, K % 64 == 0, N % 64 == 0, ldx >= K, ldy >= N, ldx/ldy % 8 == 0");
+  if (M < 1 || M > 65535 * 16 || K < 64 || K % 64 || N < 64 || N % 64 || ldx < K || ldx % 8 || ldy < N ||
+      ldy % 8)
+    return fail(SVDQ_ERR_SHAPE, "awq_linear_w4a16: need 1 <= M <= 1048560, K % 64 == 0, N % 64 == 0, ldx >= K, "
+                                "ldy >= N, ldx/ldy % 8 == 0");
   if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
       (inv_awq && !aligned16(inv_awq)) || !aligned16(Y))
     return fail(SVDQ_ERR_ALIGNMENT, "awq_linear_w4a16: pointers must be 16-byte aligned");

@@ -72,7 +72,7 @@ class SVDQLinear:
 
 
 class AWQLinear:
-    """Y = (X diag(inv_awq)) deq(W_a) + b with 4-bit group-64 weights (M <= 16)."""
+    """Y = (X diag(inv_awq)) deq(W_a) + b with 4-bit group-64 weights (any M; blocks of 16 rows)."""
 
     def __init__(self, packed, K, N, bias_bits=None, device="cuda"):
         self.K, self.N = K, N

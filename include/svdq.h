@@ -225,8 +225,9 @@ int awq_pack_weights(const uint16_t *W, int K, int N, const float *awq_scale, in
  * in fp32.  X [M][ldx] bf16; inv_awq [K] f32 or NULL (= 1); bias [N] or NULL.
  * The products run on tensor cores with X^ split into bf16 hi + lo parts
  * (relative error of the split ~2^-17).
- * Rules: 1 <= M <= 16, group == 64, K % 64 == 0, N % 64 == 0, ldx >= K,
- * ldy >= N, ldx % 8 == 0, ldy % 8 == 0.
+ * Rules: 1 <= M <= 1048560, group == 64, K % 64 == 0, N % 64 == 0, ldx >= K,
+ * ldy >= N, ldx % 8 == 0, ldy % 8 == 0.  Up to 16 rows are one pass over
+ * the weights; more rows run as blocks of 16, one pass each (from L2).
  */
 int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq,
                      const uint32_t *qweight, const void *scales, const void *zeros, int group,

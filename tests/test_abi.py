@@ -60,8 +60,10 @@ def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
     assert b"K % 64" in so.svdq_last_error_string()
     rc = so.svdq_linear_w4a4(p, p, p, p, p, p, None, 64, 256, 256, 16, 7, 0, p, 256, None)
     assert rc == lib.ERR_INVALID_ARG
-    rc = so.awq_linear_w4a16(p, 17, 256, 256, None, p, p, p, 64, None, 256, p, 256, None)
-    assert rc == lib.ERR_SHAPE
+    rc = so.awq_linear_w4a16(p, 17, 256, 256, None, p, p, p, 64, None, 96, p, 96, None)
+    assert rc == lib.ERR_SHAPE                                    # N % 64
+    rc = so.awq_linear_w4a16(p, 0, 256, 256, None, p, p, p, 64, None, 256, p, 256, None)
+    assert rc == lib.ERR_SHAPE                                    # M < 1
     odd = ctypes.c_void_p(24)
     rc = so.svdq_linear_w4a4(odd, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None)
     assert rc == lib.ERR_ALIGNMENT

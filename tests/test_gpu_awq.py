@@ -41,8 +41,8 @@ def _run(m, k, n, seed, with_bias=True, use_inv=True):
     # groups past K, more 64-column quads than SMs, 2-3 ring stages when X^ is large
     (1, 64, 64), (2, 192, 128), (5, 1024, 320), (8, 512, 64), (2, 2048, 128), (4, 4096, 192),
     (2, 6144, 64), (7, 1600, 256), (8, 1024, 12800), (8, 12288, 128),
-    # direct kernel (M > 8)
-    (9, 256, 192), (16, 3072, 512), (12, 4096, 128)])
+    # direct kernel (M > 8), and blocks of 16 rows beyond 16 (a full and a ragged last block)
+    (9, 256, 192), (16, 3072, 512), (12, 4096, 128), (32, 1024, 256), (45, 3072, 192)])
 def test_awq_parity(m, k, n):
     assert _run(m, k, n, seed=m + k + n) <= 1e-2
 

@@ -15,22 +15,22 @@
 // and every MMA is a cta_group::2 MMA of 256 x 256 x 64: CTA h of the pair
 // holds rows 128h..128h+127 of the activation tile and weight rows (output
 // columns) 128h..128h+127 of the weight tile, and its TMEM receives its own
-// 128 rows of the accumulator.  Each SM therefore loads 38 KB per k-stage
-// (its half of A and of B, plus the full 256-column block-scale slice that
-// both TMEMs need) instead of the 54 KB a one-SM 128 x 256 tile needs for the
-// same MMA time; the per-SM operand intake of the L2 fabric is what limits a
-// one-SM tile.
+// 128 rows of the accumulator.  Each SM therefore loads its half of A and
+// of B per k-stage (32 KB of codes) plus the scales: its 128 rows of A
+// scales and the B scales of all 256 weight rows that both TMEMs need.
 //
 // Roles (one CTA per SM, persistent over pair tiles, 12 warps):
-//   warp 0      producer in both CTAs: per stage three TMA copies into its
-//               own shared memory (A half with its scales, B half, B scales),
-//               all completing on the even CTA's `full` barrier
+//   warp 0      producer in both CTAs: per stage four TMA copies into its
+//               own shared memory - the A and B scales first, completing on
+//               the even CTA's `sf_loaded` barrier, then the A and B code
+//               halves, completing on its `full` barrier
 //   warp 1      owns TMEM (pair allocation); in the even CTA it issues the
 //               MMAs from one thread and commits each stage to both CTAs'
 //               `empty` barriers
 //   warp 2      even CTA: moves each stage's block scales from both CTAs'
-//               shared memory into their TMEM (tcgen05.cp, cta_group::2);
-//               from its own warp the copies overlap the MMAs
+//               shared memory into their TMEM (tcgen05.cp, cta_group::2) as
+//               soon as `sf_loaded` completes; from its own warp the copies
+//               overlap the MMAs and the codes' transfer
 //   warps 4..11 epilogue in both CTAs: drain the CTA's 128 x 256 fp32
 //               accumulator, hand TMEM back (to the even CTA's barrier),
 //               then scale, add bias, GELU, round to bf16 into a

@@ -3,8 +3,8 @@
 // The pages give these precision-sensitive, low-compute projections 4-bit
 // weights and 16-bit activations (web page "Nunchaku Diffusers 支持降低显存占用，
 // 但硬件仍决定适用范围", remio.ai, section "Nunchaku Diffusers 支持改变了加载路径").
-// With M <= 16 rows the layer is one pass over the weights and the kernel is
-// bound by how many weight bytes are in flight:
+// With up to 16 rows the layer is one pass over the weights and the kernel
+// is bound by how many weight bytes are in flight:
 //   * one CTA per quad of 64 output columns, its 16 warps split K by groups
 //     of 64; before any arithmetic each warp requests all of its groups'
 //     weights (4 x 16 bytes per lane and group: the four 16-column blocks),

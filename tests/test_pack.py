@@ -25,7 +25,7 @@ def _case(m, k, n, seed, x_out=4, x_fac=30.0, w_out=2, w_fac=8.0):
     return xb, wb, x, amax
 
 
-@pytest.mark.parametrize("k,n,rank", [(256, 256, 16), (128, 64, 0), (192, 128, 32)])
+@pytest.mark.parametrize("k,n,rank", [(256, 256, 16), (128, 64, 0), (192, 128, 32), (320, 264, 16)])
 def test_pack_matches_oracle(k, n, rank):
     xb, wb, x, amax = _case(64, k, n, seed=k + n + rank)
     p = lib.svdq_pack_weights(wb, amax, rank, want_residual=True)
@@ -90,6 +90,7 @@ def test_host_quantizer_matches_oracle_bit_exactly():
         gc, gsf = layouts.bundle_unpack(bundle, 70, 320, th)
         np.testing.assert_array_equal(gc, oc)
         np.testing.assert_array_equal(gsf, osf)
+        assert layouts.scale_replicas_agree(bundle, 70, 320, th)
         assert layouts.bundle_padding_is_zero(bundle, 70, 320, th)
     oc1, osf1 = nvfp4.quantize_blocks(t[3:4], F32(1.0))
     c1, _ = layouts.bundle_unpack(lib.svdq_quantize_host(t[3:4].copy(), 1.0), 1, 320, 128)

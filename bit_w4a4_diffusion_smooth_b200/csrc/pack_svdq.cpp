@@ -122,19 +122,26 @@ void parallel_for(int n, int threads, const std::function<void(int, int)> &fn) {
 }
 
 // Dense row-major helpers.  A is [rows][cols].
-// Y[rows][p] = A . X, X [cols][p]
+// Y[rows][p] = A . X, X [cols][p].  Four rows of A share each pass over X;
+// every output still sums its terms in order j = 0, 1, ...
 void mul_a_x(const double *A, int rows, int cols, const double *X, int p, double *Y, int threads) {
-  parallel_for(rows, threads, [&](int b, int e) {
-    std::vector<double> acc(p);
-    for (int i = b; i < e; ++i) {
+  parallel_for((rows + 3) / 4, threads, [&](int b, int e) {
+    std::vector<double> acc(4 * static_cast<size_t>(p));
+    for (int i0 = 4 * b; i0 < std::min(rows, 4 * e); i0 += 4) {
+      const int nr = std::min(4, rows - i0);
       std::fill(acc.begin(), acc.end(), 0.0);
-      const double *a = A + static_cast<size_t>(i) * cols;
+      const double *a = A + static_cast<size_t>(i0) * cols;
       for (int j = 0; j < cols; ++j) {
-        double aij = a[j];
         const double *x = X + static_cast<size_t>(j) * p;
-        for (int t = 0; t < p; ++t) acc[t] += aij * x[t];
+        for (int r = 0; r < nr; ++r) {
+          const double arj = a[static_cast<size_t>(r) * cols + j];
+          double *ac = acc.data() + static_cast<size_t>(r) * p;
+          for (int t = 0; t < p; ++t) ac[t] += arj * x[t];
+        }
       }
-      std::copy(acc.begin(), acc.end(), Y + static_cast<size_t>(i) * p);
+      for (int r = 0; r < nr; ++r)
+        std::copy(acc.begin() + static_cast<size_t>(r) * p, acc.begin() + static_cast<size_t>(r + 1) * p,
+                  Y + static_cast<size_t>(i0 + r) * p);
     }
   });
 }
@@ -161,22 +168,31 @@ void mul_at_q(const double *A, int rows, int cols, const double *Q, int p, doubl
 }
 
 // Orthonormalize the p columns of Y [rows][p] in place (modified Gram-Schmidt,
-// applied twice for stability).  Columns that vanish are left zero.
+// applied twice for stability).  Columns that vanish are left zero.  The
+// columns are worked on in a column-major copy, so that every dot product and
+// update streams contiguous memory (the sums run over rows in the same order).
 void orthonormalize(double *Y, int rows, int p) {
+  std::vector<double> colmaj(static_cast<size_t>(rows) * p);
+  for (int i = 0; i < rows; ++i)
+    for (int c = 0; c < p; ++c) colmaj[static_cast<size_t>(c) * rows + i] = Y[static_cast<size_t>(i) * p + c];
   for (int pass = 0; pass < 2; ++pass) {
     for (int c = 0; c < p; ++c) {
+      double *yc = colmaj.data() + static_cast<size_t>(c) * rows;
       for (int d = 0; d < c; ++d) {
+        const double *yd = colmaj.data() + static_cast<size_t>(d) * rows;
         double dot = 0.0;
-        for (int i = 0; i < rows; ++i) dot += Y[static_cast<size_t>(i) * p + c] * Y[static_cast<size_t>(i) * p + d];
-        for (int i = 0; i < rows; ++i) Y[static_cast<size_t>(i) * p + c] -= dot * Y[static_cast<size_t>(i) * p + d];
+        for (int i = 0; i < rows; ++i) dot += yc[i] * yd[i];
+        for (int i = 0; i < rows; ++i) yc[i] -= dot * yd[i];
       }
       double nrm = 0.0;
-      for (int i = 0; i < rows; ++i) nrm += Y[static_cast<size_t>(i) * p + c] * Y[static_cast<size_t>(i) * p + c];
+      for (int i = 0; i < rows; ++i) nrm += yc[i] * yc[i];
       nrm = std::sqrt(nrm);
       double inv = nrm > 0.0 ? 1.0 / nrm : 0.0;
-      for (int i = 0; i < rows; ++i) Y[static_cast<size_t>(i) * p + c] *= inv;
+      for (int i = 0; i < rows; ++i) yc[i] *= inv;
     }
   }
+  for (int i = 0; i < rows; ++i)
+    for (int c = 0; c < p; ++c) Y[static_cast<size_t>(i) * p + c] = colmaj[static_cast<size_t>(c) * rows + i];
 }
 
 // Eigen-decomposition of the symmetric p x p matrix C (row-major) by cyclic

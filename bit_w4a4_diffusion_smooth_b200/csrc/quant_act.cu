@@ -10,10 +10,11 @@
 //     written as 128-row swizzled tiles.
 //
 // Design (X is read once, ~0.3 B written per byte read):
-//   * one CTA per 32 rows, 16 compute warps + 1 TMA warp; a ring of stages,
-//     each a [32 rows x 256 cols] bf16 tile of X, an [r x 256] tile of L1^T
-//     (one 3-D TMA copy each, as four 64-column boxes with the 128-byte
-//     swizzle) and the stage's 256-float slice of inv_lambda (a bulk copy);
+//   * one CTA per 32 rows, 16 compute warps + 1 TMA warp + 1 store warp; a
+//     ring of stages, each a [32 rows x 256 cols] bf16 tile of X, an
+//     [r x 256] tile of L1^T (one 3-D TMA copy each, as four 64-column boxes
+//     with the 128-byte swizzle), the stage's 256-float slice of inv_lambda
+//     (a bulk copy) and a staging area for the stage's codes and scales;
 //   * compute warp w owns the 16-column slice w of every stage for all 32
 //     rows.  It loads the slice once, with ldmatrix, straight into the
 //     m16n8k16 A-fragment layout: lane (g, t) holds columns 2t, 2t+1, 2t+8,
@@ -27,11 +28,14 @@
 //     call, so f32(1 / f32(e4m3 * s_a)) has only 128 values); the four
 //     1/scale values come back by shuffles, every lane converts its 16
 //     elements, and a second butterfly gathers each block's 8 code bytes in
-//     its owner lane for one 8-byte store (plus one scale byte);
+//     its owner lane, which puts them (and the scale byte) into the staging
+//     area in the bundle's byte order;
+//   * the store warp copies each staged stage out with full-line stores (a
+//     CTA's code rows are 4 KB of contiguous bundle) and frees the stage;
 //   * warps never meet inside the loop: each waits for its stage with a
 //     bounded mbarrier wait (decided warp-uniformly; a warp whose wait runs
-//     out records SVDQ_ERR_TIMEOUT and leaves the loop) and releases it with
-//     one arrive.  At the end the 16 per-slice partial U tiles are added in
+//     out records SVDQ_ERR_TIMEOUT and leaves the loop) and signals the store
+//     warp with one arrive.  At the end the 16 per-slice partial U tiles are added in
 //     shared memory and written as 128-row swizzled tiles.
 #include <cuda.h>
 #include <cuda_runtime.h>

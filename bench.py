@@ -1,24 +1,34 @@
 """Throughput of the SVDQuant W4A4 linear (+ AWQ W4A16 projection) on B200.
 
-One step = the whole hot path over one batch of synthetic input:
-  K1  activation quantize + low-rank down-projection   X [4608 x 3072] bf16
-  K2  tcgen05 NVFP4 GEMM + low-rank up-projection      -> Y [4608 x 9216] bf16
-  K3  AWQ W4A16 projection                             [2 x 3072] -> [2 x 18432]
-(the attention-QKV-shaped layer of a 12B-class DiT at 1024x1024: 4096 image +
-512 text tokens, rank 32; and its adaLN modulation projection).
+One step = the whole hot path over one batch of synthetic input, on the layer
+shapes of one block of a 12B-class DiT at 1024x1024 (4096 image + 512 text
+tokens, rank 32):
+  qkv   K1 + K2    X [4608 x 3072] -> [4608 x 9216]
+  fc1   K1 + K2    X [4608 x 3072] -> H [4608 x 12288], GELU (erf) epilogue
+  fc2   K1 + K2    H [4608 x 12288] -> [4608 x 3072]   (fc1's output re-quantized)
+  adaLN K3         [2 x 3072] -> [2 x 18432]           (AWQ W4A16, group 64)
+K1 = activation quantize + low-rank down-projection, K2 = tcgen05 NVFP4 GEMM +
+low-rank up-projection + epilogue, K3 = W4A16 GEMV.
 
 value = algorithmic FLOPs of the step / step time (TFLOP/s, all ranks).
-Inputs rotate over buffer sets that together exceed twice the L2 cache, so no
-step reads what the previous one left in L2.  Multi-GPU runs are independent
-replicas (the layer needs no exchange between GPUs): weak scaling.
+Weights, inputs, intermediates and outputs rotate over buffer sets that
+together exceed twice the L2 cache, so no step reads what the previous one
+left in L2.  Multi-GPU runs are independent replicas (the layer needs no
+exchange between GPUs): weak scaling.
+
+After the timed region every kernel of the step is timed alone, back to back
+over the rotating sets, so that the per-kernel figures carry no event between
+two different kernels; the roofline object reports the fc1 GEMM
+(4608 x 3072 x 12288 with GELU), the largest kernel of the step.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                       [--workload qkv|dit-step]
+                       [--workload layers|dit-step]
 
 --workload dit-step times every projection linear of one denoising step of a
 12B-class DiT (228 W4A4 layers + 76 AWQ projections) as one CUDA graph.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -32,32 +42,52 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-M, K, N, RANK = 4608, 3072, 9216, 32
-AM, AK, AN = 2, 3072, 18432
-WORKLOAD = ("attention-QKV SVDQ W4A4 linear 4608x3072->9216 rank 32 (NVFP4, group 16) "
+RANK = 32
+TOKENS, HIDDEN, MLP = 4608, 3072, 12288
+# name -> (M, K, N, GELU epilogue); fc2 reads fc1's output
+LAYERS = {"qkv": (TOKENS, HIDDEN, 3 * HIDDEN, False),
+          "fc1": (TOKENS, HIDDEN, MLP, True),
+          "fc2": (TOKENS, MLP, HIDDEN, False)}
+AM, AK, AN = 2, HIDDEN, 6 * HIDDEN
+WORKLOAD = ("one 12B-class DiT block's SVDQ W4A4 linears at 4608 tokens, rank 32 (NVFP4, group 16): "
+            "QKV 3072->9216, MLP fc1 3072->12288 +GELU then fc2 12288->3072 on fc1's output; "
             "+ AWQ W4A16 adaLN projection 2x3072->18432 (INT4, group 64)")
 METRIC = "SVDQ W4A4 linear TFLOPS and % of B200 dense-FP4 peak; W4A16 GB/s vs HBM"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FP4_OVER_BF16 = 4.0  # nominal dense FP4 / dense bf16 ratio (9 / 2.25 PFLOP/s)
+FP4_OVER_BF16 = 4.0            # nominal dense FP4 / dense bf16 ratio (9 / 2.25 PFLOP/s)
+FP4_NOMINAL_TFLOPS = 9000.0    # NVIDIA's dense FP4 figure for B200
 
-W4A4_FLOPS = 2 * M * K * N                # 4-bit main branch
-LOWRANK_FLOPS = 2 * M * K * RANK + 2 * M * RANK * N
+
+def gemm_flops(m, k, n, r=RANK):
+    """FP4 main branch + the low-rank up-projection done inside K2."""
+    return 2 * m * k * n + 2 * m * r * n
+
+
+def layer_flops(m, k, n, r=RANK):
+    """The whole SVDQ layer: K2's work + K1's low-rank down-projection."""
+    return gemm_flops(m, k, n, r) + 2 * m * k * r
+
+
 AWQ_FLOPS = 2 * AM * AK * AN
-STEP_FLOPS = W4A4_FLOPS + LOWRANK_FLOPS + AWQ_FLOPS
-# Algorithmic bytes per launch (each byte the kernel must move once).
-K1_BYTES = (M * K * 2 + K * RANK * 2 + K * 4            # X, L1T, inv_lambda
-            + M * K // 2 + M * K // 16 + M * RANK * 2)  # codes, scales, U
-K2_BYTES = (M * K // 2 + M * K // 16 + M * RANK * 2     # activation codes, scales, U
-            + N * K // 2 + N * K // 16 + N * RANK * 2   # weight codes, scales, L2T
-            + N * 2 + M * N * 2)                        # bias, Y
-K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2    # qweight, scales + zeros
+STEP_FLOPS = sum(layer_flops(m, k, n) for m, k, n, _ in LAYERS.values()) + AWQ_FLOPS
+
+
+def k1_bytes(m, k, r=RANK):
+    """Algorithmic bytes of K1: X, L1T, inv_lambda in; codes, scales, U out."""
+    return m * k * 2 + k * r * 2 + k * 4 + m * k // 2 + m * k // 16 + m * r * 2
+
+
+def k2_bytes(m, k, n, r=RANK):
+    return (m * k // 2 + m * k // 16 + m * r * 2 + n * k // 2 + n * k // 16 + n * r * 2 + n * 2 + m * n * 2)
+
+
+K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2      # qweight, scales + zeros
             + AM * AK * 2 + AK * 4 + AN * 2 + AM * AN * 2)
-# DRAM bytes of one K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the ncu capture
-# summarised in profiles/gemm_w4a4_qkv_4608x3072x9216.md; None until that capture matches the
-# current K2 again.
-K2_TRAFFIC_BYTES = 33_172_992 + 46_266_880
-# Steps of the timed region that carry per-kernel CUDA events (1 in EV_EVERY).
-EV_EVERY = 16
+
+# DRAM traffic of one fc1-shaped K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
+# ncu capture summarised in profiles/, and the hash of the GEMM source it was taken on: when the
+# source has changed since, the counters no longer describe the kernel and `traffic` is null.
+K2_TRAFFIC = {"bytes": None, "source_sha16": None}
 
 
 def peaks():
@@ -67,6 +97,12 @@ def peaks():
         return p, "measured"
     except (OSError, ValueError):
         return PEAKS_FALLBACK, "fallback"
+
+
+def source_sha16(name):
+    path = os.path.join(ROOT, "bit_w4a4_diffusion_smooth_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
 def dist_env():
@@ -102,7 +138,7 @@ def aggregate_tflops(flops_per_replica_step, world, ms_per_step):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU is under the bench's load."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -157,60 +193,196 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ our arm
-def setup(device, sets):
+def _bf(bits):
     import torch
-
-    from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
-
-    lib.svdq_init(device.index)
-    c = synthetic.QKV
-    xb, wb, bb = c.make()
-    x = synthetic.bf16_bits_to_f32(xb)
-    amax = np.max(np.abs(x), axis=0).astype(np.float32)
-    packed = lib.svdq_pack_weights(wb, amax, RANK, seed=c.seed)
-    a = synthetic.AWQ
-    axb, awb, abb, asc = a.make()
-    apk = lib.awq_pack_weights(awb, asc)
-
-    def bf(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
-
-    def t(arr):
-        return torch.from_numpy(np.ascontiguousarray(arr))
-
-    host = dict(X=bf(xb).pin_memory(), AX=bf(axb).pin_memory())
-    sz = lib.svdq_act_sizes(M, K)
-    S = []
-    for _ in range(sets):
-        S.append(dict(
-            X=bf(xb).to(device), inv_lambda=t(packed["inv_lambda"]).to(device), l1t=bf(packed["l1t"]).to(device),
-            l2t=t(packed["l2t"]).to(device), w_bundle=t(packed["w_bundle"]).to(device),
-            s_w=t(packed["s_w"]).to(device), s_a=t(packed["s_a"]).to(device), bias=bf(bb).to(device),
-            a_bundle=torch.empty(sz["a_bundle"], dtype=torch.uint8, device=device),
-            U=torch.empty(sz["u"], dtype=torch.uint8, device=device),
-            Y=torch.empty((M, N), dtype=torch.bfloat16, device=device),
-            AX=bf(axb).to(device), qweight=t(apk["qweight"]).to(device), ascales=bf(apk["scales"]).to(device),
-            azeros=bf(apk["zeros"]).to(device), inv_awq=t(apk["inv_awq"]).to(device), abias=bf(abb).to(device),
-            AY=torch.empty((AM, AN), dtype=torch.bfloat16, device=device)))
-    set_bytes = sum(v.numel() * v.element_size() for v in S[0].values())
-    return S, host, set_bytes
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
 
 
-def step(S, i, ev=None):
+def _t(arr):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(arr))
+
+
+class Workload:
+    """Packed weights (host pack of the library), inputs and buffers of the step, on one device,
+    as `sets` rotating copies."""
+
+    def __init__(self, device):
+        import torch
+
+        from bit_w4a4_diffusion_smooth_b200 import lib, synthetic
+
+        self.device = device
+        lib.svdq_init(device.index)
+        cases = {"qkv": synthetic.QKV, "fc1": synthetic.MLP_FC1, "fc2": synthetic.MLP_FC2}
+        self.host_w = {}
+        self.x_bits = {}
+        for name in ("qkv", "fc1"):
+            c = cases[name]
+            xb, wb, bb = c.make()
+            amax = np.max(np.abs(synthetic.bf16_bits_to_f32(xb)), axis=0).astype(np.float32)
+            self.x_bits[name] = xb
+            self.host_w[name] = (lib.svdq_pack_weights(wb, amax, RANK, seed=c.seed), bb)
+        # fc2: calibrated on fc1's output for this input (one untimed fc1 pass on the device)
+        c2 = cases["fc2"]
+        wb2, _ = synthetic.weight(c2.k, c2.n, c2.seed, 0.02, c2.w_outlier_rows, c2.w_factor)
+        bb2 = synthetic.bias(c2.n, c2.seed + 100)
+        one = self._layer_dev("fc1")
+        xs = _bf(self.x_bits["fc1"]).to(device)
+        sz = lib.svdq_act_sizes(TOKENS, HIDDEN)
+        ab = torch.empty(sz["a_bundle"], dtype=torch.uint8, device=device)
+        u = torch.empty(sz["u"], dtype=torch.uint8, device=device)
+        h = torch.empty((TOKENS, MLP), dtype=torch.bfloat16, device=device)
+        lib.svdq_quantize_act(xs, one["inv_lambda"], one["l1t"], RANK, one["s_a"], one["s_w"], ab, u)
+        lib.svdq_linear_w4a4(ab, u, one["s_a"], one["w_bundle"], one["l2t"], one["s_w"], one["bias"],
+                             TOKENS, MLP, HIDDEN, RANK, lib.EPILOGUE_GELU_ERF, 0, h)
+        amax2 = h.float().abs().amax(dim=0).cpu().numpy().astype(np.float32)
+        self.host_w["fc2"] = (lib.svdq_pack_weights(wb2, amax2, RANK, seed=c2.seed), bb2)
+        del one, xs, ab, u, h
+        a = synthetic.AWQ
+        axb, awb, abb, asc = a.make()
+        self.awq_x_bits = axb
+        self.host_awq = (lib.awq_pack_weights(awb, asc), abb)
+        self.sets = []
+
+    def _layer_dev(self, name):
+        p, bb = self.host_w[name]
+        d = self.device
+        return dict(inv_lambda=_t(p["inv_lambda"]).to(d), l1t=_bf(p["l1t"]).to(d), l2t=_t(p["l2t"]).to(d),
+                    w_bundle=_t(p["w_bundle"]).to(d), s_w=_t(p["s_w"]).to(d), s_a=_t(p["s_a"]).to(d),
+                    bias=_bf(bb).to(d))
+
+    def add_set(self):
+        import torch
+
+        from bit_w4a4_diffusion_smooth_b200 import lib
+        d = self.device
+        s = {}
+        for name, (m, k, n, _) in LAYERS.items():
+            L = self._layer_dev(name)
+            sz = lib.svdq_act_sizes(m, k)
+            L["a_bundle"] = torch.empty(sz["a_bundle"], dtype=torch.uint8, device=d)
+            L["U"] = torch.empty(sz["u"], dtype=torch.uint8, device=d)
+            L["Y"] = torch.empty((m, n), dtype=torch.bfloat16, device=d)
+            s[name] = L
+        s["qkv"]["X"] = _bf(self.x_bits["qkv"]).to(d)
+        s["fc1"]["X"] = _bf(self.x_bits["fc1"]).to(d)
+        s["fc2"]["X"] = s["fc1"]["Y"]                    # fc2 re-quantizes fc1's output
+        apk, abb = self.host_awq
+        s["awq"] = dict(X=_bf(self.awq_x_bits).to(d), qweight=_t(apk["qweight"]).to(d),
+                        scales=_bf(apk["scales"]).to(d), zeros=_bf(apk["zeros"]).to(d),
+                        inv_awq=_t(apk["inv_awq"]).to(d), bias=_bf(abb).to(d),
+                        Y=torch.empty((AM, AN), dtype=torch.bfloat16, device=d))
+        self.sets.append(s)
+        seen, total = set(), 0
+        for part in s.values():
+            for v in part.values():
+                if v.data_ptr() not in seen:
+                    seen.add(v.data_ptr())
+                    total += v.numel() * v.element_size()
+        return total
+
+
+def k1(L, name):
     from bit_w4a4_diffusion_smooth_b200 import lib
-    s = S[i % len(S)]
-    if ev is not None:
-        ev[0].record()
-    lib.svdq_quantize_act(s["X"], s["inv_lambda"], s["l1t"], RANK, s["s_a"], s["s_w"], s["a_bundle"], s["U"])
-    if ev is not None:
-        ev[1].record()
-    lib.svdq_linear_w4a4(s["a_bundle"], s["U"], s["s_a"], s["w_bundle"], s["l2t"], s["s_w"], s["bias"],
-                         M, N, K, RANK, 0, 0, s["Y"])
-    if ev is not None:
-        ev[2].record()
-    lib.awq_linear_w4a16(s["AX"], s["inv_awq"], s["qweight"], s["ascales"], s["azeros"], s["abias"], AN, s["AY"])
-    if ev is not None:
-        ev[3].record()
+    m, k, n, _ = LAYERS[name]
+    lib.svdq_quantize_act(L["X"], L["inv_lambda"], L["l1t"], RANK, L["s_a"], L["s_w"], L["a_bundle"], L["U"],
+                          M=m, K=k)
+
+
+def k2(L, name):
+    from bit_w4a4_diffusion_smooth_b200 import lib
+    m, k, n, gelu = LAYERS[name]
+    lib.svdq_linear_w4a4(L["a_bundle"], L["U"], L["s_a"], L["w_bundle"], L["l2t"], L["s_w"], L["bias"], m, n, k,
+                         RANK, lib.EPILOGUE_GELU_ERF if gelu else lib.EPILOGUE_NONE, 0, L["Y"])
+
+
+def k3(A):
+    from bit_w4a4_diffusion_smooth_b200 import lib
+    lib.awq_linear_w4a16(A["X"], A["inv_awq"], A["qweight"], A["scales"], A["zeros"], A["bias"], AN, A["Y"])
+
+
+# the step's kernels in order: (label, function of one buffer set)
+STEP_KERNELS = [
+    ("K1 qkv", lambda s: k1(s["qkv"], "qkv")), ("K2 qkv", lambda s: k2(s["qkv"], "qkv")),
+    ("K1 fc1", lambda s: k1(s["fc1"], "fc1")), ("K2 fc1", lambda s: k2(s["fc1"], "fc1")),
+    ("K1 fc2", lambda s: k1(s["fc2"], "fc2")), ("K2 fc2", lambda s: k2(s["fc2"], "fc2")),
+    ("K3 adaLN", lambda s: k3(s["awq"])),
+]
+
+
+def step(sets, i):
+    s = sets[i % len(sets)]
+    for _, fn in STEP_KERNELS:
+        fn(s)
+
+
+def kernel_table(pk):
+    """label -> (algorithmic amount per launch, unit, bound, peak)."""
+    fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
+    t = {}
+    for name, (m, k, n, _) in LAYERS.items():
+        t[f"K1 {name}"] = (k1_bytes(m, k), "GB/s", "hbm", pk["hbm_gbs"])
+        t[f"K2 {name}"] = (gemm_flops(m, k, n), "TFLOP/s", "tensor", fp4_peak)
+    t["K3 adaLN"] = (K3_BYTES, "GB/s", "hbm", pk["hbm_gbs"])
+    return t
+
+
+def time_back_to_back(fn, sets, reps):
+    """Mean device time (ms) of `fn` launched `reps` times in a row over the rotating sets."""
+    import torch
+    for i in range(2):
+        fn(sets[i % len(sets)])
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        fn(sets[i % len(sets)])
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def copy_floor(device, nbytes, pairs=8, reps=24):
+    """A library copy of `nbytes` (torch, device to device) from cold buffers: the HBM rate a plain
+    stream of this size reaches on this GPU, as (GB/s counting read + write, us per copy)."""
+    import torch
+    n = nbytes // 2
+    src = [torch.empty(n, dtype=torch.bfloat16, device=device).fill_(1.0) for _ in range(pairs)]
+    dst = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(pairs)]
+    bufs = list(zip(src, dst))
+    ms = time_back_to_back(lambda b: b[1].copy_(b[0]), bufs, reps)
+    del src, dst, bufs
+    return 2 * nbytes / (ms * 1e-3) / 1e9, ms * 1e3
+
+
+def fp4_library_point(device, m, k, n, reps=20):
+    """torch._scaled_mm (cuBLASLt) on NVFP4 operands of the same shape as a library reference
+    point: e2m1 A [m, k] and B [n, k], ue4m3 block scales of 16 in the blocked layout.  Returns
+    (TFLOP/s of the 2mkn product, us) or an error string when the call is not supported here."""
+    import torch
+    try:
+        fp4 = torch.float4_e2m1fn_x2
+        sets = []
+        for i in range(6):          # > L2 in total
+            a = (torch.randint(0, 256, (m, k // 2), dtype=torch.uint8, device=device) & 0x77).view(fp4)
+            b = (torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=device) & 0x77).view(fp4)
+            rm, rn, rk = (m + 127) // 128 * 128, (n + 127) // 128 * 128, (k // 16 + 3) // 4 * 4
+            sa = torch.full((rm * rk,), 0x38, dtype=torch.uint8, device=device).view(torch.float8_e4m3fn)
+            sb = torch.full((rn * rk,), 0x38, dtype=torch.uint8, device=device).view(torch.float8_e4m3fn)
+            sets.append((a, b, sa, sb))
+
+        def run(s):
+            return torch._scaled_mm(s[0], s[1].t(), s[2], s[3], out_dtype=torch.bfloat16)
+
+        y = run(sets[0])
+        torch.cuda.synchronize()
+        if tuple(y.shape) != (m, n):
+            return f"unexpected output shape {tuple(y.shape)}"
+        ms = time_back_to_back(run, sets, reps)
+        return 2 * m * k * n / (ms * 1e-3) / 1e12, ms * 1e3
+    except Exception as e:  # noqa: BLE001 - a reference point only: record why it is missing
+        return f"{type(e).__name__}: {str(e).splitlines()[0][:200]}"
 
 
 def run_ours(args):
@@ -224,11 +396,11 @@ def run_ours(args):
     torch.cuda.set_device(device)
     init_replicas(world, "nccl", device)
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    sets = 4
-    S, host, set_bytes = setup(device, sets)
-    while sets * set_bytes < 2 * l2:
-        sets += 1
-        S, host, set_bytes = setup(device, sets)
+    W = Workload(device)
+    set_bytes = W.add_set()
+    while len(W.sets) < 2 or len(W.sets) * set_bytes < 2 * l2:
+        W.add_set()
+    sets = W.sets
 
     def barrier():
         if world > 1:
@@ -236,14 +408,12 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     for i in range(args.warmup):
-        step(S, i)
+        step(sets, i)
     rc = lib.svdq_check_status()
     if rc != lib.OK:
         raise RuntimeError(f"device status after warm-up: {lib.status_name(rc)}")
 
-    # ---- device-timed region: K steps; per-kernel events on every EV_EVERY-th step only, since an
-    # event between two kernels keeps the next one from launching early (dependent launches)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(0, args.steps, EV_EVERY)]
+    # ---- device-timed region: exactly K steps between two events on the launching stream
     clocks = ClockSampler(local)
     clocks.start()
     barrier()
@@ -251,14 +421,14 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for i in range(args.steps):
-        step(S, i, evs[i // EV_EVERY] if i % EV_EVERY == 0 else None)
+        step(sets, i)
     t1.record()
     barrier()
-    clk = clocks.stop()
     ms = t0.elapsed_time(t1)
-    k1 = sum(e[0].elapsed_time(e[1]) for e in evs) / len(evs)
-    k2 = sum(e[1].elapsed_time(e[2]) for e in evs) / len(evs)
-    k3 = sum(e[2].elapsed_time(e[3]) for e in evs) / len(evs)
+    # ---- each kernel alone, back to back over the rotating sets (no event between two different
+    # kernels); the clock sampler keeps running under this load
+    per = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in STEP_KERNELS}
+    clk = clocks.stop()
     rc = lib.svdq_check_status()
     if rc != lib.OK:
         raise RuntimeError(f"device status after timing: {lib.status_name(rc)}")
@@ -267,8 +437,11 @@ def run_ours(args):
     # inputs in from pinned host memory and its outputs back out; the uploads, the kernels and
     # the downloads of consecutive steps run on three streams (the two DMA directions and the
     # compute stream), ordered by events, over the rotating device buffer sets.
-    yh = [torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
-    ayh = [torch.empty((AM, AN), dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    host_in = {"qkv": _bf(W.x_bits["qkv"]).pin_memory(), "fc1": _bf(W.x_bits["fc1"]).pin_memory(),
+               "awq": _bf(W.awq_x_bits).pin_memory()}
+    outs = (("qkv", (TOKENS, 3 * HIDDEN)), ("fc2", (TOKENS, HIDDEN)), ("awq", (AM, AN)))
+    host_out = [{k: torch.empty(shape, dtype=torch.bfloat16, pin_memory=True) for k, shape in outs}
+                for _ in range(2)]
     e_steps = max(3, min(args.steps, 20))
     main_s = torch.cuda.current_stream(device)
     in_s, out_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
@@ -282,30 +455,40 @@ def run_ours(args):
     in_s.wait_event(e0)
     out_s.wait_event(e0)
     for i in range(e_steps):
-        s = S[i % len(S)]
+        s = sets[i % len(sets)]
         with torch.cuda.stream(in_s):
-            if i >= len(S):
-                in_s.wait_event(ev_done[i - len(S)])    # the set's previous inputs have been consumed
-            s["X"].copy_(host["X"], non_blocking=True)
-            s["AX"].copy_(host["AX"], non_blocking=True)
+            if i >= len(sets):
+                in_s.wait_event(ev_done[i - len(sets)])    # the set's previous inputs have been consumed
+            for k, v in host_in.items():
+                s[k]["X"].copy_(v, non_blocking=True)
             ev_in[i].record(in_s)
         main_s.wait_event(ev_in[i])
-        if i >= len(S):
-            main_s.wait_event(ev_out[i - len(S)])       # the set's previous outputs have been read out
-        step(S, i)
+        if i >= len(sets):
+            main_s.wait_event(ev_out[i - len(sets)])       # the set's previous outputs have been read out
+        step(sets, i)
         ev_done[i].record(main_s)
         with torch.cuda.stream(out_s):
             out_s.wait_event(ev_done[i])
-            yh[i % 2].copy_(s["Y"], non_blocking=True)
-            ayh[i % 2].copy_(s["AY"], non_blocking=True)
+            for k, _ in outs:
+                host_out[i % 2][k].copy_(s[k]["Y"], non_blocking=True)
             ev_out[i].record(out_s)
     main_s.wait_event(ev_out[e_steps - 1])
     e1.record(main_s)
     barrier()
     e2e_ms = e0.elapsed_time(e1) / e_steps
+    h2d = sum(v.numel() * 2 for v in host_in.values())
+    d2h = sum(v.numel() * 2 for v in host_out[0].values())
+
+    # ---- reference points on this GPU: a library copy of the activation's size, and cuBLASLt's
+    # NVFP4 GEMM on the fc1 shape
+    floor_gbs, floor_us = copy_floor(device, TOKENS * HIDDEN * 2)
+    fp4_lib = fp4_library_point(device, *LAYERS["fc1"][:3]) if not args.no_library_points else "skipped"
 
     # ---- max over ranks
-    ms, k1, k2, k3, e2e_ms = max_over_ranks([ms, k1, k2, k3, e2e_ms], world, device)
+    labels = [label for label, _ in STEP_KERNELS]
+    vals = max_over_ranks([ms, e2e_ms] + [per[x] for x in labels], world, device)
+    ms, e2e_ms = vals[0], vals[1]
+    per = dict(zip(labels, vals[2:]))
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -313,7 +496,20 @@ def run_ours(args):
     pk, how = peaks()
     fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
     ms_step = ms / args.steps
-    k2_tflops = (W4A4_FLOPS + 2 * M * RANK * N) / (k2 * 1e-3) / 1e12
+    table = kernel_table(pk)
+    kernels = {}
+    for label in labels:
+        amount, unit, bound, peak = table[label]
+        us = per[label] * 1e3
+        rate = amount / (us * 1e-6) / (1e9 if unit == "GB/s" else 1e12)
+        kernels[label] = {"us": round(us, 2), unit: round(rate, 1), "frac": round(rate / peak, 4)}
+    kernels["sum_us"] = round(sum(per.values()) * 1e3, 2)
+    kernels["timing"] = (f"each kernel alone, {args.kernel_reps} launches back to back over the rotating "
+                         "sets, after the timed region")
+    m, k, n, _ = LAYERS["fc1"]
+    k2_us = per["K2 fc1"] * 1e3
+    k2_tflops = gemm_flops(m, k, n) / (k2_us * 1e-6) / 1e12
+    traffic = K2_TRAFFIC["bytes"] if K2_TRAFFIC["source_sha16"] == source_sha16("gemm_w4a4.cu") else None
     line = {
         "metric": METRIC,
         "value": round(aggregate_tflops(STEP_FLOPS, world, ms_step), 2),
@@ -328,68 +524,83 @@ def run_ours(args):
         "dtype": "nvfp4 (e2m1 x e4m3-scaled, fp32 accumulate); bf16 low-rank; int4 x bf16",
         "data": "synthetic (seeded; outlier channels/rows as in the workload)",
         "config": {"workload": WORKLOAD, "parallelism": f"replicas x{world}",
-                   "l2": f"{len(S)} rotating input/output sets, {len(S) * set_bytes / 1e6:.0f} MB > 2x L2",
-                   "flops_per_step": STEP_FLOPS},
-        "roofline": {"bound": "tensor", "kernel": "svdq_linear_w4a4 (K2)",
+                   "l2": f"inputs larger than L2; {len(sets)} rotating sets of weights, inputs and outputs, "
+                         f"{len(sets) * set_bytes / 1e6:.0f} MB > 2x L2",
+                   "flops_per_step": STEP_FLOPS, "launches_per_step": len(STEP_KERNELS)},
+        "roofline": {"bound": "tensor", "kernel": "svdq_linear_w4a4, fc1 4608x3072x12288 +GELU",
                      "achieved": round(k2_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
-                     "frac": round(k2_tflops / fp4_peak, 4), "traffic": K2_TRAFFIC_BYTES,
+                     "frac": round(k2_tflops / fp4_peak, 4), "traffic": traffic,
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
-                     "peak_source": f"{how} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16)"},
-        "kernels": {
-            "K1_quantize_act": {"us": round(k1 * 1e3, 2), "GB/s": round(K1_BYTES / (k1 * 1e-3) / 1e9, 1),
-                                "frac_hbm": round(K1_BYTES / (k1 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-            "K2_linear_w4a4": {"us": round(k2 * 1e3, 2), "TFLOP/s": round(k2_tflops, 1),
-                               "frac_fp4": round(k2_tflops / fp4_peak, 4)},
-            "K3_awq_w4a16": {"us": round(k3 * 1e3, 2), "GB/s": round(K3_BYTES / (k3 * 1e-3) / 1e9, 1),
-                             "frac_hbm": round(K3_BYTES / (k3 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
-            "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how,
-            "events_on": f"{len(evs)} of {args.steps} timed steps (per-kernel CUDA events)",
-        },
+                     "peak_source": f"{how} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16)",
+                     "frac_of_nominal_9pf": round(k2_tflops / FP4_NOMINAL_TFLOPS, 4),
+                     "algorithmic": "2MKN (FP4) + 2MrN (low-rank up-projection) per launch"},
+        "kernels": kernels,
+        "reference_points": {
+            "hbm_copy_same_bytes": {"GB/s": round(floor_gbs, 1), "us": round(floor_us, 2),
+                                    "what": f"torch copy of {TOKENS}x{HIDDEN} bf16 (cold, read + write)"},
+            "cublaslt_nvfp4_fc1_shape": (
+                {"TFLOP/s": round(fp4_lib[0], 1), "us": round(fp4_lib[1], 2),
+                 "what": "torch._scaled_mm, NVFP4 A/B, block-16 e4m3 scales, bf16 out, no low-rank branch"}
+                if isinstance(fp4_lib, tuple) else {"unavailable": fp4_lib}),
+            "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how},
         "e2e": {"value": round(aggregate_tflops(STEP_FLOPS, world, e2e_ms), 3), "unit": "TFLOP/s",
-                "h2d_bytes_per_step": M * K * 2 + AM * AK * 2, "d2h_bytes_per_step": M * N * 2 + AM * AN * 2},
-        "gpu_launches": 3 * args.steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(STEP_KERNELS) * args.steps,
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(rows=64, reps=2)
+        line["cpu_baseline"] = cpu_baseline(rows=16, reps=1)
     print(json.dumps(line))
 
 
 # ------------------------------------------------------------------ oracle timing
-def oracle_sample(rows, x, packed, bb, awq_case):
-    """One bounded sample of the step on the CPU oracle; returns (flops, seconds)."""
-    from oracle import awq as oawq
-    from oracle import formats, svdquant
+class OracleWorkload:
+    """The oracle's own packs of the step's layers (untimed) and its bounded samples (timed)."""
 
-    def bf(bits):
-        return formats.bf16_bits_to_float(np.asarray(bits, np.uint16))
+    def __init__(self):
+        from bit_w4a4_diffusion_smooth_b200 import synthetic
+        from oracle import awq as oawq
+        from oracle import formats, svdquant
 
-    l1, l2, w_codes, w_sf = packed["l1"], packed["l2"], packed["w_codes"], packed["w_sf"]
-    axb, ainv, aq, as_, az, abias = awq_case
-    t = time.perf_counter()
-    codes, sf, u = svdquant.quantize_act(x[:rows], packed["inv_lambda"], l1, packed["s_a"], packed["s_w"])
-    svdquant.w4a4_linear(codes, sf, packed["s_a"], w_codes, w_sf, packed["s_w"], u, l2, bf(bb))
-    oawq.linear(axb, ainv, aq, as_, az, abias)
-    dt = time.perf_counter() - t
-    flops = rows / M * (W4A4_FLOPS + LOWRANK_FLOPS) + AWQ_FLOPS
-    return flops, dt
+        self.f = formats
+        self.sq = svdquant
+        self.oawq = oawq
+        self.x = {}
+        self.p = {}
+        self.b = {}
+        for name, c in (("qkv", synthetic.QKV), ("fc1", synthetic.MLP_FC1)):
+            xb, wb, bb = c.make()
+            x = formats.bf16_bits_to_float(xb)
+            self.x[name] = x
+            self.p[name] = svdquant.pack(formats.bf16_bits_to_float(wb),
+                                         np.max(np.abs(x), axis=0).astype(np.float32), RANK)
+            self.b[name] = formats.bf16_bits_to_float(bb)
+        c2 = synthetic.MLP_FC2
+        wb2, _ = synthetic.weight(c2.k, c2.n, c2.seed, 0.02, c2.w_outlier_rows, c2.w_factor)
+        self.b["fc2"] = formats.bf16_bits_to_float(synthetic.bias(c2.n, c2.seed + 100))
+        # fc2's calibration: the oracle's own fc1 output on a sample of rows
+        h = formats.bf16_round(svdquant.forward(self.x["fc1"][::36], self.p["fc1"], self.b["fc1"],
+                                                svdquant.EPILOGUE_GELU_ERF))
+        self.p["fc2"] = svdquant.pack(formats.bf16_bits_to_float(wb2),
+                                      np.max(np.abs(h), axis=0).astype(np.float32), RANK)
+        a = synthetic.AWQ
+        axb, awb, abb, asc = a.make()
+        ap = oawq.pack(formats.bf16_bits_to_float(awb), asc)
+        self.awq = (formats.bf16_bits_to_float(axb), ap["inv_a"], ap["q"], ap["s"], ap["z"],
+                    formats.bf16_bits_to_float(abb))
 
-
-def _oracle_inputs():
-    from bit_w4a4_diffusion_smooth_b200 import synthetic
-    from oracle import awq as oawq
-    from oracle import formats, svdquant
-
-    c = synthetic.QKV
-    xb, wb, bb = c.make()
-    x = formats.bf16_bits_to_float(xb)
-    # the oracle's own pack; its cost is not part of the timed sample
-    packed = svdquant.pack(formats.bf16_bits_to_float(wb), np.max(np.abs(x), axis=0).astype(np.float32), RANK)
-    a = synthetic.AWQ
-    axb, awb, abb, asc = a.make()
-    ap = oawq.pack(formats.bf16_bits_to_float(awb), asc)
-    awq_case = (formats.bf16_bits_to_float(axb), ap["inv_a"], ap["q"], ap["s"], ap["z"], formats.bf16_bits_to_float(abb))
-    return x, packed, bb, awq_case
+    def sample(self, rows):
+        """`rows` rows of every SVDQ layer (fc2 on the oracle's fc1 output of those rows) and the
+        whole AWQ projection; returns (FLOPs it stands for, seconds)."""
+        sq, f = self.sq, self.f
+        t = time.perf_counter()
+        sq.forward(self.x["qkv"][:rows], self.p["qkv"], self.b["qkv"])
+        h = sq.forward(self.x["fc1"][:rows], self.p["fc1"], self.b["fc1"], sq.EPILOGUE_GELU_ERF)
+        sq.forward(f.bf16_round(h), self.p["fc2"], self.b["fc2"])
+        self.oawq.linear(*self.awq)
+        dt = time.perf_counter() - t
+        flops = rows / TOKENS * sum(layer_flops(m, k, n) for m, k, n, _ in LAYERS.values()) + AWQ_FLOPS
+        return flops, dt
 
 
 def _cores():
@@ -400,29 +611,30 @@ def _cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(rows=64, reps=2):
-    x, packed, bb, awq_case = _oracle_inputs()
+def cpu_baseline(rows=16, reps=1):
+    ow = OracleWorkload()
     flops = secs = 0.0
     for _ in range(reps):
-        f, s = oracle_sample(rows, x, packed, bb, awq_case)
+        f, s = ow.sample(rows)
         flops += f
         secs += s
     return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
-            "sample": f"{rows} of {M} rows of the QKV layer (quantize + two-branch float64 GEMM) + the full "
-                      f"2x3072->18432 AWQ projection, {reps} repetitions"}
+            "sample": f"{rows} of {TOKENS} rows of each SVDQ layer (QKV, fc1, fc2 on fc1's output: quantize + "
+                      f"two-branch float64 GEMM) + the full 2x3072->18432 AWQ projection, {reps} repetition(s); "
+                      "the oracle's packs are untimed"}
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    x, packed, bb, awq_case = _oracle_inputs()
-    rows = 32
+    ow = OracleWorkload()
+    rows = 8
     for _ in range(args.warmup):
-        oracle_sample(rows, x, packed, bb, awq_case)
+        ow.sample(rows)
     flops = secs = 0.0
     for _ in range(args.steps):
-        f, s = oracle_sample(rows, x, packed, bb, awq_case)
+        f, s = ow.sample(rows)
         flops += f
         secs += s
     v = round(flops / secs / 1e12, 6)
@@ -432,7 +644,8 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (CPU oracle)",
         "data": "synthetic", "config": {"workload": WORKLOAD, "parallelism": "single host process"},
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
-                         "sample": f"{rows} of {M} rows of the QKV layer + the full AWQ projection per step"},
+                         "sample": f"{rows} of {TOKENS} rows of each SVDQ layer + the full AWQ projection per "
+                                   "step"},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -638,16 +851,20 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None,
-                    help="timed steps (default: 3000 for the layer step, about 0.4 s timed, so that the clock "
-                         "sampler sees the timed region; 200 for --workload dit-step and --impl reference)")
+                    help="timed steps (default: 300 for the layer step; 200 for --workload dit-step; 10 for "
+                         "--impl reference)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=("qkv", "dit-step"), default="qkv",
-                    help="qkv: the QKV layer + AWQ projection (default); dit-step: one whole DiT step")
+    ap.add_argument("--no-library-points", action="store_true",
+                    help="skip the cuBLASLt NVFP4 reference point")
+    ap.add_argument("--kernel-reps", type=int, default=20,
+                    help="back-to-back launches per kernel for the per-kernel times")
+    ap.add_argument("--workload", choices=("layers", "dit-step"), default="layers",
+                    help="layers: QKV + MLP pair + AWQ projection (default); dit-step: one whole DiT step")
     args = ap.parse_args()
     if args.steps is None:
-        args.steps = 3000 if (args.impl == "ours" and args.workload == "qkv") else 200
+        args.steps = {"reference": 10}.get(args.impl, 300 if args.workload == "layers" else 200)
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":

@@ -1,11 +1,33 @@
 """User-facing layers on top of the C ABI: SVDQLinear (W4A4 + low-rank branch)
 and AWQLinear (W4A16).  They hold the packed weights on the GPU and reuse
 activation buffers per row count; all arithmetic runs in the library.
+
+A layer instance keeps one set of activation buffers per row count, shared by
+all its calls: use an instance from one stream at a time (two calls with the
+same row count that overlap on different streams would race on them).
 """
 import numpy as np
 import torch
 
 from . import lib
+
+
+def _resolve(device):
+    """torch.device with an explicit index ('cuda' means the caller's current device)."""
+    d = torch.device(device)
+    if d.type != "cuda":
+        raise ValueError(f"the layers run on a CUDA device, got {d}")
+    return d if d.index is not None else torch.device("cuda", torch.cuda.current_device())
+
+
+def _init_on(device):
+    """svdq_init for `device` (it validates the GPU and makes it current), then restores the
+    caller's current device."""
+    prev = torch.cuda.current_device()
+    try:
+        lib.svdq_init(device.index)
+    finally:
+        torch.cuda.set_device(prev)
 
 
 def _dev(a, device, dtype=None):
@@ -15,19 +37,34 @@ def _dev(a, device, dtype=None):
     return t.to(device)
 
 
+def _check_input(X, K, device, name):
+    if X.dim() != 2 or X.shape[1] != K:
+        raise ValueError(f"{name}: X must be [M, {K}], got {tuple(X.shape)}")
+    if X.dtype != torch.bfloat16 or X.device != device:
+        raise ValueError(f"{name}: X must be bf16 on {device}, got {X.dtype} on {X.device}")
+
+
+def _check_output(Y, M, N, device, name):
+    if tuple(Y.shape) != (M, N) or Y.dtype != torch.bfloat16 or Y.device != device:
+        raise ValueError(f"{name}: Y must be bf16 [{M}, {N}] on {device}, got {Y.dtype} {tuple(Y.shape)} "
+                         f"on {Y.device}")
+
+
 class SVDQLinear:
     """Y = (X^ L1) L2 + Q(X^) Q(R) + b  (one SVDQuant linear layer).
 
     Build with `from_weight` (offline host pack of a bf16 weight [K, N] and
-    calibration maxima) or `from_packed` (a dict from lib.svdq_pack_weights).
+    calibration maxima) or with the constructor from a dict returned by
+    lib.svdq_pack_weights.
     """
 
     def __init__(self, packed, K, N, rank, bias_bits=None, epilogue=lib.EPILOGUE_NONE, gelu_col_begin=0,
                  device="cuda"):
         self.K, self.N, self.rank = K, N, rank
         self.epilogue, self.gelu_col_begin = epilogue, gelu_col_begin
-        self.device = torch.device(device)
-        lib.svdq_init(self.device.index or 0)
+        self.device = _resolve(device)
+        _init_on(self.device)
+        device = self.device
         self.inv_lambda = _dev(packed["inv_lambda"], device)
         self.l1t = _dev(packed["l1t"], device, torch.bfloat16) if rank else None
         self.l2t = _dev(packed["l2t"], device)
@@ -35,6 +72,8 @@ class SVDQLinear:
         self.s_w = _dev(np.asarray(packed["s_w"], np.float32).reshape(1), device)
         self.s_a = _dev(np.asarray(packed["s_a"], np.float32).reshape(1), device)
         self.bias = _dev(bias_bits, device, torch.bfloat16) if bias_bits is not None else None
+        if self.bias is not None and self.bias.numel() != N:
+            raise ValueError(f"SVDQLinear: bias must have {N} elements")
         self._bufs = {}
 
     @classmethod
@@ -45,7 +84,7 @@ class SVDQLinear:
         return cls(packed, K, N, rank, bias_bits, epilogue, gelu_col_begin, device)
 
     def buffers(self, M):
-        """Activation-side buffers for M rows (allocated once per M)."""
+        """Activation-side buffers for M rows (allocated once per M, shared by every call)."""
         if M not in self._bufs:
             sz = lib.svdq_act_sizes(M, self.K)
             self._bufs[M] = dict(
@@ -54,17 +93,20 @@ class SVDQLinear:
         return self._bufs[M]
 
     def quantize(self, X, stream=None):
+        _check_input(X, self.K, self.device, "SVDQLinear")
         b = self.buffers(X.shape[0])
         lib.svdq_quantize_act(X, self.inv_lambda, self.l1t, self.rank, self.s_a, self.s_w,
                               b["a_bundle"], b["U"], stream=stream)
         return b
 
     def gemm(self, b, M, Y, stream=None):
+        _check_output(Y, M, self.N, self.device, "SVDQLinear")
         lib.svdq_linear_w4a4(b["a_bundle"], b["U"], self.s_a, self.w_bundle, self.l2t, self.s_w, self.bias,
                              M, self.N, self.K, self.rank, self.epilogue, self.gelu_col_begin, Y, stream=stream)
         return Y
 
     def __call__(self, X, Y=None, stream=None):
+        _check_input(X, self.K, self.device, "SVDQLinear")
         M = X.shape[0]
         if Y is None:
             Y = torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device)
@@ -76,13 +118,16 @@ class AWQLinear:
 
     def __init__(self, packed, K, N, bias_bits=None, device="cuda"):
         self.K, self.N = K, N
-        self.device = torch.device(device)
-        lib.svdq_init(self.device.index or 0)
+        self.device = _resolve(device)
+        _init_on(self.device)
+        device = self.device
         self.qweight = _dev(packed["qweight"], device)
         self.scales = _dev(packed["scales"], device, torch.bfloat16)
         self.zeros = _dev(packed["zeros"], device, torch.bfloat16)
         self.inv_awq = _dev(packed["inv_awq"], device)
         self.bias = _dev(bias_bits, device, torch.bfloat16) if bias_bits is not None else None
+        if self.bias is not None and self.bias.numel() != N:
+            raise ValueError(f"AWQLinear: bias must have {N} elements")
 
     @classmethod
     def from_weight(cls, W_bits, awq_scale, bias_bits=None, device="cuda"):
@@ -90,8 +135,10 @@ class AWQLinear:
         return cls(lib.awq_pack_weights(W_bits, awq_scale), K, N, bias_bits, device)
 
     def __call__(self, X, Y=None, stream=None):
+        _check_input(X, self.K, self.device, "AWQLinear")
         if Y is None:
             Y = torch.empty((X.shape[0], self.N), dtype=torch.bfloat16, device=self.device)
+        _check_output(Y, X.shape[0], self.N, self.device, "AWQLinear")
         lib.awq_linear_w4a16(X, self.inv_awq, self.qweight, self.scales, self.zeros, self.bias, self.N, Y,
                              stream=stream)
         return Y

@@ -101,6 +101,22 @@ def _dptr(t, name, dtype=None, allow_none=False):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def _need_bytes(t, nbytes, name):
+    """Raises unless device buffer `t` holds at least `nbytes` bytes (checked before any call, so a
+    short buffer is never handed to a kernel)."""
+    if t is not None and _nbytes(t) < nbytes:
+        raise ValueError(f"{name} holds {_nbytes(t)} bytes; {nbytes} are needed")
+
+
+def _need_2d(t, rows, cols, name):
+    if t.dim() != 2 or t.shape[0] < rows or t.shape[1] < cols:
+        raise ValueError(f"{name} must be 2-D with at least {rows} rows and {cols} columns, got {tuple(t.shape)}")
+
+
 def _stream(stream):
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
@@ -187,6 +203,15 @@ def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M=None, K
     M = X.shape[0] if M is None else M
     K = X.shape[1] if K is None else K
     ldx = X.stride(0)
+    _need_2d(X, M, K, "X")
+    sz = svdq_act_sizes(M, K)
+    _need_bytes(a_bundle, sz["a_bundle"], "a_bundle")
+    _need_bytes(U, sz["u"], "U")
+    _need_bytes(inv_lambda, 4 * K, "inv_lambda")
+    if rank:
+        _need_bytes(l1t, 2 * rank * K, "l1t")
+    _need_bytes(s_a, 4, "s_a")
+    _need_bytes(s_w, 4, "s_w")
     _check("svdq_quantize_act", load().svdq_quantize_act(
         _dptr(X, "X", torch.bfloat16), M, K, ldx, _dptr(inv_lambda, "inv_lambda", torch.float32),
         _dptr(l1t, "l1t", allow_none=rank == 0), rank, _dptr(s_a, "s_a", torch.float32),
@@ -198,6 +223,17 @@ def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, 
                      stream=None):
     """Enqueues the W4A4 GEMM.  Y: bf16 CUDA [M, ldy]."""
     import torch
+    asz = svdq_act_sizes(M, K)
+    wsz = svdq_weight_sizes(K, N, rank)
+    _need_bytes(a_bundle, asz["a_bundle"], "a_bundle")
+    _need_bytes(w_bundle, wsz["w_bundle"], "w_bundle")
+    if rank:
+        _need_bytes(U, asz["u"], "U")
+        _need_bytes(l2t, wsz["l2t"], "l2t")
+    _need_bytes(bias, 2 * N, "bias")
+    _need_bytes(s_a, 4, "s_a")
+    _need_bytes(s_w, 4, "s_w")
+    _need_2d(Y, M, N, "Y")
     _check("svdq_linear_w4a4", load().svdq_linear_w4a4(
         _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U", allow_none=rank == 0),
         _dptr(s_a, "s_a", torch.float32), _dptr(w_bundle, "w_bundle", torch.uint8),
@@ -226,6 +262,13 @@ def awq_linear_w4a16(X, inv_awq, qweight, scales, zeros, bias, N, Y, group=64, M
     import torch
     M = X.shape[0] if M is None else M
     K = X.shape[1] if K is None else K
+    _need_2d(X, M, K, "X")
+    _need_2d(Y, M, N, "Y")
+    _need_bytes(qweight, N * K // 2, "qweight")
+    _need_bytes(scales, 2 * N * (K // group), "scales")
+    _need_bytes(zeros, 2 * N * (K // group), "zeros")
+    _need_bytes(inv_awq, 4 * K, "inv_awq")
+    _need_bytes(bias, 2 * N, "bias")
     _check("awq_linear_w4a16", load().awq_linear_w4a16(
         _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_awq, "inv_awq", allow_none=True),
         _dptr(qweight, "qweight"), _dptr(scales, "scales"), _dptr(zeros, "zeros"), group,

@@ -237,6 +237,11 @@ int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq,
  * Waits for `stream`, then returns and clears the device status word of the
  * current device: SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel's bounded wait ran
  * out since the last check (SVDQ_ERR_CUDA if the stream itself failed).
+ * There is one status word per device, shared by the kernels of every stream:
+ * a check synchronizes only `stream`, so a timeout recorded by a kernel still
+ * running on another stream may be reported by a later check, or cleared by
+ * this one if it lands between the read and the clear.  Callers that use
+ * several streams and need an exact attribution synchronize the device first.
  */
 int svdq_check_status(svdq_stream_t stream);
 

@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests: moving seeded inputs to the device,
 reading results back, and the normalised error of the parity bar."""
+import os
+
 import numpy as np
 import torch
 
@@ -70,6 +72,25 @@ def excess_error(got, want):
     rms = np.where(rms == 0, 1.0, rms)
     d = np.maximum(0.0, np.abs(got - want) - 0.5 * bf16_ulp(got))
     return float(np.max(d / rms[:, None]))
+
+
+# Every parity comparison of the session: both measures, for the report printed at the end of the
+# run (tests/conftest.py) and written as JSON to $PARITY_REPORT when that is set.
+PARITY = []
+
+
+def parity(label, got, want, tol=1e-2):
+    """Asserts the parity bar (excess_error <= tol) and records it together with the raw
+    row_rms_error, so a reader sees whether the raw bar holds as well."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    ex, raw = excess_error(got, want), row_rms_error(got, want)
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    PARITY.append({"test": test, "case": label, "excess": ex, "raw": raw, "tol": tol,
+                   "raw_within_tol": raw <= tol})
+    print(f"parity {test} {label}: excess {ex:.3e}  raw {raw:.3e}  (tol {tol:g})")
+    assert ex <= tol, f"{label}: excess error {ex:.3e} > {tol:g} (raw {raw:.3e})"
+    return ex, raw
 
 
 def check_ok():

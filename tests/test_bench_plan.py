@@ -33,5 +33,20 @@ def test_dit_step_plan_orders_fc1_before_its_fc2():
         assert all(a < b for a, b in zip(fc1, fc2))
 
 
-def test_qkv_step_flops():
-    assert bench.STEP_FLOPS == 2 * 4608 * 3072 * 9216 + 2 * 4608 * 32 * (3072 + 9216) + 2 * 2 * 3072 * 18432
+def test_layer_step_flops_and_kernels():
+    """The default step: QKV, MLP fc1 (+GELU) and fc2 on fc1's output, each K1 + K2, then K3."""
+    def layer(m, k, n, r=32):
+        return 2 * m * k * n + 2 * m * r * (k + n)
+    want = layer(4608, 3072, 9216) + layer(4608, 3072, 12288) + layer(4608, 12288, 3072) + 2 * 2 * 3072 * 18432
+    assert bench.STEP_FLOPS == want
+    labels = [label for label, _ in bench.STEP_KERNELS]
+    assert labels == ["K1 qkv", "K2 qkv", "K1 fc1", "K2 fc1", "K1 fc2", "K2 fc2", "K3 adaLN"]
+    assert bench.LAYERS["fc1"] == (4608, 3072, 12288, True)
+
+
+def test_kernel_table_units():
+    t = bench.kernel_table({"hbm_gbs": 6000.0, "bf16_tflops": 1500.0})
+    assert t["K2 fc1"] == (2 * 4608 * 3072 * 12288 + 2 * 4608 * 32 * 12288, "TFLOP/s", "tensor", 6000.0)
+    assert t["K1 qkv"][0] == 4608 * 3072 * 2 + 3072 * 32 * 2 + 3072 * 4 + 4608 * 3072 // 2 + 4608 * 3072 // 16 \
+        + 4608 * 32 * 2
+    assert t["K3 adaLN"][1:] == ("GB/s", "hbm", 6000.0)

@@ -33,7 +33,7 @@ def _run(m, k, n, seed, with_bias=True, use_inv=True):
     G.check_ok()
     x = formats.bf16_bits_to_float(xb)
     want = oawq.linear(x, p["inv_a"], p["q"], p["s"], p["z"], formats.bf16_bits_to_float(bb) if with_bias else None)
-    return G.excess_error(G.bf16_host(Y), want)
+    return G.parity(f"{m}x{k}->{n}", G.bf16_host(Y), want)[0]
 
 
 @pytest.mark.parametrize("m,k,n", [
@@ -66,4 +66,4 @@ def test_awq_layer_from_host_pack():
     p = oawq.pack(formats.bf16_bits_to_float(wb), a)
     want = oawq.linear(formats.bf16_bits_to_float(xb), p["inv_a"], p["q"], p["s"], p["z"],
                        formats.bf16_bits_to_float(bb))
-    assert G.excess_error(y, want) <= 1e-2
+    G.parity("layer", y, want)

@@ -8,7 +8,8 @@ the library's layouts.  Nothing computed by the GPU is fed back to the oracle.
 Bar: NVFP4 codes and block scales bit-exact; U and Y within 1e-2 of the
 oracle, measured as the largest error in a row beyond the rounding of the
 result to its bf16 output type, divided by the RMS of the oracle's row
-(gpu_util.excess_error).  K2 is run on the oracle's own quantized operands
+(gpu_util.excess_error); the raw largest error over the row RMS
+(gpu_util.row_rms_error) is recorded beside it for every comparison.  K2 is run on the oracle's own quantized operands
 (identical on both sides; U enters as the bf16 buffer K1 writes).  Sizes span several tiles plus ragged tails in M, N and K; the
 full-size workloads are checked on sampled rows.
 """
@@ -63,7 +64,7 @@ def _check_k1(x, p, rank, bundle, U, rows=None):
     pad = L.lowrank_unpack(G.u8(U), (M + 127) // 128 * 128, 128)[M:]
     assert (pad == 0).all()
     if rank:
-        assert G.excess_error(L.bf16_bits_to_f64(gubits[:, :rank]), ou) <= TOL
+        G.parity("U", L.bf16_bits_to_f64(gubits[:, :rank]), ou, TOL)
 
 
 K1_CASES = [
@@ -125,8 +126,7 @@ def test_linear_w4a4_parity(case, epilogue, begin, with_bias):
     oc, osf, ou = _oracle_operands(x, p, rank)
     bias = bb if with_bias else None
     Y, _ = _run_k2(oc, osf, ou, d, bias, m, n, k, rank, epilogue, begin)
-    err = G.excess_error(G.bf16_host(Y), _want_k2(oc, osf, ou, p, bias, epilogue, begin))
-    assert err <= TOL, err
+    G.parity("Y", G.bf16_host(Y), _want_k2(oc, osf, ou, p, bias, epilogue, begin), TOL)
 
 
 def test_linear_w4a4_strided_output_and_repeat():
@@ -138,7 +138,7 @@ def test_linear_w4a4_strided_output_and_repeat():
     Y2, _ = _run_k2(oc, osf, ou, d, bb, 64, 256, 256, 16, 0, 0, ldy=272)
     assert torch.equal(Y1, Y2)                            # deterministic
     assert torch.isnan(full1[:, 256:].float()).all()       # padding columns untouched
-    assert G.excess_error(G.bf16_host(Y1), _want_k2(oc, osf, ou, p, bb, 0, 0)) <= TOL
+    G.parity("Y", G.bf16_host(Y1), _want_k2(oc, osf, ou, p, bb, 0, 0), TOL)
 
 
 def _sample_rows(m, count=192, seed=0):
@@ -167,13 +167,13 @@ def test_full_size_qkv_sampled():
     Y, _ = _run_k2(oc, osf, ou, d, bb, c.m, c.n, c.k, c.rank, 0, 0)
     assert not torch.isnan(Y.float()).any()
     want = _want_k2(oc[rows], osf[rows], ou[rows], p, bb, 0, 0)
-    assert G.excess_error(G.bf16_host(Y)[rows], want) <= TOL
+    G.parity("Y on oracle operands", G.bf16_host(Y)[rows], want, TOL)
 
     Y2 = G.poisoned_bf16(c.m, c.n)
     lib.svdq_linear_w4a4(bundle, U, d["s_a"], d["w_bundle"], d["l2t"], d["s_w"], G.bf16_dev(bb),
                          c.m, c.n, c.k, c.rank, 0, 0, Y2)
     G.check_ok()
-    assert G.excess_error(G.bf16_host(Y2)[rows], want) <= TOL   # the GPU's own K1 -> K2 chain
+    G.parity("Y of the GPU's K1 -> K2 chain", G.bf16_host(Y2)[rows], want, TOL)
 
 
 def test_full_size_mlp_pair_sampled():
@@ -194,7 +194,7 @@ def test_full_size_mlp_pair_sampled():
     G.check_ok()
     oc1, osf1, ou1 = _oracle_operands(x, p1, c1.rank)
     h_oracle = _want_k2(oc1, osf1, ou1, p1, bb1, lib.EPILOGUE_GELU_ERF, 0)
-    assert G.excess_error(G.bf16_host(H)[rows], h_oracle[rows]) <= TOL
+    G.parity("fc1 H", G.bf16_host(H)[rows], h_oracle[rows], TOL)
     # fc2 on the oracle's fc1 output (rounded to bf16, the layer's output type)
     h = formats.bf16_round(h_oracle)
     hb = L.bf16_bits(h)
@@ -210,7 +210,7 @@ def test_full_size_mlp_pair_sampled():
     G.check_ok()
     oc2, osf2, ou2 = _oracle_operands(h, p2, c2.rank, rows)
     want = _want_k2(oc2, osf2, ou2, p2, bb2, 0, 0)
-    assert G.excess_error(G.bf16_host(Y)[rows], want) <= TOL
+    G.parity("fc2 Y", G.bf16_host(Y)[rows], want, TOL)
 
 
 def test_layer_tracks_unquantized_product():
@@ -226,3 +226,26 @@ def test_layer_tracks_unquantized_product():
     y = G.bf16_host(layer(G.bf16_dev(xb)))
     ref = x @ w + formats.bf16_bits_to_float(bb)
     assert np.linalg.norm(y - ref) / np.linalg.norm(ref) < 0.1
+
+
+def test_layer_and_binding_reject_mismatched_buffers():
+    """A short buffer or a wrong input width raises on the host before anything is launched."""
+    from bit_w4a4_diffusion_smooth_b200.layer import SVDQLinear
+    c = synthetic.TINY
+    xb, wb, bb = c.make()
+    x = formats.bf16_bits_to_float(xb)
+    layer = SVDQLinear.from_weight(wb, np.max(np.abs(x), axis=0).astype(np.float32), c.rank, bb)
+    X = G.bf16_dev(xb)
+    with pytest.raises(ValueError):
+        layer(X[:, : c.k - 64].contiguous())            # narrower than the layer's K
+    with pytest.raises(ValueError):
+        layer(X, Y=torch.empty((c.m, c.n - 8), dtype=torch.bfloat16, device=G.DEV))
+    b = layer.buffers(c.m)
+    with pytest.raises(ValueError):
+        lib.svdq_quantize_act(X, layer.inv_lambda, layer.l1t, c.rank, layer.s_a, layer.s_w,
+                              b["a_bundle"][:-16], b["U"])
+    with pytest.raises(ValueError):
+        lib.svdq_linear_w4a4(b["a_bundle"], b["U"], layer.s_a, layer.w_bundle[:-16], layer.l2t, layer.s_w,
+                             layer.bias, c.m, c.n, c.k, c.rank, 0, 0,
+                             torch.empty((c.m, c.n), dtype=torch.bfloat16, device=G.DEV))
+    G.check_ok()

@@ -57,6 +57,20 @@ def test_pack_matches_oracle(k, n, rank):
 @pytest.mark.parametrize("k,n,rank,tol", [(256, 256, 16, 1e-3), (512, 1536, 32, 1e-3)])
 def test_pack_svd_eckart_young(k, n, rank, tol):
     xb, wb, x, amax = _case(64, k, n, seed=3, x_out=max(1, k // 64), x_fac=50.0, w_out=max(1, k // 200))
+    _check_eckart_young(wb, amax, rank, tol)
+
+
+@pytest.mark.slow
+def test_pack_svd_eckart_young_full_size_qkv():
+    """The pack the benchmark uses: the attention-QKV weight 3072 x 9216 at rank 32, calibrated
+    on its 4608-row activation, against the exact spectrum of W'."""
+    c = synthetic.QKV
+    xb, wb, _ = c.make()
+    amax = np.max(np.abs(formats.bf16_bits_to_float(xb)), axis=0).astype(F32)
+    _check_eckart_young(wb, amax, c.rank, 1e-3)
+
+
+def _check_eckart_young(wb, amax, rank, tol):
     w = formats.bf16_bits_to_float(wb)
     p = lib.svdq_pack_weights(wb, amax, rank, want_residual=True)
     wp = svdquant.smoothed_weight(w, p["inv_lambda"])

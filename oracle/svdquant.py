@@ -85,6 +85,22 @@ def activation_tensor_scale(amax_x, inv_lambda):
     return nvfp4.tensor_scale(np.max(prod) if prod.size else F32(0.0))
 
 
+def dynamic_activation_scale(x, inv_lambda):
+    """s_A of one activation tensor, taken from that tensor itself: f32(max |X^|) / 2688 with
+    X^ = f32(x * inv_lambda), 1 when that maximum is 0.
+
+    The static reading calibrates s_A once from calibration data; the pages only say that
+    calibration decides the scales ([Remio] "基准测试展示了性能提升，但并非普遍结论"), so the
+    per-call (dynamic) scale is the other reading, offered as an optional pre-pass.  Calibrated on
+    the same tensor, the two agree: f32 multiplication by inv_j >= 0 is monotonic, so the largest
+    f32(|x_mj| inv_j) of a column is f32(max_m |x_mj| inv_j).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    inv = np.asarray(inv_lambda, dtype=F32)
+    x_hat32 = (x.astype(F32) * inv[None, :]).astype(F32)
+    return nvfp4.tensor_scale(np.max(np.abs(x_hat32)) if x_hat32.size else F32(0.0))
+
+
 def pack(w, amax_x, rank, round_bf16=True):
     """Offline quantization of one layer ([Donmalab] "自行量化模型的流程": quantize
     the weights to 4 bits and produce the low-rank branch).

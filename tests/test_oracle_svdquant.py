@@ -234,3 +234,30 @@ def test_forward_is_close_to_unquantized_layer():
     p0 = svdquant.pack(w, amax_x, 0)
     rel0 = np.linalg.norm(svdquant.forward(x, p0, b) - ref) / np.linalg.norm(ref)
     assert rel <= rel0 * 1.05
+
+
+def test_dynamic_activation_scale_pins():
+    """The per-tensor (dynamic) activation scale: brute force over every element of a small input,
+    the all-zero tensor (scale 1), and agreement with the static scale calibrated on the same
+    tensor's per-channel maxima (a different formulation of the same maximum)."""
+    from oracle import nvfp4
+    rng = np.random.default_rng(11)
+    x = formats.bf16_round(rng.standard_normal((7, 48)) * np.exp(rng.uniform(-3, 3, 48)))
+    x[3, 5] = -x[3, 5] * 40.0                    # a negative outlier decides the maximum
+    x = formats.bf16_round(x)
+    inv = np.exp(rng.uniform(-2, 2, 48)).astype(np.float32)
+    best = np.float32(0.0)
+    for i in range(x.shape[0]):
+        for j in range(x.shape[1]):
+            v = abs(np.float32(np.float32(x[i, j]) * inv[j]))
+            best = max(best, v)
+    assert svdquant.dynamic_activation_scale(x, inv) == np.float32(best / np.float32(2688.0))
+    amax = np.max(np.abs(x), axis=0).astype(np.float32)
+    assert svdquant.dynamic_activation_scale(x, inv) == svdquant.activation_tensor_scale(amax, inv)
+    assert svdquant.dynamic_activation_scale(np.zeros((3, 16)), np.ones(16, np.float32)) == np.float32(1.0)
+    # a tensor whose largest |x^| is 2688 has scale exactly 1 (the largest block scale then lands on 448)
+    z = np.zeros((2, 16))
+    z[1, 7] = -2688.0
+    assert svdquant.dynamic_activation_scale(z, np.ones(16, np.float32)) == np.float32(1.0)
+    codes, sf = nvfp4.quantize_blocks(z.astype(np.float32), np.float32(1.0))
+    assert sf[1, 0] == 0x7E and codes[1, 7] == 0xF   # e4m3 448, e2m1 -6

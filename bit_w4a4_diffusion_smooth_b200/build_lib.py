@@ -20,7 +20,9 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsvdq_b200.so")
 
-SOURCES = ["api.cu", "quant_act.cu", "gemm_w4a4.cu", "gemv_w4a16.cu", "pack_svdq.cpp", "pack_awq.cpp"]
+SOURCES = ["api.cu", "quant_act.cu", "act_amax.cu", "gemm_w4a4.cu", "gemm_w4a4_requant.cu", "gemv_w4a16.cu",
+           "pack_svdq.cpp", "pack_awq.cpp"]
+LINK_LIBS = ["-lpthread"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # Host code: no fused multiply-add contraction and no fast-math, so the
 # float32 quantization decisions of the host pack follow IEEE one rounding per
@@ -73,7 +75,7 @@ def build(force=False, verbose=False):
             if log:
                 print(f"--- {src}\n{log}", file=sys.stderr)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc(), "-shared"] + ARCH + ["-Xcompiler", "-fPIC", "-o", LIB] + objs + ["-lpthread"]
+        cmd = [nvcc(), "-shared"] + ARCH + ["-Xcompiler", "-fPIC", "-o", LIB] + objs + LINK_LIBS
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"linking failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")

@@ -429,6 +429,27 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
       : "f"(hi), "f"(lo));
   return static_cast<uint32_t>(r) & 0xFFu;
 }
+// e2m1 codes of four values in the two low bytes: byte 0 = e2m1(a1) << 4 | e2m1(a0),
+// byte 1 = e2m1(a3) << 4 | e2m1(a2) (RNE, satfinite); bytes 2 and 3 are 0.
+__device__ __forceinline__ uint32_t cvt_e2m1x4(float a0, float a1, float a2, float a3) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "mov.b32 %0, {t0, t1, 0, 0};\n\t}"
+      : "=r"(r)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return r;
+}
+// Two IEEE single-precision products, each rounded to nearest even on its
+// own (one packed f32x2 instruction; identical to two __fmul_rn).
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
 // e4m3 code of v (RNE, satfinite) in bits 0..7.
 __device__ __forceinline__ uint32_t cvt_e4m3(float v) {
   uint16_t r;

@@ -1,531 +1,19 @@
-// K2: W4A4 GEMM with the low-rank up-projection fused in.
-//
-// The pages fuse the 16-bit low-rank up-projection into the 4-bit GEMM so the
-// correction branch does not eat the W4A4 gain (web page "Nunchaku Diffusers
-// 支持降低显存占用，但硬件仍决定适用范围", remio.ai, section "SVDQuant 将棘手数值移出
-// 4 位路径").  Per 256 x 256 output tile:
-//   acc  = U_tile . L2T_tile^T                 tcgen05.mma kind::f16 (bf16)
-//   acc += sum_k (qa sa)(qw sw)                tcgen05.mma kind::mxf4nvf4,
-//                                               block16 ue4m3 scales in TMEM
-//   Y    = bf16( epilogue( s_a s_w acc + bias ) )
-// U arrives pre-divided by s_a s_w, so both branches share one fp32
-// accumulator and one scale in the epilogue.
-//
-// SM pairs.  The kernel runs in clusters of two CTAs, one per SM of a TPC,
-// and every MMA is a cta_group::2 MMA of 256 x 256 x 64: CTA h of the pair
-// holds rows 128h..128h+127 of the activation tile and weight rows (output
-// columns) 128h..128h+127 of the weight tile, and its TMEM receives its own
-// 128 rows of the accumulator.  Each SM therefore loads its half of A and
-// of B per k-stage (32 KB of codes) plus the scales: its 128 rows of A
-// scales and the B scales of all 256 weight rows that both TMEMs need.
-//
-// Roles (one CTA per SM, persistent over pair tiles, 12 warps):
-//   warp 0      producer in both CTAs: per stage four TMA copies into its
-//               own shared memory - the A and B scales first, completing on
-//               the even CTA's `sf_loaded` barrier, then the A and B code
-//               halves, completing on its `full` barrier
-//   warp 1      owns TMEM (pair allocation); in the even CTA it issues the
-//               MMAs from one thread and commits each stage to both CTAs'
-//               `empty` barriers
-//   warp 2      even CTA: moves each stage's block scales from both CTAs'
-//               shared memory into their TMEM (tcgen05.cp, cta_group::2) as
-//               soon as `sf_loaded` completes; from its own warp the copies
-//               overlap the MMAs and the codes' transfer
-//   warps 4..11 epilogue in both CTAs: drain the CTA's 128 x 256 fp32
-//               accumulator, hand TMEM back (to the even CTA's barrier),
-//               then scale, add bias, GELU, round to bf16 into a
-//               64-byte-swizzled 32 x 32 staging tile and write it with TMA
-//               stores
-// Pipeline: 4 stages of 50 KB per CTA; TMEM holds the accumulator (256
-// columns) and 4 x 48 columns of block scales.  A pair walks a contiguous
-// run of tiles, n fastest (one row block's A tiles stay hot in L2 while its
-// output columns are swept).
-// Measured limit: every tcgen05.cp of block scales takes ~115 cycles of the
-// SM's copy engine whatever its size (a 512-byte 32x128b.warpx4 atom or a
-// 4 KB 128x256b block alike).  The weight bundle therefore stores each B-scale
-// atom four times over, the image of its warpx4 copy, so one 128x256b copy
-// moves a k-block's scales for all 256 weight rows: a k-stage needs 8 copies
-// (A: 1, B: 1 per k-block) instead of 12, against 4 MMAs of ~128 cycles.
-// Every wait is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT and
-// raises the abort flag of both CTAs; in-flight work is drained, the pair
-// meets at a cluster barrier and frees TMEM.
-#include <cuda.h>
-#include <cuda_runtime.h>
-
-#include <algorithm>
-#include <mutex>
-#include <string>
-
-#include "device_common.cuh"
-#include "svdq_internal.h"
-
-namespace svdq {
-namespace {
-
-constexpr int BM = 128;                       // rows per CTA (256 per pair)
-constexpr int BN = 256;                       // output columns per pair tile
-constexpr int STAGES = 4;
-constexpr int ROW = 2048;                     // bytes per row of the bundle tensor maps
-constexpr int A_BYTES = BM * 144;             // activation tile: codes 16 KB + scales 2 KB
-constexpr int SFA_OFF = BM * 128;
-constexpr int A_CODE_BYTES = BM * 128;
-constexpr int SFA_BYTES = BM * 16;
-constexpr int B_OFF = A_BYTES;                // 18432, a multiple of 1024
-constexpr int B_BYTES = 128 * 128;            // this CTA's 128 weight rows of codes
-constexpr int SFB_OFF = B_OFF + B_BYTES;      // scales of all 256 weight rows, each atom 4 times
-constexpr int SFB_BYTES = 4 * 4096;           // per k-block: [rows 0-127: 4 x 512 B][rows 128-255: 4 x 512 B]
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFB_BYTES;  // 51200
-constexpr int LR_BYTES = 128 * 128;           // U (this CTA's rows) and L2T (its columns), 16 KB each
-constexpr int EPI_WARPS = 8;
-constexpr int EPI_TILE_BYTES = 32 * 64;       // 32 rows x 32 bf16, 64-byte swizzle
-constexpr int EPI_OFF = STAGES * STAGE_BYTES;
-constexpr int BAR_OFF = EPI_OFF + EPI_WARPS * EPI_TILE_BYTES;
-constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
-constexpr int THREADS = (4 + EPI_WARPS) * 32;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL = 256;              // stage s: SFA at +48s (+4 kb), SFB at +48s+16 (+8 kb, +4 per row block)
-static_assert(STAGE_BYTES % 1024 == 0 && B_OFF % 1024 == 0, "MMA operand tiles start on 1024-byte boundaries");
-static_assert(A_CODE_BYTES % ROW == 0 && SFA_BYTES % ROW == 0 && B_BYTES % ROW == 0 && SFB_BYTES % ROW == 0 &&
-                  LR_BYTES % ROW == 0,
-              "copies are whole tensor-map rows");
-static_assert(SF_COL + 48 * STAGES <= TMEM_COLS, "scale columns fit in TMEM");
-
-// Instruction descriptors (tcgen05 instruction-descriptor bit fields):
-// [4,6) accumulator format (1 = f32), [7,10) A format, [10,13) B format,
-// [17,23) N >> 3, [24,29) M >> 4 (M = 256: the pair); block-scaled: [23]
-// scale format (0 = ue4m3), scale-factor ids 0; A/B K-major (bits 15/16 = 0).
-constexpr uint32_t IDESC_BF16 = (1u << 4) | (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((256 >> 4) << 24);
-constexpr uint32_t IDESC_NVFP4 = (1u << 7) | (1u << 10) | ((BN >> 3) << 17) | ((256 >> 4) << 24);
-
-__device__ __forceinline__ uint32_t sfa_col(int s, int kb) { return SF_COL + 48 * s + 4 * kb; }
-__device__ __forceinline__ uint32_t sfb_col(int s, int kb) { return SF_COL + 48 * s + 16 + 8 * kb; }
-
-struct Params {
-  int M, N, rank, epilogue, gelu_col_begin;
-  int num_m2, num_n, num_tiles, k_stages, lr_stages, kb_total;
-  const float *s_a, *s_w;
-  const uint16_t *bias;
-  unsigned int *status;
-  unsigned long long limit_ns;
-};
-
-struct Maps {
-  CUtensorMap a, sfa, b, sfb, u, l2, y;
-};
-
-
-// Raises the abort flag of this CTA and of its partner, records the timeout.
-__device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t peer_abort, unsigned int *status) {
-  *abort_flag = 1;
-  dev::st_cluster_u32(peer_abort, 1u);
-  dev::report(status, SVDQ_ERR_TIMEOUT);
-}
-
-// EPI: the epilogue (SVDQ_EPILOGUE_*), a template parameter so that each
-// instantiation holds only its own, fully unrolled epilogue: with both GELU
-// forms behind runtime branches the kernel's code outgrew the instruction
-// cache and every role stalled on instruction fetch.
-template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    gemm_w4a4_kernel(const __grid_constant__ Maps maps, Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);  // even CTA: both CTAs' bytes
-  uint64_t *sf_full = full + STAGES;                               // even CTA: scales in TMEM
-  uint64_t *empty = sf_full + STAGES;                              // both CTAs: stage free again
-  uint64_t *tmem_full = empty + STAGES;                            // both CTAs: accumulator ready
-  uint64_t *tmem_empty = tmem_full + 1;                            // even CTA: both CTAs drained it
-  uint64_t *drain_mma = tmem_empty + 1;
-  uint64_t *drain_cp = drain_mma + 1;
-  uint64_t *sf_loaded = drain_cp + 1;                              // even CTA: both CTAs' scale bytes
-  uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(sf_loaded + STAGES);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t h = dev::cluster_ctarank();         // 0: even CTA (issues the MMAs), 1: odd
-  const int pair = static_cast<int>(dev::cluster_id_x());
-  const int num_pairs = static_cast<int>(dev::num_clusters_x());
-  // this pair's tiles: a contiguous run of tile ids, n fastest
-  const int t_begin = static_cast<int>((static_cast<long long>(pair) * p.num_tiles) / num_pairs);
-  const int t_end = static_cast<int>((static_cast<long long>(pair + 1) * p.num_tiles) / num_pairs);
-  const int stages_per_tile = p.lr_stages + p.k_stages;
-  const uint32_t peer_abort = dev::mapa(dev::smem_u32(const_cast<int *>(abort_flag)), h ^ 1u);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      dev::mbar_init(&full[s], 1);            // the even CTA's producer arrival (+ the bytes of both CTAs)
-      dev::mbar_init(&sf_full[s], 1);
-      dev::mbar_init(&empty[s], 1);
-      dev::mbar_init(&sf_loaded[s], 1);
-    }
-    dev::mbar_init(tmem_full, 1);
-    dev::mbar_init(tmem_empty, 2 * EPI_WARPS);
-    dev::mbar_init(drain_mma, 1);
-    dev::mbar_init(drain_cp, 1);
-    *abort_flag = 0;
-    dev::fence_mbar_init();
-  }
-  if (warp == 1) {
-    dev::tmem_alloc_pair(tmem_base_slot, TMEM_COLS);
-    dev::tmem_relinquish_pair();
-  }
-  dev::tc_fence_before();
-  __syncwarp();
-  dev::cluster_sync();                        // both CTAs' barriers exist before anyone arrives remotely
-  dev::tc_fence_after();
-  const uint32_t tmem = *tmem_base_slot;
-  dev::grid_dependency_wait();                // the operands written by the previous kernel are visible
-  dev::grid_launch_dependents();
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      dev::prefetch_tmap(&maps.a);
-      dev::prefetch_tmap(&maps.b);
-      dev::prefetch_tmap(&maps.sfb);
-      if (p.lr_stages) {
-        dev::prefetch_tmap(&maps.u);
-        dev::prefetch_tmap(&maps.l2);
-      }
-      int it = 0;
-      bool ok = true;
-      for (int tile = t_begin; tile < t_end && ok; ++tile) {
-        const int m_blk = 2 * (tile / p.num_n) + static_cast<int>(h);  // this CTA's 128-row block
-        const int n_blk = tile % p.num_n;
-        for (int st = 0; st < stages_per_tile; ++st, ++it) {
-          const int s = it % STAGES;
-          if (!dev::mbar_wait_cluster(&empty[s], ((it / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const uint32_t bar = dev::mapa(dev::smem_u32(&full[s]), 0);
-          uint8_t *dst = smem + s * STAGE_BYTES;
-          if (st < p.lr_stages) {
-            if (h == 0) {
-              dev::mbar_arrive(&sf_loaded[s]);    // no scales in the low-rank stage
-              dev::mbar_arrive_expect_tx(&full[s], 2u * 2u * LR_BYTES);
-            }
-            dev::tma_load_2d_pair(dst, &maps.u, bar, 0, m_blk * (LR_BYTES / ROW));
-            dev::tma_load_2d_pair(dst + B_OFF, &maps.l2, bar, 0, (2 * n_blk + static_cast<int>(h)) * (LR_BYTES / ROW));
-          } else {
-            const int ks = st - p.lr_stages;
-            const int wrow = (n_blk * p.k_stages + ks) * ((2 * B_BYTES + SFB_BYTES) / ROW);
-            const int arow = (m_blk * p.k_stages + ks) * (A_BYTES / ROW);
-            const uint32_t sbar = dev::mapa(dev::smem_u32(&sf_loaded[s]), 0);
-            if (h == 0) {
-              dev::mbar_arrive_expect_tx(&sf_loaded[s], 2u * (SFA_BYTES + SFB_BYTES));
-              dev::mbar_arrive_expect_tx(&full[s], 2u * (A_CODE_BYTES + B_BYTES));
-            }
-            // the scales first, on their own barrier: their copies into TMEM
-            // then overlap the transfer of the codes
-            dev::tma_load_2d_pair(dst + SFA_OFF, &maps.sfa, sbar, 0, arow + SFA_OFF / ROW);
-            dev::tma_load_2d_pair(dst + SFB_OFF, &maps.sfb, sbar, 0, wrow + 2 * B_BYTES / ROW);
-            dev::tma_load_2d_pair(dst, &maps.a, bar, 0, arow);
-            dev::tma_load_2d_pair(dst + B_OFF, &maps.b, bar, 0, wrow + static_cast<int>(h) * (B_BYTES / ROW));
-          }
-        }
-      }
-      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
-      // Before the pair may leave: the even CTA waits for every stage it
-      // armed to complete (that covers the odd CTA's copies as well).
-      if (h == 0) {
-        for (int j = max(0, it - STAGES); j < it; ++j) {
-          dev::mbar_wait_cluster(&full[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
-          dev::mbar_wait_cluster(&sf_loaded[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (h == 0 && lane == 0) {
-      int it = 0, tcount = 0;
-      bool ok = true, issued_any = false;
-      for (int tile = t_begin; tile < t_end && ok; ++tile, ++tcount) {
-        if (!dev::mbar_wait_cluster(tmem_empty, (tcount & 1) ^ 1, p.limit_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        dev::tc_fence_after();
-        uint32_t accumulate = 0;
-        for (int st = 0; st < stages_per_tile; ++st, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!dev::mbar_wait(&sf_full[s], ph, p.limit_ns, abort_flag) ||
-              !dev::mbar_wait_cluster(&full[s], ph, p.limit_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          dev::tc_fence_after();
-          const uint32_t sa = dev::smem_u32(smem + s * STAGE_BYTES);
-          const uint32_t sb = sa + B_OFF;
-          if (st < p.lr_stages) {
-            for (int j = 0; j < p.rank / 16; ++j) {  // K = 16 bf16 = 32 bytes per MMA
-              dev::umma_bf16_pair(tmem, dev::desc_sw128(sa + 32 * j), dev::desc_sw128(sb + 32 * j), IDESC_BF16,
-                                  accumulate);
-              accumulate = 1;
-            }
-          } else {
-            const int nkb = min(4, p.kb_total - 4 * (st - p.lr_stages));
-            for (int kb = 0; kb < nkb; ++kb) {  // K = 64 e2m1 = 32 bytes per MMA
-              dev::umma_nvfp4_pair(tmem, dev::desc_sw128(sa + 32 * kb), dev::desc_sw128(sb + 32 * kb), IDESC_NVFP4,
-                                   tmem + sfa_col(s, kb), tmem + sfb_col(s, kb), accumulate);
-              accumulate = 1;
-            }
-          }
-          issued_any = true;
-          dev::tc_commit_pair_mc(&empty[s], 0x3);  // both CTAs' stage s free once these MMAs finish
-        }
-        if (!ok) break;
-        dev::tc_commit_pair_mc(tmem_full, 0x3);    // both halves of the accumulator ready
-      }
-      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
-      if (issued_any) {  // the tensor cores must be idle before TMEM is freed
-        dev::tc_commit_pair(drain_mma);
-        dev::mbar_wait(drain_mma, 0, p.limit_ns, nullptr);
-      }
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ scale-factor copies (even CTA)
-    if (h == 0 && lane == 0) {
-      int it = 0;
-      bool ok = true, issued_any = false;
-      for (int tile = t_begin; tile < t_end && ok; ++tile) {
-        for (int st = 0; st < stages_per_tile; ++st, ++it) {
-          const int s = it % STAGES;
-          if (!dev::mbar_wait_cluster(&sf_loaded[s], (it / STAGES) & 1, p.limit_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (st >= p.lr_stages) {
-            const int nkb = min(4, p.kb_total - 4 * (st - p.lr_stages));
-            const uint32_t ssfa = dev::smem_u32(smem + s * STAGE_BYTES + SFA_OFF);
-            const uint32_t ssfb = dev::smem_u32(smem + s * STAGE_BYTES + SFB_OFF);
-            for (int kb = 0; kb < nkb; ++kb) {
-              dev::tmem_cp_32x128b_x4_pair(tmem + sfa_col(s, kb), dev::desc_sf(ssfa + 512 * kb));
-              // both 128-row halves of the B scales in one copy: the four replicas of an
-              // atom fill the four lane quarters as one warpx4 copy of it would
-              dev::tmem_cp_128x256b_pair(tmem + sfb_col(s, kb), dev::desc_sf_2x(ssfb + 4096 * kb));
-            }
-            issued_any = true;
-          }
-          dev::tc_commit_pair(&sf_full[s]);  // arrives once this stage's copies have landed
-        }
-      }
-      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
-      if (issued_any) {
-        dev::tc_commit_pair(drain_cp);
-        dev::mbar_wait(drain_cp, 0, p.limit_ns, nullptr);
-      }
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ epilogue (both CTAs)
-    const int e = warp - 4;
-    const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int half = e >> 2;                // which 128 of the 256 columns
-    uint8_t *stage_out = smem + EPI_OFF + e * EPI_TILE_BYTES;
-    const uint32_t tmem_empty_even = dev::mapa(dev::smem_u32(tmem_empty), 0);
-    const float alpha = __fmul_rn(__ldg(p.s_a), __ldg(p.s_w));
-    int tcount = 0;
-    for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
-      const int m_blk = 2 * (tile / p.num_n) + static_cast<int>(h);
-      const int n_blk = tile % p.num_n;
-      if (!dev::mbar_wait_cluster(tmem_full, tcount & 1, p.limit_ns, abort_flag)) {
-        abort_pair(abort_flag, peer_abort, p.status);
-        break;
-      }
-      dev::tc_fence_after();
-      uint32_t v[4][32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(half * 128);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) dev::tmem_ld_32x32b_x32(taddr + 32 * c, v[c]);
-      dev::tmem_wait_ld();
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive_cluster(tmem_empty_even);  // the MMA thread may start the next tile
-
-      const int row0 = m_blk * BM + 32 * q;
-      const int col0 = n_blk * BN + half * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {           // four 32-column chunks
-        if (lane == 0) dev::bulk_wait_group_read<0>();  // staging tile free again
-        __syncwarp();
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {         // 8 columns (16 bytes) at a time
-          const int col = col0 + 32 * c + 8 * g;
-          float b[8];
-          if (p.bias && col + 8 <= p.N) {
-            const uint4 bb = __ldg(reinterpret_cast<const uint4 *>(p.bias + col));
-            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              b[2 * j] = __uint_as_float(bw[j] << 16);
-              b[2 * j + 1] = __uint_as_float(bw[j] & 0xFFFF0000u);
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) b[j] = 0.0f;
-          }
-          uint32_t out[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float y0 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j]), b[2 * j]);
-            float y1 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j + 1]), b[2 * j + 1]);
-            if constexpr (EPI != SVDQ_EPILOGUE_NONE) {
-              // computed for every column and selected: straight-line code lets the
-              // independent GELU chains of a chunk interleave (a branch per element
-              // serialised them)
-              const bool act0 = col + 2 * j >= p.gelu_col_begin, act1 = col + 2 * j + 1 >= p.gelu_col_begin;
-              float g0, g1;
-              if constexpr (EPI == SVDQ_EPILOGUE_GELU_ERF) {
-                g0 = dev::gelu_erf(y0);
-                g1 = dev::gelu_erf(y1);
-              } else {
-                g0 = dev::gelu_tanh(y0);
-                g1 = dev::gelu_tanh(y1);
-              }
-              y0 = act0 ? g0 : y0;
-              y1 = act1 ? g1 : y1;
-            }
-            __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
-            out[j] = *reinterpret_cast<uint32_t *>(&hv);
-          }
-          // row `lane` of the 32 x 32 staging tile, 16-byte chunk g, 64-byte swizzle
-          *reinterpret_cast<uint4 *>(stage_out + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) =
-              make_uint4(out[0], out[1], out[2], out[3]);
-        }
-        dev::fence_proxy_async();  // make the generic writes visible to the TMA store
-        __syncwarp();
-        if (lane == 0 && row0 < p.M && col0 + 32 * c < p.N) {  // the TMA clips the ragged edges
-          dev::tma_store_2d(&maps.y, stage_out, col0 + 32 * c, row0);
-          dev::bulk_commit_group();
-        }
-      }
-    }
-    if (lane == 0) dev::bulk_wait_group<0>();
-  }
-
-  dev::tc_fence_before();
-  __syncwarp();
-  dev::cluster_sync();                        // no MMA or copy of the pair is still running
-  if (warp == 1) {
-    dev::tc_fence_after();
-    dev::tmem_dealloc_pair(tmem, TMEM_COLS);
-  }
-}
-
-// Per device, once: the shared-memory opt-in of the kernel and the number of
-// SM pairs that can hold one CTA each at that size.
-int prepare_device(int sm_count, int *pairs_out) {
-  static std::mutex mu;
-  static int cached[64] = {0};
-  int dev_id = 0;
-  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64)
-    return fail(SVDQ_ERR_CUDA, "svdq_linear_w4a4: no current device");
-  std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev_id] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               SMEM_BYTES);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4: ") + cudaGetErrorString(e));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(sm_count & ~1), 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE>, &cfg) != cudaSuccess || n < 1) {
-      cudaGetLastError();
-      n = sm_count / 2;
-    }
-    cached[dev_id] = n;
-  }
-  *pairs_out = cached[dev_id];
-  return SVDQ_OK;
-}
-
-}  // namespace
-}  // namespace svdq
+// K2: the W4A4 GEMM with the low-rank up-projection fused in - entry point
+// of the plain variant (the kernel itself is in gemm_w4a4_kernel.cuh).
+#include "gemm_w4a4_kernel.cuh"
 
 using namespace svdq;
+using namespace svdq::w4a4;
 
 extern "C" int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const float *s_a, const uint8_t *w_bundle,
                                 const void *l2t, const float *s_w, const void *bias, int M, int N, int K, int rank,
                                 int epilogue, int gelu_col_begin, void *Y, int ldy, svdq_stream_t stream) {
-  if (!a_bundle || !s_a || !w_bundle || !s_w || !Y || (rank > 0 && (!U || !l2t)))
-    return fail(SVDQ_ERR_INVALID_ARG, "svdq_linear_w4a4: null pointer");
-  if (epilogue < SVDQ_EPILOGUE_NONE || epilogue > SVDQ_EPILOGUE_GELU_TANH)
-    return fail(SVDQ_ERR_INVALID_ARG, "svdq_linear_w4a4: unknown epilogue");
-  if (M < 1 || K < 64 || K % 64 || N < 8 || N % 8 || ldy < N || ldy % 8)
-    return fail(SVDQ_ERR_SHAPE, "svdq_linear_w4a4: need M >= 1, K % 64 == 0, N % 8 == 0, ldy >= N, ldy % 8 == 0");
-  if (rank < 0 || rank > SVDQ_LR_STRIDE || rank % 16)
-    return fail(SVDQ_ERR_SHAPE, "svdq_linear_w4a4: rank must be a multiple of 16 in [0, 64]");
-  if (gelu_col_begin < 0 || gelu_col_begin > N)
-    return fail(SVDQ_ERR_SHAPE, "svdq_linear_w4a4: gelu_col_begin outside [0, N]");
-  if (!aligned16(a_bundle) || !aligned16(w_bundle) || !aligned16(Y) || (bias && !aligned16(bias)) ||
-      (rank > 0 && (!aligned16(U) || !aligned16(l2t))))
-    return fail(SVDQ_ERR_ALIGNMENT, "svdq_linear_w4a4: pointers must be 16-byte aligned");
-  DeviceState *st = current_device_state();
-  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
-
-  Params p;
-  p.M = M;
-  p.N = N;
-  p.rank = rank;
-  p.epilogue = epilogue;
-  p.gelu_col_begin = gelu_col_begin;
-  p.num_m2 = (M + 2 * BM - 1) / (2 * BM);
-  p.num_n = (N + BN - 1) / BN;
-  p.num_tiles = p.num_m2 * p.num_n;
-  p.kb_total = K / 64;
-  p.k_stages = bundle_ks(K);
-  p.lr_stages = rank > 0 ? 1 : 0;
-  p.s_a = s_a;
-  p.s_w = s_w;
-  p.bias = static_cast<const uint16_t *>(bias);
-  p.status = st->status_word;
-  p.limit_ns = kWaitLimitNs;
-
-  // The bundles are read as rows of 2 KB (256 x 8-byte elements); a copy is
-  // a box of whole rows.  Rows past the end of a buffer (the odd half of a
-  // pair tile whose rows lie beyond M) read as zeros.
   Maps maps;
-  const auto u64 = CU_TENSOR_MAP_DATA_TYPE_UINT64;
-  const auto none = CU_TENSOR_MAP_SWIZZLE_NONE;
-  const uint64_t a_rows = bundle_bytes(M, K, 128) / ROW, w_rows = bundle_bytes(N, K, 256) / ROW;
-  int rc = encode_tmap_2d(&maps.a, u64, a_bundle, ROW / 8, a_rows, ROW, ROW / 8, A_CODE_BYTES / ROW, none);
-  if (rc == SVDQ_OK) rc = encode_tmap_2d(&maps.sfa, u64, a_bundle, ROW / 8, a_rows, ROW, ROW / 8, SFA_BYTES / ROW, none);
-  if (rc == SVDQ_OK) rc = encode_tmap_2d(&maps.b, u64, w_bundle, ROW / 8, w_rows, ROW, ROW / 8, B_BYTES / ROW, none);
-  if (rc == SVDQ_OK)
-    rc = encode_tmap_2d(&maps.sfb, u64, w_bundle, ROW / 8, w_rows, ROW, ROW / 8, SFB_BYTES / ROW, none);
-  if (rc == SVDQ_OK && rank > 0) {
-    rc = encode_tmap_2d(&maps.u, u64, U, ROW / 8, lowrank_bytes(M, 128) / ROW, ROW, ROW / 8, LR_BYTES / ROW, none);
-    if (rc == SVDQ_OK)
-      rc = encode_tmap_2d(&maps.l2, u64, l2t, ROW / 8, lowrank_bytes(N, 256) / ROW, ROW, ROW / 8, LR_BYTES / ROW,
-                          none);
-  } else {
-    maps.u = maps.a;  // unused without the low-rank stage
-    maps.l2 = maps.a;
-  }
-  if (rc == SVDQ_OK)
-    rc = encode_tmap_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, static_cast<uint64_t>(N),
-                        static_cast<uint64_t>(M), static_cast<uint64_t>(ldy) * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+  Params p;
+  DeviceState *st = nullptr;
+  int rc = setup_gemm("svdq_linear_w4a4", a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue,
+                      gelu_col_begin, Y, ldy, false, &maps, &p, &st);
   if (rc != SVDQ_OK) return rc;
-
-  int resident = 0;
-  rc = prepare_device(st->sm_count, &resident);
-  if (rc != SVDQ_OK) return rc;
-  const int pairs = std::min(p.num_tiles, resident);
-  DependentLaunch dl(dim3(2 * pairs), dim3(THREADS), SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream));
-  cudaError_t e = epilogue == SVDQ_EPILOGUE_GELU_ERF
-                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF>, maps, p)
-                  : epilogue == SVDQ_EPILOGUE_GELU_TANH
-                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH>, maps, p)
-                      : cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE>, maps, p);
-  if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4 launch: ") + cudaGetErrorString(e));
-  return ok();
+  rc = launch_gemm<-1>("svdq_linear_w4a4", maps, p, st->sm_count, reinterpret_cast<cudaStream_t>(stream));
+  return rc == SVDQ_OK ? ok() : rc;
 }

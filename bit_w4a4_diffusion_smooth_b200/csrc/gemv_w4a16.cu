@@ -5,10 +5,16 @@
 // 但硬件仍决定适用范围", remio.ai, section "Nunchaku Diffusers 支持改变了加载路径").
 // With up to 16 rows the layer is one pass over the weights and the kernel
 // is bound by how many weight bytes are in flight:
-//   * one CTA per quad of 64 output columns, its 16 warps split K by groups
-//     of 64; before any arithmetic each warp requests all of its groups'
-//     weights (4 x 16 bytes per lane and group: the four 16-column blocks),
-//     scales and zero points, so a CTA has 48 KB in flight (K = 3072);
+//   * one CTA of 8 warps per quad of 64 output columns, two CTAs per SM (at
+//     the adaLN widths every CTA of the grid is resident at once).  A quad's
+//     weights are contiguous (quad-major layout), so one thread requests them
+//     at the start with bulk copies into a shared-memory ring of chunks of 8
+//     groups of 64 along K (16 KB of codes + 1 KB of scales + 1 KB of zero
+//     points each, 6 chunks = K 3072 in flight per CTA, ~200 KB per SM);
+//     longer K refills a chunk once all 8 warps have consumed it;
+//   * warp w takes group w of every chunk, reading its four 16-column blocks
+//     (512 bytes each, lane-contiguous) from shared memory as soon as the
+//     chunk's barrier completes;
 //   * the products run on the tensor cores as Y^T = W^T . X^T (mma.sync
 //     m16n8k16: 16 output columns x 16 k per instruction, the rows of X in
 //     the 8-wide slot); X^ = f32(x * inv_awq) is split into bf16 hi + lo
@@ -17,7 +23,7 @@
 //     (128 + q) by one mask-and-or, one bf16x2 subtraction of (128 + z)
 //     gives (q - z) exactly;
 //   * per group the fp32 partial is scaled by s in registers; the warps'
-//     partials are added through shared memory.
+//     partials are added through shared memory (the ring, once drained).
 // More than 16 rows (a batch of modulation vectors) run as blocks of 16 rows
 // on the grid's second dimension; each block is one more pass over the
 // weights, mostly from L2.
@@ -49,11 +55,6 @@ __device__ __forceinline__ void a_frags(uint32_t w, uint32_t (&a)[4]) {
   a[3] = nib_pair(w >> 12);   // column g+8, k 2t+8, 2t+9
 }
 
-// ===========================================================================
-// Direct kernel: one CTA per quad and block of 8 NT rows, 16 warps split K by groups.
-constexpr int D_THREADS = 512;
-constexpr int D_WARPS = D_THREADS / 32;
-
 struct Params {
   int M, K, N, ldx, ldy, G;
   const uint16_t *X;
@@ -61,6 +62,8 @@ struct Params {
   const uint4 *qw;
   const uint16_t *scales, *zeros, *bias;
   uint16_t *Y;
+  unsigned int *status;
+  unsigned long long limit_ns;
 };
 
 // B fragments (hi and lo bf16 parts of X^) of one k16 step for rows nt*8+g.
@@ -103,20 +106,61 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t w, int s, uint32_t z12
   return *reinterpret_cast<uint32_t *>(&d);
 }
 
-template <int NT, int GPW>
-__global__ void __launch_bounds__(D_THREADS, 1) awq_gemv_kernel(Params p) {
-  extern __shared__ float red[];  // [WARPS][4][NT][32][4]
+// ===========================================================================
+// One CTA per quad (64 output columns) and block of 8 NT rows.
+constexpr int S_THREADS = 256;
+constexpr int S_WARPS = S_THREADS / 32;
+constexpr int CHUNK_G = S_WARPS;                 // groups per chunk: one per warp
+constexpr int CHUNK_QW = CHUNK_G * 2048;         // codes: 2 KB per group (four 16-column blocks)
+constexpr int CHUNK_SZ = CHUNK_G * 128;          // scales (and zero points): 64 bf16 per group
+constexpr int CHUNK_BYTES = CHUNK_QW + 2 * CHUNK_SZ;
+constexpr int RING = 6;
+constexpr int BAR_OFF = RING * CHUNK_BYTES;
+constexpr int SMEM_BYTES = BAR_OFF + 2 * RING * 8 + 16;
+static_assert(S_WARPS * 4 * 2 * 32 * 4 * 4 <= BAR_OFF, "the partial sums fit the drained ring");
+
+template <int NT>
+__global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);
+  uint64_t *empty = full + RING;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + RING);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t = lane & 3;
   const int quad = blockIdx.x;
+  const int nchunks = (p.G + CHUNK_G - 1) / CHUNK_G;
   {  // this CTA's block of 8 NT rows
     const int r0 = static_cast<int>(blockIdx.y) * 8 * NT;
     p.X += static_cast<size_t>(r0) * p.ldx;
     p.Y += static_cast<size_t>(r0) * p.ldy;
     p.M = min(8 * NT, p.M - r0);
   }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RING; ++s) {
+      dev::mbar_init(&full[s], 1);
+      dev::mbar_init(&empty[s], S_WARPS);
+    }
+    *abort_flag = 0;
+    dev::fence_mbar_init();
+  }
+  __syncthreads();
   dev::grid_dependency_wait();
   dev::grid_launch_dependents();
+
+  // chunk c: groups 8c .. 8c+7 of the quad, into ring slot c % RING
+  auto issue = [&](int c) {
+    uint8_t *dst = smem + (c % RING) * CHUNK_BYTES;
+    const int g0 = c * CHUNK_G, ng = min(CHUNK_G, p.G - g0);
+    const size_t blk = static_cast<size_t>(quad) * p.G + g0;
+    uint64_t *bar = &full[c % RING];
+    dev::mbar_arrive_expect_tx(bar, static_cast<uint32_t>(ng * (2048 + 2 * 128)));
+    dev::bulk_load(dst, p.qw + blk * 128, static_cast<uint32_t>(ng * 2048), bar);
+    dev::bulk_load(dst + CHUNK_QW, p.scales + blk * 64, static_cast<uint32_t>(ng * 128), bar);
+    dev::bulk_load(dst + CHUNK_QW + CHUNK_SZ, p.zeros + blk * 64, static_cast<uint32_t>(ng * 128), bar);
+  };
+  int issued = 0;
+  if (threadIdx.x == 0)
+    for (; issued < min(RING, nchunks); ++issued) issue(issued);
 
   float tot[4][NT][4];
 #pragma unroll
@@ -127,81 +171,90 @@ __global__ void __launch_bounds__(D_THREADS, 1) awq_gemv_kernel(Params p) {
       for (int e = 0; e < 4; ++e) tot[a][b][e] = 0.0f;
 
 #pragma unroll 1
-  for (int base = 0; base < p.G; base += D_WARPS * GPW) {
-  // every weight, scale and zero point of this slice, requested before any arithmetic:
-  // groups base + warp, base + warp + 16, ... of the quad, 4 column blocks each
-  uint4 wq[GPW][4];
-  uint32_t sp[GPW][4], zp[GPW][4];  // bf16 of columns g (low half) and g + 8 (high half)
-#pragma unroll
-  for (int i = 0; i < GPW; ++i) {
-    const int grp = base + warp + D_WARPS * i;
-    const size_t blk = static_cast<size_t>(quad) * p.G + (grp < p.G ? grp : 0);
-#pragma unroll
-    for (int cb = 0; cb < 4; ++cb) {
-      if (grp < p.G) {
-        wq[i][cb] = __ldg(p.qw + (blk * 4 + cb) * 32 + lane);
-        const size_t gb = blk * 64 + cb * 16 + g8;
-        sp[i][cb] = static_cast<uint32_t>(__ldg(p.scales + gb)) | (static_cast<uint32_t>(__ldg(p.scales + gb + 8)) << 16);
-        zp[i][cb] = static_cast<uint32_t>(__ldg(p.zeros + gb)) | (static_cast<uint32_t>(__ldg(p.zeros + gb + 8)) << 16);
-      } else {
-        wq[i][cb] = make_uint4(0, 0, 0, 0);
-        sp[i][cb] = zp[i][cb] = 0;
-      }
+  for (int c = 0; c < nchunks; ++c) {
+    const int slot = c % RING;
+    if (!dev::mbar_wait_warp(&full[slot], (c / RING) & 1, p.limit_ns, abort_flag)) {
+      *abort_flag = 1;
+      dev::report(p.status, SVDQ_ERR_TIMEOUT);
+      break;
     }
-  }
-
-#pragma unroll
-  for (int i = 0; i < GPW; ++i) {
-    const int grp = base + warp + D_WARPS * i;
-    if (grp >= p.G) break;
-    uint32_t z_lo[4], z_hi[4];
-#pragma unroll
-    for (int cb = 0; cb < 4; ++cb) {
-      const float zl = bf16_bits_to_float(zp[i][cb] & 0xFFFFu), zh = bf16_bits_to_float(zp[i][cb] >> 16);
-      z_lo[cb] = pack_bf16x2(128.0f + zl, 128.0f + zl);
-      z_hi[cb] = pack_bf16x2(128.0f + zh, 128.0f + zh);
-    }
-    float c[4][NT][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < NT; ++b)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) c[a][b][e] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t bh[NT][2], bl[NT][2];
-      load_x_frag<NT>(p, grp * 64 + 16 * j + 2 * t, g8, bh, bl);
+    const int grp = c * CHUNK_G + warp;
+    if (grp < p.G) {
+      const uint8_t *src = smem + slot * CHUNK_BYTES;
+      uint4 wq[4];
+      uint32_t sp[4], zp[4];  // bf16 of columns g (low half) and g + 8 (high half) of each block
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
-        const uint4 &w4 = wq[i][cb];
-        const uint32_t w = j == 0 ? w4.x : j == 1 ? w4.y : j == 2 ? w4.z : w4.w;
-        uint32_t a[4];
-        a[0] = dequant_pair(w, 0, z_lo[cb]);
-        a[1] = dequant_pair(w, 4, z_hi[cb]);
-        a[2] = dequant_pair(w, 8, z_lo[cb]);
-        a[3] = dequant_pair(w, 12, z_hi[cb]);
+        wq[cb] = reinterpret_cast<const uint4 *>(src + warp * 2048)[cb * 32 + lane];
+        const uint16_t *sc = reinterpret_cast<const uint16_t *>(src + CHUNK_QW + warp * 128) + cb * 16 + g8;
+        const uint16_t *zc = reinterpret_cast<const uint16_t *>(src + CHUNK_QW + CHUNK_SZ + warp * 128) + cb * 16 + g8;
+        sp[cb] = static_cast<uint32_t>(sc[0]) | (static_cast<uint32_t>(sc[8]) << 16);
+        zp[cb] = static_cast<uint32_t>(zc[0]) | (static_cast<uint32_t>(zc[8]) << 16);
+      }
+      uint32_t z_lo[4], z_hi[4];
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        const float zl = bf16_bits_to_float(zp[cb] & 0xFFFFu), zh = bf16_bits_to_float(zp[cb] >> 16);
+        z_lo[cb] = pack_bf16x2(128.0f + zl, 128.0f + zl);
+        z_hi[cb] = pack_bf16x2(128.0f + zh, 128.0f + zh);
+      }
+      float acc[4][NT][4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < NT; ++b)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t bh[NT][2], bl[NT][2];
+        load_x_frag<NT>(p, grp * 64 + 16 * j + 2 * t, g8, bh, bl);
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb) {
+          const uint32_t w = j == 0 ? wq[cb].x : j == 1 ? wq[cb].y : j == 2 ? wq[cb].z : wq[cb].w;
+          uint32_t a[4];
+          a[0] = dequant_pair(w, 0, z_lo[cb]);
+          a[1] = dequant_pair(w, 4, z_hi[cb]);
+          a[2] = dequant_pair(w, 8, z_lo[cb]);
+          a[3] = dequant_pair(w, 12, z_hi[cb]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            dev::mma_bf16_16816(acc[cb][nt], a, bh[nt][0], bh[nt][1]);
+            dev::mma_bf16_16816(acc[cb][nt], a, bl[nt][0], bl[nt][1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        const float s_lo = bf16_bits_to_float(sp[cb] & 0xFFFFu), s_hi = bf16_bits_to_float(sp[cb] >> 16);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          dev::mma_bf16_16816(c[cb][nt], a, bh[nt][0], bh[nt][1]);
-          dev::mma_bf16_16816(c[cb][nt], a, bl[nt][0], bl[nt][1]);
+          tot[cb][nt][0] = __fmaf_rn(s_lo, acc[cb][nt][0], tot[cb][nt][0]);
+          tot[cb][nt][1] = __fmaf_rn(s_lo, acc[cb][nt][1], tot[cb][nt][1]);
+          tot[cb][nt][2] = __fmaf_rn(s_hi, acc[cb][nt][2], tot[cb][nt][2]);
+          tot[cb][nt][3] = __fmaf_rn(s_hi, acc[cb][nt][3], tot[cb][nt][3]);
         }
       }
     }
-#pragma unroll
-    for (int cb = 0; cb < 4; ++cb) {
-      const float s_lo = bf16_bits_to_float(sp[i][cb] & 0xFFFFu), s_hi = bf16_bits_to_float(sp[i][cb] >> 16);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        tot[cb][nt][0] = __fmaf_rn(s_lo, c[cb][nt][0], tot[cb][nt][0]);
-        tot[cb][nt][1] = __fmaf_rn(s_lo, c[cb][nt][1], tot[cb][nt][1]);
-        tot[cb][nt][2] = __fmaf_rn(s_hi, c[cb][nt][2], tot[cb][nt][2]);
-        tot[cb][nt][3] = __fmaf_rn(s_hi, c[cb][nt][3], tot[cb][nt][3]);
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(&empty[slot]);
+    // a longer K: refill this slot with chunk c + RING once every warp has read it
+    if (threadIdx.x == 0 && issued < nchunks) {
+      if (!dev::mbar_wait(&empty[slot], (c / RING) & 1, p.limit_ns, abort_flag)) {
+        *abort_flag = 1;
+        dev::report(p.status, SVDQ_ERR_TIMEOUT);
+      } else {
+        issue(issued++);
       }
     }
   }
-  }
+  // every copy this CTA issued has landed before its shared memory is reused or released
+  if (threadIdx.x == 0)
+    for (int c = max(0, issued - RING); c < issued; ++c)
+      dev::mbar_wait(&full[c % RING], (c / RING) & 1, p.limit_ns, nullptr);
+  __syncthreads();
 
+  float *red = reinterpret_cast<float *>(smem);  // [WARPS][4][NT][32][4]
 #pragma unroll
   for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
@@ -209,12 +262,13 @@ __global__ void __launch_bounds__(D_THREADS, 1) awq_gemv_kernel(Params p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) red[(((warp * 4 + cb) * NT + nt) * 32 + lane) * 4 + e] = tot[cb][nt][e];
   __syncthreads();
+  if (*abort_flag) return;                        // Y is left as it was; the status word has the error
 
   constexpr int SLOTS = 4 * NT * 32 * 4;
-  for (int slot = threadIdx.x; slot < SLOTS; slot += D_THREADS) {
+  for (int slot = threadIdx.x; slot < SLOTS; slot += S_THREADS) {
     float v = 0.0f;
-#pragma unroll 4
-    for (int w = 0; w < D_WARPS; ++w) v += red[w * SLOTS + slot];
+#pragma unroll
+    for (int w = 0; w < S_WARPS; ++w) v += red[w * SLOTS + slot];
     const int e = slot & 3, ln = (slot >> 2) & 31, nt = (slot >> 7) % NT, cb = (slot >> 7) / NT;
     const int n = quad * 64 + cb * 16 + (ln >> 2) + (e >= 2 ? 8 : 0);
     const int m = nt * 8 + 2 * (ln & 3) + (e & 1);
@@ -226,28 +280,15 @@ __global__ void __launch_bounds__(D_THREADS, 1) awq_gemv_kernel(Params p) {
   }
 }
 
-template <int NT, int GPW>
-int launch_direct(const Params &p, cudaStream_t stream) {
-  const int smem = D_WARPS * 4 * NT * 32 * 4 * static_cast<int>(sizeof(float));
-  cudaError_t e =
-      cudaFuncSetAttribute(awq_gemv_kernel<NT, GPW>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16: ") + cudaGetErrorString(e));
-  DependentLaunch dl(dim3(p.N / 64, (p.M + 8 * NT - 1) / (8 * NT)), dim3(D_THREADS), smem, stream);
-  e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT, GPW>, p);
+template <int NT>
+int launch(const Params &p, cudaStream_t stream) {
+  const int rc = smem_optin_once<awq_gemv_kernel<NT>>(SMEM_BYTES, "awq_linear_w4a16");
+  if (rc != SVDQ_OK) return rc;
+  DependentLaunch dl(dim3(p.N / 64, (p.M + 8 * NT - 1) / (8 * NT)), dim3(S_THREADS), SMEM_BYTES, stream);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT>, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16 launch: ") + cudaGetErrorString(e));
   return ok();
-}
-
-// Groups per warp (G / 16 rounded up, at most 3 for one row block of X and 1
-// for two, which keeps every operand in registers) picks the instantiation;
-// a longer K is walked in slices.
-int launch_direct_g(const Params &p, cudaStream_t stream) {
-  if (p.M > 8) return launch_direct<2, 1>(p, stream);
-  const int gpw = (p.G + D_WARPS - 1) / D_WARPS;
-  if (gpw <= 1) return launch_direct<1, 1>(p, stream);
-  if (gpw == 2) return launch_direct<1, 2>(p, stream);
-  return launch_direct<1, 3>(p, stream);
 }
 
 }  // namespace
@@ -286,5 +327,8 @@ extern "C" int awq_linear_w4a16(const void *X, int M, int K, int ldx, const floa
   p.zeros = static_cast<const uint16_t *>(zeros);
   p.bias = static_cast<const uint16_t *>(bias);
   p.Y = static_cast<uint16_t *>(Y);
-  return launch_direct_g(p, s);
+  p.status = st->status_word;
+  p.limit_ns = kWaitLimitNs;
+  // up to 8 rows: one block of rows; more: blocks of 16 rows, one pass over the weights each
+  return M > 8 ? launch<2>(p, s) : launch<1>(p, s);
 }

@@ -112,3 +112,18 @@ extern "C" int awq_pack_weights(const uint16_t *W, int K, int N, const float *aw
   for (int k = 0; k < K; ++k) inv_awq[k] = 1.0f / awq_scale[k];
   return ok();
 }
+
+extern "C" int awq_packed_sizes(int K, int N, int group, size_t *qweight_bytes, size_t *scales_bytes,
+                                size_t *zeros_bytes, size_t *inv_awq_bytes) {
+  using svdq::fail;
+  if (!qweight_bytes || !scales_bytes || !zeros_bytes || !inv_awq_bytes)
+    return fail(SVDQ_ERR_INVALID_ARG, "awq_packed_sizes: null pointer");
+  if (group != 64 || K < 64 || K % 64 || N < 64 || N % 64)
+    return fail(SVDQ_ERR_SHAPE, "awq_packed_sizes: need group == 64, K % 64 == 0, N % 64 == 0");
+  const size_t k = static_cast<size_t>(K), n = static_cast<size_t>(N);
+  *qweight_bytes = n * k / 2;
+  *scales_bytes = n * (k / 64) * 2;
+  *zeros_bytes = n * (k / 64) * 2;
+  *inv_awq_bytes = k * 4;
+  return svdq::ok();
+}

@@ -195,6 +195,8 @@ void orthonormalize(double *Y, int rows, int p) {
     for (int c = 0; c < p; ++c) Y[static_cast<size_t>(i) * p + c] = colmaj[static_cast<size_t>(c) * rows + i];
 }
 
+}  // namespace
+
 // Eigen-decomposition of the symmetric p x p matrix C (row-major) by cyclic
 // Jacobi rotations.  On return the eigenvalues are on C's diagonal and the
 // eigenvectors are the columns of V.
@@ -234,6 +236,8 @@ void jacobi_eigen(std::vector<double> &C, int p, std::vector<double> &V) {
     }
   }
 }
+
+namespace {
 
 // Standard normal draws from a fully specified engine (mt19937_64) through
 // Box-Muller, so the pack is reproducible across C++ libraries.

@@ -265,10 +265,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int q = 0; q < 4; ++q) {
         const uint32_t lo = (q >> 1) ? a1[q & 1] : a0[q & 1];
         const uint32_t hi = (q >> 1) ? a1[2 + (q & 1)] : a0[2 + (q & 1)];
-        xs[q][0] = __fmul_rn(bf16_lo(lo), i0.x);
-        xs[q][1] = __fmul_rn(bf16_hi(lo), i0.y);
-        xs[q][2] = __fmul_rn(bf16_lo(hi), i1.x);
-        xs[q][3] = __fmul_rn(bf16_hi(hi), i1.y);
+        const float2 p0 = dev::mul2_rn(make_float2(bf16_lo(lo), bf16_hi(lo)), i0);
+        const float2 p1 = dev::mul2_rn(make_float2(bf16_lo(hi), bf16_hi(hi)), i1);
+        xs[q][0] = p0.x;
+        xs[q][1] = p0.y;
+        xs[q][2] = p1.x;
+        xs[q][3] = p1.y;
       }
       if (RANK > 0) {
         // down-projection of this slice: A = bf16(x^), B = L1^T rows (ldmatrix of 2 tiles x 2 k-halves)
@@ -321,8 +323,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t cq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      cq[q] = dev::cvt_e2m1x2(__fmul_rn(xs[q][0], rq[q]), __fmul_rn(xs[q][1], rq[q])) |
-              (dev::cvt_e2m1x2(__fmul_rn(xs[q][2], rq[q]), __fmul_rn(xs[q][3], rq[q])) << 8);
+    {
+      const float2 r2 = make_float2(rq[q], rq[q]);
+      const float2 c0 = dev::mul2_rn(make_float2(xs[q][0], xs[q][1]), r2);
+      const float2 c1 = dev::mul2_rn(make_float2(xs[q][2], xs[q][3]), r2);
+      cq[q] = dev::cvt_e2m1x4(c0.x, c0.y, c1.x, c1.y);
+    }
     // gather: after the xor-1 step a lane holds bytes {e, e+1, e+4, e+5} (e = t & 2) of its
     // two kept blocks, after the xor-2 step all 8 bytes of the block it owns
     const uint32_t keep = o1 ? (cq[2] | (cq[3] << 16)) : (cq[0] | (cq[1] << 16));
@@ -379,10 +385,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 template <int RANK>
 int launch(const CUtensorMap &tx, const CUtensorMap &tl, const Params &p, int grid, cudaStream_t stream) {
   const int smem = smem_bytes<RANK>();
-  cudaError_t e = cudaFuncSetAttribute(quant_act_kernel<RANK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_quantize_act: ") + cudaGetErrorString(e));
+  const int rc = smem_optin_once<quant_act_kernel<RANK>>(smem, "svdq_quantize_act");
+  if (rc != SVDQ_OK) return rc;
   DependentLaunch dl(dim3(grid), dim3(THREADS), smem, stream);
-  e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK>, tx, tl, p);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK>, tx, tl, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_quantize_act launch: ") + cudaGetErrorString(e));
   return ok();

@@ -3,7 +3,9 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -87,6 +89,11 @@ SVDQ_HD size_t lowrank_offset(int m, int j, int th) {
          static_cast<size_t>((((j >> 3) ^ r) & 7) << 4) + static_cast<size_t>(j & 7) * 2u;
 }
 
+// Eigen-decomposition of the symmetric p x p matrix C (row-major, float64) by
+// cyclic Jacobi rotations: eigenvalues on C's diagonal, eigenvectors in the
+// columns of V (host; used by the host and the device packs).
+void jacobi_eigen(std::vector<double> &C, int p, std::vector<double> &V);
+
 // Per-device state filled by svdq_init.
 struct DeviceState {
   bool initialized = false;
@@ -117,6 +124,28 @@ struct DependentLaunch {
     cfg.numAttrs = 1;
   }
 };
+#endif
+
+#ifdef __CUDACC__
+// Raises a kernel's dynamic shared-memory limit to `bytes`, once per device
+// (a host call that need not be repeated on every launch).
+template <auto Kernel>
+int smem_optin_once(int bytes, const char *fn) {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return fail(SVDQ_ERR_CUDA, std::string(fn) + ": no current device");
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + ": " + cudaGetErrorString(e));
+    done[dev] = true;
+  }
+  return SVDQ_OK;
+}
 #endif
 
 // Bounded-wait limit handed to every kernel, in nanoseconds.

@@ -26,6 +26,7 @@ EPILOGUE_NONE = 0
 EPILOGUE_GELU_ERF = 1
 EPILOGUE_GELU_TANH = 2
 LR_STRIDE = 64
+AMAX_WORKSPACE_BYTES = 256
 
 _lib = None
 
@@ -43,6 +44,11 @@ _SIGNATURES = {
     "svdq_quantize_host": (_I, [_P, _I, _I, ctypes.c_float, _I, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P]),
     "svdq_linear_w4a4": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_linear_w4a4_requant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I,
+                                      _P, _P, _I, _P, _P, _P, _P, _P, _P]),
+    "svdq_requant_workspace_size": (_I, [_I, _I, _SZ]),
+    "svdq_act_amax": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
+    "awq_packed_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ]),
     "awq_pack_weights": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "awq_linear_w4a16": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P]),
     "svdq_check_status": (_I, [_P]),
@@ -240,6 +246,72 @@ def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, 
         _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
         _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue, gelu_col_begin,
         _dptr(Y, "Y", torch.bfloat16), Y.stride(0), _stream(stream)))
+
+
+def svdq_act_amax(X, inv_lambda, workspace, s_a, M=None, K=None, stream=None):
+    """Enqueues the dynamic activation-scale pass: s_a (f32 CUDA, 1 element) = f32(max |X^|) / 2688."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    _need_2d(X, M, K, "X")
+    _need_bytes(inv_lambda, 4 * K, "inv_lambda")
+    _need_bytes(workspace, AMAX_WORKSPACE_BYTES, "workspace")
+    _need_bytes(s_a, 4, "s_a")
+    _check("svdq_act_amax", load().svdq_act_amax(
+        _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_lambda, "inv_lambda", torch.float32),
+        _dptr(workspace, "workspace"), _dptr(s_a, "s_a", torch.float32), _stream(stream)))
+
+
+def awq_packed_sizes(K, N, group=64):
+    s = [ctypes.c_size_t() for _ in range(4)]
+    _check("awq_packed_sizes", load().awq_packed_sizes(K, N, group, *[ctypes.byref(x) for x in s]))
+    return dict(zip(("qweight", "scales", "zeros", "inv_awq"), (x.value for x in s)))
+
+
+def svdq_requant_workspace_size(M, next_rank):
+    n = ctypes.c_size_t()
+    _check("svdq_requant_workspace_size", load().svdq_requant_workspace_size(M, next_rank, ctypes.byref(n)))
+    return n.value
+
+
+def svdq_linear_w4a4_requant(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue, gelu_col_begin,
+                             Y, next_inv_lambda, next_l1t, next_rank, next_s_a, next_s_w, next_a_bundle, next_U,
+                             workspace, stream=None):
+    """Enqueues the W4A4 GEMM that re-quantizes its output for the next SVDQ layer (K_next = N).
+    Y: bf16 CUDA [M, ldy] or None (no bf16 output)."""
+    import torch
+    asz = svdq_act_sizes(M, K)
+    wsz = svdq_weight_sizes(K, N, rank)
+    nsz = svdq_act_sizes(M, N)
+    _need_bytes(a_bundle, asz["a_bundle"], "a_bundle")
+    _need_bytes(w_bundle, wsz["w_bundle"], "w_bundle")
+    if rank:
+        _need_bytes(U, asz["u"], "U")
+        _need_bytes(l2t, wsz["l2t"], "l2t")
+    _need_bytes(bias, 2 * N, "bias")
+    _need_bytes(s_a, 4, "s_a")
+    _need_bytes(s_w, 4, "s_w")
+    if Y is not None:
+        _need_2d(Y, M, N, "Y")
+    _need_bytes(next_inv_lambda, 4 * N, "next_inv_lambda")
+    _need_bytes(next_s_a, 4, "next_s_a")
+    _need_bytes(next_s_w, 4, "next_s_w")
+    _need_bytes(next_a_bundle, nsz["a_bundle"], "next_a_bundle")
+    if next_rank:
+        _need_bytes(next_l1t, 2 * next_rank * N, "next_l1t")
+        _need_bytes(next_U, nsz["u"], "next_U")
+        _need_bytes(workspace, svdq_requant_workspace_size(M, next_rank), "workspace")
+    _check("svdq_linear_w4a4_requant", load().svdq_linear_w4a4_requant(
+        _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U", allow_none=rank == 0),
+        _dptr(s_a, "s_a", torch.float32), _dptr(w_bundle, "w_bundle", torch.uint8),
+        _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
+        _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue, gelu_col_begin,
+        _dptr(Y, "Y", torch.bfloat16, allow_none=True), Y.stride(0) if Y is not None else N,
+        _dptr(next_inv_lambda, "next_inv_lambda", torch.float32),
+        _dptr(next_l1t, "next_l1t", allow_none=next_rank == 0), next_rank,
+        _dptr(next_s_a, "next_s_a", torch.float32), _dptr(next_s_w, "next_s_w", torch.float32),
+        _dptr(next_a_bundle, "next_a_bundle", torch.uint8), _dptr(next_U, "next_U", allow_none=next_rank == 0),
+        _dptr(workspace, "workspace", torch.float32, allow_none=next_rank == 0), _stream(stream)))
 
 
 def awq_pack_weights(W_bits, awq_scale, group=64):

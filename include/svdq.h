@@ -98,6 +98,7 @@ enum svdq_epilogue {
 
 #define SVDQ_LR_STRIDE 64  /* row stride (elements) of U and L2T; max rank */
 #define SVDQ_GROUP 16      /* NVFP4 block size along K */
+#define SVDQ_AMAX_WORKSPACE_BYTES 256  /* workspace of svdq_act_amax */
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int svdq_version(void);
@@ -189,6 +190,23 @@ int svdq_quantize_act(const void *X, int M, int K, int ldx, const float *inv_lam
                       uint8_t *a_bundle, void *U, svdq_stream_t stream);
 
 /*
+ * Dynamic activation scale (optional pre-pass of svdq_quantize_act).  The
+ * pages say calibration decides the quantization scales (remio.ai, section
+ * "基准测试展示了性能提升，但并非普遍结论"); svdq_pack_weights calibrates a static
+ * s_a once, this call takes it from the tensor being quantized instead:
+ *   s_a = f32(max_{m,k} |f32(x[m][k] * inv_lambda[k])|) / 2688   (1 if that max is 0)
+ * written to the device scalar *s_a, in the f32 steps svdq_quantize_act uses;
+ * pass the same scalar to svdq_quantize_act and svdq_linear_w4a4.
+ * Args: X [M][ldx] bf16, inv_lambda [K] f32, workspace: device buffer of
+ * SVDQ_AMAX_WORKSPACE_BYTES (cleared and used by the call; free again when
+ * the call's stream work is done), s_a: one f32 (device).  Enqueues a memset
+ * of the workspace and one kernel.
+ * Rules: M >= 1, K % 64 == 0, ldx >= K, ldx % 8 == 0.
+ */
+int svdq_act_amax(const void *X, int M, int K, int ldx, const float *inv_lambda, void *workspace, float *s_a,
+                  svdq_stream_t stream);
+
+/*
  * The W4A4 GEMM with the low-rank up-projection fused in (the second fused
  * kernel on the pages, remio.ai, section "SVDQuant 将棘手数值移出 4 位路径"):
  *   acc = U . L2T^T + sum_k qa sa qw sw     (tcgen05 block-scaled FP4, fp32)
@@ -207,6 +225,45 @@ int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const float *s_a,
                      int ldy, svdq_stream_t stream);
 
 /*
+ * The W4A4 GEMM of a layer whose output is the input of the next SVDQ layer
+ * (MLP fc1 -> fc2), re-quantizing its output for that layer in the same
+ * kernel.  The pages fuse the quantization of a layer's input with its
+ * low-rank down-projection (remio.ai, section "SVDQuant 将棘手数值移出 4 位路径");
+ * this call moves that fusion into the epilogue of the producing GEMM, so the
+ * 16-bit activation between the two layers is never written out and the next
+ * layer needs no svdq_quantize_act.  With y = the layer's output (after the
+ * epilogue, as svdq_linear_w4a4 computes it), for the next layer:
+ *   x^      = f32(bf16(y) * next_inv_lambda[n])          (n < N; K_next = N)
+ *   next_a_bundle, next_U = exactly what svdq_quantize_act would write for an
+ *             input X = bf16(y) with next_inv_lambda, next_l1t, next_rank,
+ *             next_s_a and next_s_w (codes and block scales bit-identical;
+ *             U's fp32 sum is formed in another order, so it may differ in
+ *             the last bit of its bf16 rounding).
+ * Args: the first fifteen as svdq_linear_w4a4, except that Y may be NULL (the
+ * bf16 output is then not written at all, ldy ignored).  next_inv_lambda [N]
+ * f32, next_l1t [next_rank][N] bf16, next_s_a / next_s_w device scalars of
+ * the next layer; next_a_bundle (128-row bundle of M x N, size from
+ * svdq_act_sizes(M, N)), next_U (128-row low-rank tiles); workspace: device
+ * buffer of svdq_requant_workspace_size(M, next_rank) bytes (fp32 partial
+ * sums), cleared and used by the call, free again when the call's stream
+ * work is done; next_l1t, next_U and workspace may be NULL when next_rank
+ * is 0.  The call enqueues a memset of the workspace, the GEMM and one small
+ * kernel that turns the sums into next_U.
+ * Rules: those of svdq_linear_w4a4, plus N % 64 == 0 and next_rank a
+ * multiple of 16 in [0, 64].
+ */
+int svdq_linear_w4a4_requant(const uint8_t *a_bundle, const void *U, const float *s_a,
+                             const uint8_t *w_bundle, const void *l2t, const float *s_w, const void *bias,
+                             int M, int N, int K, int rank, int epilogue, int gelu_col_begin, void *Y,
+                             int ldy, const float *next_inv_lambda, const void *next_l1t, int next_rank,
+                             const float *next_s_a, const float *next_s_w, uint8_t *next_a_bundle,
+                             void *next_U, float *workspace, svdq_stream_t stream);
+
+/* Bytes of the workspace svdq_linear_w4a4_requant needs: M * next_rank * 4
+ * (host, no GPU).  Rules: M >= 1, next_rank a multiple of 16 in [0, 64]. */
+int svdq_requant_workspace_size(int M, int next_rank, size_t *bytes);
+
+/*
  * Offline AWQ quantization on the host (asymmetric INT4 per group along K):
  *   W_a = diag(awq_scale) W;  per group and output column:
  *   lo = min(0, min W_a), hi = max(0, max W_a), s = bf16((hi - lo) / 15),
@@ -218,6 +275,14 @@ int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const float *s_a,
  */
 int awq_pack_weights(const uint16_t *W, int K, int N, const float *awq_scale, int group,
                      uint32_t *qweight, uint16_t *scales, uint16_t *zeros, float *inv_awq);
+
+/*
+ * Byte sizes of the packed AWQ buffers of a K x N weight (host, no GPU):
+ * qweight N*K/2, scales and zeros N*K/group*2 each, inv_awq K*4.
+ * Rules: group == 64, K % 64 == 0, N % 64 == 0.
+ */
+int awq_packed_sizes(int K, int N, int group, size_t *qweight_bytes, size_t *scales_bytes,
+                     size_t *zeros_bytes, size_t *inv_awq_bytes);
 
 /*
  * AWQ W4A16 projection for small row counts (the modulation / adaLN layers):

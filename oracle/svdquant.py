@@ -24,7 +24,8 @@ Readings where the pages are silent (each also in the design notes):
   * The activation tensor scale is static: calibrated from the per-channel
     absolute maxima of X (the pages: calibration samples decide the scales,
     section "基准测试展示了性能提升，但并非普遍结论").
-  * The low-rank branch is a 16-bit branch ("一个小型 16 位低秩分支"): its input
+  * The low-rank branch is a small 16-bit branch ([Remio], section "SVDQuant
+    将棘手数值移出 4 位路径"): its input
     is the smoothed activation rounded to bf16 (RNE of the float32 X^), its
     factors are bf16; products and sums are exact here (float64).
   * The low-rank up-projection enters the 4-bit GEMM's accumulator divided by

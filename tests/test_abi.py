@@ -64,6 +64,26 @@ def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
     assert rc == lib.ERR_SHAPE                                    # N % 64
     rc = so.awq_linear_w4a16(p, 0, 256, 256, None, p, p, p, 64, None, 256, p, 256, None)
     assert rc == lib.ERR_SHAPE                                    # M < 1
+    # the re-quantizing GEMM: N is the next layer's K (multiple of 64), next_rank in {0, 16, .., 64}
+    rc = so.svdq_linear_w4a4_requant(p, p, p, p, p, p, None, 64, 200, 256, 16, 0, 0, None, 0,
+                                     p, p, 16, p, p, p, p, p, None)
+    assert rc == lib.ERR_SHAPE
+    rc = so.svdq_linear_w4a4_requant(p, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, None, 0,
+                                     p, p, 24, p, p, p, p, p, None)
+    assert rc == lib.ERR_SHAPE
+    rc = so.svdq_linear_w4a4_requant(p, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, None, 0,
+                                     p, None, 16, p, p, p, p, p, None)
+    assert rc == lib.ERR_INVALID_ARG                              # next_l1t missing with next_rank > 0
+    assert lib.svdq_requant_workspace_size(4608, 32) == 4608 * 32 * 4
+    assert lib.svdq_requant_workspace_size(100, 0) == 0
+    rc = so.svdq_act_amax(p, 4, 96, 96, p, p, p, None)
+    assert rc == lib.ERR_SHAPE                                    # K % 64
+    rc = so.svdq_act_amax(p, 4, 128, 128, p, None, p, None)
+    assert rc == lib.ERR_INVALID_ARG                              # no workspace
+    assert lib.awq_packed_sizes(3072, 18432) == {"qweight": 3072 * 18432 // 2, "scales": 18432 * 48 * 2,
+                                                 "zeros": 18432 * 48 * 2, "inv_awq": 3072 * 4}
+    with pytest.raises(lib.SvdqError):
+        lib.awq_packed_sizes(3072, 100)
     odd = ctypes.c_void_p(24)
     rc = so.svdq_linear_w4a4(odd, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None)
     assert rc == lib.ERR_ALIGNMENT

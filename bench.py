@@ -315,25 +315,38 @@ def k3(A):
     lib.awq_linear_w4a16(A["X"], A["inv_awq"], A["qweight"], A["scales"], A["zeros"], A["bias"], AN, A["Y"])
 
 
-# the step's kernels in order: (label, function of one buffer set).  The MLP pair runs fused: fc1's
-# GEMM re-quantizes its GELU output for fc2 in its epilogue, so fc2 needs no K1 pass and the
-# 4608 x 12288 bf16 activation between the two layers never travels through memory.
-STEP_KERNELS = [
-    ("K1 qkv", lambda s: k1(s["qkv"], "qkv")), ("K2 qkv", lambda s: k2(s["qkv"], "qkv")),
-    ("K1 fc1", lambda s: k1(s["fc1"], "fc1")), ("K2 fc1 -> fc2 operands", k2_requant),
-    ("K2 fc2", lambda s: k2(s["fc2"], "fc2")),
-    ("K3 adaLN", lambda s: k3(s["awq"])),
-]
-# my kernels per step: the re-quantizing call launches the GEMM and a small finalize kernel (plus a memset)
-LAUNCHES_PER_STEP = len(STEP_KERNELS) + 1
-# the unfused MLP pair, timed alone for comparison: fc1's plain GEMM (bf16 output) and fc2's K1 on it
-UNFUSED_KERNELS = [("K2 fc1 (plain, bf16 out)", lambda s: k2(s["fc1"], "fc1")),
-                   ("K1 fc2 (on fc1's bf16 out)", lambda s: k1(s["fc2"], "fc2"))]
+# The step's kernels in order: (label, function of one buffer set).  The MLP pair runs either
+# fused - fc1's GEMM re-quantizes its GELU output for fc2 in its epilogue, so fc2 needs no K1 pass
+# and the 4608 x 12288 bf16 activation between the two layers never travels through memory - or
+# unfused (fc1's plain GEMM writes the bf16 activation, fc2's K1 reads it back); the other form is
+# timed alone for comparison.
+def step_kernels(mlp):
+    head = [("K1 qkv", lambda s: k1(s["qkv"], "qkv")), ("K2 qkv", lambda s: k2(s["qkv"], "qkv")),
+            ("K1 fc1", lambda s: k1(s["fc1"], "fc1"))]
+    tail = [("K2 fc2", lambda s: k2(s["fc2"], "fc2")), ("K3 adaLN", lambda s: k3(s["awq"]))]
+    if mlp == "fused":
+        return head + FUSED_MLP + tail
+    return head + UNFUSED_MLP + tail
 
 
-def step(sets, i):
+FUSED_MLP = [("K2 fc1 -> fc2 operands", k2_requant)]
+UNFUSED_MLP = [("K2 fc1 (plain, bf16 out)", lambda s: k2(s["fc1"], "fc1")),
+               ("K1 fc2 (on fc1's bf16 out)", lambda s: k1(s["fc2"], "fc2"))]
+MLP_DEFAULT = "unfused"   # measured faster on B200 (the fused epilogue is the longer path)
+STEP_KERNELS = step_kernels(MLP_DEFAULT)
+
+
+def launches_per_step(mlp):
+    """My kernels per step; the re-quantizing call launches the GEMM and a small finalize kernel."""
+    return len(step_kernels(mlp)) + (1 if mlp == "fused" else 0)
+
+
+LAUNCHES_PER_STEP = launches_per_step(MLP_DEFAULT)
+
+
+def step(sets, i, kernels=None):
     s = sets[i % len(sets)]
-    for _, fn in STEP_KERNELS:
+    for _, fn in (kernels or STEP_KERNELS):
         fn(s)
 
 
@@ -436,8 +449,10 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
 
+    kernels = step_kernels(args.mlp)
+    other = UNFUSED_MLP if args.mlp == "fused" else FUSED_MLP
     for i in range(args.warmup):
-        step(sets, i)
+        step(sets, i, kernels)
     rc = lib.svdq_check_status()
     if rc != lib.OK:
         raise RuntimeError(f"device status after warm-up: {lib.status_name(rc)}")
@@ -450,14 +465,14 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
     for i in range(args.steps):
-        step(sets, i)
+        step(sets, i, kernels)
     t1.record()
     barrier()
     ms = t0.elapsed_time(t1)
     # ---- each kernel alone, back to back over the rotating sets (no event between two different
     # kernels); the clock sampler keeps running under this load
-    per = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in STEP_KERNELS}
-    extra = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in UNFUSED_KERNELS}
+    per = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in kernels}
+    extra = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in other}
     clk = clocks.stop()
     rc = lib.svdq_check_status()
     if rc != lib.OK:
@@ -495,7 +510,7 @@ def run_ours(args):
         main_s.wait_event(ev_in[i])
         if i >= len(sets):
             main_s.wait_event(ev_out[i - len(sets)])       # the set's previous outputs have been read out
-        step(sets, i)
+        step(sets, i, kernels)
         ev_done[i].record(main_s)
         with torch.cuda.stream(out_s):
             out_s.wait_event(ev_done[i])
@@ -515,8 +530,8 @@ def run_ours(args):
     fp4_lib = fp4_library_point(device, *LAYERS["fc1"][:3]) if not args.no_library_points else "skipped"
 
     # ---- max over ranks
-    labels = [label for label, _ in STEP_KERNELS]
-    xlabels = [label for label, _ in UNFUSED_KERNELS]
+    labels = [label for label, _ in kernels]
+    xlabels = [label for label, _ in other]
     vals = max_over_ranks([ms, e2e_ms] + [per[x] for x in labels] + [extra[x] for x in xlabels], world, device)
     ms, e2e_ms = vals[0], vals[1]
     per = dict(zip(labels, vals[2:2 + len(labels)]))
@@ -535,13 +550,19 @@ def run_ours(args):
         rate = amount / (us * 1e-6) / (1e9 if unit == "GB/s" else 1e12)
         return {"us": round(us, 2), unit: round(rate, 1), "frac": round(rate / peak, 4)}
 
-    kernels = {label: entry(label, per[label]) for label in labels}
-    kernels["sum_us"] = round(sum(per.values()) * 1e3, 2)
-    kernels["timing"] = (f"each kernel alone, {args.kernel_reps} launches back to back over the rotating "
+    ktab = {label: entry(label, per[label]) for label in labels}
+    ktab["sum_us"] = round(sum(per.values()) * 1e3, 2)
+    ktab["timing"] = (f"each kernel alone, {args.kernel_reps} launches back to back over the rotating "
                          "sets, after the timed region")
-    kernels["unfused_mlp_for_comparison"] = {label: entry(label, extra[label]) for label in xlabels}
-    k2_us = per["K2 fc1 -> fc2 operands"] * 1e3
-    k2_tflops = requant_flops() / (k2_us * 1e-6) / 1e12
+    ktab[f"{'unfused' if args.mlp == 'fused' else 'fused'}_mlp_for_comparison"] = {
+        label: entry(label, extra[label]) for label in xlabels}
+    m, k, n, _ = LAYERS["fc1"]
+    if args.mlp == "fused":
+        k2_label, k2_flops = "K2 fc1 -> fc2 operands", requant_flops()
+    else:
+        k2_label, k2_flops = "K2 fc1 (plain, bf16 out)", gemm_flops(m, k, n)
+    k2_us = per[k2_label] * 1e3
+    k2_tflops = k2_flops / (k2_us * 1e-6) / 1e12
     traffic = K2_TRAFFIC["bytes"] if K2_TRAFFIC["source_sha16"] == source_sha16("gemm_w4a4_kernel.cuh") else None
     line = {
         "metric": METRIC,
@@ -559,18 +580,21 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2; {len(sets)} rotating sets of weights, inputs and outputs, "
                          f"{len(sets) * set_bytes / 1e6:.0f} MB > 2x L2",
-                   "flops_per_step": STEP_FLOPS, "launches_per_step": LAUNCHES_PER_STEP,
-                   "mlp": "fused: fc1's GEMM writes fc2's NVFP4 operands and U (no bf16 activation, no K1 for fc2)"},
+                   "flops_per_step": STEP_FLOPS, "launches_per_step": launches_per_step(args.mlp),
+                   "mlp": ("fused: fc1's GEMM writes fc2's NVFP4 operands and U (no bf16 activation, no K1 for fc2)"
+                           if args.mlp == "fused" else "unfused: fc1 writes its bf16 output, fc2's K1 reads it")},
         "roofline": {"bound": "tensor",
-                     "kernel": "svdq_linear_w4a4_requant, fc1 4608x3072x12288 +GELU re-quantized for fc2",
+                     "kernel": ("svdq_linear_w4a4_requant, fc1 4608x3072x12288 +GELU re-quantized for fc2"
+                                if args.mlp == "fused" else "svdq_linear_w4a4, fc1 4608x3072x12288 +GELU"),
                      "achieved": round(k2_tflops, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(k2_tflops / fp4_peak, 4), "traffic": traffic,
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{how} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16)",
                      "frac_of_nominal_9pf": round(k2_tflops / FP4_NOMINAL_TFLOPS, 4),
-                     "algorithmic": "2MKN (FP4) + 2MrN (low-rank up-projection) + 2MNr (fc2's low-rank "
-                                    "down-projection in the epilogue) per launch"},
-        "kernels": kernels,
+                     "algorithmic": ("2MKN (FP4) + 2MrN (low-rank up-projection) + 2MNr (fc2's low-rank "
+                                     "down-projection in the epilogue) per launch" if args.mlp == "fused" else
+                                     "2MKN (FP4) + 2MrN (low-rank up-projection) per launch")},
+        "kernels": ktab,
         "reference_points": {
             "hbm_copy_same_bytes": {"GB/s": round(floor_gbs, 1), "us": round(floor_us, 2),
                                     "what": f"torch copy of {TOKENS}x{HIDDEN} bf16 (cold, read + write)"},
@@ -581,7 +605,7 @@ def run_ours(args):
             "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how},
         "e2e": {"value": round(aggregate_tflops(STEP_FLOPS, world, e2e_ms), 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": launches_per_step(args.mlp) * args.steps,
         "clocks": clk,
     }
     if world == 1 and not args.no_cpu_baseline:
@@ -896,6 +920,8 @@ def main():
                     help="skip the cuBLASLt NVFP4 reference point")
     ap.add_argument("--kernel-reps", type=int, default=20,
                     help="back-to-back launches per kernel for the per-kernel times")
+    ap.add_argument("--mlp", choices=("fused", "unfused"), default=MLP_DEFAULT,
+                    help="MLP pair: fc1's GEMM re-quantizing for fc2 (fused) or fc1 bf16 out + fc2 K1 (unfused)")
     ap.add_argument("--workload", choices=("layers", "dit-step"), default="layers",
                     help="layers: QKV + MLP pair + AWQ projection (default); dit-step: one whole DiT step")
     args = ap.parse_args()

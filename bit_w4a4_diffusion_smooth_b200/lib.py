@@ -48,6 +48,9 @@ _SIGNATURES = {
                                       _P, _P, _I, _P, _P, _P, _P, _P, _P]),
     "svdq_requant_workspace_size": (_I, [_I, _I, _SZ]),
     "svdq_act_amax": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
+    "svdq_calibrate_absmax": (_I, [_P, _I, _I, _I, _P, _P]),
+    "svdq_pack_device_workspace_size": (_I, [_I, _I, _I, _SZ]),
+    "svdq_pack_weights_device": (_I, [_P, _I, _I, _P, _I, ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "awq_packed_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ]),
     "awq_pack_weights": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "awq_linear_w4a16": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P]),
@@ -260,6 +263,54 @@ def svdq_act_amax(X, inv_lambda, workspace, s_a, M=None, K=None, stream=None):
     _check("svdq_act_amax", load().svdq_act_amax(
         _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_lambda, "inv_lambda", torch.float32),
         _dptr(workspace, "workspace"), _dptr(s_a, "s_a", torch.float32), _stream(stream)))
+
+
+def svdq_calibrate_absmax(X, act_absmax, M=None, K=None, stream=None):
+    """act_absmax (f32 CUDA [K]) = max(act_absmax, max over rows of |X|) for a bf16 CUDA X [M, ldx]."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    _need_2d(X, M, K, "X")
+    _need_bytes(act_absmax, 4 * K, "act_absmax")
+    _check("svdq_calibrate_absmax", load().svdq_calibrate_absmax(
+        _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(act_absmax, "act_absmax", torch.float32),
+        _stream(stream)))
+
+
+def svdq_pack_device_workspace_size(K, N, rank):
+    n = ctypes.c_size_t()
+    _check("svdq_pack_device_workspace_size", load().svdq_pack_device_workspace_size(K, N, rank, ctypes.byref(n)))
+    return n.value
+
+
+def svdq_pack_weights_device(W, act_absmax, rank, seed=0, want_residual=False, stream=None):
+    """GPU pack of a bf16 CUDA weight W [K, N] with calibration maxima act_absmax (f32 CUDA [K]).
+
+    Returns CUDA tensors: inv_lambda [K] f32, l1t [rank, K] bf16, l2t (u8 tiles), w_bundle (u8),
+    s_w, s_a ([1] f32), and residual [K, N] f32 if asked.
+    """
+    import torch
+    K, N = W.shape
+    dev = W.device
+    sz = svdq_weight_sizes(K, N, rank)
+    out = dict(inv_lambda=torch.empty(K, dtype=torch.float32, device=dev),
+               l1t=torch.empty((rank, K), dtype=torch.bfloat16, device=dev),
+               l2t=torch.empty(sz["l2t"], dtype=torch.uint8, device=dev),
+               w_bundle=torch.empty(sz["w_bundle"], dtype=torch.uint8, device=dev),
+               s_w=torch.empty(1, dtype=torch.float32, device=dev), s_a=torch.empty(1, dtype=torch.float32, device=dev))
+    residual = torch.empty((K, N), dtype=torch.float32, device=dev) if want_residual else None
+    ws = torch.empty(svdq_pack_device_workspace_size(K, N, rank), dtype=torch.uint8, device=dev)
+    _need_2d(W, K, N, "W")
+    _need_bytes(act_absmax, 4 * K, "act_absmax")
+    _check("svdq_pack_weights_device", load().svdq_pack_weights_device(
+        _dptr(W, "W", torch.bfloat16), K, N, _dptr(act_absmax, "act_absmax", torch.float32), rank, seed,
+        _dptr(out["inv_lambda"], "inv_lambda"), _dptr(out["l1t"], "l1t") if rank else None,
+        _dptr(out["l2t"], "l2t"), _dptr(out["w_bundle"], "w_bundle"), _dptr(out["s_w"], "s_w"),
+        _dptr(out["s_a"], "s_a"), _dptr(residual, "residual", allow_none=True), _dptr(ws, "workspace"),
+        _stream(stream)))
+    if want_residual:
+        out["residual"] = residual
+    return out
 
 
 def awq_packed_sizes(K, N, group=64):

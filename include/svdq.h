@@ -164,6 +164,40 @@ int svdq_pack_weights(const uint16_t *W, int K, int N, const float *act_absmax, 
                       uint8_t *l2t, uint8_t *w_bundle, float *s_w, float *s_a, float *residual);
 
 /*
+ * Calibration on the GPU: act_absmax[k] = max(act_absmax[k], max_m |X[m][k]|)
+ * for k < K (device buffers; act_absmax accumulates over calls: zero it
+ * before the first batch).  The pages' offline quantize step derives the
+ * scales from calibration data (remio.ai, section
+ * "基准测试展示了性能提升，但并非普遍结论"); the result is svdq_pack_weights' /
+ * svdq_pack_weights_device's act_absmax.
+ * Rules: M >= 1, K % 8 == 0, ldx >= K, ldx % 8 == 0.
+ */
+int svdq_calibrate_absmax(const void *X, int M, int K, int ldx, float *act_absmax, svdq_stream_t stream);
+
+/* Bytes of the device workspace svdq_pack_weights_device needs (host, no GPU):
+ * the float64 W' [K][N] plus the subspace iteration's blocks. */
+int svdq_pack_device_workspace_size(int K, int N, int rank, size_t *bytes);
+
+/*
+ * The offline pack of svdq_pack_weights, on the GPU (donmalab.com, section
+ * "自行量化模型的流程": quantize the weights to 4 bits and produce the low-rank
+ * branch).  Same arguments and results, in device memory, except:
+ *   - the top-r subspace comes from the same randomized subspace iteration
+ *     (oversampling 48, 10 power iterations, float64) with a counter-based
+ *     random test matrix, so L1, L2 (and therefore R and its codes) differ
+ *     from the host pack's within the freedom of the SVD; inv_lambda and s_a
+ *     are identical;
+ *   - residual is NULL or [K][N] f32 (device); workspace is a device buffer
+ *     of svdq_pack_device_workspace_size bytes.
+ * The float64 products run on cuBLAS; the small p x p factorizations between
+ * them on the host, so the call synchronizes `stream` (an offline step, not
+ * the hot path).  Rules: those of svdq_pack_weights; rank <= min(K, N).
+ */
+int svdq_pack_weights_device(const void *W, int K, int N, const float *act_absmax, int rank, uint64_t seed,
+                             float *inv_lambda, void *l1t, uint8_t *l2t, uint8_t *w_bundle, float *s_w,
+                             float *s_a, float *residual, void *workspace, svdq_stream_t stream);
+
+/*
  * NVFP4 quantization of a host float32 matrix T [rows][K] (host, no GPU),
  * blocks of 16 along K under tensor scale s_t, into a bundle of tile height
  * tile_rows (128 or 256; bundle_bytes from the layout above).  Used by the

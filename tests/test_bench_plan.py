@@ -39,10 +39,14 @@ def test_layer_step_flops_and_kernels():
         return 2 * m * k * n + 2 * m * r * (k + n)
     want = layer(4608, 3072, 9216) + layer(4608, 3072, 12288) + layer(4608, 12288, 3072) + 2 * 2 * 3072 * 18432
     assert bench.STEP_FLOPS == want
-    labels = [label for label, _ in bench.STEP_KERNELS]
+    labels = [label for label, _ in bench.step_kernels("fused")]
     assert labels == ["K1 qkv", "K2 qkv", "K1 fc1", "K2 fc1 -> fc2 operands", "K2 fc2", "K3 adaLN"]
+    labels = [label for label, _ in bench.step_kernels("unfused")]
+    assert labels == ["K1 qkv", "K2 qkv", "K1 fc1", "K2 fc1 (plain, bf16 out)", "K1 fc2 (on fc1's bf16 out)",
+                      "K2 fc2", "K3 adaLN"]
     assert bench.LAYERS["fc1"] == (4608, 3072, 12288, True)
-    assert bench.LAUNCHES_PER_STEP == 7                    # the re-quantizing call also runs its finalize kernel
+    assert bench.launches_per_step("fused") == 7           # the re-quantizing call also runs its finalize kernel
+    assert bench.launches_per_step("unfused") == 7
     assert bench.requant_flops() == 2 * 4608 * 3072 * 12288 + 2 * 4608 * 32 * 12288 * 2
 
 

@@ -107,3 +107,61 @@ extern "C" int svdq_linear_w4a4_requant(const uint8_t *a_bundle, const void *U, 
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return ok();
 }
+
+// Allocation-free form of svdq_linear_w4a4_requant: the fp32 partial sums of
+// the next layer's low-rank input live in a fixed array of this library's
+// device image instead of a caller buffer.  It serves callers that can hand
+// the library only the tensors of the layer and no scratch buffer: plugins of
+// an inference engine whose interface passes inputs and outputs alone, or
+// code that must not call cudaMalloc in the middle of a pipeline (it can
+// synchronize the device) and keeps no memory pool of its own.
+constexpr size_t kStaticScratchFloats = 262144;   // 1 MiB: M * next_rank <= 262144
+static __device__ __align__(256) float g_requant_scratch[kStaticScratchFloats];
+
+namespace {
+// Device address of g_requant_scratch, looked up once per device (with that
+// device current): in host code the array's name is only a host-side stand-in.
+float *static_scratch_address(int *status_out) {
+  static std::mutex mu;
+  static float *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    *status_out = fail(SVDQ_ERR_CUDA, "svdq_linear_w4a4_requant_noalloc: no current device");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_requant_scratch);
+    if (e != cudaSuccess) {
+      *status_out = fail(SVDQ_ERR_CUDA, std::string("svdq_linear_w4a4_requant_noalloc: cudaGetSymbolAddress: ") +
+                                            cudaGetErrorString(e));
+      return nullptr;
+    }
+    addr[dev] = static_cast<float *>(p);
+  }
+  *status_out = SVDQ_OK;
+  return addr[dev];
+}
+}  // namespace
+
+extern "C" int svdq_linear_w4a4_requant_noalloc(const uint8_t *a_bundle, const void *U, const float *s_a,
+                                                const uint8_t *w_bundle, const void *l2t, const float *s_w,
+                                                const void *bias, int M, int N, int K, int rank, int epilogue,
+                                                int gelu_col_begin, void *Y, int ldy, const float *next_inv_lambda,
+                                                const void *next_l1t, int next_rank, const float *next_s_a,
+                                                const float *next_s_w, uint8_t *next_a_bundle, void *next_U,
+                                                svdq_stream_t stream) {
+  if (M < 1 || next_rank < 0 || static_cast<size_t>(M) * static_cast<size_t>(next_rank > 0 ? next_rank : 0) >
+                                    kStaticScratchFloats)
+    return fail(SVDQ_ERR_SHAPE, "svdq_linear_w4a4_requant_noalloc: M * next_rank must be at most " +
+                                    std::to_string(kStaticScratchFloats) + " (the fixed scratch array)");
+  if (current_device_state() == nullptr) return SVDQ_ERR_NOT_INITIALIZED;
+  int rc = SVDQ_OK;
+  float *scratch = static_scratch_address(&rc);
+  if (!scratch) return rc;
+  return svdq_linear_w4a4_requant(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue,
+                                  gelu_col_begin, Y, ldy, next_inv_lambda, next_l1t, next_rank, next_s_a, next_s_w,
+                                  next_a_bundle, next_U, scratch, stream);
+}

@@ -47,6 +47,8 @@ _SIGNATURES = {
     "svdq_linear_w4a4_requant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I,
                                       _P, _P, _I, _P, _P, _P, _P, _P, _P]),
     "svdq_requant_workspace_size": (_I, [_I, _I, _SZ]),
+    "svdq_linear_w4a4_requant_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I,
+                                              _P, _P, _I, _P, _P, _P, _P, _P]),
     "svdq_act_amax": (_I, [_P, _I, _I, _I, _P, _P, _P, _P]),
     "svdq_calibrate_absmax": (_I, [_P, _I, _I, _I, _P, _P]),
     "svdq_pack_device_workspace_size": (_I, [_I, _I, _I, _SZ]),
@@ -363,6 +365,41 @@ def svdq_linear_w4a4_requant(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K
         _dptr(next_s_a, "next_s_a", torch.float32), _dptr(next_s_w, "next_s_w", torch.float32),
         _dptr(next_a_bundle, "next_a_bundle", torch.uint8), _dptr(next_U, "next_U", allow_none=next_rank == 0),
         _dptr(workspace, "workspace", torch.float32, allow_none=next_rank == 0), _stream(stream)))
+
+
+def svdq_linear_w4a4_requant_noalloc(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue,
+                                     gelu_col_begin, Y, next_inv_lambda, next_l1t, next_rank, next_s_a, next_s_w,
+                                     next_a_bundle, next_U, stream=None):
+    """svdq_linear_w4a4_requant for callers that cannot allocate: the partial sums use the library's
+    fixed device array (M * next_rank <= 262144), so no workspace is passed."""
+    import torch
+    asz = svdq_act_sizes(M, K)
+    wsz = svdq_weight_sizes(K, N, rank)
+    nsz = svdq_act_sizes(M, N)
+    _need_bytes(a_bundle, asz["a_bundle"], "a_bundle")
+    _need_bytes(w_bundle, wsz["w_bundle"], "w_bundle")
+    if rank:
+        _need_bytes(U, asz["u"], "U")
+        _need_bytes(l2t, wsz["l2t"], "l2t")
+    _need_bytes(bias, 2 * N, "bias")
+    if Y is not None:
+        _need_2d(Y, M, N, "Y")
+    _need_bytes(next_inv_lambda, 4 * N, "next_inv_lambda")
+    _need_bytes(next_a_bundle, nsz["a_bundle"], "next_a_bundle")
+    if next_rank:
+        _need_bytes(next_l1t, 2 * next_rank * N, "next_l1t")
+        _need_bytes(next_U, nsz["u"], "next_U")
+    _check("svdq_linear_w4a4_requant_noalloc", load().svdq_linear_w4a4_requant_noalloc(
+        _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U", allow_none=rank == 0),
+        _dptr(s_a, "s_a", torch.float32), _dptr(w_bundle, "w_bundle", torch.uint8),
+        _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
+        _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue, gelu_col_begin,
+        _dptr(Y, "Y", torch.bfloat16, allow_none=True), Y.stride(0) if Y is not None else N,
+        _dptr(next_inv_lambda, "next_inv_lambda", torch.float32),
+        _dptr(next_l1t, "next_l1t", allow_none=next_rank == 0), next_rank,
+        _dptr(next_s_a, "next_s_a", torch.float32), _dptr(next_s_w, "next_s_w", torch.float32),
+        _dptr(next_a_bundle, "next_a_bundle", torch.uint8), _dptr(next_U, "next_U", allow_none=next_rank == 0),
+        _stream(stream)))
 
 
 def awq_pack_weights(W_bits, awq_scale, group=64):

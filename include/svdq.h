@@ -293,6 +293,32 @@ int svdq_linear_w4a4_requant(const uint8_t *a_bundle, const void *U, const float
                              const float *next_s_a, const float *next_s_w, uint8_t *next_a_bundle,
                              void *next_U, float *workspace, svdq_stream_t stream);
 
+/*
+ * svdq_linear_w4a4_requant without the workspace argument, for callers that
+ * cannot allocate device memory: a plugin of an inference engine whose
+ * interface hands over only a layer's inputs and outputs, or code that must
+ * not call cudaMalloc between kernels (the call can synchronize the device)
+ * and keeps no memory pool of its own.  No counterpart on the pages: it is an
+ * interface variant of this library, the arithmetic is that of
+ * svdq_linear_w4a4_requant.
+ * The fp32 partial sums live in one fixed array in the library's device image
+ * (1 MiB, every GPU that loads the library holds it until the process exits):
+ * M * next_rank must be at most 262144, else SVDQ_ERR_SHAPE.  Every call on a
+ * device shares that array and the call clears it first, so calls whose
+ * stream work overlaps on the GPU (other streams, other threads) race on it;
+ * serialize them.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture.  It allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ */
+int svdq_linear_w4a4_requant_noalloc(const uint8_t *a_bundle, const void *U, const float *s_a,
+                                     const uint8_t *w_bundle, const void *l2t, const float *s_w,
+                                     const void *bias, int M, int N, int K, int rank, int epilogue,
+                                     int gelu_col_begin, void *Y, int ldy, const float *next_inv_lambda,
+                                     const void *next_l1t, int next_rank, const float *next_s_a,
+                                     const float *next_s_w, uint8_t *next_a_bundle, void *next_U,
+                                     svdq_stream_t stream);
+
 /* Bytes of the workspace svdq_linear_w4a4_requant needs: M * next_rank * 4
  * (host, no GPU).  Rules: M >= 1, next_rank a multiple of 16 in [0, 64]. */
 int svdq_requant_workspace_size(int M, int next_rank, size_t *bytes);

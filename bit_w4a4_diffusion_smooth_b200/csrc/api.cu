@@ -200,7 +200,7 @@ namespace svdq {
 namespace {
 __global__ void gelu_probe_kernel(const float *in, int n, int kind, float *out) {
   int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) out[i] = kind == SVDQ_EPILOGUE_GELU_TANH ? dev::gelu_tanh(in[i]) : dev::gelu_erf(in[i]);
+  if (i < n) out[i] = kind == SVDQ_EPILOGUE_GELU_TANH ? dev::gelu_tanh(in[i]) : dev::gelu_erf2(make_float2(in[i], 0.0f)).x;
 }
 }  // namespace
 }  // namespace svdq

@@ -395,24 +395,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 }
 
 // ---------------------------------------------------------------- GELU
-// erf(x) by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
-// 7.1.26: for x >= 0, erf(x) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5)
-// exp(-x^2) with t = 1 / (1 + p x), |error| <= 1.5e-7; odd in x.  Evaluated
-// with the fast exp and division (a few 1e-7 more), it is far below the bf16
-// rounding of the GEMM output it feeds, at a third of the instructions of a
-// correctly rounded erf - the GELU epilogue runs once per output element.
-__device__ __forceinline__ float erf_as7126(float x) {
-  const float ax = fabsf(x);
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, ax, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  return copysignf(1.0f - poly * __expf(-ax * ax), x);
-}
-// GELU, erf form: y * Phi(y) = 0.5 y (1 + erf(y / sqrt 2)).
-__device__ __forceinline__ float gelu_erf(float y) { return 0.5f * y * (1.0f + erf_as7126(y * 0.70710678118654752f)); }
 // GELU, tanh form: 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))).
 __device__ __forceinline__ float gelu_tanh(float y) {
   return 0.5f * y * (1.0f + tanhf(0.79788456080286536f * (y + 0.044715f * y * y * y)));
@@ -464,5 +446,41 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
                 : __uint2float_rn(8u + m) * __uint_as_float((e + 117u) << 23);
 }
 
+// Two IEEE single-precision fused multiply-adds, each rounded on its own
+// (one packed f32x2 instruction).
+__device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t *>(&a)), "l"(*reinterpret_cast<const uint64_t *>(&b)),
+        "l"(*reinterpret_cast<const uint64_t *>(&c)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+// GELU, erf form, of two values at once: y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)).
+// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
+// 7.1.26: for x >= 0, 1 - erf(x) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5)
+// exp(-x^2) = q with t = 1 / (1 + p x), |error| <= 1.5e-7; erf is odd, so
+// 1 + erf(x) = 2 - q(|x|) for x >= 0 and q(|x|) for x < 0 - taken directly, with
+// no cancellation, so GELU of a negative input keeps its (tiny) negative value.
+// Evaluated with the fast exp and reciprocal (a few 1e-7 more), it is far below
+// the bf16 rounding of the GEMM output it feeds, at a third of the instructions
+// of a correctly rounded erf; the multiply-adds run on f32x2 instructions, two
+// elements per issue slot - the GELU epilogue runs once per output element.
+__device__ __forceinline__ float2 gelu_erf2(float2 y) {
+  const float2 x = mul2_rn(y, make_float2(0.70710678118654752f, 0.70710678118654752f));
+  const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
+  const float2 den = fma2_rn(make_float2(0.3275911f, 0.3275911f), ax, make_float2(1.0f, 1.0f));
+  const float2 t = make_float2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
+  float2 poly = fma2_rn(make_float2(1.061405429f, 1.061405429f), t, make_float2(-1.453152027f, -1.453152027f));
+  poly = fma2_rn(poly, t, make_float2(1.421413741f, 1.421413741f));
+  poly = fma2_rn(poly, t, make_float2(-0.284496736f, -0.284496736f));
+  poly = fma2_rn(poly, t, make_float2(0.254829592f, 0.254829592f));
+  poly = mul2_rn(poly, t);
+  const float2 xx = mul2_rn(ax, ax);
+  const float2 q = mul2_rn(poly, make_float2(__expf(-xx.x), __expf(-xx.y)));   // 1 - erf(|x|)
+  const float2 two_minus_q = fma2_rn(make_float2(-1.0f, -1.0f), q, make_float2(2.0f, 2.0f));
+  const float2 one_plus_erf = make_float2(x.x >= 0.0f ? two_minus_q.x : q.x, x.y >= 0.0f ? two_minus_q.y : q.y);
+  return mul2_rn(mul2_rn(y, make_float2(0.5f, 0.5f)), one_plus_erf);
+}
 }  // namespace dev
 }  // namespace svdq

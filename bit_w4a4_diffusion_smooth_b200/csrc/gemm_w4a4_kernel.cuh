@@ -413,8 +413,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            float y0 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j]), b[2 * j]);
-            float y1 = __fmaf_rn(alpha, __uint_as_float(v[c][8 * g + 2 * j + 1]), b[2 * j + 1]);
+            const float2 yy = dev::fma2_rn(make_float2(alpha, alpha),
+                                           make_float2(__uint_as_float(v[c][8 * g + 2 * j]),
+                                                       __uint_as_float(v[c][8 * g + 2 * j + 1])),
+                                           make_float2(b[2 * j], b[2 * j + 1]));
+            float y0 = yy.x, y1 = yy.y;
             if constexpr (EPI != SVDQ_EPILOGUE_NONE) {
               // computed for every column and selected: straight-line code lets the
               // independent GELU chains of a chunk interleave (a branch per element
@@ -422,8 +425,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
               const bool act0 = col + 2 * j >= p.gelu_col_begin, act1 = col + 2 * j + 1 >= p.gelu_col_begin;
               float g0, g1;
               if constexpr (EPI == SVDQ_EPILOGUE_GELU_ERF) {
-                g0 = dev::gelu_erf(y0);
-                g1 = dev::gelu_erf(y1);
+                const float2 gg = dev::gelu_erf2(yy);
+                g0 = gg.x;
+                g1 = gg.y;
               } else {
                 g0 = dev::gelu_tanh(y0);
                 g1 = dev::gelu_tanh(y1);

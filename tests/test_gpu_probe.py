@@ -109,6 +109,12 @@ def test_gelu_erf_matches_definition():
     err = np.abs(got - want)
     assert np.all(err <= 1e-6 * np.abs(xd) + 1e-30), float(np.max(err / (np.abs(xd) + 1e-30)))
     assert got[x == 30.0][0] == 30.0 and got[x == -30.0][0] == 0.0
+    # GELU of a negative input is negative: the sign survives down to the smallest results (it
+    # decides the sign of a zero e2m1 code when the output is re-quantized), and results the
+    # format can hold are not flushed to zero
+    neg = x < 0
+    assert np.signbit(got[neg]).all()
+    assert (got[(x < -1.0) & (x > -12.0)] < 0).all()
 
 
 def test_gelu_tanh_matches_definition():

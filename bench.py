@@ -370,31 +370,45 @@ def kernel_table(pk):
     return t
 
 
-def time_back_to_back(fn, sets, reps):
-    """Mean device time (ms) of `fn` launched `reps` times in a row over the rotating sets."""
+class L2Flush:
+    """Writes a buffer of twice the L2 size, so that the next kernel finds none of its data in L2."""
+
+    def __init__(self, device):
+        import torch
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        self.buf = torch.empty(2 * l2 // 4, dtype=torch.int32, device=device)
+
+    def __call__(self):
+        self.buf.fill_(0)
+
+
+def time_cold(fn, sets, reps, flush):
+    """Mean device time (ms) of one launch of `fn` with L2 flushed before it: each launch sits alone
+    between two events on the stream, after a write of twice the L2 size."""
     import torch
     for i in range(2):
         fn(sets[i % len(sets)])
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
     for i in range(reps):
+        flush()
+        ev[i][0].record()
         fn(sets[i % len(sets)])
-    e1.record()
+        ev[i][1].record()
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps
+    return sum(a.elapsed_time(b) for a, b in ev) / reps
 
 
-def copy_floor(device, nbytes, pairs=8, reps=24):
-    """A library copy of `nbytes` (torch, device to device) from cold buffers: the HBM rate a plain
-    stream of this size reaches on this GPU, as (GB/s counting read + write, us per copy)."""
+def copy_floor(device, nbytes, reps=24):
+    """A library copy of `nbytes` (torch, device to device) with L2 flushed before it, timed like the
+    kernels: the HBM rate a plain stream of this size reaches on this GPU, as (GB/s counting read +
+    write, us per copy)."""
     import torch
     n = nbytes // 2
-    src = [torch.empty(n, dtype=torch.bfloat16, device=device).fill_(1.0) for _ in range(pairs)]
-    dst = [torch.empty(n, dtype=torch.bfloat16, device=device) for _ in range(pairs)]
-    bufs = list(zip(src, dst))
-    ms = time_back_to_back(lambda b: b[1].copy_(b[0]), bufs, reps)
-    del src, dst, bufs
+    src = torch.empty(n, dtype=torch.bfloat16, device=device).fill_(1.0)
+    dst = torch.empty(n, dtype=torch.bfloat16, device=device)
+    flush = L2Flush(device)
+    ms = time_cold(lambda b: b[1].copy_(b[0]), [(src, dst)], reps, flush)
+    del src, dst, flush
     return 2 * nbytes / (ms * 1e-3) / 1e9, ms * 1e3
 
 
@@ -406,7 +420,7 @@ def fp4_library_point(device, m, k, n, reps=20):
     try:
         fp4 = torch.float4_e2m1fn_x2
         sets = []
-        for i in range(6):          # > L2 in total
+        for i in range(2):
             a = (torch.randint(0, 256, (m, k // 2), dtype=torch.uint8, device=device) & 0x77).view(fp4)
             b = (torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=device) & 0x77).view(fp4)
             rm, rn, rk = (m + 127) // 128 * 128, (n + 127) // 128 * 128, (k // 16 + 3) // 4 * 4
@@ -421,7 +435,8 @@ def fp4_library_point(device, m, k, n, reps=20):
         torch.cuda.synchronize()
         if tuple(y.shape) != (m, n):
             return f"unexpected output shape {tuple(y.shape)}"
-        ms = time_back_to_back(run, sets, reps)
+        flush = L2Flush(device)
+        ms = time_cold(run, sets, reps, flush)
         return 2 * m * k * n / (ms * 1e-3) / 1e12, ms * 1e3
     except Exception as e:  # noqa: BLE001 - a reference point only: record why it is missing
         return f"{type(e).__name__}: {str(e).splitlines()[0][:200]}"
@@ -471,8 +486,10 @@ def run_ours(args):
     ms = t0.elapsed_time(t1)
     # ---- each kernel alone, back to back over the rotating sets (no event between two different
     # kernels); the clock sampler keeps running under this load
-    per = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in kernels}
-    extra = {label: time_back_to_back(fn, sets, args.kernel_reps) for label, fn in other}
+    flush = L2Flush(device)
+    per = {label: time_cold(fn, sets, args.kernel_reps, flush) for label, fn in kernels}
+    extra = {label: time_cold(fn, sets, args.kernel_reps, flush) for label, fn in other}
+    del flush
     clk = clocks.stop()
     rc = lib.svdq_check_status()
     if rc != lib.OK:
@@ -552,8 +569,10 @@ def run_ours(args):
 
     ktab = {label: entry(label, per[label]) for label in labels}
     ktab["sum_us"] = round(sum(per.values()) * 1e3, 2)
-    ktab["timing"] = (f"each kernel alone, {args.kernel_reps} launches back to back over the rotating "
-                         "sets, after the timed region")
+    ktab["timing"] = (f"each kernel alone, mean of {args.kernel_reps} launches, each after an L2 flush (a write "
+                      "of twice the L2 size) and between its own two events, after the timed region; the "
+                      "step's kernels run back to back, so their sum exceeds ms_per_step by the launch "
+                      "overlap and the events")
     ktab[f"{'unfused' if args.mlp == 'fused' else 'fused'}_mlp_for_comparison"] = {
         label: entry(label, extra[label]) for label in xlabels}
     m, k, n, _ = LAYERS["fc1"]
@@ -597,10 +616,12 @@ def run_ours(args):
         "kernels": ktab,
         "reference_points": {
             "hbm_copy_same_bytes": {"GB/s": round(floor_gbs, 1), "us": round(floor_us, 2),
-                                    "what": f"torch copy of {TOKENS}x{HIDDEN} bf16 (cold, read + write)"},
+                                    "what": f"torch copy of {TOKENS}x{HIDDEN} bf16, timed like the kernels "
+                                            "(L2 flushed first; read + write)"},
             "cublaslt_nvfp4_fc1_shape": (
                 {"TFLOP/s": round(fp4_lib[0], 1), "us": round(fp4_lib[1], 2),
-                 "what": "torch._scaled_mm, NVFP4 A/B, block-16 e4m3 scales, bf16 out, no low-rank branch"}
+                 "what": "torch._scaled_mm, NVFP4 A/B, block-16 e4m3 scales, bf16 out, no low-rank branch; timed "
+                        "like the kernels (L2 flushed first)"}
                 if isinstance(fp4_lib, tuple) else {"unavailable": fp4_lib}),
             "hbm_peak_gbs": pk["hbm_gbs"], "peak_source": how},
         "e2e": {"value": round(aggregate_tflops(STEP_FLOPS, world, e2e_ms), 3), "unit": "TFLOP/s",

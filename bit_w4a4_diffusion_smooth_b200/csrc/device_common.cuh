@@ -456,28 +456,43 @@ __device__ __forceinline__ float2 fma2_rn(float2 a, float2 b, float2 c) {
         "l"(*reinterpret_cast<const uint64_t *>(&c)));
   return *reinterpret_cast<float2 *>(&d);
 }
+// Hardware approximations of 2^x and 1/x (one special-function-unit
+// instruction each; subnormal inputs and results flush to zero).
+__device__ __forceinline__ float ex2_approx_ftz(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx_ftz(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 // GELU, erf form, of two values at once: y Phi(y) = 0.5 y (1 + erf(y / sqrt 2)).
 // erf by Abramowitz & Stegun, Handbook of Mathematical Functions, formula
 // 7.1.26: for x >= 0, 1 - erf(x) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5)
 // exp(-x^2) = q with t = 1 / (1 + p x), |error| <= 1.5e-7; erf is odd, so
 // 1 + erf(x) = 2 - q(|x|) for x >= 0 and q(|x|) for x < 0 - taken directly, with
 // no cancellation, so GELU of a negative input keeps its (tiny) negative value.
-// Evaluated with the fast exp and reciprocal (a few 1e-7 more), it is far below
-// the bf16 rounding of the GEMM output it feeds, at a third of the instructions
-// of a correctly rounded erf; the multiply-adds run on f32x2 instructions, two
-// elements per issue slot - the GELU epilogue runs once per output element.
+// exp(-x^2) = 2^(-x^2 log2 e) and t come from the hardware approximations (a
+// few 1e-7 more; exp(-x^2) flushes to zero only for |y| > 13.2, where GELU is
+// below 1e-38), far below the bf16 rounding of the GEMM output it feeds, at a
+// third of the instructions of a correctly rounded erf; the multiply-adds run
+// on f32x2 instructions, two elements per issue slot - the GELU epilogue runs
+// once per output element.
 __device__ __forceinline__ float2 gelu_erf2(float2 y) {
   const float2 x = mul2_rn(y, make_float2(0.70710678118654752f, 0.70710678118654752f));
   const float2 ax = make_float2(fabsf(x.x), fabsf(x.y));
   const float2 den = fma2_rn(make_float2(0.3275911f, 0.3275911f), ax, make_float2(1.0f, 1.0f));
-  const float2 t = make_float2(__fdividef(1.0f, den.x), __fdividef(1.0f, den.y));
+  const float2 t = make_float2(rcp_approx_ftz(den.x), rcp_approx_ftz(den.y));
   float2 poly = fma2_rn(make_float2(1.061405429f, 1.061405429f), t, make_float2(-1.453152027f, -1.453152027f));
   poly = fma2_rn(poly, t, make_float2(1.421413741f, 1.421413741f));
   poly = fma2_rn(poly, t, make_float2(-0.284496736f, -0.284496736f));
   poly = fma2_rn(poly, t, make_float2(0.254829592f, 0.254829592f));
   poly = mul2_rn(poly, t);
-  const float2 xx = mul2_rn(ax, ax);
-  const float2 q = mul2_rn(poly, make_float2(__expf(-xx.x), __expf(-xx.y)));   // 1 - erf(|x|)
+  // -x^2 log2(e)
+  const float2 e2 = mul2_rn(ax, mul2_rn(ax, make_float2(-1.4426950408889634f, -1.4426950408889634f)));
+  const float2 q = mul2_rn(poly, make_float2(ex2_approx_ftz(e2.x), ex2_approx_ftz(e2.y)));   // 1 - erf(|x|)
   const float2 two_minus_q = fma2_rn(make_float2(-1.0f, -1.0f), q, make_float2(2.0f, 2.0f));
   const float2 one_plus_erf = make_float2(x.x >= 0.0f ? two_minus_q.x : q.x, x.y >= 0.0f ? two_minus_q.y : q.y);
   return mul2_rn(mul2_rn(y, make_float2(0.5f, 0.5f)), one_plus_erf);

@@ -85,7 +85,7 @@ K3_BYTES = (AN * AK // 2 + 2 * AN * (AK // 64) * 2      # qweight, scales + zero
             + AM * AK * 2 + AK * 4 + AN * 2 + AM * AN * 2)
 
 # DRAM traffic of one fc1-shaped K2 launch (dram__bytes_read.sum + dram__bytes_write.sum) from the
-# ncu capture summarised in profiles/, and the hash of the GEMM source it was taken on: when the
+# ncu capture summarised in profiles/, and the hash of the GEMM sources it was taken on: when the
 # source has changed since, the counters no longer describe the kernel and `traffic` is null.
 K2_TRAFFIC = {"bytes": None, "source_sha16": None}
 
@@ -99,10 +99,16 @@ def peaks():
         return PEAKS_FALLBACK, "fallback"
 
 
-def source_sha16(name):
-    path = os.path.join(ROOT, "bit_w4a4_diffusion_smooth_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+K2_SOURCES = ("gemm_w4a4_kernel.cuh", "device_common.cuh", "svdq_internal.h")
+
+
+def source_sha16(names=K2_SOURCES):
+    """Hash of the sources a kernel is compiled from (the GEMM's by default)."""
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(ROOT, "bit_w4a4_diffusion_smooth_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def dist_env():
@@ -371,20 +377,24 @@ def kernel_table(pk):
 
 
 class L2Flush:
-    """Writes a buffer of twice the L2 size, so that the next kernel finds none of its data in L2."""
+    """Reads a buffer of twice the L2 size, so that the next kernel finds none of its data in L2.  A read
+    leaves the cache clean: a flush by writing would leave ~L2-size of dirty lines for the timed kernel
+    to write back."""
 
     def __init__(self, device):
         import torch
         l2 = torch.cuda.get_device_properties(device).L2_cache_size
-        self.buf = torch.empty(2 * l2 // 4, dtype=torch.int32, device=device)
+        self.buf = torch.zeros(2 * l2 // 4, dtype=torch.int32, device=device)
+        self.out = torch.zeros((), dtype=torch.int64, device=device)
 
     def __call__(self):
-        self.buf.fill_(0)
+        import torch
+        torch.sum(self.buf, dim=0, dtype=torch.int64, out=self.out)
 
 
 def time_cold(fn, sets, reps, flush):
     """Mean device time (ms) of one launch of `fn` with L2 flushed before it: each launch sits alone
-    between two events on the stream, after a write of twice the L2 size."""
+    between two events on the stream, after a read of twice the L2 size."""
     import torch
     for i in range(2):
         fn(sets[i % len(sets)])
@@ -484,8 +494,24 @@ def run_ours(args):
     t1.record()
     barrier()
     ms = t0.elapsed_time(t1)
-    # ---- each kernel alone, back to back over the rotating sets (no event between two different
-    # kernels); the clock sampler keeps running under this load
+    # ---- the same steps again with an event after every kernel: each kernel's mean duration inside
+    # the running step, on the launching stream.  An event between two kernels costs their launch
+    # overlap, so this pass is slower than the region above; it gives the per-kernel split and the
+    # roofline, not the headline.  The first steps after the barrier are left out (the queue is
+    # still filling).
+    skip, nb = 3, max(1, min(args.steps, 100))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)] for _ in range(skip + nb)]
+    barrier()
+    for i in range(skip + nb):
+        s = sets[i % len(sets)]
+        evs[i][0].record()
+        for j, (_, fn) in enumerate(kernels):
+            fn(s)
+            evs[i][j + 1].record()
+    barrier()
+    live = {label: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(skip, skip + nb)) / nb
+            for j, (label, _) in enumerate(kernels)}
+    # ---- each kernel alone after an L2 flush; the clock sampler keeps running under this load
     flush = L2Flush(device)
     per = {label: time_cold(fn, sets, args.kernel_reps, flush) for label, fn in kernels}
     extra = {label: time_cold(fn, sets, args.kernel_reps, flush) for label, fn in other}
@@ -549,10 +575,12 @@ def run_ours(args):
     # ---- max over ranks
     labels = [label for label, _ in kernels]
     xlabels = [label for label, _ in other]
-    vals = max_over_ranks([ms, e2e_ms] + [per[x] for x in labels] + [extra[x] for x in xlabels], world, device)
+    vals = max_over_ranks([ms, e2e_ms] + [per[x] for x in labels] + [extra[x] for x in xlabels]
+                          + [live[x] for x in labels], world, device)
     ms, e2e_ms = vals[0], vals[1]
     per = dict(zip(labels, vals[2:2 + len(labels)]))
-    extra = dict(zip(xlabels, vals[2 + len(labels):]))
+    extra = dict(zip(xlabels, vals[2 + len(labels):2 + len(labels) + len(xlabels)]))
+    live = dict(zip(labels, vals[2 + len(labels) + len(xlabels):]))
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -561,28 +589,32 @@ def run_ours(args):
     fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
     ms_step = ms / args.steps
     table = kernel_table(pk)
-    def entry(label, ms_):
+    def entry(label, ms_, cold_ms=None):
         amount, unit, bound, peak = table[label]
         us = ms_ * 1e3
         rate = amount / (us * 1e-6) / (1e9 if unit == "GB/s" else 1e12)
-        return {"us": round(us, 2), unit: round(rate, 1), "frac": round(rate / peak, 4)}
+        e = {"us": round(us, 2), unit: round(rate, 1), "frac": round(rate / peak, 4)}
+        if cold_ms is not None:
+            cold_rate = amount / (cold_ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+            e.update({"cold_us": round(cold_ms * 1e3, 2), "cold_frac": round(cold_rate / peak, 4)})
+        return e
 
-    ktab = {label: entry(label, per[label]) for label in labels}
-    ktab["sum_us"] = round(sum(per.values()) * 1e3, 2)
-    ktab["timing"] = (f"each kernel alone, mean of {args.kernel_reps} launches, each after an L2 flush (a write "
-                      "of twice the L2 size) and between its own two events, after the timed region; the "
-                      "step's kernels run back to back, so their sum exceeds ms_per_step by the launch "
-                      "overlap and the events")
-    ktab[f"{'unfused' if args.mlp == 'fused' else 'fused'}_mlp_for_comparison"] = {
-        label: entry(label, extra[label]) for label in xlabels}
+    ktab = {label: entry(label, live[label], per[label]) for label in labels}
+    ktab["sum_us"] = round(sum(live.values()) * 1e3, 2)
+    ktab["timing"] = (f"us/frac: mean over {nb} steps of the step's own launches, an event after every kernel "
+                      "on the launching stream (those events cost the launch overlap, so sum_us exceeds "
+                      f"ms_per_step); cold_us/cold_frac: each kernel alone, mean of {args.kernel_reps} launches, "
+                      "each after an L2 flush (a read of twice the L2 size) and between its own two events")
+    ktab[f"{'unfused' if args.mlp == 'fused' else 'fused'}_mlp_for_comparison"] = dict(
+        {label: entry(label, extra[label]) for label in xlabels}, timing="alone after an L2 flush, like cold_us")
     m, k, n, _ = LAYERS["fc1"]
     if args.mlp == "fused":
         k2_label, k2_flops = "K2 fc1 -> fc2 operands", requant_flops()
     else:
         k2_label, k2_flops = "K2 fc1 (plain, bf16 out)", gemm_flops(m, k, n)
-    k2_us = per[k2_label] * 1e3
+    k2_us = live[k2_label] * 1e3
     k2_tflops = k2_flops / (k2_us * 1e-6) / 1e12
-    traffic = K2_TRAFFIC["bytes"] if K2_TRAFFIC["source_sha16"] == source_sha16("gemm_w4a4_kernel.cuh") else None
+    traffic = K2_TRAFFIC["bytes"] if K2_TRAFFIC["source_sha16"] == source_sha16() else None
     line = {
         "metric": METRIC,
         "value": round(aggregate_tflops(STEP_FLOPS, world, ms_step), 2),
@@ -610,6 +642,7 @@ def run_ours(args):
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{how} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/bf16)",
                      "frac_of_nominal_9pf": round(k2_tflops / FP4_NOMINAL_TFLOPS, 4),
+                     "duration": "mean in-step duration of the launch (the kernels table's us)",
                      "algorithmic": ("2MKN (FP4) + 2MrN (low-rank up-projection) + 2MNr (fc2's low-rank "
                                      "down-projection in the epilogue) per launch" if args.mlp == "fused" else
                                      "2MKN (FP4) + 2MrN (low-rank up-projection) per launch")},

@@ -777,8 +777,8 @@ def dit_step_plan():
     for _ in range(d.dual_blocks):
         for stream in ("img", "txt"):
             plan.append(("awq", f"dual.{stream}.adaln", 2, d.hidden, 6 * d.hidden, None))
-        for stream in ("img", "txt"):
-            for name in ("qkv", "out", "fc1", "fc2"):
+        for name in ("qkv", "out", "fc1", "fc2"):   # each projection on both streams (fc2 after fc1)
+            for stream in ("img", "txt"):
                 m, k, n, gelu, gbeg = by_name[f"dual.{stream}.{name}"]
                 plan.append(("w4a4", f"dual.{stream}.{name}", m, k, n, gbeg if gelu else None))
     for _ in range(d.single_blocks):
@@ -855,16 +855,40 @@ def run_dit_step(args):
         if L["name"].endswith(".fc1"):
             prev_fc1[L["name"].rsplit(".", 1)[0]] = L["Y"]
 
-    def step():
-        for L in layers:
-            if L["kind"] == "awq":
-                lib.awq_linear_w4a16(L["X"], L["inv"], L["qw"], L["sc"], L["z"], L["b"], L["n"], L["Y"])
-                continue
+    # launch units: with --group-streams on, the image and text instances of a dual-stream block's
+    # projection run as one grouped K1 and one grouped K2 launch (adjacent in the plan)
+    units = []
+    for L in layers:
+        prev = units[-1] if units else None
+        if (args.group_streams == "on" and L["kind"] == "w4a4" and L["name"].startswith("dual.txt.") and prev
+                and prev[0]["kind"] == "w4a4" and prev[0]["name"] == L["name"].replace(".txt.", ".img.")):
+            prev.append(L)
+        else:
+            units.append([L])
+
+    def run_unit(unit):
+        L = unit[0]
+        if L["kind"] == "awq":
+            lib.awq_linear_w4a16(L["X"], L["inv"], L["qw"], L["sc"], L["z"], L["b"], L["n"], L["Y"])
+            return
+        epi = lib.EPILOGUE_GELU_ERF if L["gbeg"] is not None else lib.EPILOGUE_NONE
+        if len(unit) == 1:
             ab, U = act[(L["m"], L["k"])]
             lib.svdq_quantize_act(L["X"], L["inv"], L["l1t"], r, one_t, s_w, ab, U)
-            epi = lib.EPILOGUE_GELU_ERF if L["gbeg"] is not None else lib.EPILOGUE_NONE
             lib.svdq_linear_w4a4(ab, U, one_t, L["w"], L["l2t"], s_w, L["b"], L["m"], L["n"], L["k"], r, epi,
                                  L["gbeg"] or 0, L["Y"])
+            return
+        lib.svdq_quantize_act_grouped(
+            [dict(X=u["X"], inv_lambda=u["inv"], l1t=u["l1t"], s_a=one_t, s_w=s_w, a_bundle=act[(u["m"], u["k"])][0],
+                  U=act[(u["m"], u["k"])][1]) for u in unit], r)
+        lib.svdq_linear_w4a4_grouped(
+            [dict(a_bundle=act[(u["m"], u["k"])][0], U=act[(u["m"], u["k"])][1], s_a=one_t, w_bundle=u["w"],
+                  l2t=u["l2t"], s_w=s_w, bias=u["b"], M=u["m"], N=u["n"], K=u["k"], gelu_col_begin=u["gbeg"] or 0,
+                  Y=u["Y"]) for u in unit], r, epi)
+
+    def step():
+        for unit in units:
+            run_unit(unit)
 
     for _ in range(args.warmup):
         step()
@@ -954,9 +978,12 @@ def run_dit_step(args):
                                "3072->21504 with GELU on the last 12288 columns, 15360->3072), rank 32; "
                                "adaLN AWQ 2x3072->18432 (x38) and 2x3072->9216 (x38)",
                    "parallelism": f"replicas x{world}", "graph": "one CUDA graph per step",
+                   "group_streams": (f"{args.group_streams}: a dual-stream block's image and text instances of "
+                                     "each projection run as one grouped K1 and one grouped K2 launch"
+                                     if args.group_streams == "on" else "off: every layer its own launches"),
                    "layers": {"w4a4": n_w4a4, "awq": n_awq}, "flops_per_step": flops},
         "breakdown": breakdown,
-        "gpu_launches": args.steps * (2 * n_w4a4 + n_awq),
+        "gpu_launches": args.steps * sum(1 if u[0]["kind"] == "awq" else 2 for u in units),
         "clocks": clk,
     }))
 
@@ -978,6 +1005,8 @@ def main():
                     help="MLP pair: fc1's GEMM re-quantizing for fc2 (fused) or fc1 bf16 out + fc2 K1 (unfused)")
     ap.add_argument("--workload", choices=("layers", "dit-step"), default="layers",
                     help="layers: QKV + MLP pair + AWQ projection (default); dit-step: one whole DiT step")
+    ap.add_argument("--group-streams", choices=("on", "off"), default="on",
+                    help="dit-step: image and text instances of a dual-stream projection as one grouped launch")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {"reference": 10}.get(args.impl, 300 if args.workload == "layers" else 200)

@@ -125,6 +125,32 @@ struct Maps {
   CUtensorMap a, sfa, b, sfb, u, l2, y;
 };
 
+// One launch computes up to kMaxGroup independent GEMMs of the same epilogue
+// kind (a grouped launch): their tiles form one sequence, problem after
+// problem, which the persistent SM pairs split into contiguous runs.  A
+// single GEMM is a group of one.
+constexpr int kMaxGroup = SVDQ_MAX_GROUP;
+struct Group {
+  Maps maps[kMaxGroup];
+  Params p[kMaxGroup];
+  int tile_end[kMaxGroup];      // prefix sums of the problems' tile counts
+  int count;
+  int total_tiles;
+  unsigned int *status;
+  unsigned long long limit_ns;
+};
+
+// Problem `pi` of tile `tile` of the group's sequence, and the tile's index inside it.
+struct TileRef {
+  int pi, m2, n_blk;            // problem, 256-row pair block, 256-column block
+};
+__device__ __forceinline__ TileRef locate_tile(const Group &g, int tile) {
+  int pi = 0;
+  while (pi + 1 < g.count && tile >= g.tile_end[pi]) ++pi;
+  const int lt = tile - (pi > 0 ? g.tile_end[pi - 1] : 0);
+  return TileRef{pi, lt / g.p[pi].num_n, lt % g.p[pi].num_n};
+}
+
 
 // Raises the abort flag of this CTA and of its partner, records the timeout.
 __device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t peer_abort, unsigned int *status) {
@@ -153,7 +179,7 @@ __device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t pe
 // sums into the next layer's U once every column block is done).
 template <int EPI, int RQ>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    gemm_w4a4_kernel(const __grid_constant__ Maps maps, Params p) {
+    gemm_w4a4_kernel(const __grid_constant__ Group grp) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);  // even CTA: both CTAs' bytes
@@ -172,9 +198,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const int pair = static_cast<int>(dev::cluster_id_x());
   const int num_pairs = static_cast<int>(dev::num_clusters_x());
   // this pair's tiles: a contiguous run of tile ids, n fastest
-  const int t_begin = static_cast<int>((static_cast<long long>(pair) * p.num_tiles) / num_pairs);
-  const int t_end = static_cast<int>((static_cast<long long>(pair + 1) * p.num_tiles) / num_pairs);
-  const int stages_per_tile = p.lr_stages + p.k_stages;
+  const int t_begin = static_cast<int>((static_cast<long long>(pair) * grp.total_tiles) / num_pairs);
+  const int t_end = static_cast<int>((static_cast<long long>(pair + 1) * grp.total_tiles) / num_pairs);
+  const unsigned long long limit_ns = grp.limit_ns;
+  unsigned int *const status = grp.status;
   const uint32_t peer_abort = dev::mapa(dev::smem_u32(const_cast<int *>(abort_flag)), h ^ 1u);
 
   if (threadIdx.x == 0) {
@@ -206,21 +233,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
-      dev::prefetch_tmap(&maps.a);
-      dev::prefetch_tmap(&maps.b);
-      dev::prefetch_tmap(&maps.sfb);
-      if (p.lr_stages) {
-        dev::prefetch_tmap(&maps.u);
-        dev::prefetch_tmap(&maps.l2);
+      for (int q = 0; q < grp.count; ++q) {
+        dev::prefetch_tmap(&grp.maps[q].a);
+        dev::prefetch_tmap(&grp.maps[q].sfa);
+        dev::prefetch_tmap(&grp.maps[q].b);
+        dev::prefetch_tmap(&grp.maps[q].sfb);
+        if (grp.p[q].lr_stages) {
+          dev::prefetch_tmap(&grp.maps[q].u);
+          dev::prefetch_tmap(&grp.maps[q].l2);
+        }
       }
       int it = 0;
       bool ok = true;
       for (int tile = t_begin; tile < t_end && ok; ++tile) {
-        const int m_blk = 2 * (tile / p.num_n) + static_cast<int>(h);  // this CTA's 128-row block
-        const int n_blk = tile % p.num_n;
+        const TileRef tr = locate_tile(grp, tile);
+        const Params &p = grp.p[tr.pi];
+        const Maps &maps = grp.maps[tr.pi];
+        const int stages_per_tile = p.lr_stages + p.k_stages;
+        const int m_blk = 2 * tr.m2 + static_cast<int>(h);  // this CTA's 128-row block
+        const int n_blk = tr.n_blk;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
-          if (!dev::mbar_wait_cluster(&empty[s], ((it / STAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
+          if (!dev::mbar_wait_cluster(&empty[s], ((it / STAGES) & 1) ^ 1, limit_ns, abort_flag)) {
             ok = false;
             break;
           }
@@ -251,13 +285,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
         }
       }
-      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
+      if (!ok) abort_pair(abort_flag, peer_abort, status);
       // Before the pair may leave: the even CTA waits for every stage it
       // armed to complete (that covers the odd CTA's copies as well).
       if (h == 0) {
         for (int j = max(0, it - STAGES); j < it; ++j) {
-          dev::mbar_wait_cluster(&full[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
-          dev::mbar_wait_cluster(&sf_loaded[j % STAGES], (j / STAGES) & 1, p.limit_ns, nullptr);
+          dev::mbar_wait_cluster(&full[j % STAGES], (j / STAGES) & 1, limit_ns, nullptr);
+          dev::mbar_wait_cluster(&sf_loaded[j % STAGES], (j / STAGES) & 1, limit_ns, nullptr);
         }
       }
     }
@@ -267,7 +301,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int it = 0, tcount = 0;
       bool ok = true, issued_any = false;
       for (int tile = t_begin; tile < t_end && ok; ++tile, ++tcount) {
-        if (!dev::mbar_wait_cluster(tmem_empty, (tcount & 1) ^ 1, p.limit_ns, abort_flag)) {
+        const Params &p = grp.p[locate_tile(grp, tile).pi];
+        const int stages_per_tile = p.lr_stages + p.k_stages;
+        if (!dev::mbar_wait_cluster(tmem_empty, (tcount & 1) ^ 1, limit_ns, abort_flag)) {
           ok = false;
           break;
         }
@@ -276,8 +312,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!dev::mbar_wait(&sf_full[s], ph, p.limit_ns, abort_flag) ||
-              !dev::mbar_wait_cluster(&full[s], ph, p.limit_ns, abort_flag)) {
+          if (!dev::mbar_wait(&sf_full[s], ph, limit_ns, abort_flag) ||
+              !dev::mbar_wait_cluster(&full[s], ph, limit_ns, abort_flag)) {
             ok = false;
             break;
           }
@@ -304,10 +340,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         if (!ok) break;
         dev::tc_commit_pair_mc(tmem_full, 0x3);    // both halves of the accumulator ready
       }
-      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
+      if (!ok) abort_pair(abort_flag, peer_abort, status);
       if (issued_any) {  // the tensor cores must be idle before TMEM is freed
         dev::tc_commit_pair(drain_mma);
-        dev::mbar_wait(drain_mma, 0, p.limit_ns, nullptr);
+        dev::mbar_wait(drain_mma, 0, limit_ns, nullptr);
       }
     }
   } else if (warp == 2) {
@@ -316,9 +352,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int it = 0;
       bool ok = true, issued_any = false;
       for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        const Params &p = grp.p[locate_tile(grp, tile).pi];
+        const int stages_per_tile = p.lr_stages + p.k_stages;
         for (int st = 0; st < stages_per_tile; ++st, ++it) {
           const int s = it % STAGES;
-          if (!dev::mbar_wait_cluster(&sf_loaded[s], (it / STAGES) & 1, p.limit_ns, abort_flag)) {
+          if (!dev::mbar_wait_cluster(&sf_loaded[s], (it / STAGES) & 1, limit_ns, abort_flag)) {
             ok = false;
             break;
           }
@@ -337,10 +375,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           dev::tc_commit_pair(&sf_full[s]);  // arrives once this stage's copies have landed
         }
       }
-      if (!ok) abort_pair(abort_flag, peer_abort, p.status);
+      if (!ok) abort_pair(abort_flag, peer_abort, status);
       if (issued_any) {
         dev::tc_commit_pair(drain_cp);
-        dev::mbar_wait(drain_cp, 0, p.limit_ns, nullptr);
+        dev::mbar_wait(drain_cp, 0, limit_ns, nullptr);
       }
     }
   } else if (warp >= 4) {
@@ -350,12 +388,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int half = e >> 2;                // which 128 of the 256 columns
     uint8_t *stage_out = smem + EPI_OFF + e * EPI_TILE_BYTES;
     const uint32_t tmem_empty_even = dev::mapa(dev::smem_u32(tmem_empty), 0);
-    const float alpha = __fmul_rn(__ldg(p.s_a), __ldg(p.s_w));
     float *rinv_tab = reinterpret_cast<float *>(smem + TAB_OFF);
     float d6n = 0.0f;
     if constexpr (RQ >= 0) {
       // 1 / (block scale of code c) of the next layer: f32(e4m3(c) * s_a_next), then f32(1 / that)
-      const float s_an = __ldg(p.nx_s_a);
+      const float s_an = __ldg(grp.p[0].nx_s_a);   // a re-quantizing launch holds one problem
       d6n = __fmul_rn(6.0f, s_an);
       if (e < 4) {
         const uint32_t c = static_cast<uint32_t>(e * 32 + lane);
@@ -366,10 +403,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     int tcount = 0;
     for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
-      const int m_blk = 2 * (tile / p.num_n) + static_cast<int>(h);
-      const int n_blk = tile % p.num_n;
-      if (!dev::mbar_wait_cluster(tmem_full, tcount & 1, p.limit_ns, abort_flag)) {
-        abort_pair(abort_flag, peer_abort, p.status);
+      const TileRef tr = locate_tile(grp, tile);
+      const Params &p = grp.p[tr.pi];
+      const Maps &maps = grp.maps[tr.pi];
+      const int m_blk = 2 * tr.m2 + static_cast<int>(h);
+      const int n_blk = tr.n_blk;
+      const float alpha = __fmul_rn(__ldg(p.s_a), __ldg(p.s_w));
+      if (!dev::mbar_wait_cluster(tmem_full, tcount & 1, limit_ns, abort_flag)) {
+        abort_pair(abort_flag, peer_abort, status);
         break;
       }
       dev::tc_fence_after();
@@ -698,22 +739,39 @@ int prepare_device(const char *fn, int sm_count, int *pairs_out) {
   return SVDQ_OK;
 }
 
+// A group of one problem.
+inline Group single_group(const Maps &maps, const Params &p) {
+  Group g{};
+  g.maps[0] = maps;
+  g.p[0] = p;
+  g.tile_end[0] = p.num_tiles;
+  g.count = 1;
+  g.total_tiles = p.num_tiles;
+  g.status = p.status;
+  g.limit_ns = p.limit_ns;
+  return g;
+}
+
 // Launches the instantiation of `epilogue` on min(tiles, resident) SM pairs.
 template <int RQ>
-int launch_gemm(const char *fn, const Maps &maps, const Params &p, int sm_count, cudaStream_t stream) {
+int launch_gemm(const char *fn, const Group &g, int epilogue, int sm_count, cudaStream_t stream) {
   int resident = 0;
   int rc = prepare_device<RQ>(fn, sm_count, &resident);
   if (rc != SVDQ_OK) return rc;
-  const int pairs = p.num_tiles < resident ? p.num_tiles : resident;
+  const int pairs = g.total_tiles < resident ? g.total_tiles : resident;
   DependentLaunch dl(dim3(2 * pairs), dim3(THREADS), SMEM_BYTES, stream);
-  cudaError_t e = p.epilogue == SVDQ_EPILOGUE_GELU_ERF
-                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF, RQ>, maps, p)
-                  : p.epilogue == SVDQ_EPILOGUE_GELU_TANH
-                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH, RQ>, maps, p)
-                      : cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ>, maps, p);
+  cudaError_t e = epilogue == SVDQ_EPILOGUE_GELU_ERF
+                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF, RQ>, g)
+                  : epilogue == SVDQ_EPILOGUE_GELU_TANH
+                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH, RQ>, g)
+                      : cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ>, g);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return SVDQ_OK;
+}
+template <int RQ>
+int launch_gemm(const char *fn, const Maps &maps, const Params &p, int sm_count, cudaStream_t stream) {
+  return launch_gemm<RQ>(fn, single_group(maps, p), p.epilogue, sm_count, stream);
 }
 
 }  // namespace w4a4

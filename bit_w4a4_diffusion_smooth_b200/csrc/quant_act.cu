@@ -69,6 +69,17 @@ struct Params {
   unsigned long long limit_ns;
 };
 
+// A grouped launch: up to SVDQ_MAX_GROUP activations quantized by one grid,
+// the CTAs of problem i after those of problems 0..i-1; each CTA reads its
+// problem's tensor maps and parameters.  A single call is a group of one.
+constexpr int kMaxGroup = SVDQ_MAX_GROUP;
+struct Group {
+  CUtensorMap tx[kMaxGroup], tl[kMaxGroup];
+  Params p[kMaxGroup];
+  int blk_end[kMaxGroup];       // prefix sums of the problems' CTA counts
+  int count;
+};
+
 template <int RANK>
 __host__ __device__ constexpr int stage_bytes() {
   return X_STAGE + 4 * RANK * 128 + OUT_BYTES;
@@ -106,7 +117,7 @@ __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
 
 template <int RANK>
 __global__ void __launch_bounds__(THREADS, 1)
-    quant_act_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1, Params p) {
+    quant_act_kernel(const __grid_constant__ Group grp) {
   constexpr int STAGES = num_stages<RANK>();
   constexpr int L1_BOX = RANK * 128;
   constexpr int STAGE = stage_bytes<RANK>();
@@ -124,7 +135,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(done + STAGES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;
+  int pi = 0;
+  while (pi + 1 < grp.count && static_cast<int>(blockIdx.x) >= grp.blk_end[pi]) ++pi;
+  const CUtensorMap &tm_x = grp.tx[pi];
+  const CUtensorMap &tm_l1 = grp.tl[pi];
+  const Params &p = grp.p[pi];
+  const int m0 = (static_cast<int>(blockIdx.x) - (pi > 0 ? grp.blk_end[pi - 1] : 0)) * BM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -383,15 +399,70 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 template <int RANK>
-int launch(const CUtensorMap &tx, const CUtensorMap &tl, const Params &p, int grid, cudaStream_t stream) {
+int launch(const Group &g, int grid, cudaStream_t stream, const char *fn) {
   const int smem = smem_bytes<RANK>();
-  const int rc = smem_optin_once<quant_act_kernel<RANK>>(smem, "svdq_quantize_act");
+  const int rc = smem_optin_once<quant_act_kernel<RANK>>(smem, fn);
   if (rc != SVDQ_OK) return rc;
   DependentLaunch dl(dim3(grid), dim3(THREADS), smem, stream);
-  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK>, tx, tl, p);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK>, g);
   if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_quantize_act launch: ") + cudaGetErrorString(e));
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return ok();
+}
+
+// Checks one problem and fills its parameters; returns its CTA count in *grid.
+int check_problem(const std::string &fn, const void *X, int M, int K, int ldx, const float *inv_lambda,
+                  const void *l1t, int rank, const float *s_a, const float *s_w, uint8_t *a_bundle, void *U,
+                  Params *p, int *grid) {
+  if (!X || !inv_lambda || !s_a || !s_w || !a_bundle || !U || (rank > 0 && !l1t))
+    return fail(SVDQ_ERR_INVALID_ARG, fn + ": null pointer");
+  if (M < 1 || K < 64 || K % 64 || ldx < K || ldx % 8)
+    return fail(SVDQ_ERR_SHAPE, fn + ": need M >= 1, K % 64 == 0, ldx >= K, ldx % 8 == 0");
+  if (rank < 0 || rank > SVDQ_LR_STRIDE || rank % 16)
+    return fail(SVDQ_ERR_SHAPE, fn + ": rank must be a multiple of 16 in [0, 64]");
+  if (!aligned16(X) || !aligned16(inv_lambda) || !aligned16(a_bundle) || !aligned16(U) ||
+      (rank > 0 && !aligned16(l1t)))
+    return fail(SVDQ_ERR_ALIGNMENT, fn + ": pointers must be 16-byte aligned");
+  p->M = M;
+  p->K = K;
+  p->KS = bundle_ks(K);
+  p->inv_lambda = inv_lambda;
+  p->s_a = s_a;
+  p->s_w = s_w;
+  p->bundle = a_bundle;
+  p->U = static_cast<uint8_t *>(U);
+  p->limit_ns = kWaitLimitNs;   // p->status: the caller's device
+  *grid = (M + 127) / 128 * (128 / BM);   // every row of every 128-row tile
+  return SVDQ_OK;
+}
+
+// The tensor maps of a checked problem: X as [K/64 boxes][M rows][64 columns] and L1^T as
+// [K/64][rank][64], one copy per stage each.
+int encode_problem(const void *X, int M, int K, int ldx, const void *l1t, int rank, CUtensorMap *tx,
+                   CUtensorMap *tl) {
+  const uint64_t kb = static_cast<uint64_t>(K / 64);
+  int rc = encode_tmap_3d(tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, {64, static_cast<uint64_t>(M), kb},
+                          {static_cast<uint64_t>(ldx) * 2, 128}, {64, BM, 4}, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc != SVDQ_OK) return rc;
+  if (rank > 0) {
+    rc = encode_tmap_3d(tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l1t, {64, static_cast<uint64_t>(rank), kb},
+                        {static_cast<uint64_t>(K) * 2, 128}, {64, static_cast<uint32_t>(rank), 4},
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc != SVDQ_OK) return rc;
+  } else {
+    *tl = *tx;
+  }
+  return SVDQ_OK;
+}
+
+int launch_rank(int rank, const Group &g, int grid, cudaStream_t s, const char *fn) {
+  switch (rank) {
+    case 0: return launch<0>(g, grid, s, fn);
+    case 16: return launch<16>(g, grid, s, fn);
+    case 32: return launch<32>(g, grid, s, fn);
+    case 48: return launch<48>(g, grid, s, fn);
+    default: return launch<64>(g, grid, s, fn);
+  }
 }
 
 }  // namespace
@@ -402,51 +473,46 @@ using namespace svdq;
 extern "C" int svdq_quantize_act(const void *X, int M, int K, int ldx, const float *inv_lambda, const void *l1t,
                                  int rank, const float *s_a, const float *s_w, uint8_t *a_bundle, void *U,
                                  svdq_stream_t stream) {
-  if (!X || !inv_lambda || !s_a || !s_w || !a_bundle || !U || (rank > 0 && !l1t))
-    return fail(SVDQ_ERR_INVALID_ARG, "svdq_quantize_act: null pointer");
-  if (M < 1 || K < 64 || K % 64 || ldx < K || ldx % 8)
-    return fail(SVDQ_ERR_SHAPE, "svdq_quantize_act: need M >= 1, K % 64 == 0, ldx >= K, ldx % 8 == 0");
-  if (rank < 0 || rank > SVDQ_LR_STRIDE || rank % 16)
-    return fail(SVDQ_ERR_SHAPE, "svdq_quantize_act: rank must be a multiple of 16 in [0, 64]");
-  if (!aligned16(X) || !aligned16(inv_lambda) || !aligned16(a_bundle) || !aligned16(U) ||
-      (rank > 0 && !aligned16(l1t)))
-    return fail(SVDQ_ERR_ALIGNMENT, "svdq_quantize_act: pointers must be 16-byte aligned");
+  static const char *fn = "svdq_quantize_act";
+  Group g{};
+  int grid = 0;
+  int rc = check_problem(fn, X, M, K, ldx, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, &g.p[0], &grid);
+  if (rc != SVDQ_OK) return rc;
   DeviceState *st = current_device_state();
   if (!st) return SVDQ_ERR_NOT_INITIALIZED;
-
-  Params p;
-  p.M = M;
-  p.K = K;
-  p.KS = bundle_ks(K);
-  p.inv_lambda = inv_lambda;
-  p.s_a = s_a;
-  p.s_w = s_w;
-  p.bundle = a_bundle;
-  p.U = static_cast<uint8_t *>(U);
-  p.status = st->status_word;
-  p.limit_ns = kWaitLimitNs;
-
-  // X as [K/64 boxes][M rows][64 columns] and L1^T as [K/64][rank][64]: one copy per stage each
-  CUtensorMap tx, tl;
-  const uint64_t kb = static_cast<uint64_t>(K / 64);
-  int rc = encode_tmap_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, {64, static_cast<uint64_t>(M), kb},
-                          {static_cast<uint64_t>(ldx) * 2, 128}, {64, BM, 4}, CU_TENSOR_MAP_SWIZZLE_128B);
+  g.p[0].status = st->status_word;
+  rc = encode_problem(X, M, K, ldx, l1t, rank, &g.tx[0], &g.tl[0]);
   if (rc != SVDQ_OK) return rc;
-  if (rank > 0) {
-    rc = encode_tmap_3d(&tl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, l1t, {64, static_cast<uint64_t>(rank), kb},
-                        {static_cast<uint64_t>(K) * 2, 128}, {64, static_cast<uint32_t>(rank), 4},
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+  g.blk_end[0] = grid;
+  g.count = 1;
+  return launch_rank(rank, g, grid, reinterpret_cast<cudaStream_t>(stream), fn);
+}
+
+extern "C" int svdq_quantize_act_grouped(const svdq_quant_problem *problems, int count, int rank,
+                                         svdq_stream_t stream) {
+  static const char *fn = "svdq_quantize_act_grouped";
+  if (!problems) return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": null problem list");
+  if (count < 1 || count > kMaxGroup)
+    return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": count must be in [1, " + std::to_string(kMaxGroup) + "]");
+  Group g{};
+  int total = 0;
+  for (int i = 0; i < count; ++i) {
+    const svdq_quant_problem &q = problems[i];
+    int grid = 0;
+    const int rc = check_problem(std::string(fn) + " (problem " + std::to_string(i) + ")", q.X, q.M, q.K, q.ldx,
+                                 q.inv_lambda, q.l1t, rank, q.s_a, q.s_w, q.a_bundle, q.U, &g.p[i], &grid);
     if (rc != SVDQ_OK) return rc;
-  } else {
-    tl = tx;
+    total += grid;
+    g.blk_end[i] = total;
   }
-  const int grid = (M + 127) / 128 * (128 / BM);   // every row of every 128-row tile
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  switch (rank) {
-    case 0: return launch<0>(tx, tl, p, grid, s);
-    case 16: return launch<16>(tx, tl, p, grid, s);
-    case 32: return launch<32>(tx, tl, p, grid, s);
-    case 48: return launch<48>(tx, tl, p, grid, s);
-    default: return launch<64>(tx, tl, p, grid, s);
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  for (int i = 0; i < count; ++i) {
+    g.p[i].status = st->status_word;
+    const svdq_quant_problem &q = problems[i];
+    const int rc = encode_problem(q.X, q.M, q.K, q.ldx, q.l1t, rank, &g.tx[i], &g.tl[i]);
+    if (rc != SVDQ_OK) return rc;
   }
+  g.count = count;
+  return launch_rank(rank, g, total, reinterpret_cast<cudaStream_t>(stream), fn);
 }

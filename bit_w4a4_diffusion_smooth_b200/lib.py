@@ -27,12 +27,28 @@ EPILOGUE_GELU_ERF = 1
 EPILOGUE_GELU_TANH = 2
 LR_STRIDE = 64
 AMAX_WORKSPACE_BYTES = 256
+MAX_GROUP = 4
 
 _lib = None
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SZ = ctypes.POINTER(ctypes.c_size_t)
+class QuantProblem(ctypes.Structure):
+    """svdq_quant_problem of include/svdq.h."""
+    _fields_ = [("X", ctypes.c_void_p), ("M", ctypes.c_int), ("K", ctypes.c_int), ("ldx", ctypes.c_int),
+                ("inv_lambda", ctypes.c_void_p), ("l1t", ctypes.c_void_p), ("s_a", ctypes.c_void_p),
+                ("s_w", ctypes.c_void_p), ("a_bundle", ctypes.c_void_p), ("U", ctypes.c_void_p)]
+
+
+class W4A4Problem(ctypes.Structure):
+    """svdq_w4a4_problem of include/svdq.h."""
+    _fields_ = [("a_bundle", ctypes.c_void_p), ("U", ctypes.c_void_p), ("s_a", ctypes.c_void_p),
+                ("w_bundle", ctypes.c_void_p), ("l2t", ctypes.c_void_p), ("s_w", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int),
+                ("gelu_col_begin", ctypes.c_int), ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int)]
+
+
 _SIGNATURES = {
     "svdq_version": (_I, []),
     "svdq_last_error_string": (ctypes.c_char_p, []),
@@ -44,6 +60,8 @@ _SIGNATURES = {
     "svdq_quantize_host": (_I, [_P, _I, _I, ctypes.c_float, _I, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P]),
     "svdq_linear_w4a4": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
+    "svdq_quantize_act_grouped": (_I, [ctypes.POINTER(QuantProblem), _I, _I, _P]),
+    "svdq_linear_w4a4_grouped": (_I, [ctypes.POINTER(W4A4Problem), _I, _I, _I, _P]),
     "svdq_linear_w4a4_requant": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I,
                                       _P, _P, _I, _P, _P, _P, _P, _P, _P]),
     "svdq_requant_workspace_size": (_I, [_I, _I, _SZ]),
@@ -208,12 +226,11 @@ def svdq_quantize_host(T, s_t, tile_rows=128):
     return bundle
 
 
-def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M=None, K=None, stream=None):
-    """Enqueues the activation kernel.  X: bf16 CUDA [M, ldx] (row stride ldx)."""
+def _quant_problem(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M=None, K=None):
+    """Checks one activation problem's buffers and returns its QuantProblem."""
     import torch
     M = X.shape[0] if M is None else M
     K = X.shape[1] if K is None else K
-    ldx = X.stride(0)
     _need_2d(X, M, K, "X")
     sz = svdq_act_sizes(M, K)
     _need_bytes(a_bundle, sz["a_bundle"], "a_bundle")
@@ -223,16 +240,27 @@ def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M=None, K
         _need_bytes(l1t, 2 * rank * K, "l1t")
     _need_bytes(s_a, 4, "s_a")
     _need_bytes(s_w, 4, "s_w")
+    return QuantProblem(_dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_lambda, "inv_lambda", torch.float32),
+                        _dptr(l1t, "l1t", allow_none=rank == 0), _dptr(s_a, "s_a", torch.float32),
+                        _dptr(s_w, "s_w", torch.float32), _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U"))
+
+
+def svdq_quantize_act(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M=None, K=None, stream=None):
+    """Enqueues the activation kernel.  X: bf16 CUDA [M, ldx] (row stride ldx)."""
+    q = _quant_problem(X, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, M, K)
     _check("svdq_quantize_act", load().svdq_quantize_act(
-        _dptr(X, "X", torch.bfloat16), M, K, ldx, _dptr(inv_lambda, "inv_lambda", torch.float32),
-        _dptr(l1t, "l1t", allow_none=rank == 0), rank, _dptr(s_a, "s_a", torch.float32),
-        _dptr(s_w, "s_w", torch.float32), _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U"),
-        _stream(stream)))
+        q.X, q.M, q.K, q.ldx, q.inv_lambda, q.l1t, rank, q.s_a, q.s_w, q.a_bundle, q.U, _stream(stream)))
 
 
-def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue, gelu_col_begin, Y,
-                     stream=None):
-    """Enqueues the W4A4 GEMM.  Y: bf16 CUDA [M, ldy]."""
+def svdq_quantize_act_grouped(problems, rank, stream=None):
+    """One launch of the activation kernel over several problems (dicts of svdq_quantize_act's
+    keyword arguments X, inv_lambda, l1t, s_a, s_w, a_bundle, U and optionally M, K)."""
+    arr = (QuantProblem * len(problems))(*[_quant_problem(rank=rank, **d) for d in problems])
+    _check("svdq_quantize_act_grouped", load().svdq_quantize_act_grouped(arr, len(problems), rank, _stream(stream)))
+
+
+def _w4a4_problem(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, gelu_col_begin, Y):
+    """Checks one GEMM problem's buffers and returns its W4A4Problem."""
     import torch
     asz = svdq_act_sizes(M, K)
     wsz = svdq_weight_sizes(K, N, rank)
@@ -245,12 +273,28 @@ def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, 
     _need_bytes(s_a, 4, "s_a")
     _need_bytes(s_w, 4, "s_w")
     _need_2d(Y, M, N, "Y")
+    return W4A4Problem(_dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U", allow_none=rank == 0),
+                       _dptr(s_a, "s_a", torch.float32), _dptr(w_bundle, "w_bundle", torch.uint8),
+                       _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
+                       _dptr(bias, "bias", allow_none=True), M, N, K, gelu_col_begin,
+                       _dptr(Y, "Y", torch.bfloat16), Y.stride(0))
+
+
+def svdq_linear_w4a4(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, epilogue, gelu_col_begin, Y,
+                     stream=None):
+    """Enqueues the W4A4 GEMM.  Y: bf16 CUDA [M, ldy]."""
+    q = _w4a4_problem(a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, rank, gelu_col_begin, Y)
     _check("svdq_linear_w4a4", load().svdq_linear_w4a4(
-        _dptr(a_bundle, "a_bundle", torch.uint8), _dptr(U, "U", allow_none=rank == 0),
-        _dptr(s_a, "s_a", torch.float32), _dptr(w_bundle, "w_bundle", torch.uint8),
-        _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(s_w, "s_w", torch.float32),
-        _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue, gelu_col_begin,
-        _dptr(Y, "Y", torch.bfloat16), Y.stride(0), _stream(stream)))
+        q.a_bundle, q.U, q.s_a, q.w_bundle, q.l2t, q.s_w, q.bias, M, N, K, rank, epilogue, gelu_col_begin, q.Y,
+        q.ldy, _stream(stream)))
+
+
+def svdq_linear_w4a4_grouped(problems, rank, epilogue, stream=None):
+    """One launch of the W4A4 GEMM over several problems (dicts of svdq_linear_w4a4's keyword
+    arguments a_bundle, U, s_a, w_bundle, l2t, s_w, bias, M, N, K, gelu_col_begin, Y)."""
+    arr = (W4A4Problem * len(problems))(*[_w4a4_problem(rank=rank, **d) for d in problems])
+    _check("svdq_linear_w4a4_grouped", load().svdq_linear_w4a4_grouped(arr, len(problems), rank, epilogue,
+                                                                       _stream(stream)))
 
 
 def svdq_act_amax(X, inv_lambda, workspace, s_a, M=None, K=None, stream=None):

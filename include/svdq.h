@@ -99,6 +99,7 @@ enum svdq_epilogue {
 #define SVDQ_LR_STRIDE 64  /* row stride (elements) of U and L2T; max rank */
 #define SVDQ_GROUP 16      /* NVFP4 block size along K */
 #define SVDQ_AMAX_WORKSPACE_BYTES 256  /* workspace of svdq_act_amax */
+#define SVDQ_MAX_GROUP 4   /* problems per grouped launch */
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int svdq_version(void);
@@ -257,6 +258,50 @@ int svdq_linear_w4a4(const uint8_t *a_bundle, const void *U, const float *s_a,
                      const uint8_t *w_bundle, const void *l2t, const float *s_w, const void *bias,
                      int M, int N, int K, int rank, int epilogue, int gelu_col_begin, void *Y,
                      int ldy, svdq_stream_t stream);
+
+/*
+ * Grouped launches: several independent layers of the same kind in one
+ * launch, for a step that runs the same projection on streams of different
+ * lengths (a dual-stream DiT block's image tokens and text tokens).  The
+ * pages' pipeline runs each projection on both streams; one launch over both
+ * keeps the whole GPU busy where the short stream alone would fill a few
+ * SMs.  No counterpart on the pages beyond that: the arithmetic of every
+ * problem is exactly that of the single call with the same arguments.
+ * `problems` is a HOST array of `count` (1..SVDQ_MAX_GROUP) descriptors,
+ * read during the call; each problem's fields follow the single call's
+ * arguments, meaning and rules.  Errors name the first bad problem.
+ */
+typedef struct svdq_quant_problem {
+  const void *X;                /* [M][ldx] bf16 */
+  int M, K, ldx;
+  const float *inv_lambda;      /* [K] f32 */
+  const void *l1t;              /* [rank][K] bf16 */
+  const float *s_a, *s_w;       /* device scalars */
+  uint8_t *a_bundle;            /* out */
+  void *U;                      /* out */
+} svdq_quant_problem;
+
+typedef struct svdq_w4a4_problem {
+  const uint8_t *a_bundle;
+  const void *U;
+  const float *s_a;
+  const uint8_t *w_bundle;
+  const void *l2t;
+  const float *s_w;
+  const void *bias;             /* [N] bf16 or NULL */
+  int M, N, K;
+  int gelu_col_begin;
+  void *Y;                      /* [M][ldy] bf16 */
+  int ldy;
+} svdq_w4a4_problem;
+
+/* svdq_quantize_act on every problem; all problems share `rank`. */
+int svdq_quantize_act_grouped(const svdq_quant_problem *problems, int count, int rank, svdq_stream_t stream);
+
+/* svdq_linear_w4a4 on every problem; all share `rank` and `epilogue`.  The
+ * persistent SM pairs take the problems' 256 x 256 tiles as one sequence. */
+int svdq_linear_w4a4_grouped(const svdq_w4a4_problem *problems, int count, int rank, int epilogue,
+                             svdq_stream_t stream);
 
 /*
  * The W4A4 GEMM of a layer whose output is the input of the next SVDQ layer

@@ -75,6 +75,19 @@ def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
                                      p, None, 16, p, p, p, p, p, None)
     assert rc == lib.ERR_INVALID_ARG                              # next_l1t missing with next_rank > 0
     assert lib.svdq_requant_workspace_size(4608, 32) == 4608 * 32 * 4
+    # grouped calls: the list, its length and each problem are checked before anything is launched
+    assert so.svdq_quantize_act_grouped(None, 1, 16, None) == lib.ERR_INVALID_ARG
+    qp = (lib.QuantProblem * 2)()
+    for i in range(2):
+        qp[i] = lib.QuantProblem(p, 64, 256 if i == 0 else 100, 256, p, p, p, p, p, p)
+    assert so.svdq_quantize_act_grouped(qp, lib.MAX_GROUP + 1, 16, None) == lib.ERR_INVALID_ARG
+    assert so.svdq_quantize_act_grouped(qp, 2, 16, None) == lib.ERR_SHAPE
+    assert b"problem 1" in so.svdq_last_error_string()
+    wp = (lib.W4A4Problem * 1)()
+    wp[0] = lib.W4A4Problem(p, p, p, p, p, p, None, 64, 256, 100, 0, p, 256)
+    assert so.svdq_linear_w4a4_grouped(wp, 0, 16, 0, None) == lib.ERR_INVALID_ARG
+    assert so.svdq_linear_w4a4_grouped(wp, 1, 16, 0, None) == lib.ERR_SHAPE
+    assert b"problem 0" in so.svdq_last_error_string()
     assert lib.svdq_requant_workspace_size(100, 0) == 0
     rc = so.svdq_act_amax(p, 4, 96, 96, p, p, p, None)
     assert rc == lib.ERR_SHAPE                                    # K % 64

@@ -66,24 +66,42 @@ struct Params {
   unsigned long long limit_ns;
 };
 
-// B fragments (hi and lo bf16 parts of X^) of one k16 step for rows nt*8+g.
+// The raw X words and inv_awq pairs a lane needs for the four k16 steps of
+// one group (rows nt*8+g, columns 16j+2t, +1, +8, +9): fetched in one go,
+// before the group's weights have landed, so that their latency overlaps
+// the wait instead of stalling every k16 step.
 template <int NT>
-__device__ __forceinline__ void load_x_frag(const Params &p, int k, int g8, uint32_t (&bh)[NT][2],
-                                            uint32_t (&bl)[NT][2]) {
-  const float2 i0 = p.inv ? __ldg(reinterpret_cast<const float2 *>(p.inv + k)) : make_float2(1.f, 1.f);
-  const float2 i1 = p.inv ? __ldg(reinterpret_cast<const float2 *>(p.inv + k + 8)) : make_float2(1.f, 1.f);
+struct XRaw {
+  uint32_t w[4][NT][2];
+  float2 iv[4][2];
+};
+template <int NT>
+__device__ __forceinline__ void fetch_x(const Params &p, int k0, int g8, int j0, int j1, XRaw<NT> &r) {
+#pragma unroll
+  for (int j = j0; j < j1; ++j) {
+    const int k = k0 + 16 * j;
+    r.iv[j][0] = p.inv ? __ldg(reinterpret_cast<const float2 *>(p.inv + k)) : make_float2(1.f, 1.f);
+    r.iv[j][1] = p.inv ? __ldg(reinterpret_cast<const float2 *>(p.inv + k + 8)) : make_float2(1.f, 1.f);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int m = nt * 8 + g8;
+      r.w[j][nt][0] = m < p.M ? __ldg(reinterpret_cast<const uint32_t *>(p.X + static_cast<size_t>(m) * p.ldx + k)) : 0u;
+      r.w[j][nt][1] =
+          m < p.M ? __ldg(reinterpret_cast<const uint32_t *>(p.X + static_cast<size_t>(m) * p.ldx + k + 8)) : 0u;
+    }
+  }
+}
+// B fragments (hi and lo bf16 parts of X^ = f32(x * inv_awq)) of k16 step j.
+template <int NT>
+__device__ __forceinline__ void split_x(const XRaw<NT> &r, int j, uint32_t (&bh)[NT][2], uint32_t (&bl)[NT][2]) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    const int m = nt * 8 + g8;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
-    if (m < p.M) {
-      const uint32_t w0 = __ldg(reinterpret_cast<const uint32_t *>(p.X + static_cast<size_t>(m) * p.ldx + k));
-      const uint32_t w1 = __ldg(reinterpret_cast<const uint32_t *>(p.X + static_cast<size_t>(m) * p.ldx + k + 8));
-      x[0] = __fmul_rn(__uint_as_float(w0 << 16), i0.x);
-      x[1] = __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), i0.y);
-      x[2] = __fmul_rn(__uint_as_float(w1 << 16), i1.x);
-      x[3] = __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), i1.y);
-    }
+    const uint32_t w0 = r.w[j][nt][0], w1 = r.w[j][nt][1];
+    float x[4];
+    x[0] = __fmul_rn(__uint_as_float(w0 << 16), r.iv[j][0].x);
+    x[1] = __fmul_rn(__uint_as_float(w0 & 0xFFFF0000u), r.iv[j][0].y);
+    x[2] = __fmul_rn(__uint_as_float(w1 << 16), r.iv[j][1].x);
+    x[3] = __fmul_rn(__uint_as_float(w1 & 0xFFFF0000u), r.iv[j][1].y);
     float h[4], l[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -173,12 +191,16 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
     const int slot = c % RING;
+    const int grp = c * CHUNK_G + warp;
+    XRaw<NT> xr;
+    // one row block (the modulation layers): all four steps' X up front; two row blocks would
+    // hold twice the registers, so those fetch each step's X where it is used
+    if (NT == 1 && grp < p.G) fetch_x<NT>(p, grp * 64 + 2 * t, g8, 0, 4, xr);
     if (!dev::mbar_wait_warp(&full[slot], (c / RING) & 1, p.limit_ns, abort_flag)) {
       *abort_flag = 1;
       dev::report(p.status, SVDQ_ERR_TIMEOUT);
       break;
     }
-    const int grp = c * CHUNK_G + warp;
     if (grp < p.G) {
       const uint8_t *src = smem + slot * CHUNK_BYTES;
       uint4 wq[4];
@@ -208,7 +230,8 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t bh[NT][2], bl[NT][2];
-        load_x_frag<NT>(p, grp * 64 + 16 * j + 2 * t, g8, bh, bl);
+        if (NT > 1) fetch_x<NT>(p, grp * 64 + 2 * t, g8, j, j + 1, xr);
+        split_x<NT>(xr, j, bh, bl);
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           const uint32_t w = j == 0 ? wq[cb].x : j == 1 ? wq[cb].y : j == 2 ? wq[cb].z : wq[cb].w;

@@ -113,6 +113,61 @@ class SVDQLinear:
         return self.gemm(self.quantize(X, stream), M, Y, stream)
 
 
+class SplitProjection:
+    """A fused projection's packed checkpoint mapped onto split modules.
+
+    The pages note that a checkpoint whose query, key and value projections
+    are fused into one grouped operation does not map by itself onto a model
+    that keeps them as separate modules: the mapping needs the tensor order
+    and a small runtime adapter.  This is that adapter for an SVDQLinear
+    packed over the concatenation [W_0 | W_1 | ...] of the parts along N
+    (in that order): every part keeps the fused layer's smoothing, L1, s_a
+    and s_w, and takes its own columns of the residual codes and scales, of
+    L2^T and of the bias - views of the fused layer's device buffers, no
+    copy.  One call quantizes X once (the parts share the activation side)
+    and runs the parts' GEMMs as one grouped launch; part i's output equals
+    columns [n_i, n_i + size_i) of the fused layer's output bit for bit.
+    Part sizes must be multiples of 256 (the weight bundle's tile rows).
+    """
+
+    def __init__(self, fused, sizes, names=None):
+        if sum(sizes) != fused.N or any(sz <= 0 or sz % 256 for sz in sizes):
+            raise ValueError(f"SplitProjection: part sizes {sizes} must be positive multiples of 256 adding up to "
+                             f"N = {fused.N}")
+        if len(sizes) > lib.MAX_GROUP:
+            raise ValueError(f"SplitProjection: at most {lib.MAX_GROUP} parts")
+        self.fused = fused
+        self.names = list(names) if names is not None else [str(i) for i in range(len(sizes))]
+        tile_bytes = lib.svdq_weight_sizes(fused.K, 256, fused.rank)["w_bundle"]   # one 256-row tile row, all K
+        self.parts = []
+        n0 = 0
+        for sz in sizes:
+            n1 = n0 + sz
+            begin = min(max(fused.gelu_col_begin - n0, 0), sz)
+            self.parts.append(dict(n0=n0, N=sz, gelu_col_begin=begin,
+                                   w_bundle=fused.w_bundle[n0 // 256 * tile_bytes:n1 // 256 * tile_bytes],
+                                   l2t=fused.l2t[n0 * 2 * lib.LR_STRIDE:n1 * 2 * lib.LR_STRIDE],
+                                   bias=fused.bias[n0:n1] if fused.bias is not None else None))
+            n0 = n1
+
+    def __call__(self, X, out=None, stream=None):
+        """X: bf16 CUDA [M, K] -> {name: Y_i bf16 [M, size_i]} (or into the tensors of `out`)."""
+        f = self.fused
+        M = X.shape[0]
+        b = f.quantize(X, stream)
+        ys = {}
+        probs = []
+        for name, p in zip(self.names, self.parts):
+            Y = out[name] if out is not None else torch.empty((M, p["N"]), dtype=torch.bfloat16, device=f.device)
+            _check_output(Y, M, p["N"], f.device, "SplitProjection")
+            ys[name] = Y
+            probs.append(dict(a_bundle=b["a_bundle"], U=b["U"], s_a=f.s_a, w_bundle=p["w_bundle"], l2t=p["l2t"],
+                              s_w=f.s_w, bias=p["bias"], M=M, N=p["N"], K=f.K, gelu_col_begin=p["gelu_col_begin"],
+                              Y=Y))
+        lib.svdq_linear_w4a4_grouped(probs, f.rank, f.epilogue, stream=stream)
+        return ys
+
+
 class AWQLinear:
     """Y = (X diag(inv_awq)) deq(W_a) + b with 4-bit group-64 weights (any M; blocks of 16 rows)."""
 

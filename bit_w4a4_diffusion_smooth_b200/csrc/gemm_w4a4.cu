@@ -24,7 +24,7 @@ extern "C" int svdq_linear_w4a4_grouped(const svdq_w4a4_problem *problems, int c
   if (!problems) return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": null problem list");
   if (count < 1 || count > kMaxGroup)
     return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": count must be in [1, " + std::to_string(kMaxGroup) + "]");
-  Group g{};
+  Group<kMaxGroup> g{};
   DeviceState *st = nullptr;
   int tiles = 0;
   for (int i = 0; i < count; ++i) {
@@ -40,6 +40,6 @@ extern "C" int svdq_linear_w4a4_grouped(const svdq_w4a4_problem *problems, int c
   g.total_tiles = tiles;
   g.status = g.p[0].status;
   g.limit_ns = g.p[0].limit_ns;
-  const int rc = launch_gemm<-1>(fn, g, epilogue, st->sm_count, reinterpret_cast<cudaStream_t>(stream));
+  const int rc = launch_gemm<-1, kMaxGroup>(fn, g, epilogue, st->sm_count, reinterpret_cast<cudaStream_t>(stream));
   return rc == SVDQ_OK ? ok() : rc;
 }

@@ -125,15 +125,17 @@ struct Maps {
   CUtensorMap a, sfa, b, sfb, u, l2, y;
 };
 
-// One launch computes up to kMaxGroup independent GEMMs of the same epilogue
-// kind (a grouped launch): their tiles form one sequence, problem after
-// problem, which the persistent SM pairs split into contiguous runs.  A
-// single GEMM is a group of one.
+// One launch computes up to G independent GEMMs of the same epilogue kind
+// (a grouped launch): their tiles form one sequence, problem after problem,
+// which the persistent SM pairs split into contiguous runs.  A single GEMM is
+// a group of one, compiled with G = 1 so that it carries no group lookup and
+// the small parameter block of one problem.
 constexpr int kMaxGroup = SVDQ_MAX_GROUP;
+template <int G>
 struct Group {
-  Maps maps[kMaxGroup];
-  Params p[kMaxGroup];
-  int tile_end[kMaxGroup];      // prefix sums of the problems' tile counts
+  Maps maps[G];
+  Params p[G];
+  int tile_end[G];              // prefix sums of the problems' tile counts
   int count;
   int total_tiles;
   unsigned int *status;
@@ -144,9 +146,11 @@ struct Group {
 struct TileRef {
   int pi, m2, n_blk;            // problem, 256-row pair block, 256-column block
 };
-__device__ __forceinline__ TileRef locate_tile(const Group &g, int tile) {
+template <int G>
+__device__ __forceinline__ TileRef locate_tile(const Group<G> &g, int tile) {
   int pi = 0;
-  while (pi + 1 < g.count && tile >= g.tile_end[pi]) ++pi;
+  if constexpr (G > 1)
+    while (pi + 1 < g.count && tile >= g.tile_end[pi]) ++pi;
   const int lt = tile - (pi > 0 ? g.tile_end[pi - 1] : 0);
   return TileRef{pi, lt / g.p[pi].num_n, lt % g.p[pi].num_n};
 }
@@ -177,9 +181,9 @@ __device__ __forceinline__ void abort_pair(volatile int *abort_flag, uint32_t pe
 // and bf16(x^) . L1_next over the tile's 256 columns on mma.sync, added into
 // an fp32 [M][RQ] buffer with vector atomics (a separate kernel turns the
 // sums into the next layer's U once every column block is done).
-template <int EPI, int RQ>
+template <int EPI, int RQ, int G>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
-    gemm_w4a4_kernel(const __grid_constant__ Group grp) {
+    gemm_w4a4_kernel(const __grid_constant__ Group<G> grp) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);  // even CTA: both CTAs' bytes
@@ -706,7 +710,7 @@ inline int setup_gemm(const char *fn, const uint8_t *a_bundle, const void *U, co
 // Per device and kernel family (RQ), once: the shared-memory opt-in of the
 // three epilogue instantiations and the number of SM pairs that can hold one
 // CTA each at that size.
-template <int RQ>
+template <int RQ, int G>
 int prepare_device(const char *fn, int sm_count, int *pairs_out) {
   static std::mutex mu;
   static int cached[64] = {0};
@@ -715,13 +719,13 @@ int prepare_device(const char *fn, int sm_count, int *pairs_out) {
     return fail(SVDQ_ERR_CUDA, std::string(fn) + ": no current device");
   std::lock_guard<std::mutex> lock(mu);
   if (cached[dev_id] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ, G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF, RQ>,
+      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF, RQ, G>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH, RQ>,
+      e = cudaFuncSetAttribute(gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH, RQ, G>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + ": " + cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
@@ -729,7 +733,7 @@ int prepare_device(const char *fn, int sm_count, int *pairs_out) {
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ>, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ, G>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = sm_count / 2;
     }
@@ -740,8 +744,8 @@ int prepare_device(const char *fn, int sm_count, int *pairs_out) {
 }
 
 // A group of one problem.
-inline Group single_group(const Maps &maps, const Params &p) {
-  Group g{};
+inline Group<1> single_group(const Maps &maps, const Params &p) {
+  Group<1> g{};
   g.maps[0] = maps;
   g.p[0] = p;
   g.tile_end[0] = p.num_tiles;
@@ -753,25 +757,25 @@ inline Group single_group(const Maps &maps, const Params &p) {
 }
 
 // Launches the instantiation of `epilogue` on min(tiles, resident) SM pairs.
-template <int RQ>
-int launch_gemm(const char *fn, const Group &g, int epilogue, int sm_count, cudaStream_t stream) {
+template <int RQ, int G>
+int launch_gemm(const char *fn, const Group<G> &g, int epilogue, int sm_count, cudaStream_t stream) {
   int resident = 0;
-  int rc = prepare_device<RQ>(fn, sm_count, &resident);
+  int rc = prepare_device<RQ, G>(fn, sm_count, &resident);
   if (rc != SVDQ_OK) return rc;
   const int pairs = g.total_tiles < resident ? g.total_tiles : resident;
   DependentLaunch dl(dim3(2 * pairs), dim3(THREADS), SMEM_BYTES, stream);
   cudaError_t e = epilogue == SVDQ_EPILOGUE_GELU_ERF
-                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF, RQ>, g)
+                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_ERF, RQ, G>, g)
                   : epilogue == SVDQ_EPILOGUE_GELU_TANH
-                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH, RQ>, g)
-                      : cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ>, g);
+                      ? cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_GELU_TANH, RQ, G>, g)
+                      : cudaLaunchKernelEx(&dl.cfg, gemm_w4a4_kernel<SVDQ_EPILOGUE_NONE, RQ, G>, g);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return SVDQ_OK;
 }
 template <int RQ>
 int launch_gemm(const char *fn, const Maps &maps, const Params &p, int sm_count, cudaStream_t stream) {
-  return launch_gemm<RQ>(fn, single_group(maps, p), p.epilogue, sm_count, stream);
+  return launch_gemm<RQ, 1>(fn, single_group(maps, p), p.epilogue, sm_count, stream);
 }
 
 }  // namespace w4a4

@@ -69,14 +69,15 @@ struct Params {
   unsigned long long limit_ns;
 };
 
-// A grouped launch: up to SVDQ_MAX_GROUP activations quantized by one grid,
-// the CTAs of problem i after those of problems 0..i-1; each CTA reads its
-// problem's tensor maps and parameters.  A single call is a group of one.
+// A grouped launch: up to G activations quantized by one grid, the CTAs of
+// problem i after those of problems 0..i-1; each CTA reads its problem's
+// tensor maps and parameters.  A single call is a group of one (G = 1).
 constexpr int kMaxGroup = SVDQ_MAX_GROUP;
+template <int G>
 struct Group {
-  CUtensorMap tx[kMaxGroup], tl[kMaxGroup];
-  Params p[kMaxGroup];
-  int blk_end[kMaxGroup];       // prefix sums of the problems' CTA counts
+  CUtensorMap tx[G], tl[G];
+  Params p[G];
+  int blk_end[G];               // prefix sums of the problems' CTA counts
   int count;
 };
 
@@ -115,9 +116,9 @@ __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
 }
 
-template <int RANK>
+template <int RANK, int G>
 __global__ void __launch_bounds__(THREADS, 1)
-    quant_act_kernel(const __grid_constant__ Group grp) {
+    quant_act_kernel(const __grid_constant__ Group<G> grp) {
   constexpr int STAGES = num_stages<RANK>();
   constexpr int L1_BOX = RANK * 128;
   constexpr int STAGE = stage_bytes<RANK>();
@@ -136,7 +137,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int pi = 0;
-  while (pi + 1 < grp.count && static_cast<int>(blockIdx.x) >= grp.blk_end[pi]) ++pi;
+  if constexpr (G > 1)
+    while (pi + 1 < grp.count && static_cast<int>(blockIdx.x) >= grp.blk_end[pi]) ++pi;
   const CUtensorMap &tm_x = grp.tx[pi];
   const CUtensorMap &tm_l1 = grp.tl[pi];
   const Params &p = grp.p[pi];
@@ -398,13 +400,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int RANK>
-int launch(const Group &g, int grid, cudaStream_t stream, const char *fn) {
+template <int RANK, int G>
+int launch(const Group<G> &g, int grid, cudaStream_t stream, const char *fn) {
   const int smem = smem_bytes<RANK>();
-  const int rc = smem_optin_once<quant_act_kernel<RANK>>(smem, fn);
+  const int rc = smem_optin_once<quant_act_kernel<RANK, G>>(smem, fn);
   if (rc != SVDQ_OK) return rc;
   DependentLaunch dl(dim3(grid), dim3(THREADS), smem, stream);
-  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK>, g);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK, G>, g);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return ok();
@@ -455,13 +457,14 @@ int encode_problem(const void *X, int M, int K, int ldx, const void *l1t, int ra
   return SVDQ_OK;
 }
 
-int launch_rank(int rank, const Group &g, int grid, cudaStream_t s, const char *fn) {
+template <int G>
+int launch_rank(int rank, const Group<G> &g, int grid, cudaStream_t s, const char *fn) {
   switch (rank) {
-    case 0: return launch<0>(g, grid, s, fn);
-    case 16: return launch<16>(g, grid, s, fn);
-    case 32: return launch<32>(g, grid, s, fn);
-    case 48: return launch<48>(g, grid, s, fn);
-    default: return launch<64>(g, grid, s, fn);
+    case 0: return launch<0, G>(g, grid, s, fn);
+    case 16: return launch<16, G>(g, grid, s, fn);
+    case 32: return launch<32, G>(g, grid, s, fn);
+    case 48: return launch<48, G>(g, grid, s, fn);
+    default: return launch<64, G>(g, grid, s, fn);
   }
 }
 
@@ -474,7 +477,7 @@ extern "C" int svdq_quantize_act(const void *X, int M, int K, int ldx, const flo
                                  int rank, const float *s_a, const float *s_w, uint8_t *a_bundle, void *U,
                                  svdq_stream_t stream) {
   static const char *fn = "svdq_quantize_act";
-  Group g{};
+  Group<1> g{};
   int grid = 0;
   int rc = check_problem(fn, X, M, K, ldx, inv_lambda, l1t, rank, s_a, s_w, a_bundle, U, &g.p[0], &grid);
   if (rc != SVDQ_OK) return rc;
@@ -494,7 +497,7 @@ extern "C" int svdq_quantize_act_grouped(const svdq_quant_problem *problems, int
   if (!problems) return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": null problem list");
   if (count < 1 || count > kMaxGroup)
     return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": count must be in [1, " + std::to_string(kMaxGroup) + "]");
-  Group g{};
+  Group<kMaxGroup> g{};
   int total = 0;
   for (int i = 0; i < count; ++i) {
     const svdq_quant_problem &q = problems[i];

@@ -6,6 +6,7 @@ tensors (torch supplies device memory and streams); host arguments are numpy
 arrays.  A missing library raises immediately: there is no fallback path.
 """
 import ctypes
+import functools
 import os
 
 import numpy as np
@@ -168,16 +169,29 @@ def svdq_init(device=0):
     _check("svdq_init", load().svdq_init(int(device)))
 
 
-def svdq_weight_sizes(K, N, rank):
+@functools.lru_cache(maxsize=1024)
+def _weight_sizes(K, N, rank):
     s = [ctypes.c_size_t() for _ in range(4)]
     _check("svdq_weight_sizes", load().svdq_weight_sizes(K, N, rank, *[ctypes.byref(x) for x in s]))
-    return dict(zip(("inv_lambda", "l1t", "l2t", "w_bundle"), (x.value for x in s)))
+    return tuple(x.value for x in s)
+
+
+@functools.lru_cache(maxsize=1024)
+def _act_sizes(M, K):
+    s = [ctypes.c_size_t() for _ in range(2)]
+    _check("svdq_act_sizes", load().svdq_act_sizes(M, K, *[ctypes.byref(x) for x in s]))
+    return tuple(x.value for x in s)
+
+
+def svdq_weight_sizes(K, N, rank):
+    """Byte sizes of a packed layer's buffers (the library's answer, cached per shape: the
+    per-call argument checks of the device calls ask it every time)."""
+    return dict(zip(("inv_lambda", "l1t", "l2t", "w_bundle"), _weight_sizes(K, N, rank)))
 
 
 def svdq_act_sizes(M, K):
-    s = [ctypes.c_size_t() for _ in range(2)]
-    _check("svdq_act_sizes", load().svdq_act_sizes(M, K, *[ctypes.byref(x) for x in s]))
-    return dict(zip(("a_bundle", "u"), (x.value for x in s)))
+    """Byte sizes of an activation's bundle and U (cached per shape, like svdq_weight_sizes)."""
+    return dict(zip(("a_bundle", "u"), _act_sizes(M, K)))
 
 
 def svdq_pack_weights(W_bits, act_absmax, rank, num_threads=0, seed=0, want_residual=False):

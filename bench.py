@@ -408,6 +408,36 @@ def time_cold(fn, sets, reps, flush):
     return sum(a.elapsed_time(b) for a, b in ev) / reps
 
 
+def awq_many_rows(W, device, m=256, reps=10):
+    """The adaLN projection on a batch of m rows: K3's blocks of 16 rows against the GEMM path on weights
+    expanded once (mean device time of `reps` back-to-back launches each, after warm-up)."""
+    import torch
+    from bit_w4a4_diffusion_smooth_b200 import lib
+    A = W.sets[0]["awq"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(7)
+    X = torch.randn(m, AK, device=device, generator=gen).to(torch.bfloat16)
+    Y = torch.empty(m, AN, dtype=torch.bfloat16, device=device)
+    ws = torch.empty(lib.awq_gemm_workspace_size(m, AK, AN), dtype=torch.uint8, device=device)
+    lib.awq_expand_weights(A["inv_awq"], A["qweight"], A["scales"], A["zeros"], AK, AN, ws)
+    out = {}
+    for name, fn in (("gemv_blocks_of_16_us", lambda: lib.awq_linear_w4a16(X, A["inv_awq"], A["qweight"], A["scales"],
+                                                                           A["zeros"], A["bias"], AN, Y)),
+                     ("gemm_on_expanded_us", lambda: lib.awq_linear_w4a16_expanded(X, A["bias"], AN, Y, ws))):
+        for _ in range(3):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = round(e0.elapsed_time(e1) / reps * 1e3, 2)
+    out["what"] = f"{m}x{AK}->{AN} AWQ W4A16, {reps} launches back to back (the many-row path of the adaLN projection)"
+    return out
+
+
 def copy_floor(device, nbytes, reps=24):
     """A library copy of `nbytes` (torch, device to device) with L2 flushed before it, timed like the
     kernels: the HBM rate a plain stream of this size reaches on this GPU, as (GB/s counting read +
@@ -570,6 +600,7 @@ def run_ours(args):
     # ---- reference points on this GPU: a library copy of the activation's size, and cuBLASLt's
     # NVFP4 GEMM on the fc1 shape
     floor_gbs, floor_us = copy_floor(device, TOKENS * HIDDEN * 2)
+    awq_batch = awq_many_rows(W, device)
     fp4_lib = fp4_library_point(device, *LAYERS["fc1"][:3]) if not args.no_library_points else "skipped"
 
     # ---- max over ranks
@@ -647,6 +678,7 @@ def run_ours(args):
                                      "down-projection in the epilogue) per launch" if args.mlp == "fused" else
                                      "2MKN (FP4) + 2MrN (low-rank up-projection) per launch")},
         "kernels": ktab,
+        "awq_many_rows": awq_batch,
         "reference_points": {
             "hbm_copy_same_bytes": {"GB/s": round(floor_gbs, 1), "us": round(floor_us, 2),
                                     "what": f"torch copy of {TOKENS}x{HIDDEN} bf16, timed like the kernels "

@@ -21,10 +21,11 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsvdq_b200.so")
 
 SOURCES = ["api.cu", "quant_act.cu", "act_amax.cu", "gemm_w4a4.cu", "gemm_w4a4_requant.cu", "gemv_w4a16.cu",
-           "pack_svdq.cpp", "pack_awq.cpp", "pack_device.cu"]
-# The device pack's float64 products run on cuBLAS (plain GEMMs); the toolkit's copy is found through the rpath.
+           "awq_gemm.cu", "pack_svdq.cpp", "pack_awq.cpp", "pack_device.cu"]
+# The device pack's float64 products and the many-row AWQ GEMM run on cuBLAS / cuBLASLt (plain GEMMs); the
+# toolkit's copies are found through the rpath.
 CUDA_LIB = os.path.join(os.path.dirname(os.path.dirname(shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc")), "lib64")
-LINK_LIBS = ["-lpthread", "-lcublas", "-Xlinker", f"-rpath={CUDA_LIB}"]
+LINK_LIBS = ["-lpthread", "-lcublas", "-lcublasLt", "-Xlinker", f"-rpath={CUDA_LIB}"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # Host code: no fused multiply-add contraction and no fast-math, so the
 # float32 quantization decisions of the host pack follow IEEE one rounding per

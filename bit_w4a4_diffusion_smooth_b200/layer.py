@@ -169,7 +169,14 @@ class SplitProjection:
 
 
 class AWQLinear:
-    """Y = (X diag(inv_awq)) deq(W_a) + b with 4-bit group-64 weights (any M; blocks of 16 rows)."""
+    """Y = (X diag(inv_awq)) deq(W_a) + b with 4-bit group-64 weights, any M.
+
+    Up to `gemm_rows` rows run on the GEMV (one pass over the packed weights per
+    block of 16 rows); more rows run the GEMM path on weights expanded once into
+    a workspace the layer keeps (allocated on first use, grown with M).
+    """
+
+    gemm_rows = 48
 
     def __init__(self, packed, K, N, bias_bits=None, device="cuda"):
         self.K, self.N = K, N
@@ -194,6 +201,15 @@ class AWQLinear:
         if Y is None:
             Y = torch.empty((X.shape[0], self.N), dtype=torch.bfloat16, device=self.device)
         _check_output(Y, X.shape[0], self.N, self.device, "AWQLinear")
-        lib.awq_linear_w4a16(X, self.inv_awq, self.qweight, self.scales, self.zeros, self.bias, self.N, Y,
-                             stream=stream)
+        if X.shape[0] > self.gemm_rows:
+            need = lib.awq_gemm_workspace_size(X.shape[0], self.K, self.N)
+            if getattr(self, "_workspace", None) is None or self._workspace.numel() < need:
+                # (re)allocated: the expanded weights are written once into its head and reused
+                self._workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+                lib.awq_expand_weights(self.inv_awq, self.qweight, self.scales, self.zeros, self.K, self.N,
+                                       self._workspace, stream=stream)
+            lib.awq_linear_w4a16_expanded(X, self.bias, self.N, Y, self._workspace, stream=stream)
+        else:
+            lib.awq_linear_w4a16(X, self.inv_awq, self.qweight, self.scales, self.zeros, self.bias, self.N, Y,
+                                 stream=stream)
         return Y

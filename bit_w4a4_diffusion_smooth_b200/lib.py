@@ -75,6 +75,10 @@ _SIGNATURES = {
     "awq_packed_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ]),
     "awq_pack_weights": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "awq_linear_w4a16": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P]),
+    "awq_gemm_workspace_size": (_I, [_I, _I, _I, _SZ]),
+    "awq_linear_w4a16_gemm": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
+    "awq_expand_weights": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "awq_linear_w4a16_expanded": (_I, [_P, _I, _I, _I, _P, _I, _P, _I, _P, _P]),
     "svdq_check_status": (_I, [_P]),
     "svdq_debug_wait_timeout": (_I, [ctypes.c_uint64, _P]),
     "svdq_debug_convert": (_I, [_P, _I, _P, _P, _P]),
@@ -492,6 +496,59 @@ def awq_linear_w4a16(X, inv_awq, qweight, scales, zeros, bias, N, Y, group=64, M
         _dptr(qweight, "qweight"), _dptr(scales, "scales"), _dptr(zeros, "zeros"), group,
         _dptr(bias, "bias", allow_none=True), N, _dptr(Y, "Y", torch.bfloat16), Y.stride(0),
         _stream(stream)))
+
+
+def awq_gemm_workspace_size(M, K, N):
+    n = ctypes.c_size_t()
+    _check("awq_gemm_workspace_size", load().awq_gemm_workspace_size(M, K, N, ctypes.byref(n)))
+    return n.value
+
+
+def awq_linear_w4a16_gemm(X, inv_awq, qweight, scales, zeros, bias, N, Y, workspace, group=64, M=None, K=None,
+                          stream=None):
+    """Enqueues the many-row W4A16 path (weights expanded into `workspace`, then one bf16 GEMM)."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    _need_2d(X, M, K, "X")
+    _need_2d(Y, M, N, "Y")
+    _need_bytes(qweight, N * K // 2, "qweight")
+    _need_bytes(scales, 2 * N * (K // group), "scales")
+    _need_bytes(zeros, 2 * N * (K // group), "zeros")
+    _need_bytes(inv_awq, 4 * K, "inv_awq")
+    _need_bytes(bias, 2 * N, "bias")
+    _need_bytes(workspace, awq_gemm_workspace_size(M, K, N), "workspace")
+    _check("awq_linear_w4a16_gemm", load().awq_linear_w4a16_gemm(
+        _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_awq, "inv_awq"),
+        _dptr(qweight, "qweight"), _dptr(scales, "scales"), _dptr(zeros, "zeros"), group,
+        _dptr(bias, "bias", allow_none=True), N, _dptr(Y, "Y", torch.bfloat16), Y.stride(0),
+        _dptr(workspace, "workspace"), _stream(stream)))
+
+
+def awq_expand_weights(inv_awq, qweight, scales, zeros, K, N, workspace, group=64, stream=None):
+    """Writes the layer's expanded weights into the first 4 K N bytes of `workspace`."""
+    _need_bytes(qweight, N * K // 2, "qweight")
+    _need_bytes(scales, 2 * N * (K // group), "scales")
+    _need_bytes(zeros, 2 * N * (K // group), "zeros")
+    _need_bytes(inv_awq, 4 * K, "inv_awq")
+    _need_bytes(workspace, 4 * K * N, "workspace")
+    _check("awq_expand_weights", load().awq_expand_weights(
+        _dptr(inv_awq, "inv_awq"), _dptr(qweight, "qweight"), _dptr(scales, "scales"), _dptr(zeros, "zeros"),
+        K, N, group, _dptr(workspace, "workspace"), _stream(stream)))
+
+
+def awq_linear_w4a16_expanded(X, bias, N, Y, workspace, M=None, K=None, stream=None):
+    """The GEMM half of the many-row path, on the expansion already in `workspace`."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    _need_2d(X, M, K, "X")
+    _need_2d(Y, M, N, "Y")
+    _need_bytes(bias, 2 * N, "bias")
+    _need_bytes(workspace, awq_gemm_workspace_size(M, K, N), "workspace")
+    _check("awq_linear_w4a16_expanded", load().awq_linear_w4a16_expanded(
+        _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(bias, "bias", allow_none=True), N,
+        _dptr(Y, "Y", torch.bfloat16), Y.stride(0), _dptr(workspace, "workspace"), _stream(stream)))
 
 
 def svdq_check_status(stream=None):

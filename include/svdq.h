@@ -404,6 +404,37 @@ int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq,
                      const void *bias, int N, void *Y, int ldy, svdq_stream_t stream);
 
 /*
+ * AWQ W4A16 for many rows (the GEMM path; awq_linear_w4a16 reads the packed
+ * weights once per block of 16 rows, which suits the few rows of a
+ * modulation layer).  Same result definition as awq_linear_w4a16,
+ *   Y = (X diag(inv_awq)) deq(W) + bias,
+ * computed as: w = f32(inv_awq[k] (q - z) s) expanded into two bf16 matrices
+ * W_hi = bf16(w), W_lo = bf16(w - W_hi) (together ~16 significant bits),
+ * D = X . W_hi + X . W_lo in fp32 (two bf16 GEMMs through cuBLASLt), then
+ * Y = bf16(D + bias).  The pages have no counterpart beyond the W4A16
+ * projection itself.
+ * workspace: device scratch of awq_gemm_workspace_size(M, K, N) bytes
+ * (4 K N for W_hi and W_lo, then 4 M N for D), 16-byte aligned; its contents
+ * do not matter and are overwritten.
+ * Args and rules: those of awq_linear_w4a16 (any M >= 1), plus workspace and a
+ * 16-byte aligned bias when given.
+ */
+int awq_gemm_workspace_size(int M, int K, int N, size_t *bytes);
+/* The two halves of awq_linear_w4a16_gemm, for a layer called many times:
+ * awq_expand_weights writes W_hi and W_lo into the first 4 K N bytes of the
+ * workspace (its arguments and rules as in awq_linear_w4a16_gemm); as long as
+ * the caller keeps those bytes, awq_linear_w4a16_expanded computes Y from them
+ * (the workspace of awq_gemm_workspace_size(M, K, N) bytes: the expansion,
+ * then D). */
+int awq_expand_weights(const float *inv_awq, const uint32_t *qweight, const void *scales, const void *zeros,
+                       int K, int N, int group, void *workspace, svdq_stream_t stream);
+int awq_linear_w4a16_expanded(const void *X, int M, int K, int ldx, const void *bias, int N, void *Y, int ldy,
+                              void *workspace, svdq_stream_t stream);
+int awq_linear_w4a16_gemm(const void *X, int M, int K, int ldx, const float *inv_awq,
+                          const uint32_t *qweight, const void *scales, const void *zeros, int group,
+                          const void *bias, int N, void *Y, int ldy, void *workspace, svdq_stream_t stream);
+
+/*
  * Waits for `stream`, then returns and clears the device status word of the
  * current device: SVDQ_OK, or SVDQ_ERR_TIMEOUT if a kernel's bounded wait ran
  * out since the last check (SVDQ_ERR_CUDA if the stream itself failed).

@@ -75,6 +75,11 @@ def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
                                      p, None, 16, p, p, p, p, p, None)
     assert rc == lib.ERR_INVALID_ARG                              # next_l1t missing with next_rank > 0
     assert lib.svdq_requant_workspace_size(4608, 32) == 4608 * 32 * 4
+    # the many-row AWQ path: a workspace is required; shapes as the GEMV's
+    assert so.awq_linear_w4a16_gemm(p, 100, 256, 256, p, p, p, p, 64, None, 256, p, 256, None, None) == \
+        lib.ERR_INVALID_ARG
+    assert so.awq_linear_w4a16_gemm(p, 100, 256, 256, p, p, p, p, 64, None, 96, p, 96, p, None) == lib.ERR_SHAPE
+    assert lib.awq_gemm_workspace_size(256, 3072, 18432) == 3072 * 18432 * 4 + 256 * 18432 * 4
     # grouped calls: the list, its length and each problem are checked before anything is launched
     assert so.svdq_quantize_act_grouped(None, 1, 16, None) == lib.ERR_INVALID_ARG
     qp = (lib.QuantProblem * 2)()

@@ -18,10 +18,15 @@
 //   * the products run on the tensor cores as Y^T = W^T . X^T (mma.sync
 //     m16n8k16: 16 output columns x 16 k per instruction, the rows of X in
 //     the 8-wide slot); X^ = f32(x * inv_awq) is split into bf16 hi + lo
-//     parts (hi + lo carries ~16 significant bits), one MMA each;
+//     parts (hi + lo carries ~16 significant bits).  Up to 4 rows, the hi
+//     parts fill slots 0..3 and the lo parts slots 4..7 of one MMA, added
+//     at the end; more rows take one MMA per part;
 //   * dequantization in registers: two nibbles at a time become a bf16 pair
-//     (128 + q) by one mask-and-or, one bf16x2 subtraction of (128 + z)
-//     gives (q - z) exactly;
+//     (128 + q) by one mask-and-or.  With one block of rows the zero point
+//     leaves the inner loop: an MMA with an all-ones A fragment gives
+//     sum_k b per row, and the group's sum of (q - z) b is
+//     sum (128 + q) b - (128 + z) sum b, one f32 fma per output; two row
+//     blocks subtract 128 + z from every pair (bf16x2, exact) instead;
 //   * per group the fp32 partial is scaled by s in registers; the warps'
 //     partials are added through shared memory (the ring, once drained).
 // More than 16 rows (a batch of modulation vectors) run as blocks of 16 rows
@@ -47,13 +52,13 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_
 // bf16 (128 + q) for the two nibbles at bits [0, 4) and [16, 20) of w.
 __device__ __forceinline__ uint32_t nib_pair(uint32_t w) { return (w & 0x000F000Fu) | 0x43004300u; }
 
-// The 4 A fragments (16 columns x 16 k) of k16-step word w: (128 + q) as bf16.
-__device__ __forceinline__ void a_frags(uint32_t w, uint32_t (&a)[4]) {
-  a[0] = nib_pair(w);         // column g,   k 2t, 2t+1
-  a[1] = nib_pair(w >> 4);    // column g+8, k 2t, 2t+1
-  a[2] = nib_pair(w >> 8);    // column g,   k 2t+8, 2t+9
-  a[3] = nib_pair(w >> 12);   // column g+8, k 2t+8, 2t+9
+// (q - z) as bf16 pairs, exact: (128 + q) - (128 + z) for the two nibbles of nib_pair(w).
+__device__ __forceinline__ uint32_t minus_zero(uint32_t a128, uint32_t z128) {
+  __nv_bfloat162 d = __hsub2(*reinterpret_cast<__nv_bfloat162 *>(&a128), *reinterpret_cast<__nv_bfloat162 *>(&z128));
+  return *reinterpret_cast<uint32_t *>(&d);
 }
+// bf16 1.0 in both halves: the all-ones A fragment that sums B over k
+constexpr uint32_t kOnes = 0x3F803F80u;
 
 struct Params {
   int M, K, N, ldx, ldy, G;
@@ -75,8 +80,9 @@ struct XRaw {
   uint32_t w[4][NT][2];
   float2 iv[4][2];
 };
-template <int NT>
-__device__ __forceinline__ void fetch_x(const Params &p, int k0, int g8, int j0, int j1, XRaw<NT> &r) {
+// row(nt): the row of X whose words lane slot nt carries (rows past M read as zeros).
+template <int NT, typename RowOf>
+__device__ __forceinline__ void fetch_x(const Params &p, int k0, RowOf row, int j0, int j1, XRaw<NT> &r) {
 #pragma unroll
   for (int j = j0; j < j1; ++j) {
     const int k = k0 + 16 * j;
@@ -84,7 +90,7 @@ __device__ __forceinline__ void fetch_x(const Params &p, int k0, int g8, int j0,
     r.iv[j][1] = p.inv ? __ldg(reinterpret_cast<const float2 *>(p.inv + k + 8)) : make_float2(1.f, 1.f);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const int m = nt * 8 + g8;
+      const int m = row(nt);
       r.w[j][nt][0] = m < p.M ? __ldg(reinterpret_cast<const uint32_t *>(p.X + static_cast<size_t>(m) * p.ldx + k)) : 0u;
       r.w[j][nt][1] =
           m < p.M ? __ldg(reinterpret_cast<const uint32_t *>(p.X + static_cast<size_t>(m) * p.ldx + k + 8)) : 0u;
@@ -115,13 +121,23 @@ __device__ __forceinline__ void split_x(const XRaw<NT> &r, int j, uint32_t (&bh)
   }
 }
 
-// (q - z) for the two nibbles at bits [s, s+4) and [s+16, s+20) of w, as bf16x2.
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t w, int s, uint32_t z128) {
-  uint32_t t = nib_pair(w >> s);
-  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&t);
-  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&z128);
-  __nv_bfloat162 d = __hsub2(a, b);
-  return *reinterpret_cast<uint32_t *>(&d);
+// B fragments of k16 step j with the hi and lo parts in one MMA (up to 4
+// rows): lane (g, t) carries part g >> 2 (0: hi, 1: lo) of row g & 3, so n
+// slots 0..3 hold the rows' hi parts and 4..7 their lo parts.  lo_sel is 0
+// on hi lanes and -1 on lo lanes: x^ + lo_sel f32(bf16(x^)) is x^ itself or
+// the exact remainder x^ - hi, then rounded to bf16 like the hi part.
+__device__ __forceinline__ void split_x_merged(const XRaw<1> &r, int j, float lo_sel, uint32_t (&b)[2]) {
+  const uint32_t w0 = r.w[j][0][0], w1 = r.w[j][0][1];
+  const float2 x01 = dev::mul2_rn(make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u)),
+                                  r.iv[j][0]);
+  const float2 x23 = dev::mul2_rn(make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u)),
+                                  r.iv[j][1]);
+  const uint32_t h01 = pack_bf16x2(x01.x, x01.y), h23 = pack_bf16x2(x23.x, x23.y);
+  const float2 sel = make_float2(lo_sel, lo_sel);
+  const float2 v01 = dev::fma2_rn(make_float2(bf16_bits_to_float(h01 & 0xFFFFu), bf16_bits_to_float(h01 >> 16)), sel, x01);
+  const float2 v23 = dev::fma2_rn(make_float2(bf16_bits_to_float(h23 & 0xFFFFu), bf16_bits_to_float(h23 >> 16)), sel, x23);
+  b[0] = pack_bf16x2(v01.x, v01.y);
+  b[1] = pack_bf16x2(v23.x, v23.y);
 }
 
 // ===========================================================================
@@ -137,7 +153,8 @@ constexpr int BAR_OFF = RING * CHUNK_BYTES;
 constexpr int SMEM_BYTES = BAR_OFF + 2 * RING * 8 + 16;
 static_assert(S_WARPS * 4 * 2 * 32 * 4 * 4 <= BAR_OFF, "the partial sums fit the drained ring");
 
-template <int NT>
+// MERGED: up to 4 rows, the hi and lo parts of X^ in one MMA (NT = 1).
+template <int NT, bool MERGED>
 __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);
@@ -188,6 +205,13 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) tot[a][b][e] = 0.0f;
 
+  static_assert(!MERGED || NT == 1, "the merged form carries one block of 4 rows");
+  constexpr bool FOLD = NT == 1;
+  // the row of X a lane's B slot nt carries
+  auto row_of = [&](int nt) { return MERGED ? (g8 & 3) : nt * 8 + g8; };
+  const float lo_sel = MERGED && g8 >= 4 ? -1.0f : 0.0f;
+  const uint32_t ones[4] = {kOnes, kOnes, kOnes, kOnes};
+
 #pragma unroll 1
   for (int c = 0; c < nchunks; ++c) {
     const int slot = c % RING;
@@ -195,7 +219,7 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
     XRaw<NT> xr;
     // one row block (the modulation layers): all four steps' X up front; two row blocks would
     // hold twice the registers, so those fetch each step's X where it is used
-    if (NT == 1 && grp < p.G) fetch_x<NT>(p, grp * 64 + 2 * t, g8, 0, 4, xr);
+    if (NT == 1 && grp < p.G) fetch_x<NT>(p, grp * 64 + 2 * t, row_of, 0, 4, xr);
     if (!dev::mbar_wait_warp(&full[slot], (c / RING) & 1, p.limit_ns, abort_flag)) {
       *abort_flag = 1;
       dev::report(p.status, SVDQ_ERR_TIMEOUT);
@@ -204,7 +228,7 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
     if (grp < p.G) {
       const uint8_t *src = smem + slot * CHUNK_BYTES;
       uint4 wq[4];
-      uint32_t sp[4], zp[4];  // bf16 of columns g (low half) and g + 8 (high half) of each block
+      uint32_t sp[4], zp[4];  // bf16 s and z of columns g (low half) and g + 8 (high half) of each block
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
         wq[cb] = reinterpret_cast<const uint4 *>(src + warp * 2048)[cb * 32 + lane];
@@ -213,50 +237,71 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
         sp[cb] = static_cast<uint32_t>(sc[0]) | (static_cast<uint32_t>(sc[8]) << 16);
         zp[cb] = static_cast<uint32_t>(zc[0]) | (static_cast<uint32_t>(zc[8]) << 16);
       }
-      uint32_t z_lo[4], z_hi[4];
+      // one row block (FOLD): acc = sum_k (128 + q) b and sx = sum_k b over the group's 64 k, and
+      // sum_k (q - z) b = acc - (128 + z) sx, taken once per group in f32; two row blocks
+      // (registers for sx would spill) subtract 128 + z from every pair instead
+      uint32_t z128[4][2];
+      if constexpr (!FOLD) {
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        const float zl = bf16_bits_to_float(zp[cb] & 0xFFFFu), zh = bf16_bits_to_float(zp[cb] >> 16);
-        z_lo[cb] = pack_bf16x2(128.0f + zl, 128.0f + zl);
-        z_hi[cb] = pack_bf16x2(128.0f + zh, 128.0f + zh);
+        for (int cb = 0; cb < 4; ++cb) {
+          const float zl = 128.0f + bf16_bits_to_float(zp[cb] & 0xFFFFu), zh = 128.0f + bf16_bits_to_float(zp[cb] >> 16);
+          z128[cb][0] = pack_bf16x2(zl, zl);
+          z128[cb][1] = pack_bf16x2(zh, zh);
+        }
       }
-      float acc[4][NT][4];
+      float acc[4][NT][4], sx[NT][4];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int b = 0; b < NT; ++b)
 #pragma unroll
-        for (int b = 0; b < NT; ++b)
+        for (int e = 0; e < 4; ++e) {
+          sx[b][e] = 0.0f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.0f;
+          for (int a = 0; a < 4; ++a) acc[a][b][e] = 0.0f;
+        }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t bh[NT][2], bl[NT][2];
-        if (NT > 1) fetch_x<NT>(p, grp * 64 + 2 * t, g8, j, j + 1, xr);
-        split_x<NT>(xr, j, bh, bl);
+        if constexpr (MERGED) {
+          split_x_merged(xr, j, lo_sel, bh[0]);
+        } else {
+          if (NT > 1) fetch_x<NT>(p, grp * 64 + 2 * t, row_of, j, j + 1, xr);
+          split_x<NT>(xr, j, bh, bl);
+        }
+        if constexpr (FOLD) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            dev::mma_bf16_16816(sx[nt], ones, bh[nt][0], bh[nt][1]);
+            if (!MERGED) dev::mma_bf16_16816(sx[nt], ones, bl[nt][0], bl[nt][1]);
+          }
+        }
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
           const uint32_t w = j == 0 ? wq[cb].x : j == 1 ? wq[cb].y : j == 2 ? wq[cb].z : wq[cb].w;
-          uint32_t a[4];
-          a[0] = dequant_pair(w, 0, z_lo[cb]);
-          a[1] = dequant_pair(w, 4, z_hi[cb]);
-          a[2] = dequant_pair(w, 8, z_lo[cb]);
-          a[3] = dequant_pair(w, 12, z_hi[cb]);
+          // (128 + q) as bf16 pairs: columns g / g + 8 at k 2t, 2t+1 (a0 / a1) and 2t+8, 2t+9 (a2 / a3)
+          uint32_t a[4] = {nib_pair(w), nib_pair(w >> 4), nib_pair(w >> 8), nib_pair(w >> 12)};
+          if constexpr (!FOLD) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = minus_zero(a[i], z128[cb][i & 1]);
+          }
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             dev::mma_bf16_16816(acc[cb][nt], a, bh[nt][0], bh[nt][1]);
-            dev::mma_bf16_16816(acc[cb][nt], a, bl[nt][0], bl[nt][1]);
+            if (!MERGED) dev::mma_bf16_16816(acc[cb][nt], a, bl[nt][0], bl[nt][1]);
           }
         }
       }
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
+        // C rows g (e < 2) and g + 8 (e >= 2) are the block's columns g and g + 8
         const float s_lo = bf16_bits_to_float(sp[cb] & 0xFFFFu), s_hi = bf16_bits_to_float(sp[cb] >> 16);
+        const float z_lo = 128.0f + bf16_bits_to_float(zp[cb] & 0xFFFFu), z_hi = 128.0f + bf16_bits_to_float(zp[cb] >> 16);
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          tot[cb][nt][0] = __fmaf_rn(s_lo, acc[cb][nt][0], tot[cb][nt][0]);
-          tot[cb][nt][1] = __fmaf_rn(s_lo, acc[cb][nt][1], tot[cb][nt][1]);
-          tot[cb][nt][2] = __fmaf_rn(s_hi, acc[cb][nt][2], tot[cb][nt][2]);
-          tot[cb][nt][3] = __fmaf_rn(s_hi, acc[cb][nt][3], tot[cb][nt][3]);
-        }
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            tot[cb][nt][e] = __fmaf_rn(
+                e < 2 ? s_lo : s_hi,
+                FOLD ? __fmaf_rn(-(e < 2 ? z_lo : z_hi), sx[nt][e], acc[cb][nt][e]) : acc[cb][nt][e], tot[cb][nt][e]);
       }
     }
     __syncwarp();
@@ -277,6 +322,13 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
       dev::mbar_wait(&full[c % RING], (c / RING) & 1, p.limit_ns, nullptr);
   __syncthreads();
 
+  if constexpr (MERGED) {
+    // n slots 4..7 (lanes t = 2, 3) hold the lo parts of the rows in slots 0..3 (lanes t = 0, 1)
+#pragma unroll
+    for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tot[cb][0][e] += __shfl_xor_sync(0xFFFFFFFFu, tot[cb][0][e], 2);
+  }
   float *red = reinterpret_cast<float *>(smem);  // [WARPS][4][NT][32][4]
 #pragma unroll
   for (int cb = 0; cb < 4; ++cb)
@@ -303,12 +355,12 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
   }
 }
 
-template <int NT>
+template <int NT, bool MERGED>
 int launch(const Params &p, cudaStream_t stream) {
-  const int rc = smem_optin_once<awq_gemv_kernel<NT>>(SMEM_BYTES, "awq_linear_w4a16");
+  const int rc = smem_optin_once<awq_gemv_kernel<NT, MERGED>>(SMEM_BYTES, "awq_linear_w4a16");
   if (rc != SVDQ_OK) return rc;
   DependentLaunch dl(dim3(p.N / 64, (p.M + 8 * NT - 1) / (8 * NT)), dim3(S_THREADS), SMEM_BYTES, stream);
-  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT>, p);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT, MERGED>, p);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16 launch: ") + cudaGetErrorString(e));
   return ok();
@@ -352,6 +404,8 @@ extern "C" int awq_linear_w4a16(const void *X, int M, int K, int ldx, const floa
   p.Y = static_cast<uint16_t *>(Y);
   p.status = st->status_word;
   p.limit_ns = kWaitLimitNs;
-  // up to 8 rows: one block of rows; more: blocks of 16 rows, one pass over the weights each
-  return M > 8 ? launch<2>(p, s) : launch<1>(p, s);
+  // up to 4 rows: hi and lo parts in one MMA; up to 8: one block of rows; more: blocks of 16
+  // rows, one pass over the weights each
+  if (M <= 4) return launch<1, true>(p, s);
+  return M > 8 ? launch<2, false>(p, s) : launch<1, false>(p, s);
 }

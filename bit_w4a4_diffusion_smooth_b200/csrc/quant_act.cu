@@ -15,28 +15,27 @@
 //     [r x 256] tile of L1^T (one 3-D TMA copy each, as four 64-column boxes
 //     with the 128-byte swizzle), the stage's 256-float slice of inv_lambda
 //     (a bulk copy) and a staging area for the stage's codes and scales;
-//   * compute warp w owns the 16-column slice w of every stage for all 32
-//     rows.  It loads the slice once, with ldmatrix, straight into the
-//     m16n8k16 A-fragment layout: lane (g, t) holds columns 2t, 2t+1, 2t+8,
-//     2t+9 of rows g + 8q, q = 0..3, i.e. a quarter of four 16-element blocks;
-//   * from those registers: x^ = x * inv_lambda, the bf16 A fragments of the
-//     down-projection (mma.sync into r/2 independent accumulators per lane),
-//     and the block maxima, reduced over the 4 lanes of a row group by a
-//     butterfly that leaves each lane owning one whole block.  That lane
-//     takes the f32 division for the block scale and looks 1/scale up in a
-//     per-CTA table of all 128 scale codes (the tensor scale is fixed per
-//     call, so f32(1 / f32(e4m3 * s_a)) has only 128 values); the four
-//     1/scale values come back by shuffles, every lane converts its 16
-//     elements, and a second butterfly gathers each block's 8 code bytes in
-//     its owner lane, which puts them (and the scale byte) into the staging
-//     area in the bundle's byte order;
+//   * compute warp w owns rows 16 (w >> 3) .. +15 and the 32-column slice
+//     w & 7 of every stage; lane l of it owns one whole 16-element block
+//     (row 16 (w >> 3) + (l & 15), block l >> 4 of the slice), read as two
+//     16-byte chunks of the swizzled box.  The lane alone forms x^ = x *
+//     inv_lambda, the block maximum, the f32 division for the block scale,
+//     1/scale from a per-CTA table of all 128 scale codes (the tensor scale
+//     is fixed per call, so f32(1 / f32(e4m3 * s_a)) has only 128 values)
+//     and the block's 8 code bytes, which it puts (with the scale byte)
+//     into the staging area in the bundle's byte order: no shuffles;
+//   * the lane writes bf16(x^) back over its x; the warp then loads its
+//     16 x 32 tile of it with ldmatrix as m16n8k16 A fragments for the
+//     down-projection (mma.sync into r/8 accumulators per lane, B = L1^T
+//     rows by ldmatrix);
 //   * the store warp copies each staged stage out with full-line stores (a
 //     CTA's code rows are 4 KB of contiguous bundle) and frees the stage;
 //   * warps never meet inside the loop: each waits for its stage with a
 //     bounded mbarrier wait (decided warp-uniformly; a warp whose wait runs
 //     out records SVDQ_ERR_TIMEOUT and leaves the loop) and signals the store
-//     warp with one arrive.  At the end the 16 per-slice partial U tiles are added in
-//     shared memory and written as 128-row swizzled tiles.
+//     warp with one arrive.  At the end the 8 per-slice partial U tiles of
+//     each 16-row half are added in shared memory and written as 128-row
+//     swizzled tiles.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -51,7 +50,7 @@ namespace {
 
 constexpr int BM = 32;             // rows per CTA
 constexpr int KC = kStageK;        // columns per stage (one bundle k-stage)
-constexpr int CWARPS = 16;         // compute warps: one 16-column slice each
+constexpr int CWARPS = 16;         // compute warps: 16 rows x one 32-column slice each
 constexpr int THREADS = (CWARPS + 2) * 32;   // + TMA warp + store warp
 constexpr int X_BOX = BM * 128;    // one [32 x 64] bf16 box, 128-byte rows
 constexpr int X_STAGE = 4 * X_BOX;
@@ -94,7 +93,7 @@ __host__ __device__ constexpr int smem_bytes() {
   return 1024 + num_stages<RANK>() * stage_bytes<RANK>() + 128 * 4 + 512;
 }
 // the per-slice partial U tiles reuse the ring at the end
-static_assert(CWARPS * BM * (64 + 4) * 4 <= num_stages<64>() * stage_bytes<64>(), "partials must fit the ring");
+static_assert(CWARPS * 16 * (64 + 4) * 4 <= num_stages<64>() * stage_bytes<64>(), "partials must fit the ring");
 
 // Byte offset of the 16-byte chunk holding column c (0..63, multiple of 8) of
 // row r inside a 128-byte-swizzled box of 128-byte rows.
@@ -106,11 +105,6 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
-}
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
 }
 __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
@@ -229,33 +223,30 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   // -------------------------------------------------------------- compute warps
-  const int g = lane >> 2, t = lane & 3;
-  const int bx = warp >> 2;                     // 64-column box of this warp's slice
-  const int kc = (warp & 3) * 16;               // slice offset inside the box
-  const bool o1 = (t & 1) != 0, o2 = (t & 2) != 0;
-  // the block this lane owns after the butterflies: rows g + 8 q, q = 2 o1 + o2
-  const int row_own = 8 * (2 * (t & 1) + ((t >> 1) & 1)) + g;
-  // staged like the bundle tile: code chunk (warp >> 1) of the row, 128-byte swizzle on the row
-  // inside the 128-row tile (m0 is a multiple of 32, so that row and row_own agree mod 8)
-  const uint32_t code_off =
-      static_cast<uint32_t>(CODE_OFF + row_own * 128 + ((((warp >> 1) ^ row_own) & 7) << 4) + 8 * (warp & 1));
-  const uint32_t scale_off = static_cast<uint32_t>(SC_OFF + (bx * 32 + row_own) * 4 + (warp & 3));
+  // warp w: rows 16 (w >> 3) .. +15 of the CTA and the 32-column slice w & 7 of every stage;
+  // lane l: row 16 (w >> 3) + (l & 15) and the 16-column block l >> 4 of that slice, which it
+  // quantizes on its own
+  const int rh = warp >> 3, cs = warp & 7;
+  const int bx = cs >> 1;                                   // 64-column box of the slice
+  const int row = 16 * rh + (lane & 15), blk = lane >> 4;
+  const int col = 32 * (cs & 1) + 16 * blk;                 // the block's first column inside the box
+  const uint32_t x_off0 = sw_off(row, col), x_off1 = sw_off(row, col + 8);
+  // staged like the bundle tile: 16-byte code chunk cs of the row, half blk; scale byte 2 cs + blk
+  // of the row's 16 (m0 is a multiple of 32, so row and the bundle row agree mod 8)
+  const uint32_t code_off = static_cast<uint32_t>(CODE_OFF + row * 128 + (((cs ^ row) & 7) << 4) + 8 * blk);
+  const uint32_t scale_off = static_cast<uint32_t>(SC_OFF + (bx * 32 + row) * 4 + ((2 * cs + blk) & 3));
   const float d6 = __fmul_rn(6.0f, s_a);
-  // ldmatrix lane addresses: A rows (per 16-row half), B rows of L1^T (per pair of 8-column tiles)
-  const uint32_t a_off0 = sw_off((lane & 7) + ((lane >> 3) & 1) * 8, kc + (lane >> 4) * 8);
-  const uint32_t a_off1 = sw_off(16 + (lane & 7) + ((lane >> 3) & 1) * 8, kc + (lane >> 4) * 8);
-  const int lsrc = lane & ~3;
-  // prmt selectors of the code-byte gather (they depend on the lane's parity bits)
-  const uint32_t sel_a = o1 ? 0x1504u : 0x5140u, sel_b = o1 ? 0x3726u : 0x7362u;
-  const uint32_t sel_w0 = o2 ? 0x1054u : 0x5410u, sel_w1 = o2 ? 0x3276u : 0x7632u;
+  // ldmatrix lane addresses of the down-projection: A = the warp's 16 rows of bf16(x^) (written
+  // back in place), B = rows of L1^T (per pair of 8-column tiles), each per k16 step kk
+  const int arow = 16 * rh + (lane & 15);
+  const int acol = 32 * (cs & 1) + 8 * (lane >> 4);
+  const int brow = (lane >> 4) * 8 + (lane & 7), bcol = 32 * (cs & 1) + ((lane >> 3) & 1) * 8;
 
-  float acc[2][NT > 0 ? NT : 1][4];
+  float acc[NT > 0 ? NT : 1][4];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int n = 0; n < (NT > 0 ? NT : 1); ++n)
 #pragma unroll
-    for (int n = 0; n < (NT > 0 ? NT : 1); ++n)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[mt][n][i] = 0.0f;
+    for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
   bool failed = false;
 
   for (int c = 0; c < p.KS; ++c) {
@@ -268,129 +259,101 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     const int nbox = min(4, (p.K - c * KC) / 64);
     uint8_t *st = smem + s * STAGE;
-    // x^ of the lane's 16 elements: xs[q][0..3] = row g + 8q, columns 2t, 2t+1, 2t+8, 2t+9
-    float xs[4][4];
-    if (bx < nbox) {
-      const uint32_t xbase = dev::smem_u32(st + bx * X_BOX);
-      uint32_t a0[4], a1[4];
-      dev::ldmatrix_x4(xbase + a_off0, a0[0], a0[1], a0[2], a0[3]);
-      dev::ldmatrix_x4(xbase + a_off1, a1[0], a1[1], a1[2], a1[3]);
-      const float *iv = reinterpret_cast<const float *>(st + INV_OFF) + bx * 64 + kc + 2 * t;
-      const float2 i0 = *reinterpret_cast<const float2 *>(iv);
-      const float2 i1 = *reinterpret_cast<const float2 *>(iv + 8);
-      // fragment register h of half mt: rows g (h even) / g + 8 (h odd), columns 2t.. (h < 2) / 2t+8.. (h >= 2)
+    uint32_t sb = 0, code0 = 0, code1 = 0;
+    if (bx < nbox) {   // warp-uniform: columns past K quantize as zeros (code and scale 0)
+      uint8_t *xb = st + bx * X_BOX;
+      const uint4 w0 = *reinterpret_cast<const uint4 *>(xb + x_off0);
+      const uint4 w1 = *reinterpret_cast<const uint4 *>(xb + x_off1);
+      const float4 *iv = reinterpret_cast<const float4 *>(st + INV_OFF) + (bx * 64 + col) / 4;
+      const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      // x^ of the block's 16 elements, in column order
+      float xs[16];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t lo = (q >> 1) ? a1[q & 1] : a0[q & 1];
-        const uint32_t hi = (q >> 1) ? a1[2 + (q & 1)] : a0[2 + (q & 1)];
-        const float2 p0 = dev::mul2_rn(make_float2(bf16_lo(lo), bf16_hi(lo)), i0);
-        const float2 p1 = dev::mul2_rn(make_float2(bf16_lo(hi), bf16_hi(hi)), i1);
-        xs[q][0] = p0.x;
-        xs[q][1] = p0.y;
-        xs[q][2] = p1.x;
-        xs[q][3] = p1.y;
+      for (int i = 0; i < 4; ++i) {
+        const float4 v = iv[i];
+        const float2 p0 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i]), bf16_hi(wv[2 * i])), make_float2(v.x, v.y));
+        const float2 p1 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i + 1]), bf16_hi(wv[2 * i + 1])), make_float2(v.z, v.w));
+        xs[4 * i] = p0.x;
+        xs[4 * i + 1] = p0.y;
+        xs[4 * i + 2] = p1.x;
+        xs[4 * i + 3] = p1.y;
       }
-      if (RANK > 0) {
-        // down-projection of this slice: A = bf16(x^), B = L1^T rows (ldmatrix of 2 tiles x 2 k-halves)
-        uint32_t af[2][4];
+      float amax = absmax4(xs[0], xs[1], xs[2], xs[3]);
+      amax = fmaxf(amax, absmax4(xs[4], xs[5], xs[6], xs[7]));
+      amax = fmaxf(amax, absmax4(xs[8], xs[9], xs[10], xs[11]));
+      amax = fmaxf(amax, absmax4(xs[12], xs[13], xs[14], xs[15]));
+      sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
+      const float rinv = rinv_tab[sb];
+      const float2 r2 = make_float2(rinv, rinv);
+      uint32_t cw[4];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          af[mt][0] = bf16x2(xs[2 * mt][0], xs[2 * mt][1]);
-          af[mt][1] = bf16x2(xs[2 * mt + 1][0], xs[2 * mt + 1][1]);
-          af[mt][2] = bf16x2(xs[2 * mt][2], xs[2 * mt][3]);
-          af[mt][3] = bf16x2(xs[2 * mt + 1][2], xs[2 * mt + 1][3]);
-        }
+      for (int i = 0; i < 4; ++i) {
+        const float2 c0 = dev::mul2_rn(make_float2(xs[4 * i], xs[4 * i + 1]), r2);
+        const float2 c1 = dev::mul2_rn(make_float2(xs[4 * i + 2], xs[4 * i + 3]), r2);
+        cw[i] = dev::cvt_e2m1x4(c0.x, c0.y, c1.x, c1.y);     // code bytes 2i, 2i + 1
+      }
+      code0 = cw[0] | (cw[1] << 16);
+      code1 = cw[2] | (cw[3] << 16);
+      if (RANK > 0) {
+        // bf16(x^) back in place of x, as the A operand of the down-projection
+        *reinterpret_cast<uint4 *>(xb + x_off0) =
+            make_uint4(bf16x2(xs[0], xs[1]), bf16x2(xs[2], xs[3]), bf16x2(xs[4], xs[5]), bf16x2(xs[6], xs[7]));
+        *reinterpret_cast<uint4 *>(xb + x_off1) =
+            make_uint4(bf16x2(xs[8], xs[9]), bf16x2(xs[10], xs[11]), bf16x2(xs[12], xs[13]), bf16x2(xs[14], xs[15]));
+        __syncwarp();
+        const uint32_t xbase = dev::smem_u32(xb);
         const uint32_t lbase = dev::smem_u32(st + X_STAGE + bx * L1_BOX);
 #pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-          uint32_t b[4];
-          dev::ldmatrix_x4(lbase + sw_off(np * 16 + (lane >> 4) * 8 + (lane & 7), kc + ((lane >> 3) & 1) * 8), b[0],
-                           b[1], b[2], b[3]);
+        for (int kk = 0; kk < 2; ++kk) {
+          uint32_t af[4];
+          dev::ldmatrix_x4(xbase + sw_off(arow, acol + 16 * kk), af[0], af[1], af[2], af[3]);
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            dev::mma_bf16_16816(acc[mt][2 * np], af[mt], b[0], b[1]);
-            dev::mma_bf16_16816(acc[mt][2 * np + 1], af[mt], b[2], b[3]);
+          for (int np = 0; np < NT / 2; ++np) {
+            uint32_t bq[4];
+            dev::ldmatrix_x4(lbase + sw_off(np * 16 + brow, bcol + 16 * kk), bq[0], bq[1], bq[2], bq[3]);
+            dev::mma_bf16_16816(acc[2 * np], af, bq[0], bq[1]);
+            dev::mma_bf16_16816(acc[2 * np + 1], af, bq[2], bq[3]);
           }
         }
       }
-    } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xs[q][i] = 0.0f;   // columns past K quantize as zeros
     }
-
-    // block maxima: lane partials, then a butterfly over the row group's 4 lanes
-    const float m0q = absmax4(xs[0][0], xs[0][1], xs[0][2], xs[0][3]);
-    const float m1q = absmax4(xs[1][0], xs[1][1], xs[1][2], xs[1][3]);
-    const float m2q = absmax4(xs[2][0], xs[2][1], xs[2][2], xs[2][3]);
-    const float m3q = absmax4(xs[3][0], xs[3][1], xs[3][2], xs[3][3]);
-    float ka = o1 ? m2q : m0q, kb = o1 ? m3q : m1q;       // keep blocks {2 o1, 2 o1 + 1}
-    ka = fmaxf(ka, __shfl_xor_sync(0xFFFFFFFFu, o1 ? m0q : m2q, 1));
-    kb = fmaxf(kb, __shfl_xor_sync(0xFFFFFFFFu, o1 ? m1q : m3q, 1));
-    const float amax = fmaxf(o2 ? kb : ka, __shfl_xor_sync(0xFFFFFFFFu, o2 ? ka : kb, 2));   // block 2 o1 + o2
-    const uint32_t sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
-    const float rown = rinv_tab[sb];
-    // 1/scale of blocks 0..3 from their owners (lanes t = 0, 2, 1, 3)
-    float rq[4];
-    rq[0] = __shfl_sync(0xFFFFFFFFu, rown, lsrc);
-    rq[1] = __shfl_sync(0xFFFFFFFFu, rown, lsrc + 2);
-    rq[2] = __shfl_sync(0xFFFFFFFFu, rown, lsrc + 1);
-    rq[3] = __shfl_sync(0xFFFFFFFFu, rown, lsrc + 3);
-    // code bytes t (columns 2t, 2t+1) and t + 4 (columns 2t+8, 2t+9) of each block
-    uint32_t cq[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-    {
-      const float2 r2 = make_float2(rq[q], rq[q]);
-      const float2 c0 = dev::mul2_rn(make_float2(xs[q][0], xs[q][1]), r2);
-      const float2 c1 = dev::mul2_rn(make_float2(xs[q][2], xs[q][3]), r2);
-      cq[q] = dev::cvt_e2m1x4(c0.x, c0.y, c1.x, c1.y);
-    }
-    // gather: after the xor-1 step a lane holds bytes {e, e+1, e+4, e+5} (e = t & 2) of its
-    // two kept blocks, after the xor-2 step all 8 bytes of the block it owns
-    const uint32_t keep = o1 ? (cq[2] | (cq[3] << 16)) : (cq[0] | (cq[1] << 16));
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, o1 ? (cq[0] | (cq[1] << 16)) : (cq[2] | (cq[3] << 16)), 1);
-    const uint32_t da = prmt(keep, recv, sel_a), db = prmt(keep, recv, sel_b);
-    const uint32_t mine = o2 ? db : da;
-    const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, o2 ? da : db, 2);
-    *reinterpret_cast<uint2 *>(st + code_off) = make_uint2(prmt(mine, other, sel_w0), prmt(mine, other, sel_w1));
+    *reinterpret_cast<uint2 *>(st + code_off) = make_uint2(code0, code1);
     st[scale_off] = static_cast<uint8_t>(sb);
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(&done[s]);
   }
 
-  // ---- U = (sum of the 16 slices' partial products) / (s_a s_w), bf16, 128-row tiles
+  // ---- U = (sum of the 8 slices' partial products of each row half) / (s_a s_w), bf16, 128-row tiles
   const int tid = threadIdx.x;  // 0..511
   constexpr int RS = RANK + 4;   // padded row of a partial tile
+  constexpr int SLICES = CWARPS / 2;
   if (RANK > 0) {
     dev::named_barrier(1, (CWARPS + 1) * 32);      // the ring is no longer read (store warp included)
-    float *red = reinterpret_cast<float *>(smem) + warp * BM * RS;   // [CWARPS][BM][RS]
+    float *red = reinterpret_cast<float *>(smem) + warp * 16 * RS;   // [CWARPS][16][RS]
     if (!failed) {
+      const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int n = 0; n < (NT > 0 ? NT : 1); ++n) {
-          const int row = mt * 16 + g, col = n * 8 + 2 * t;
-          *reinterpret_cast<float2 *>(red + row * RS + col) = make_float2(acc[mt][n][0], acc[mt][n][1]);
-          *reinterpret_cast<float2 *>(red + (row + 8) * RS + col) = make_float2(acc[mt][n][2], acc[mt][n][3]);
-        }
+      for (int n = 0; n < (NT > 0 ? NT : 1); ++n) {
+        const int cc = n * 8 + 2 * t;
+        *reinterpret_cast<float2 *>(red + g * RS + cc) = make_float2(acc[n][0], acc[n][1]);
+        *reinterpret_cast<float2 *>(red + (g + 8) * RS + cc) = make_float2(acc[n][2], acc[n][3]);
+      }
     }
     dev::named_barrier(2, CWARPS * 32);
   }
   // a wait that ran out anywhere leaves U zero (the status word carries the error)
   const bool any_failed = RANK > 0 && *abort_flag != 0;
   const float alpha = __fmul_rn(s_a, __ldg(p.s_w));
-  // every thread: column pairs (2 cp, 2 cp + 1) of the CTA's rows, the 16 partials added in order
+  // every thread: column pairs (2 cp, 2 cp + 1) of the CTA's rows, the slices' partials added in order
   for (int idx = tid; idx < BM * (SVDQ_LR_STRIDE / 2); idx += CWARPS * 32) {
     const int rr = idx / (SVDQ_LR_STRIDE / 2), cp = idx % (SVDQ_LR_STRIDE / 2);
     uint32_t o = 0;
     if (RANK > 0 && 2 * cp < RANK && !any_failed) {
-      const float *red = reinterpret_cast<const float *>(smem) + rr * RS + 2 * cp;
+      const float *red = reinterpret_cast<const float *>(smem) + ((rr >> 4) * SLICES * 16 + (rr & 15)) * RS + 2 * cp;
       float2 sum = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int w = 0; w < CWARPS; ++w) {
-        const float2 v = *reinterpret_cast<const float2 *>(red + w * BM * RS);
+      for (int w = 0; w < SLICES; ++w) {
+        const float2 v = *reinterpret_cast<const float2 *>(red + w * 16 * RS);
         sum.x += v.x;
         sum.y += v.y;
       }

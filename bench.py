@@ -49,6 +49,7 @@ LAYERS = {"qkv": (TOKENS, HIDDEN, 3 * HIDDEN, False),
           "fc1": (TOKENS, HIDDEN, MLP, True),
           "fc2": (TOKENS, MLP, HIDDEN, False)}
 AM, AK, AN = 2, HIDDEN, 6 * HIDDEN
+MIN_SETS = 6                   # rotating buffer sets: 6 x 32 MB (the AWQ weights) > 1.5 x L2
 WORKLOAD = ("one 12B-class DiT block's SVDQ W4A4 linears at 4608 tokens, rank 32 (NVFP4, group 16): "
             "QKV 3072->9216, MLP fc1 3072->12288 +GELU then fc2 12288->3072 on fc1's output; "
             "+ AWQ W4A16 adaLN projection 2x3072->18432 (INT4, group 64)")
@@ -392,6 +393,22 @@ class L2Flush:
         torch.sum(self.buf, dim=0, dtype=torch.int64, out=self.out)
 
 
+def time_back_to_back(fn, sets, reps, barrier):
+    """Mean device time (ms) per launch of `fn` launched `reps` times back to back over the rotating
+    sets, with one event before the first launch and one after the last."""
+    import torch
+    for i in range(2):
+        fn(sets[i % len(sets)])
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        fn(sets[i % len(sets)])
+    b.record()
+    barrier()
+    return a.elapsed_time(b) / reps
+
+
 def time_cold(fn, sets, reps, flush):
     """Mean device time (ms) of one launch of `fn` with L2 flushed before it: each launch sits alone
     between two events on the stream, after a read of twice the L2 size."""
@@ -495,7 +512,9 @@ def run_ours(args):
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     W = Workload(device)
     set_bytes = W.add_set()
-    while len(W.sets) < 2 or len(W.sets) * set_bytes < 2 * l2:
+    # enough sets that a kernel run back to back over them (the smallest one touches ~32 MB of a
+    # set) finds its data evicted from L2 each time, as it does inside the step
+    while len(W.sets) < MIN_SETS or len(W.sets) * set_bytes < 2 * l2:
         W.add_set()
     sets = W.sets
 
@@ -541,6 +560,10 @@ def run_ours(args):
     barrier()
     live = {label: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(skip, skip + nb)) / nb
             for j, (label, _) in enumerate(kernels)}
+    # ---- each kernel back to back: its launches over the rotating sets between two events and none
+    # in between, so consecutive launches keep their overlap as in the step; these per-kernel times
+    # add up to about the step time
+    b2b = {label: time_back_to_back(fn, sets, max(8, min(args.steps, 50)), barrier) for label, fn in kernels}
     # ---- each kernel alone after an L2 flush; the clock sampler keeps running under this load
     flush = L2Flush(device)
     per = {label: time_cold(fn, sets, args.kernel_reps, flush) for label, fn in kernels}
@@ -607,11 +630,13 @@ def run_ours(args):
     labels = [label for label, _ in kernels]
     xlabels = [label for label, _ in other]
     vals = max_over_ranks([ms, e2e_ms] + [per[x] for x in labels] + [extra[x] for x in xlabels]
-                          + [live[x] for x in labels], world, device)
+                          + [live[x] for x in labels] + [b2b[x] for x in labels], world, device)
     ms, e2e_ms = vals[0], vals[1]
-    per = dict(zip(labels, vals[2:2 + len(labels)]))
-    extra = dict(zip(xlabels, vals[2 + len(labels):2 + len(labels) + len(xlabels)]))
-    live = dict(zip(labels, vals[2 + len(labels) + len(xlabels):]))
+    nl, nx = len(labels), len(xlabels)
+    per = dict(zip(labels, vals[2:2 + nl]))
+    extra = dict(zip(xlabels, vals[2 + nl:2 + nl + nx]))
+    live = dict(zip(labels, vals[2 + nl + nx:2 + 2 * nl + nx]))
+    b2b = dict(zip(labels, vals[2 + 2 * nl + nx:]))
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
@@ -620,22 +645,28 @@ def run_ours(args):
     fp4_peak = pk["bf16_tflops"] * FP4_OVER_BF16
     ms_step = ms / args.steps
     table = kernel_table(pk)
-    def entry(label, ms_, cold_ms=None):
+    def entry(label, ms_, cold_ms=None, b2b_ms=None):
         amount, unit, bound, peak = table[label]
-        us = ms_ * 1e3
-        rate = amount / (us * 1e-6) / (1e9 if unit == "GB/s" else 1e12)
-        e = {"us": round(us, 2), unit: round(rate, 1), "frac": round(rate / peak, 4)}
+
+        def rate(t_ms):
+            return amount / (t_ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+        e = {"us": round(ms_ * 1e3, 2), unit: round(rate(ms_), 1), "frac": round(rate(ms_) / peak, 4)}
+        if b2b_ms is not None:
+            e.update({"b2b_us": round(b2b_ms * 1e3, 2), "b2b_frac": round(rate(b2b_ms) / peak, 4)})
         if cold_ms is not None:
-            cold_rate = amount / (cold_ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
-            e.update({"cold_us": round(cold_ms * 1e3, 2), "cold_frac": round(cold_rate / peak, 4)})
+            e.update({"cold_us": round(cold_ms * 1e3, 2), "cold_frac": round(rate(cold_ms) / peak, 4)})
         return e
 
-    ktab = {label: entry(label, live[label], per[label]) for label in labels}
+    ktab = {label: entry(label, live[label], per[label], b2b[label]) for label in labels}
     ktab["sum_us"] = round(sum(live.values()) * 1e3, 2)
+    ktab["b2b_sum_us"] = round(sum(b2b.values()) * 1e3, 2)
     ktab["timing"] = (f"us/frac: mean over {nb} steps of the step's own launches, an event after every kernel "
                       "on the launching stream (those events cost the launch overlap, so sum_us exceeds "
-                      f"ms_per_step); cold_us/cold_frac: each kernel alone, mean of {args.kernel_reps} launches, "
-                      "each after an L2 flush (a read of twice the L2 size) and between its own two events")
+                      "ms_per_step); b2b_us/b2b_frac: the kernel's own launches back to back over the rotating "
+                      f"sets ({len(sets)}, each launch's data evicted from L2 by the others), between two events "
+                      f"and none in between; cold_us/cold_frac: each kernel alone, mean of {args.kernel_reps} "
+                      "launches, each after an L2 flush (a read of twice the L2 size) and between its own two "
+                      "events")
     ktab[f"{'unfused' if args.mlp == 'fused' else 'fused'}_mlp_for_comparison"] = dict(
         {label: entry(label, extra[label]) for label in xlabels}, timing="alone after an L2 flush, like cold_us")
     m, k, n, _ = LAYERS["fc1"]

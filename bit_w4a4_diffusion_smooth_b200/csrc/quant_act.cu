@@ -57,12 +57,18 @@ constexpr int X_STAGE = 4 * X_BOX;
 constexpr int INV_BYTES = KC * 4;
 constexpr int OUT_BYTES = 6144;   // inv_lambda slice (1 KB), code rows (4 KB), scale words (512 B), padded
 constexpr int RING_BYTES = 224 * 1024;
+// INT4 form: each compute warp's 16 row maxima of its two blocks, per stage parity, for the warp
+// that holds the other half of the 64-column groups
+constexpr int XCH_BYTES = 2 * 16 * 16 * 4;
 
 struct Params {
   int M, K, KS;
   const float *inv_lambda;
-  const float *s_a, *s_w;
-  uint8_t *bundle;
+  const float *s_a, *s_w;       // NVFP4 tensor scales (unused by the INT4 form)
+  uint8_t *bundle;              // NVFP4 codes and scales
+  uint8_t *codes4;              // INT4 form: codes [rows][K/2] and group scales [K/64][ld_s] (bf16)
+  uint16_t *scales4;
+  int ld_s;
   uint8_t *U;
   unsigned int *status;
   unsigned long long limit_ns;
@@ -90,7 +96,7 @@ __host__ __device__ constexpr int num_stages() {
 }
 template <int RANK>
 __host__ __device__ constexpr int smem_bytes() {
-  return 1024 + num_stages<RANK>() * stage_bytes<RANK>() + 128 * 4 + 512;
+  return 1024 + num_stages<RANK>() * stage_bytes<RANK>() + 128 * 4 + 512 + XCH_BYTES;
 }
 // the per-slice partial U tiles reuse the ring at the end
 static_assert(CWARPS * 16 * (64 + 4) * 4 <= num_stages<64>() * stage_bytes<64>(), "partials must fit the ring");
@@ -106,11 +112,24 @@ __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
 }
+// Named barrier over nthreads threads that also ORs a predicate across them: every
+// participant gets the same answer (used to leave a loop together).
+__device__ __forceinline__ bool barrier_or(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, %2, %3, q;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(r)
+               : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+               : "memory");
+  return r != 0;
+}
 __device__ __forceinline__ float absmax4(float a, float b, float c, float d) {
   return fmaxf(fmaxf(fabsf(a), fabsf(b)), fmaxf(fabsf(c), fabsf(d)));
 }
 
-template <int RANK, int G>
+// INT4: the form of the INT4 W4A4 variant (groups of 64 along K, bf16 group scales, codes in
+// plain rows); otherwise NVFP4 into the operand bundle.
+template <int RANK, int G, bool INT4>
 __global__ void __launch_bounds__(THREADS, 1)
     quant_act_kernel(const __grid_constant__ Group<G> grp) {
   constexpr int STAGES = num_stages<RANK>();
@@ -128,6 +147,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t *empty = full + STAGES;   // the store warp has written the stage out
   uint64_t *done = empty + STAGES;   // the compute warps have staged the stage's codes and scales
   volatile int *abort_flag = reinterpret_cast<volatile int *>(done + STAGES);
+  float *xch = reinterpret_cast<float *>(smem + STAGES * STAGE + 1024);   // [2][CWARPS][16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int pi = 0;
@@ -149,8 +169,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   dev::grid_dependency_wait();
   dev::grid_launch_dependents();
-  const float s_a = __ldg(p.s_a);
-  if (threadIdx.x < 128) {
+  const float s_a = INT4 ? 1.0f : __ldg(p.s_a);
+  if (!INT4 && threadIdx.x < 128) {
     // 1 / (scale of code c): the same two f32 roundings as the quantizer
     // definition, f32(e4m3(c) * s_a) then f32(1 / that)
     const uint32_t c = threadIdx.x;
@@ -202,6 +222,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       const uint8_t *st = smem + s * STAGE;
+      if constexpr (INT4) {
+        // code rows: 32 rows x 8 chunks of 16 bytes (staged with the chunk index xor the row);
+        // scales: 4 groups x 32 rows of bf16.  Only the stage's groups inside K are written.
+        const int ngrp = min(4, (p.K - c * KC) / 64);
+        uint4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = i * 32 + lane, r = j >> 3, ch = j & 7;
+          v[i] = *reinterpret_cast<const uint4 *>(st + CODE_OFF + r * 128 + (((ch ^ r) & 7) << 4));
+        }
+        const uint2 sc = *reinterpret_cast<const uint2 *>(st + SC_OFF + ((lane >> 3) * 32 + 4 * (lane & 7)) * 2);
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(&empty[s]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int j = i * 32 + lane, r = j >> 3, ch = j & 7;
+          if (ch < 2 * ngrp)
+            *reinterpret_cast<uint4 *>(p.codes4 + static_cast<size_t>(m0 + r) * (p.K / 2) + c * (KC / 2) + ch * 16) = v[i];
+        }
+        if ((lane >> 3) < ngrp)
+          *reinterpret_cast<uint2 *>(p.scales4 + static_cast<size_t>(4 * c + (lane >> 3)) * p.ld_s + m0 +
+                                     4 * (lane & 7)) = sc;
+        continue;
+      }
       uint8_t *tile = p.bundle + (static_cast<size_t>(m_blk) * p.KS + c) * bundle_tile_bytes(128);
       uint4 v[8];
       uint32_t w[4];
@@ -249,52 +293,71 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < 4; ++i) acc[n][i] = 0.0f;
   bool failed = false;
 
-  for (int c = 0; c < p.KS; ++c) {
-    const int s = c % STAGES;
-    if (!dev::mbar_wait_warp(&full[s], (c / STAGES) & 1, p.limit_ns, abort_flag)) {
-      *abort_flag = 1;
-      dev::report(p.status, SVDQ_ERR_TIMEOUT);
-      failed = true;
-      break;
-    }
-    const int nbox = min(4, (p.K - c * KC) / 64);
-    uint8_t *st = smem + s * STAGE;
-    uint32_t sb = 0, code0 = 0, code1 = 0;
-    if (bx < nbox) {   // warp-uniform: columns past K quantize as zeros (code and scale 0)
+  if constexpr (INT4) {
+    // A 64-column group is box bx of the stage: this lane's block and the other block of the
+    // same row in this warp (lane ^ 16), and the two blocks of the row in the pair warp w ^ 1.
+    // The pair exchanges its row maxima through shared memory at a barrier of its own (ids
+    // 3..10), whose OR-reduced predicate also carries a wait that ran out, so both warps of the
+    // pair leave the loop together.
+    const int pair_bar = 3 + (warp >> 1);
+    for (int c = 0; c < p.KS; ++c) {
+      const int s = c % STAGES;
+      const bool got = dev::mbar_wait_warp(&full[s], (c / STAGES) & 1, p.limit_ns, abort_flag);
+      if (!got) {
+        *abort_flag = 1;
+        dev::report(p.status, SVDQ_ERR_TIMEOUT);
+      }
+      const int nbox = min(4, (p.K - c * KC) / 64);
+      uint8_t *st = smem + s * STAGE;
       uint8_t *xb = st + bx * X_BOX;
-      const uint4 w0 = *reinterpret_cast<const uint4 *>(xb + x_off0);
-      const uint4 w1 = *reinterpret_cast<const uint4 *>(xb + x_off1);
-      const float4 *iv = reinterpret_cast<const float4 *>(st + INV_OFF) + (bx * 64 + col) / 4;
-      const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      // x^ of the block's 16 elements, in column order
+      const bool live = got && bx < nbox;   // warp-uniform: groups past K quantize as zeros
       float xs[16];
+      float bmax = 0.0f;
+      if (live) {
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(xb + x_off0);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(xb + x_off1);
+        const float4 *iv = reinterpret_cast<const float4 *>(st + INV_OFF) + (bx * 64 + col) / 4;
+        const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = iv[i];
-        const float2 p0 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i]), bf16_hi(wv[2 * i])), make_float2(v.x, v.y));
-        const float2 p1 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i + 1]), bf16_hi(wv[2 * i + 1])), make_float2(v.z, v.w));
-        xs[4 * i] = p0.x;
-        xs[4 * i + 1] = p0.y;
-        xs[4 * i + 2] = p1.x;
-        xs[4 * i + 3] = p1.y;
-      }
-      float amax = absmax4(xs[0], xs[1], xs[2], xs[3]);
-      amax = fmaxf(amax, absmax4(xs[4], xs[5], xs[6], xs[7]));
-      amax = fmaxf(amax, absmax4(xs[8], xs[9], xs[10], xs[11]));
-      amax = fmaxf(amax, absmax4(xs[12], xs[13], xs[14], xs[15]));
-      sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
-      const float rinv = rinv_tab[sb];
-      const float2 r2 = make_float2(rinv, rinv);
-      uint32_t cw[4];
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = iv[i];
+          const float2 p0 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i]), bf16_hi(wv[2 * i])), make_float2(v.x, v.y));
+          const float2 p1 =
+              dev::mul2_rn(make_float2(bf16_lo(wv[2 * i + 1]), bf16_hi(wv[2 * i + 1])), make_float2(v.z, v.w));
+          xs[4 * i] = p0.x;
+          xs[4 * i + 1] = p0.y;
+          xs[4 * i + 2] = p1.x;
+          xs[4 * i + 3] = p1.y;
+        }
+        bmax = absmax4(xs[0], xs[1], xs[2], xs[3]);
+        bmax = fmaxf(bmax, absmax4(xs[4], xs[5], xs[6], xs[7]));
+        bmax = fmaxf(bmax, absmax4(xs[8], xs[9], xs[10], xs[11]));
+        bmax = fmaxf(bmax, absmax4(xs[12], xs[13], xs[14], xs[15]));
+      } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 c0 = dev::mul2_rn(make_float2(xs[4 * i], xs[4 * i + 1]), r2);
-        const float2 c1 = dev::mul2_rn(make_float2(xs[4 * i + 2], xs[4 * i + 3]), r2);
-        cw[i] = dev::cvt_e2m1x4(c0.x, c0.y, c1.x, c1.y);     // code bytes 2i, 2i + 1
+        for (int i = 0; i < 16; ++i) xs[i] = 0.0f;
       }
-      code0 = cw[0] | (cw[1] << 16);
-      code1 = cw[2] | (cw[3] << 16);
-      if (RANK > 0) {
+      bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 16));
+      float *xw = xch + (c & 1) * CWARPS * 16;
+      if (lane < 16) xw[warp * 16 + lane] = bmax;
+      if (barrier_or(pair_bar, 64, !got || *abort_flag != 0)) {
+        failed = true;
+        break;
+      }
+      const float gmax = fmaxf(bmax, xw[(warp ^ 1) * 16 + (lane & 15)]);
+      // s = bf16(f32(gmax / 7)) (0 below 2^-120), q = clamp(rne(f32(x^ * f32(1 / s))), -8, 7)
+      const float sv = gmax < 0x1.0p-120f ? 0.0f : __bfloat162float(__float2bfloat16_rn(__fdiv_rn(gmax, 7.0f)));
+      const float rcp = sv == 0.0f ? 0.0f : __frcp_rn(sv);
+      uint32_t cw[2] = {0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int q = min(7, max(-8, __float2int_rn(__fmul_rn(xs[i], rcp))));
+        cw[i >> 3] |= (static_cast<uint32_t>(q) & 0xFu) << (4 * (i & 7));
+      }
+      *reinterpret_cast<uint2 *>(st + code_off) = make_uint2(cw[0], cw[1]);
+      if ((cs & 1) == 0 && blk == 0)   // one writer per row and group
+        reinterpret_cast<uint16_t *>(st + SC_OFF)[bx * 32 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(sv));
+      if (RANK > 0 && live) {
         // bf16(x^) back in place of x, as the A operand of the down-projection
         *reinterpret_cast<uint4 *>(xb + x_off0) =
             make_uint4(bf16x2(xs[0], xs[1]), bf16x2(xs[2], xs[3]), bf16x2(xs[4], xs[5]), bf16x2(xs[6], xs[7]));
@@ -316,11 +379,83 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&done[s]);
     }
-    *reinterpret_cast<uint2 *>(st + code_off) = make_uint2(code0, code1);
-    st[scale_off] = static_cast<uint8_t>(sb);
-    __syncwarp();
-    if (lane == 0) dev::mbar_arrive(&done[s]);
+  } else {
+    for (int c = 0; c < p.KS; ++c) {
+      const int s = c % STAGES;
+      if (!dev::mbar_wait_warp(&full[s], (c / STAGES) & 1, p.limit_ns, abort_flag)) {
+        *abort_flag = 1;
+        dev::report(p.status, SVDQ_ERR_TIMEOUT);
+        failed = true;
+        break;
+      }
+      const int nbox = min(4, (p.K - c * KC) / 64);
+      uint8_t *st = smem + s * STAGE;
+      uint32_t sb = 0, code0 = 0, code1 = 0;
+      if (bx < nbox) {   // warp-uniform: columns past K quantize as zeros (code and scale 0)
+        uint8_t *xb = st + bx * X_BOX;
+        const uint4 w0 = *reinterpret_cast<const uint4 *>(xb + x_off0);
+        const uint4 w1 = *reinterpret_cast<const uint4 *>(xb + x_off1);
+        const float4 *iv = reinterpret_cast<const float4 *>(st + INV_OFF) + (bx * 64 + col) / 4;
+        const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        // x^ of the block's 16 elements, in column order
+        float xs[16];
+  #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 v = iv[i];
+          const float2 p0 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i]), bf16_hi(wv[2 * i])), make_float2(v.x, v.y));
+          const float2 p1 = dev::mul2_rn(make_float2(bf16_lo(wv[2 * i + 1]), bf16_hi(wv[2 * i + 1])), make_float2(v.z, v.w));
+          xs[4 * i] = p0.x;
+          xs[4 * i + 1] = p0.y;
+          xs[4 * i + 2] = p1.x;
+          xs[4 * i + 3] = p1.y;
+        }
+        float amax = absmax4(xs[0], xs[1], xs[2], xs[3]);
+        amax = fmaxf(amax, absmax4(xs[4], xs[5], xs[6], xs[7]));
+        amax = fmaxf(amax, absmax4(xs[8], xs[9], xs[10], xs[11]));
+        amax = fmaxf(amax, absmax4(xs[12], xs[13], xs[14], xs[15]));
+        sb = dev::cvt_e4m3(__fdiv_rn(amax, d6));
+        const float rinv = rinv_tab[sb];
+        const float2 r2 = make_float2(rinv, rinv);
+        uint32_t cw[4];
+  #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 c0 = dev::mul2_rn(make_float2(xs[4 * i], xs[4 * i + 1]), r2);
+          const float2 c1 = dev::mul2_rn(make_float2(xs[4 * i + 2], xs[4 * i + 3]), r2);
+          cw[i] = dev::cvt_e2m1x4(c0.x, c0.y, c1.x, c1.y);     // code bytes 2i, 2i + 1
+        }
+        code0 = cw[0] | (cw[1] << 16);
+        code1 = cw[2] | (cw[3] << 16);
+        if (RANK > 0) {
+          // bf16(x^) back in place of x, as the A operand of the down-projection
+          *reinterpret_cast<uint4 *>(xb + x_off0) =
+              make_uint4(bf16x2(xs[0], xs[1]), bf16x2(xs[2], xs[3]), bf16x2(xs[4], xs[5]), bf16x2(xs[6], xs[7]));
+          *reinterpret_cast<uint4 *>(xb + x_off1) =
+              make_uint4(bf16x2(xs[8], xs[9]), bf16x2(xs[10], xs[11]), bf16x2(xs[12], xs[13]), bf16x2(xs[14], xs[15]));
+          __syncwarp();
+          const uint32_t xbase = dev::smem_u32(xb);
+          const uint32_t lbase = dev::smem_u32(st + X_STAGE + bx * L1_BOX);
+  #pragma unroll
+          for (int kk = 0; kk < 2; ++kk) {
+            uint32_t af[4];
+            dev::ldmatrix_x4(xbase + sw_off(arow, acol + 16 * kk), af[0], af[1], af[2], af[3]);
+  #pragma unroll
+            for (int np = 0; np < NT / 2; ++np) {
+              uint32_t bq[4];
+              dev::ldmatrix_x4(lbase + sw_off(np * 16 + brow, bcol + 16 * kk), bq[0], bq[1], bq[2], bq[3]);
+              dev::mma_bf16_16816(acc[2 * np], af, bq[0], bq[1]);
+              dev::mma_bf16_16816(acc[2 * np + 1], af, bq[2], bq[3]);
+            }
+          }
+        }
+      }
+      *reinterpret_cast<uint2 *>(st + code_off) = make_uint2(code0, code1);
+      st[scale_off] = static_cast<uint8_t>(sb);
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&done[s]);
+    }
   }
 
   // ---- U = (sum of the 8 slices' partial products of each row half) / (s_a s_w), bf16, 128-row tiles
@@ -343,7 +478,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   // a wait that ran out anywhere leaves U zero (the status word carries the error)
   const bool any_failed = RANK > 0 && *abort_flag != 0;
-  const float alpha = __fmul_rn(s_a, __ldg(p.s_w));
+  const float alpha = INT4 ? 1.0f : __fmul_rn(s_a, __ldg(p.s_w));
   // every thread: column pairs (2 cp, 2 cp + 1) of the CTA's rows, the slices' partials added in order
   for (int idx = tid; idx < BM * (SVDQ_LR_STRIDE / 2); idx += CWARPS * 32) {
     const int rr = idx / (SVDQ_LR_STRIDE / 2), cp = idx % (SVDQ_LR_STRIDE / 2);
@@ -363,13 +498,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-template <int RANK, int G>
+template <int RANK, int G, bool INT4>
 int launch(const Group<G> &g, int grid, cudaStream_t stream, const char *fn) {
   const int smem = smem_bytes<RANK>();
-  const int rc = smem_optin_once<quant_act_kernel<RANK, G>>(smem, fn);
+  const int rc = smem_optin_once<quant_act_kernel<RANK, G, INT4>>(smem, fn);
   if (rc != SVDQ_OK) return rc;
   DependentLaunch dl(dim3(grid), dim3(THREADS), smem, stream);
-  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK, G>, g);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, quant_act_kernel<RANK, G, INT4>, g);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return ok();
@@ -420,14 +555,14 @@ int encode_problem(const void *X, int M, int K, int ldx, const void *l1t, int ra
   return SVDQ_OK;
 }
 
-template <int G>
+template <int G, bool INT4 = false>
 int launch_rank(int rank, const Group<G> &g, int grid, cudaStream_t s, const char *fn) {
   switch (rank) {
-    case 0: return launch<0, G>(g, grid, s, fn);
-    case 16: return launch<16, G>(g, grid, s, fn);
-    case 32: return launch<32, G>(g, grid, s, fn);
-    case 48: return launch<48, G>(g, grid, s, fn);
-    default: return launch<64, G>(g, grid, s, fn);
+    case 0: return launch<0, G, INT4>(g, grid, s, fn);
+    case 16: return launch<16, G, INT4>(g, grid, s, fn);
+    case 32: return launch<32, G, INT4>(g, grid, s, fn);
+    case 48: return launch<48, G, INT4>(g, grid, s, fn);
+    default: return launch<64, G, INT4>(g, grid, s, fn);
   }
 }
 
@@ -481,4 +616,38 @@ extern "C" int svdq_quantize_act_grouped(const svdq_quant_problem *problems, int
   }
   g.count = count;
   return launch_rank(rank, g, total, reinterpret_cast<cudaStream_t>(stream), fn);
+}
+
+extern "C" int svdq_quantize_act_int4(const void *X, int M, int K, int ldx, const float *inv_lambda, const void *l1t,
+                                      int rank, uint8_t *a_codes, void *a_scales, void *U, svdq_stream_t stream) {
+  static const char *fn = "svdq_quantize_act_int4";
+  if (!X || !inv_lambda || !a_codes || !a_scales || !U || (rank > 0 && !l1t))
+    return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": null pointer");
+  if (M < 1 || K < 64 || K % 64 || ldx < K || ldx % 8)
+    return fail(SVDQ_ERR_SHAPE, std::string(fn) + ": need M >= 1, K % 64 == 0, ldx >= K, ldx % 8 == 0");
+  if (rank < 0 || rank > SVDQ_LR_STRIDE || rank % 16)
+    return fail(SVDQ_ERR_SHAPE, std::string(fn) + ": rank must be a multiple of 16 in [0, 64]");
+  if (!aligned16(X) || !aligned16(inv_lambda) || !aligned16(a_codes) || !aligned16(a_scales) || !aligned16(U) ||
+      (rank > 0 && !aligned16(l1t)))
+    return fail(SVDQ_ERR_ALIGNMENT, std::string(fn) + ": pointers must be 16-byte aligned");
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  Group<1> g{};
+  Params &p = g.p[0];
+  p.M = M;
+  p.K = K;
+  p.KS = bundle_ks(K);
+  p.inv_lambda = inv_lambda;
+  p.codes4 = a_codes;
+  p.scales4 = static_cast<uint16_t *>(a_scales);
+  p.ld_s = (M + 127) / 128 * 128;
+  p.U = static_cast<uint8_t *>(U);
+  p.status = st->status_word;
+  p.limit_ns = kWaitLimitNs;
+  const int rc = encode_problem(X, M, K, ldx, l1t, rank, &g.tx[0], &g.tl[0]);
+  if (rc != SVDQ_OK) return rc;
+  const int grid = (M + 127) / 128 * (128 / BM);
+  g.blk_end[0] = grid;
+  g.count = 1;
+  return launch_rank<1, true>(rank, g, grid, reinterpret_cast<cudaStream_t>(stream), fn);
 }

@@ -59,6 +59,11 @@ _SIGNATURES = {
     "svdq_act_sizes": (_I, [_I, _I, _SZ, _SZ]),
     "svdq_pack_weights": (_I, [_P, _I, _I, _P, _I, _I, ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _P]),
     "svdq_quantize_host": (_I, [_P, _I, _I, ctypes.c_float, _I, _P]),
+    "svdq_int4_weight_sizes": (_I, [_I, _I, _SZ, _SZ]),
+    "svdq_int4_act_sizes": (_I, [_I, _I, _SZ, _SZ]),
+    "svdq_quantize_int4_host": (_I, [_P, _I, _I, _I, _P, _P]),
+    "svdq_quantize_act_int4": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]),
+    "svdq_linear_int4": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "svdq_quantize_act": (_I, [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P]),
     "svdq_linear_w4a4": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P]),
     "svdq_quantize_act_grouped": (_I, [ctypes.POINTER(QuantProblem), _I, _I, _P]),
@@ -229,6 +234,82 @@ def svdq_pack_weights(W_bits, act_absmax, rank, num_threads=0, seed=0, want_resi
     if want_residual:
         out["residual"] = residual
     return out
+
+
+def svdq_int4_weight_sizes(K, N):
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("svdq_int4_weight_sizes", load().svdq_int4_weight_sizes(K, N, ctypes.byref(a), ctypes.byref(b)))
+    return dict(codes=a.value, scales=b.value)
+
+
+def svdq_int4_act_sizes(M, K):
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check("svdq_int4_act_sizes", load().svdq_int4_act_sizes(M, K, ctypes.byref(a), ctypes.byref(b)))
+    return dict(codes=a.value, scales=b.value)
+
+
+def svdq_quantize_int4_host(T, ld_s=None):
+    """INT4 groups of 64 of float32 rows T [rows, K] (host): codes u8 [rows, K/2], scales u16 (bf16)
+    [K/64, ld_s]."""
+    T = np.ascontiguousarray(T, dtype=np.float32)
+    rows, K = T.shape
+    ld_s = rows if ld_s is None else ld_s
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((max(K // 64, 1), max(ld_s, 1)), np.uint16)
+    _check("svdq_quantize_int4_host", load().svdq_quantize_int4_host(
+        _hptr(T, np.float32, "T"), rows, K, ld_s, _hptr(codes, np.uint8, "codes"),
+        _hptr(scales, np.uint16, "scales")))
+    return codes, scales
+
+
+def svdq_pack_weights_int4(W_bits, act_absmax, rank, num_threads=0, seed=0):
+    """Host pack of the INT4 layer: svdq_pack_weights' smoothing, low-rank branch and residual, the
+    residual in INT4 groups along K per output column.  Returns inv_lambda, l1t, l2t (as
+    svdq_pack_weights), w_codes u8 [N, K/2], w_scales u16 (bf16) [K/64, N] and the residual."""
+    p = svdq_pack_weights(W_bits, act_absmax, rank, num_threads, seed, want_residual=True)
+    codes, scales = svdq_quantize_int4_host(np.ascontiguousarray(p["residual"].T))
+    return dict(inv_lambda=p["inv_lambda"], l1t=p["l1t"], l2t=p["l2t"], w_codes=codes, w_scales=scales,
+                residual=p["residual"])
+
+
+def svdq_quantize_act_int4(X, inv_lambda, l1t, rank, a_codes, a_scales, U, M=None, K=None, stream=None):
+    """Enqueues the INT4 activation kernel.  X: bf16 CUDA [M, ldx]."""
+    import torch
+    M = X.shape[0] if M is None else M
+    K = X.shape[1] if K is None else K
+    _need_2d(X, M, K, "X")
+    sz = svdq_int4_act_sizes(M, K)
+    _need_bytes(a_codes, sz["codes"], "a_codes")
+    _need_bytes(a_scales, sz["scales"], "a_scales")
+    _need_bytes(U, _act_sizes(M, K)[1], "U")
+    _need_bytes(inv_lambda, 4 * K, "inv_lambda")
+    if rank:
+        _need_bytes(l1t, 2 * rank * K, "l1t")
+    _check("svdq_quantize_act_int4", load().svdq_quantize_act_int4(
+        _dptr(X, "X", torch.bfloat16), M, K, X.stride(0), _dptr(inv_lambda, "inv_lambda", torch.float32),
+        _dptr(l1t, "l1t", allow_none=rank == 0), rank, _dptr(a_codes, "a_codes", torch.uint8),
+        _dptr(a_scales, "a_scales"), _dptr(U, "U"), _stream(stream)))
+
+
+def svdq_linear_int4(a_codes, a_scales, U, w_codes, w_scales, l2t, bias, M, N, K, rank, epilogue, gelu_col_begin, Y,
+                     stream=None):
+    """Enqueues the INT4 GEMM.  Y: bf16 CUDA [M, ldy]."""
+    import torch
+    asz, wsz = svdq_int4_act_sizes(M, K), svdq_int4_weight_sizes(K, N)
+    _need_bytes(a_codes, asz["codes"], "a_codes")
+    _need_bytes(a_scales, asz["scales"], "a_scales")
+    _need_bytes(w_codes, wsz["codes"], "w_codes")
+    _need_bytes(w_scales, wsz["scales"], "w_scales")
+    if rank:
+        _need_bytes(U, _act_sizes(M, K)[1], "U")
+        _need_bytes(l2t, _weight_sizes(K, N, rank)[2], "l2t")
+    _need_bytes(bias, 2 * N, "bias")
+    _need_2d(Y, M, N, "Y")
+    _check("svdq_linear_int4", load().svdq_linear_int4(
+        _dptr(a_codes, "a_codes", torch.uint8), _dptr(a_scales, "a_scales"), _dptr(U, "U", allow_none=rank == 0),
+        _dptr(w_codes, "w_codes", torch.uint8), _dptr(w_scales, "w_scales"),
+        _dptr(l2t, "l2t", allow_none=rank == 0), _dptr(bias, "bias", allow_none=True), M, N, K, rank, epilogue,
+        gelu_col_begin, _dptr(Y, "Y", torch.bfloat16), Y.stride(0), _stream(stream)))
 
 
 def svdq_quantize_host(T, s_t, tile_rows=128):

@@ -446,6 +446,65 @@ int awq_linear_w4a16_gemm(const void *X, int M, int K, int ldx, const float *inv
  */
 int svdq_check_status(svdq_stream_t stream);
 
+/* ------------------------------------------------------------- INT4 W4A4
+ * The pages ship an INT4 W4A4 variant beside NVFP4 for GPUs without NVFP4
+ * (donmalab.com, "Diffusers × Nunchaku 4-bit", section "實務上的影響與硬體要求";
+ * remio.ai, section "硬件支持划分了最快路径与最广泛路径") and give no layout.
+ * This library's reading: the NVFP4 layer (smoothing, low-rank branch,
+ * residual; svdq_pack_weights) with its 4-bit branch in signed integers,
+ * groups of 64 along K, one bf16 scale per row (activations) or output column
+ * (weights) and group:
+ *   s = bf16(f32(amax / 7)),   q = clamp(rne(f32(v * f32(1 / s))), -8, 7)
+ * with s = 0 and q = 0 for a group whose amax is below 2^-120.
+ * Layouts: codes [rows][K/2] bytes, element k in byte k/2 (low nibble for
+ * even k), two's complement; scales [K/64][ld] bf16 (group-major), ld = N for
+ * weights and the activation rows rounded up to 128 for activations.  U and
+ * L2T keep the low-rank tile layouts of the NVFP4 calls.
+ */
+
+/* Byte sizes of the INT4 weight codes and scales.  Rules: K % 64 == 0, N % 128 == 0. */
+int svdq_int4_weight_sizes(int K, int N, size_t *codes_bytes, size_t *scales_bytes);
+
+/* Byte sizes of the INT4 activation codes and scales (rows rounded up to 128).
+ * Rules: M >= 1, K % 64 == 0. */
+int svdq_int4_act_sizes(int M, int K, size_t *codes_bytes, size_t *scales_bytes);
+
+/*
+ * Group quantization of host float32 rows T [rows][K] (host, no GPU) into
+ * codes [rows][K/2] and scales [K/64][ld_s] (ld_s >= rows): the weight side of
+ * the INT4 pack, applied to the transposed residual R^T [N][K] that
+ * svdq_pack_weights returns.  Rules: rows >= 1, K % 64 == 0, ld_s >= rows.
+ */
+int svdq_quantize_int4_host(const float *T, int rows, int K, int ld_s, uint8_t *codes, uint16_t *scales);
+
+/*
+ * Activation side of the INT4 layer, one pass over X like svdq_quantize_act:
+ *   x^ = f32(x * inv_lambda[k]);  codes and scales of x^ as above;
+ *   U[m][j] = bf16( sum_k bf16(x^[m][k]) * L1T[j][k] )   (no tensor scale)
+ * Args: X [M][ldx] bf16 (device); inv_lambda [K] f32; l1t [rank][K] bf16
+ * (ignored when rank == 0); outputs a_codes, a_scales (sizes from
+ * svdq_int4_act_sizes; padding rows written as 0) and U (128-row low-rank
+ * tiles).  Rules: those of svdq_quantize_act.
+ */
+int svdq_quantize_act_int4(const void *X, int M, int K, int ldx, const float *inv_lambda, const void *l1t,
+                           int rank, uint8_t *a_codes, void *a_scales, void *U, svdq_stream_t stream);
+
+/*
+ * The INT4 GEMM with the low-rank up-projection fused in:
+ *   Y = bf16( epilogue( sum_g (s_a[m,g] s_w[n,g]) sum_{k in g} q_a q_w
+ *                       + U . L2T^T + bias ) )
+ * B200 has no 4-bit integer MMA: the kernel unpacks the codes to 8 bits and
+ * runs 8-bit warp MMAs (exact int32 per group), rescaling each group in
+ * fp32.  Args: a_codes, a_scales, U from svdq_quantize_act_int4; w_codes,
+ * w_scales from svdq_quantize_int4_host, l2t from svdq_pack_weights
+ * (uploaded); bias [N] bf16 or NULL; Y [M][ldy] bf16.
+ * Rules: M >= 1, K % 64 == 0, N % 128 == 0, ldy >= N, ldy % 8 == 0,
+ * 0 <= rank <= 64, rank % 16 == 0, 0 <= gelu_col_begin <= N.
+ */
+int svdq_linear_int4(const uint8_t *a_codes, const void *a_scales, const void *U, const uint8_t *w_codes,
+                     const void *w_scales, const void *l2t, const void *bias, int M, int N, int K, int rank,
+                     int epilogue, int gelu_col_begin, void *Y, int ldy, svdq_stream_t stream);
+
 /*
  * Self-test of the bounded wait used by every kernel: launches one block that
  * waits on a shared-memory barrier nothing will ever complete, with a limit

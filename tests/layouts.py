@@ -180,3 +180,34 @@ def bf16_bits(values):
     if (u & 0xFFFF).any():
         raise ValueError("not bf16 values")
     return (u >> 16).astype(np.uint16)
+
+
+# ---- INT4 W4A4 operands: codes [rows][K/2] (element k in byte k/2, low nibble for even k, two's
+# complement), scales [K/64][ld] bf16 (group-major)
+def int4_pack(q):
+    q = np.asarray(q, dtype=np.int8)
+    u = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    return (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+
+
+def int4_unpack(codes, rows, K):
+    c = np.asarray(codes, dtype=np.uint8).reshape(-1, K // 2)[:rows]
+    lo = (c & 0xF).astype(np.int16)
+    hi = (c >> 4).astype(np.int16)
+    q = np.empty((rows, K), np.int8)
+    q[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    q[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return q
+
+
+def int4_scales_pack(s, ld):
+    """s: float64 [rows, K/64] holding bf16 values -> uint16 [K/64, ld] (columns past rows 0)."""
+    rows, groups = s.shape
+    out = np.zeros((groups, ld), np.uint16)
+    out[:, :rows] = bf16_bits(s.T)
+    return out
+
+
+def int4_scales_unpack(buf, rows, groups, ld):
+    b = np.asarray(buf, dtype=np.uint16).reshape(groups, ld)
+    return bf16_bits_to_f64(b[:, :rows].T)

@@ -105,6 +105,18 @@ def test_device_calls_reject_bad_arguments_before_touching_a_gpu():
     odd = ctypes.c_void_p(24)
     rc = so.svdq_linear_w4a4(odd, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None)
     assert rc == lib.ERR_ALIGNMENT
+    # the INT4 variant: sizes, then the same argument rules before any device access
+    assert lib.svdq_int4_weight_sizes(3072, 9216) == {"codes": 9216 * 1536, "scales": 48 * 9216 * 2}
+    assert lib.svdq_int4_act_sizes(200, 320) == {"codes": 256 * 160, "scales": 5 * 256 * 2}
+    with pytest.raises(lib.SvdqError) as e:
+        lib.svdq_int4_weight_sizes(3072, 200)                     # N % 128
+    assert e.value.status == lib.ERR_SHAPE
+    assert so.svdq_quantize_act_int4(p, 64, 256, 256, p, None, 16, p, p, p, None) == lib.ERR_INVALID_ARG
+    assert so.svdq_quantize_act_int4(p, 64, 200, 256, p, p, 16, p, p, p, None) == lib.ERR_SHAPE
+    assert so.svdq_linear_int4(p, p, p, p, p, p, None, 64, 200, 256, 16, 0, 0, p, 256, None) == lib.ERR_SHAPE
+    assert so.svdq_linear_int4(p, p, None, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None) == lib.ERR_INVALID_ARG
+    assert so.svdq_linear_int4(p, p, p, p, p, p, None, 64, 256, 256, 16, 5, 0, p, 256, None) == lib.ERR_INVALID_ARG
+    assert so.svdq_linear_int4(odd, p, p, p, p, p, None, 64, 256, 256, 16, 0, 0, p, 256, None) == lib.ERR_ALIGNMENT
 
 
 def test_init_without_a_b200_is_an_error():

@@ -17,9 +17,11 @@
 //     tiles in shared memory (16-byte chunks xor-swizzled by row pairs, so the
 //     ldmatrix reads are conflict-free) and multiplied with the 8-bit warp MMA
 //     (mma.sync m16n8k32 s8, int32 accumulation: exact, |partial| <= 4096);
-//   * the group's int32 partial is converted exactly (the int32 + 1.5 * 2^23
-//     float trick, |partial| < 2^22) and added into fp32 accumulators with
-//     the two scales: acc += s_a * (s_w * partial);
+//   * the group's first MMA starts from the integer bits of the float
+//     1.5 * 2^23 instead of zero, so the int32 result is the bit pattern of
+//     1.5 * 2^23 + partial (exact, |partial| < 2^22): one subtraction gives
+//     the partial as a float, added into fp32 accumulators with the two
+//     scales: acc += s_a * (s_w * partial);
 //   * after the last group, U . L2 (bf16 warp MMAs from the 128-row tiles of
 //     U and the 256-row tiles of L2T, into the same accumulators), bias,
 //     GELU and bf16 stores.
@@ -79,6 +81,14 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
+}
+// The first k32 step of a group: D = A . B + C with C = the bits of 1.5 * 2^23 in every element, so
+// that after the group D holds the bits of the float 1.5 * 2^23 + partial (exact for |partial| < 2^22).
+__device__ __forceinline__ void mma_s8_biased(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%10,%10,%10,%10};"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0x4B400000));
 }
 __device__ __forceinline__ void mma_s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -166,25 +176,25 @@ __global__ void __launch_bounds__(THREADS, 1) int4_gemm_kernel(const Params p) {
     }
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
-      int part[4][4];
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) part[nt][e] = 0;
+      int part[4][4];   // bits of the float 1.5 * 2^23 + the group's int32 partial
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         uint32_t af[4];
         ldmatrix_x4(a8 + i8_off(wm + mt * 16 + (lane & 15), 2 * kk + (lane >> 4)), af);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) mma_s8(part[nt], af, bf[nt][kk][0], bf[nt][kk][1]);
+        for (int nt = 0; nt < 4; ++nt) {
+          if (kk == 0)
+            mma_s8_biased(part[nt], af, bf[nt][kk][0], bf[nt][kk][1]);
+          else
+            mma_s8(part[nt], af, bf[nt][kk][0], bf[nt][kk][1]);
+        }
       }
       const float sa0 = bf16f(sa[wm + mt * 16 + g8]), sa1 = bf16f(sa[wm + mt * 16 + g8 + 8]);
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          // exact int32 -> f32 for |partial| < 2^22: the float with bits (partial + bits of 1.5 * 2^23)
-          const float f = __int_as_float(part[nt][e] + 0x4B400000) - 12582912.0f;
+          const float f = __int_as_float(part[nt][e]) - 12582912.0f;   // the partial, exactly
           acc[mt][nt][e] = __fmaf_rn(e < 2 ? sa0 : sa1, __fmul_rn(swc[nt][e & 1], f), acc[mt][nt][e]);
         }
     }

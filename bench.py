@@ -56,6 +56,7 @@ WORKLOAD = ("one 12B-class DiT block's SVDQ W4A4 linears at 4608 tokens, rank 32
 METRIC = "SVDQ W4A4 linear TFLOPS and % of B200 dense-FP4 peak; W4A16 GB/s vs HBM"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0            # nominal dense FP4 / dense bf16 ratio (9 / 2.25 PFLOP/s)
+INT8_OVER_BF16 = 2.0           # nominal dense int8 / dense bf16 ratio (4.5 / 2.25 POPS)
 FP4_NOMINAL_TFLOPS = 9000.0    # NVIDIA's dense FP4 figure for B200
 
 
@@ -224,11 +225,13 @@ class Workload:
         cases = {"qkv": synthetic.QKV, "fc1": synthetic.MLP_FC1, "fc2": synthetic.MLP_FC2}
         self.host_w = {}
         self.x_bits = {}
+        self.w_bits = {}
         for name in ("qkv", "fc1"):
             c = cases[name]
             xb, wb, bb = c.make()
             amax = np.max(np.abs(synthetic.bf16_bits_to_f32(xb)), axis=0).astype(np.float32)
             self.x_bits[name] = xb
+            self.w_bits[name] = (wb, amax, bb)
             self.host_w[name] = (lib.svdq_pack_weights(wb, amax, RANK, seed=c.seed), bb)
         # fc2: calibrated on fc1's output for this input (one untimed fc1 pass on the device)
         c2 = cases["fc2"]
@@ -455,6 +458,53 @@ def awq_many_rows(W, device, m=256, reps=10):
     return out
 
 
+def int4_variant(W, device, pk, reps=20):
+    """The INT4 W4A4 variant on the MLP fc1 layer (4608 x 3072 -> 12288, erf GELU, rank 32): its
+    activation kernel and its GEMM, each launched back to back over rotating copies of every buffer
+    (six: each launch's data evicted from L2 by the others), beside the NVFP4 kernels of the step."""
+    import torch
+    from bit_w4a4_diffusion_smooth_b200 import lib
+    m, k, n, _ = LAYERS["fc1"]
+    wb, amax, bb = W.w_bits["fc1"]
+    pack = lib.svdq_pack_weights_int4(wb, amax, RANK, seed=11)
+    asz = lib.svdq_int4_act_sizes(m, k)
+    sets = []
+    for s in W.sets[:MIN_SETS]:
+        sets.append(dict(X=s["fc1"]["X"], inv=_t(pack["inv_lambda"]).to(device), l1t=_bf(pack["l1t"]).to(device),
+                         l2t=_t(pack["l2t"]).to(device), wc=_t(pack["w_codes"]).to(device),
+                         ws=_t(pack["w_scales"]).to(device), bias=s["fc1"]["bias"],
+                         ac=torch.empty(asz["codes"], dtype=torch.uint8, device=device),
+                         asc=torch.empty(asz["scales"], dtype=torch.uint8, device=device),
+                         U=torch.empty(lib.svdq_act_sizes(m, k)["u"], dtype=torch.uint8, device=device),
+                         Y=s["fc1"]["Y"]))
+
+    def k1(d):
+        lib.svdq_quantize_act_int4(d["X"], d["inv"], d["l1t"], RANK, d["ac"], d["asc"], d["U"], M=m, K=k)
+
+    def k2(d):
+        lib.svdq_linear_int4(d["ac"], d["asc"], d["U"], d["wc"], d["ws"], d["l2t"], d["bias"], m, n, k, RANK,
+                             lib.EPILOGUE_GELU_ERF, 0, d["Y"])
+
+    def sync():
+        torch.cuda.synchronize()
+    k1_ms = time_back_to_back(k1, sets, reps, sync)
+    k2_ms = time_back_to_back(k2, sets, reps, sync)
+    rc = lib.svdq_check_status()
+    if rc != lib.OK:
+        raise RuntimeError(f"device status after the INT4 pass: {lib.status_name(rc)}")
+    int8_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    k1_gbs = k1_bytes(m, k) / (k1_ms * 1e-3) / 1e9
+    k2_tops = gemm_flops(m, k, n) / (k2_ms * 1e-3) / 1e12
+    return {"K1 int4 fc1": {"us": round(k1_ms * 1e3, 2), "GB/s": round(k1_gbs, 1),
+                            "frac": round(k1_gbs / pk["hbm_gbs"], 4)},
+            "K2 int4 fc1 +GELU": {"us": round(k2_ms * 1e3, 2), "TOPS": round(k2_tops, 1),
+                                  "frac_of_int8_peak": round(k2_tops / int8_peak, 4)},
+            "int8_peak_tops": round(int8_peak, 1),
+            "what": "INT4 W4A4 (groups of 64, bf16 scales) on the fc1 layer: back-to-back launches over 6 rotating "
+                    "buffer sets; the GEMM runs 8-bit warp MMAs (B200 has no 4-bit integer MMA) against the "
+                    "int8 peak taken as the bf16 peak x 2 (nominal dense int8 : bf16)"}
+
+
 def copy_floor(device, nbytes, reps=24):
     """A library copy of `nbytes` (torch, device to device) with L2 flushed before it, timed like the
     kernels: the HBM rate a plain stream of this size reaches on this GPU, as (GB/s counting read +
@@ -624,6 +674,8 @@ def run_ours(args):
     # NVFP4 GEMM on the fc1 shape
     floor_gbs, floor_us = copy_floor(device, TOKENS * HIDDEN * 2)
     awq_batch = awq_many_rows(W, device)
+    pk_local, _ = peaks()
+    int4_pass = int4_variant(W, device, pk_local)
     fp4_lib = fp4_library_point(device, *LAYERS["fc1"][:3]) if not args.no_library_points else "skipped"
 
     # ---- max over ranks
@@ -710,6 +762,7 @@ def run_ours(args):
                                      "2MKN (FP4) + 2MrN (low-rank up-projection) per launch")},
         "kernels": ktab,
         "awq_many_rows": awq_batch,
+        "int4_w4a4": int4_pass,
         "reference_points": {
             "hbm_copy_same_bytes": {"GB/s": round(floor_gbs, 1), "us": round(floor_us, 2),
                                     "what": f"torch copy of {TOKENS}x{HIDDEN} bf16, timed like the kernels "

@@ -21,7 +21,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsvdq_b200.so")
 
 SOURCES = ["api.cu", "quant_act.cu", "act_amax.cu", "gemm_w4a4.cu", "gemm_w4a4_requant.cu", "gemv_w4a16.cu",
-           "awq_gemm.cu", "int4_gemm.cu", "pack_svdq.cpp", "pack_awq.cpp", "pack_int4.cpp", "pack_device.cu"]
+           "awq_gemm.cu", "int4_gemm.cu", "int4_gemm_tc.cu", "pack_svdq.cpp", "pack_awq.cpp", "pack_int4.cpp", "pack_device.cu"]
 # The device pack's float64 products and the many-row AWQ GEMM run on cuBLAS / cuBLASLt (plain GEMMs); the
 # toolkit's copies are found through the rpath.
 CUDA_LIB = os.path.join(os.path.dirname(os.path.dirname(shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc")), "lib64")

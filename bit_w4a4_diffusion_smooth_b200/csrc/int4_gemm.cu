@@ -299,7 +299,14 @@ extern "C" int svdq_linear_int4(const uint8_t *a_codes, const void *a_scales, co
   if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(Y) ||
       (bias && !aligned16(bias)) || (rank > 0 && (!aligned16(U) || !aligned16(l2t))))
     return fail(SVDQ_ERR_ALIGNMENT, "svdq_linear_int4: pointers must be 16-byte aligned");
-  if (!current_device_state()) return SVDQ_ERR_NOT_INITIALIZED;
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // widths in whole 256-column tiles: the tcgen05 kernel (fp16 operands from the codes, no per-group
+  // rescale); otherwise the 8-bit warp-MMA kernel below
+  if (N % 256 == 0)
+    return launch_int4_tc(a_codes, a_scales, U, w_codes, w_scales, l2t, bias, M, N, K, rank, epilogue, gelu_col_begin,
+                          Y, ldy, st->status_word, s);
   Params p;
   p.a_codes = a_codes;
   p.w_codes = w_codes;
@@ -316,7 +323,6 @@ extern "C" int svdq_linear_int4(const uint8_t *a_codes, const void *a_scales, co
   p.ld_sa = (M + 127) / 128 * 128;
   p.rank = rank;
   p.gelu_col_begin = gelu_col_begin;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (epilogue) {
     case SVDQ_EPILOGUE_GELU_ERF: return launch<SVDQ_EPILOGUE_GELU_ERF>(p, s);
     case SVDQ_EPILOGUE_GELU_TANH: return launch<SVDQ_EPILOGUE_GELU_TANH>(p, s);

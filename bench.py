@@ -56,7 +56,6 @@ WORKLOAD = ("one 12B-class DiT block's SVDQ W4A4 linears at 4608 tokens, rank 32
 METRIC = "SVDQ W4A4 linear TFLOPS and % of B200 dense-FP4 peak; W4A16 GB/s vs HBM"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_OVER_BF16 = 4.0            # nominal dense FP4 / dense bf16 ratio (9 / 2.25 PFLOP/s)
-INT8_OVER_BF16 = 2.0           # nominal dense int8 / dense bf16 ratio (4.5 / 2.25 POPS)
 FP4_NOMINAL_TFLOPS = 9000.0    # NVIDIA's dense FP4 figure for B200
 
 
@@ -492,17 +491,18 @@ def int4_variant(W, device, pk, reps=20):
     rc = lib.svdq_check_status()
     if rc != lib.OK:
         raise RuntimeError(f"device status after the INT4 pass: {lib.status_name(rc)}")
-    int8_peak = pk["bf16_tflops"] * INT8_OVER_BF16
+    f16_peak = pk["bf16_tflops"]           # the GEMM's tensor-core arithmetic is fp16 x fp16 -> fp32
     k1_gbs = k1_bytes(m, k) / (k1_ms * 1e-3) / 1e9
     k2_tops = gemm_flops(m, k, n) / (k2_ms * 1e-3) / 1e12
     return {"K1 int4 fc1": {"us": round(k1_ms * 1e3, 2), "GB/s": round(k1_gbs, 1),
                             "frac": round(k1_gbs / pk["hbm_gbs"], 4)},
-            "K2 int4 fc1 +GELU": {"us": round(k2_ms * 1e3, 2), "TOPS": round(k2_tops, 1),
-                                  "frac_of_int8_peak": round(k2_tops / int8_peak, 4)},
-            "int8_peak_tops": round(int8_peak, 1),
+            "K2 int4 fc1 +GELU": {"us": round(k2_ms * 1e3, 2), "TFLOP/s": round(k2_tops, 1),
+                                  "frac_of_fp16_tensor_peak": round(k2_tops / f16_peak, 4)},
+            "fp16_tensor_peak_tflops": round(f16_peak, 1),
             "what": "INT4 W4A4 (groups of 64, bf16 scales) on the fc1 layer: back-to-back launches over 6 rotating "
-                    "buffer sets; the GEMM runs 8-bit warp MMAs (B200 has no 4-bit integer MMA) against the "
-                    "int8 peak taken as the bf16 peak x 2 (nominal dense int8 : bf16)"}
+                    "buffer sets; B200 has no 4-bit integer MMA, so the GEMM turns the codes into exact fp16 "
+                    "operands q*s in shared memory and runs tcgen05 kind::f16 (fp32 accumulation), against the "
+                    "16-bit tensor peak"}
 
 
 def copy_floor(device, nbytes, reps=24):

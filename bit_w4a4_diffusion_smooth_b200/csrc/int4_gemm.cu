@@ -1,4 +1,6 @@
-// INT4 W4A4 GEMM with the low-rank up-projection, bias and GELU fused in.
+// INT4 W4A4 GEMM with the low-rank up-projection, bias and GELU fused in:
+// the entry point, and the kernel for widths that are not whole 256-column
+// tiles (the others run on the tensor cores, int4_gemm_tc.cu).
 //
 // The pages ship an INT4 W4A4 variant beside NVFP4 for GPUs without NVFP4
 // tensor cores (web page "Diffusers × Nunchaku 4-bit", donmalab.com, section

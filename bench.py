@@ -30,6 +30,7 @@ Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|referenc
 import argparse
 import hashlib
 import json
+import platform
 import os
 import statistics
 import subprocess
@@ -841,6 +842,17 @@ def _cores():
         return os.cpu_count() or 1
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(rows=16, reps=1):
     ow = OracleWorkload()
     flops = secs = 0.0
@@ -848,7 +860,16 @@ def cpu_baseline(rows=16, reps=1):
         f, s = ow.sample(rows)
         flops += f
         secs += s
+    # the same sample with numpy's BLAS held to one thread
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(1):
+            f1, s1 = ow.sample(rows)
+        one = round(f1 / s1 / 1e12, 6)
+    except Exception:
+        one = None
     return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": _cores(), "kind": "oracle",
+            "one_thread_value": one, "cpu_model": _cpu_model(),
             "sample": f"{rows} of {TOKENS} rows of each SVDQ layer (QKV, fc1, fc2 on fc1's output: quantize + "
                       f"two-branch float64 GEMM) + the full 2x3072->18432 AWQ projection, {reps} repetition(s); "
                       "the oracle's packs are untimed"}

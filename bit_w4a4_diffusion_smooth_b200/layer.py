@@ -1,5 +1,5 @@
-"""User-facing layers on top of the C ABI: SVDQLinear (W4A4 + low-rank branch)
-and AWQLinear (W4A16).  They hold the packed weights on the GPU and reuse
+"""User-facing layers on top of the C ABI: SVDQLinear (W4A4 + low-rank branch),
+SVDQLinearInt4 (its INT4 variant) and AWQLinear (W4A16).  They hold the packed weights on the GPU and reuse
 activation buffers per row count; all arithmetic runs in the library.
 
 A layer instance keeps one set of activation buffers per row count, shared by
@@ -111,6 +111,63 @@ class SVDQLinear:
         if Y is None:
             Y = torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device)
         return self.gemm(self.quantize(X, stream), M, Y, stream)
+
+
+class SVDQLinearInt4:
+    """The INT4 W4A4 variant of SVDQLinear: the same smoothing and low-rank branch, the 4-bit
+    branch in INT4 groups of 64 along K with bf16 scales (svdq_quantize_act_int4 +
+    svdq_linear_int4).
+
+    Build with `from_weight` (host pack) or from a dict returned by lib.svdq_pack_weights_int4.
+    N must be a multiple of 128 (a multiple of 256 runs on the tensor cores).
+    """
+
+    def __init__(self, packed, K, N, rank, bias_bits=None, epilogue=lib.EPILOGUE_NONE, gelu_col_begin=0,
+                 device="cuda"):
+        self.K, self.N, self.rank = K, N, rank
+        self.epilogue, self.gelu_col_begin = epilogue, gelu_col_begin
+        self.device = _resolve(device)
+        _init_on(self.device)
+        device = self.device
+        self.inv_lambda = _dev(packed["inv_lambda"], device)
+        self.l1t = _dev(packed["l1t"], device, torch.bfloat16) if rank else None
+        self.l2t = _dev(packed["l2t"], device)
+        self.w_codes = _dev(packed["w_codes"], device)
+        self.w_scales = _dev(packed["w_scales"], device)
+        self.bias = _dev(bias_bits, device, torch.bfloat16) if bias_bits is not None else None
+        if self.bias is not None and self.bias.numel() != N:
+            raise ValueError(f"SVDQLinearInt4: bias must have {N} elements")
+        self._bufs = {}
+
+    @classmethod
+    def from_weight(cls, W_bits, act_absmax, rank, bias_bits=None, epilogue=lib.EPILOGUE_NONE,
+                    gelu_col_begin=0, device="cuda", seed=0):
+        K, N = W_bits.shape
+        packed = lib.svdq_pack_weights_int4(W_bits, act_absmax, rank, seed=seed)
+        return cls(packed, K, N, rank, bias_bits, epilogue, gelu_col_begin, device)
+
+    def buffers(self, M):
+        """Activation-side buffers for M rows (allocated once per M, shared by every call)."""
+        if M not in self._bufs:
+            sz = lib.svdq_int4_act_sizes(M, self.K)
+            self._bufs[M] = dict(
+                codes=torch.empty(sz["codes"], dtype=torch.uint8, device=self.device),
+                scales=torch.empty(sz["scales"], dtype=torch.uint8, device=self.device),
+                U=torch.empty(lib.svdq_act_sizes(M, self.K)["u"], dtype=torch.uint8, device=self.device))
+        return self._bufs[M]
+
+    def __call__(self, X, Y=None, stream=None):
+        _check_input(X, self.K, self.device, "SVDQLinearInt4")
+        M = X.shape[0]
+        if Y is None:
+            Y = torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device)
+        _check_output(Y, M, self.N, self.device, "SVDQLinearInt4")
+        b = self.buffers(M)
+        lib.svdq_quantize_act_int4(X, self.inv_lambda, self.l1t, self.rank, b["codes"], b["scales"], b["U"],
+                                   stream=stream)
+        lib.svdq_linear_int4(b["codes"], b["scales"], b["U"], self.w_codes, self.w_scales, self.l2t, self.bias, M,
+                             self.N, self.K, self.rank, self.epilogue, self.gelu_col_begin, Y, stream=stream)
+        return Y
 
 
 class SplitProjection:

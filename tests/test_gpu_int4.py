@@ -136,3 +136,22 @@ def test_int4_chain_mlp_fc1_full_size():
     want = int4.int4_linear(q[rows], s[rows], qw, sw, L.bf16_bits_to_f64(u[rows, :rank]), l2,
                             formats.bf16_bits_to_float(bb), svdquant.EPILOGUE_GELU_ERF, 0)
     G.parity("INT4 chain Y (GPU operands)", G.bf16_host(Y)[rows], want, TOL)
+
+
+def test_int4_layer_from_weight():
+    """The user-facing INT4 layer (host pack, K1, GEMM) against the oracle on the layer's own packed values."""
+    from bit_w4a4_diffusion_smooth_b200.layer import SVDQLinearInt4
+    m, k, n, rank = 130, 512, 256, 32
+    xb, x, wb, amax = _data(m, k, n, 77)
+    bb = synthetic.bias(n, 78)
+    layer = SVDQLinearInt4.from_weight(wb, amax, rank, bias_bits=bb, epilogue=svdquant.EPILOGUE_GELU_ERF)
+    y = G.bf16_host(layer(G.bf16_dev(xb)))
+    G.check_ok()
+    pk = lib.svdq_pack_weights_int4(wb, amax, rank)
+    l1 = L.bf16_bits_to_f64(pk["l1t"]).T
+    qa, sa, u = int4.quantize_act(x, pk["inv_lambda"], l1)
+    want = int4.int4_linear(qa, sa, L.int4_unpack(pk["w_codes"], n, k),
+                            L.int4_scales_unpack(pk["w_scales"], n, k // 64, n), formats.bf16_round(u),
+                            L.bf16_bits_to_f64(L.lowrank_unpack(pk["l2t"], n, 256))[:, :rank].T,
+                            formats.bf16_bits_to_float(bb), svdquant.EPILOGUE_GELU_ERF, 0)
+    G.parity("INT4 layer", y, want, TOL)

@@ -26,6 +26,8 @@
 //                the 128-byte-swizzled K-major layout (16 KB of A, 32 KB of B)
 //   warps 12..15 epilogue: TMEM -> registers (lane quarter = warp % 4), bias,
 //                GELU, bf16 rows to global memory
+// The pair form below (a cluster of 2 CTAs per 256 x 256 tile, cta_group::2
+// MMAs) is the one launched: each SM converts a third less per group.
 // Inside every 8-element chunk both operands hold k in the same permuted order
 // (k, k+4 pairs, so one mask-and-or makes a pair), which leaves the products'
 // sum unchanged.  Every wait is bounded: a wait that runs out records
@@ -300,6 +302,278 @@ __global__ void __launch_bounds__(THREADS, 1) int4_gemm_tc_kernel(const __grid_c
   }
 }
 
+// ---------------------------------------------------------------------------
+// Pair form: a cluster of 2 CTAs per 256 x 256 tile (cta_group::2 MMAs, M 256).
+// CTA h holds rows 128 h .. of the tile's A and output columns 128 h .. of its
+// B, converts only those (128 + 128 rows per group instead of 128 + 256) and
+// serves only its half of B to the tensor cores: a third less shared-memory
+// traffic per group than the single-CTA form.  The even CTA's thread issues
+// the MMAs once both CTAs' converters have arrived on its barrier; commits
+// multicast to both CTAs; each CTA drains its own 128 accumulator rows.
+constexpr int P_LSTAGES = 4, P_CSTAGES = 3;
+constexpr int P_A4 = 128 * 32, P_B4 = 128 * 32, P_SA = 256, P_SB = 256;
+constexpr int P_LSTAGE = 9216;                                   // 8,704 bytes used
+constexpr int P_HALF16 = 128 * 128;                              // 16 KB: 128 rows of 64 fp16
+constexpr int P_CSTAGE = 2 * P_HALF16;
+constexpr int P_CONV_OFF = 0;
+constexpr int P_LR_OFF = P_CONV_OFF + P_CSTAGES * P_CSTAGE;      // U rows + L2T half, 16 KB each
+constexpr int P_LOAD_OFF = P_LR_OFF + 2 * P_HALF16;
+constexpr int P_BAR_OFF = P_LOAD_OFF + P_LSTAGES * P_LSTAGE;
+constexpr int P_SMEM_BYTES = 1024 + P_BAR_OFF + 256;
+static_assert(P_A4 + P_B4 + P_SA + P_SB <= P_LSTAGE, "a pair load slot holds one group");
+static_assert(P_SMEM_BYTES <= 227 * 1024, "shared memory");
+constexpr bool kPair = true;   // the pair form runs the tcgen05 INT4 GEMM
+constexpr uint32_t IDESC_F16_PAIR = (1u << 4) | ((256 >> 3) << 17) | ((256 >> 4) << 24);
+constexpr uint32_t IDESC_BF16_PAIR = IDESC_F16_PAIR | (1u << 7) | (1u << 10);
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    int4_gemm_pair_kernel(const __grid_constant__ TcMaps maps, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *load_full = reinterpret_cast<uint64_t *>(smem + P_BAR_OFF);   // local
+  uint64_t *load_empty = load_full + P_LSTAGES;                          // local
+  uint64_t *conv_full = load_empty + P_LSTAGES;                          // even CTA: both CTAs' converters
+  uint64_t *conv_empty = conv_full + P_CSTAGES;                          // both: the multicast commit
+  uint64_t *lr_local = conv_empty + P_CSTAGES;                           // local low-rank bytes
+  uint64_t *lr_pair = lr_local + 1;                                      // even CTA: both CTAs' low-rank rows
+  uint64_t *tmem_full = lr_pair + 1;                                     // both
+  uint64_t *drain = tmem_full + 1;                                       // even CTA
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t h = dev::cluster_ctarank();
+  const int n0 = blockIdx.y * BN, m0 = static_cast<int>(blockIdx.x) * BM;    // blockIdx.x = 2 * pair + h
+  const int nb0 = n0 + 128 * static_cast<int>(h);                            // this CTA's B rows
+  const bool a_live = m0 < p.ld_sa;          // the odd CTA of a last, half pair has no rows
+  const int G = p.K / 64;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_LSTAGES; ++s) {
+      dev::mbar_init(&load_full[s], 1);
+      dev::mbar_init(&load_empty[s], 8);
+    }
+    for (int c = 0; c < P_CSTAGES; ++c) {
+      dev::mbar_init(&conv_full[c], 16);
+      dev::mbar_init(&conv_empty[c], 1);
+    }
+    dev::mbar_init(lr_local, 1);
+    dev::mbar_init(lr_pair, 2);
+    dev::mbar_init(tmem_full, 1);
+    dev::mbar_init(drain, 1);
+    *abort_flag = 0;
+    dev::fence_mbar_init();
+  }
+  if (warp == 1) {
+    dev::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    dev::tmem_relinquish_pair();
+  }
+  dev::tc_fence_before();
+  __syncwarp();
+  dev::cluster_sync();                       // both CTAs' barriers exist before anyone arrives remotely
+  dev::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  dev::grid_dependency_wait();
+  dev::grid_launch_dependents();
+  const uint32_t peer_abort = dev::mapa(dev::smem_u32(const_cast<int *>(abort_flag)), h ^ 1u);
+  auto fail_wait = [&]() {
+    *abort_flag = 1;
+    dev::st_cluster_u32(peer_abort, 1u);
+    dev::report(p.status, SVDQ_ERR_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      dev::prefetch_tmap(&maps.a);
+      dev::prefetch_tmap(&maps.b);
+      if (p.rank > 0) {
+        dev::mbar_arrive_expect_tx(lr_local, (a_live ? P_HALF16 : 0) + P_HALF16);
+        if (a_live) dev::bulk_load(smem + P_LR_OFF, p.U + static_cast<size_t>(m0) * 128, P_HALF16, lr_local);
+        dev::bulk_load(smem + P_LR_OFF + P_HALF16, p.l2t + static_cast<size_t>(nb0) * 128, P_HALF16, lr_local);
+      }
+      int issued = 0;
+      bool lr_sent = p.rank == 0;
+      for (int g = 0; g < G; ++g) {
+        const int s = g % P_LSTAGES;
+        if (!lr_sent && g == P_LSTAGES) {
+          // the first ring of loads is in flight: once this CTA's low-rank rows have landed, tell the
+          // even CTA, whose MMA thread starts with them (it must not wait for the whole loop, which
+          // itself waits on slots that only those MMAs free)
+          if (!dev::mbar_wait(lr_local, 0, p.limit_ns, abort_flag)) {
+            fail_wait();
+            break;
+          }
+          dev::mbar_arrive_cluster(dev::mapa(dev::smem_u32(lr_pair), 0));
+          lr_sent = true;
+        }
+        if (!dev::mbar_wait(&load_empty[s], ((g / P_LSTAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
+          fail_wait();
+          break;
+        }
+        uint8_t *st = smem + P_LOAD_OFF + s * P_LSTAGE;
+        // a CTA without rows loads no A codes or scales: its converters use scale 0, so its codes never count
+        dev::mbar_arrive_expect_tx(&load_full[s], (a_live ? P_A4 + P_SA : 0) + P_B4 + P_SB);
+        if (a_live) dev::tma_load_2d(st, &maps.a, &load_full[s], g * 32, m0);
+        dev::tma_load_2d(st + P_A4, &maps.b, &load_full[s], g * 32, nb0);
+        if (a_live)
+          dev::bulk_load(st + P_A4 + P_B4, p.a_scales + static_cast<size_t>(g) * p.ld_sa + m0, P_SA, &load_full[s]);
+        dev::bulk_load(st + P_A4 + P_B4 + P_SA, p.w_scales + static_cast<size_t>(g) * p.N + nb0, P_SB, &load_full[s]);
+        ++issued;
+      }
+      if (!lr_sent && issued == G) {   // G <= P_LSTAGES: the loop never reached the hand-off
+        if (dev::mbar_wait(lr_local, 0, p.limit_ns, abort_flag))
+          dev::mbar_arrive_cluster(dev::mapa(dev::smem_u32(lr_pair), 0));
+        else
+          fail_wait();
+      }
+      for (int g = max(0, issued - P_LSTAGES); g < issued; ++g)
+        dev::mbar_wait(&load_full[g % P_LSTAGES], (g / P_LSTAGES) & 1, p.limit_ns, nullptr);
+      if (p.rank > 0) dev::mbar_wait(lr_local, 0, p.limit_ns, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (h == 0 && lane == 0) {
+      bool ok = true, issued_any = false;
+      uint32_t accumulate = 0;
+      if (p.rank > 0) {
+        if (!dev::mbar_wait_cluster(lr_pair, 0, p.limit_ns, abort_flag)) {
+          fail_wait();
+          ok = false;
+        } else {
+          dev::tc_fence_after();
+          const uint32_t ua = dev::smem_u32(smem + P_LR_OFF), lb = ua + P_HALF16;
+          for (int j = 0; j < p.rank / 16; ++j) {
+            dev::umma_bf16_pair(tmem, dev::desc_sw128(ua + 32 * j), dev::desc_sw128(lb + 32 * j), IDESC_BF16_PAIR,
+                                accumulate);
+            accumulate = 1;
+          }
+          issued_any = true;
+        }
+      }
+      for (int g = 0; g < G && ok; ++g) {
+        const int c = g % P_CSTAGES;
+        if (!dev::mbar_wait(&conv_full[c], (g / P_CSTAGES) & 1, p.limit_ns, abort_flag)) {
+          fail_wait();
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        const uint32_t sa = dev::smem_u32(smem + P_CONV_OFF + c * P_CSTAGE), sb = sa + P_HALF16;
+        for (int j = 0; j < 4; ++j) {
+          dev::umma_bf16_pair(tmem, dev::desc_sw128(sa + 32 * j), dev::desc_sw128(sb + 32 * j), IDESC_F16_PAIR,
+                              accumulate);
+          accumulate = 1;
+        }
+        issued_any = true;
+        dev::tc_commit_pair_mc(&conv_empty[c], 0x3);   // both CTAs' slot c is free once these MMAs have read it
+      }
+      if (ok) dev::tc_commit_pair_mc(tmem_full, 0x3);
+      if (issued_any) {
+        dev::tc_commit_pair(drain);
+        dev::mbar_wait(drain, 0, p.limit_ns, nullptr);
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ converters (both CTAs)
+    const int ct = (warp - 4) * 32 + lane;           // 0..255
+    for (int g = 0; g < G; ++g) {
+      const int s = g % P_LSTAGES, c = g % P_CSTAGES;
+      if (!dev::mbar_wait_warp(&load_full[s], (g / P_LSTAGES) & 1, p.limit_ns, abort_flag) ||
+          !dev::mbar_wait_warp(&conv_empty[c], ((g / P_CSTAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
+        fail_wait();
+        break;
+      }
+      const uint8_t *st = smem + P_LOAD_OFF + s * P_LSTAGE;
+      const uint16_t *sc = reinterpret_cast<const uint16_t *>(st + P_A4 + P_B4);   // A then B scales
+      uint8_t *cv = smem + P_CONV_OFF + c * P_CSTAGE;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        // half-row hr of the 256 rows (A 0..127, B 128..255): 32 codes, k 32 h .. 32 h + 31
+        const int hr = ct + 256 * j, row = hr >> 1, hh = hr & 1;
+        const uint4 q = *reinterpret_cast<const uint4 *>(st + row * 32 + hh * 16);
+        const uint16_t sbits = (row < 128 && !a_live) ? 0 : sc[row];
+        const __half s16 = __float2half_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));
+        const __half2 s2 = __halves2half2(s16, s16);
+        const int r = row & 127;
+        uint8_t *tile = cv + (row < 128 ? 0 : P_HALF16) + r * 128;
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int chunk = 4 * hh + w;
+          *reinterpret_cast<uint4 *>(tile + (((chunk ^ r) & 7) << 4)) = dequant8(words[w], s2);
+        }
+      }
+      dev::fence_proxy_async();                      // the tensor cores read what the threads wrote
+      __syncwarp();
+      if (lane == 0) {
+        dev::mbar_arrive(&load_empty[s]);
+        dev::mbar_arrive_remote(dev::mapa(dev::smem_u32(&conv_full[c]), 0));
+      }
+    }
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    if (dev::mbar_wait_warp(tmem_full, 0, p.limit_ns, abort_flag)) {
+      dev::tc_fence_after();
+      const int row = 32 * q + lane, grow = m0 + row;
+#pragma unroll 1
+      for (int cb = 0; cb < BN / 32; ++cb) {
+        uint32_t v[32];
+        dev::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + 32 * cb, v);
+        dev::tmem_wait_ld();
+        const int c0 = n0 + 32 * cb;
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + 2 * i;
+          float2 y = make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          if (p.bias) {
+            const uint32_t bb = __ldg(reinterpret_cast<const uint32_t *>(p.bias + c));
+            y.x += __uint_as_float(bb << 16);
+            y.y += __uint_as_float(bb & 0xFFFF0000u);
+          }
+          if constexpr (EPI == SVDQ_EPILOGUE_GELU_ERF) {
+            const float2 gy = dev::gelu_erf2(y);
+            y = make_float2(c >= p.gelu_col_begin ? gy.x : y.x, c + 1 >= p.gelu_col_begin ? gy.y : y.y);
+          } else if constexpr (EPI == SVDQ_EPILOGUE_GELU_TANH) {
+            y = make_float2(c >= p.gelu_col_begin ? dev::gelu_tanh(y.x) : y.x,
+                            c + 1 >= p.gelu_col_begin ? dev::gelu_tanh(y.y) : y.y);
+          }
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(y.x, y.y);
+          packed[i] = *reinterpret_cast<uint32_t *>(&h2);
+        }
+        if (grow < p.M) {
+          uint4 *dst = reinterpret_cast<uint4 *>(p.Y + static_cast<size_t>(grow) * p.ldy + c0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+    } else {
+      fail_wait();
+    }
+  }
+  dev::tc_fence_before();
+  __syncwarp();
+  dev::cluster_sync();                       // no MMA of the pair still reads either CTA's shared memory
+  if (warp == 1) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+template <int EPI>
+int launch_pair(const TcMaps &maps, const TcParams &p, cudaStream_t stream) {
+  const int rc = smem_optin_once<int4_gemm_pair_kernel<EPI>>(P_SMEM_BYTES, "svdq_linear_int4");
+  if (rc != SVDQ_OK) return rc;
+  DependentLaunch dl(dim3(2 * ((p.ld_sa + 255) / 256), p.N / BN), dim3(THREADS), P_SMEM_BYTES, stream);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, int4_gemm_pair_kernel<EPI>, maps, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("svdq_linear_int4 launch: ") + cudaGetErrorString(e));
+  return ok();
+}
+
 template <int EPI>
 int launch(const TcMaps &maps, const TcParams &p, cudaStream_t stream) {
   const int rc = smem_optin_once<int4_gemm_tc_kernel<EPI>>(SMEM_BYTES, "svdq_linear_int4");
@@ -323,7 +597,8 @@ int launch_int4_tc(const uint8_t *a_codes, const void *a_scales, const void *U, 
                           static_cast<uint64_t>(mp), static_cast<uint64_t>(K / 2), 32, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc != SVDQ_OK) return rc;
   rc = encode_tmap_2d(&maps.b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, static_cast<uint64_t>(K / 2),
-                      static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 32, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
+                      static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 32, kPair ? 128 : BN,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
   if (rc != SVDQ_OK) return rc;
   TcParams p;
   p.a_scales = static_cast<const uint16_t *>(a_scales);
@@ -341,6 +616,13 @@ int launch_int4_tc(const uint8_t *a_codes, const void *a_scales, const void *U, 
   p.gelu_col_begin = gelu_col_begin;
   p.status = status;
   p.limit_ns = kWaitLimitNs;
+  if (kPair) {
+    switch (epilogue) {
+      case SVDQ_EPILOGUE_GELU_ERF: return launch_pair<SVDQ_EPILOGUE_GELU_ERF>(maps, p, stream);
+      case SVDQ_EPILOGUE_GELU_TANH: return launch_pair<SVDQ_EPILOGUE_GELU_TANH>(maps, p, stream);
+      default: return launch_pair<SVDQ_EPILOGUE_NONE>(maps, p, stream);
+    }
+  }
   switch (epilogue) {
     case SVDQ_EPILOGUE_GELU_ERF: return launch<SVDQ_EPILOGUE_GELU_ERF>(maps, p, stream);
     case SVDQ_EPILOGUE_GELU_TANH: return launch<SVDQ_EPILOGUE_GELU_TANH>(maps, p, stream);

@@ -112,6 +112,23 @@ def test_int4_gemm_matches_oracle(m, k, n, rank, epilogue, begin, with_bias):
     G.parity(f"INT4 K2 Y, M={m} K={k} N={n} r={rank}", y, want, TOL)
 
 
+def test_int4_gemm_many_tiles_sampled():
+    """Several 256 x 256 tiles per SM pair (both accumulators in turn), a last half pair, rank 16, tanh GELU
+    from column 1000: sampled rows against the oracle on the same operands."""
+    m, k, n, rank = 4480, 1024, 5120, 16
+    xb, x, wb, amax = _data(m, k, n, 55)
+    p = int4.pack(formats.bf16_bits_to_float(wb), amax, rank)
+    qa, sa, u = int4.quantize_act(x, p["inv_lambda"], p["l1"])
+    ub = formats.bf16_round(u)
+    bb = synthetic.bias(n, 56)
+    y = _k2(qa, sa, L.bf16_bits(ub), p["qw"], p["sw"], p["l2"], bb, m, n, k, rank, svdquant.EPILOGUE_GELU_TANH, 1000)
+    rows = np.sort(np.random.default_rng(57).choice(m, 24, replace=False))
+    rows[-1] = m - 1                                                 # a row of the last, half pair
+    want = int4.int4_linear(qa[rows], sa[rows], p["qw"], p["sw"], ub[rows], p["l2"],
+                            formats.bf16_bits_to_float(bb), svdquant.EPILOGUE_GELU_TANH, 1000)
+    G.parity("INT4 K2 Y many tiles (sampled rows)", y[rows], want, TOL)
+
+
 def test_int4_chain_mlp_fc1_full_size():
     """4608 x 3072 -> 12288 with the erf GELU: the library's host pack, K1 then K2 on the GPU."""
     m, k, n, rank = 4608, 3072, 12288, 32

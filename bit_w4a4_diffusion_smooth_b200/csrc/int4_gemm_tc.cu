@@ -29,15 +29,18 @@
 //                issues per tile the low-rank MMAs (kind::f16, bf16, straight
 //                from the U and L2T tiles, whose layout is the operand image)
 //                and then 4 MMAs per group (kind::f16, fp16 operands) from a
-//                ring of 3 converted slots, committing each slot back to both
+//                ring of 4 converted slots, committing each slot back to both
 //                CTAs (multicast commit)
 //   warp 2       low-rank loader: per tile the CTA's U rows and L2T rows, then
 //                tells the even CTA they have landed
-//   warps 4..19  converters: half-precision q * s of the slot's 256 rows into
-//                the 128-byte-swizzled K-major layout, one 32-code half row
-//                per thread and group; then a CTA-scope arrive on the even
-//                CTA's barrier (the hand-off CUTLASS's SM100 mixed-input
-//                pipeline makes: no cluster-scope fence per group)
+//   warps 4..19  converters, 4 teams of 4 warps; team j takes the groups
+//                g = j mod 4, so four groups are converted at once: half-
+//                precision q * s of the group's 256 rows into the
+//                128-byte-swizzled K-major layout (4 half rows of 32 codes per
+//                thread), then a CTA-scope arrive on the even CTA's barrier
+//                (the hand-off CUTLASS's SM100 mixed-input pipeline makes: no
+//                cluster-scope fence per group).  With all 16 warps on one
+//                group at a time the conversion was a latency chain per group
 //   warps 20..23 epilogue: TMEM -> registers (lane quarter = warp % 4), bias,
 //                GELU, bf16 rows to global memory, then the accumulator is
 //                handed back to the even CTA
@@ -61,12 +64,14 @@ namespace svdq {
 namespace {
 
 constexpr int BN = 256;                                          // output columns per pair tile
-constexpr int LSTAGES = 4, CSTAGES = 3;
+constexpr int LSTAGES = 4, CSTAGES = 4;
 constexpr int NCONV = 16;                                        // converter warps per CTA
+constexpr int TEAMS = 4;                                         // teams of converters take groups in turn
+constexpr int TEAM_WARPS = NCONV / TEAMS;
 constexpr int CONV_WARP0 = 4, EPI_WARP0 = CONV_WARP0 + NCONV;
 constexpr int THREADS = (EPI_WARP0 + 4) * 32;
 constexpr int HALF_ROWS = 512;                                   // 256 rows x 2 halves of 32 codes per group
-constexpr int HR_PER_THREAD = HALF_ROWS / (NCONV * 32);
+constexpr int HR_PER_THREAD = HALF_ROWS / (TEAM_WARPS * 32);
 constexpr int A4 = 128 * 32, B4 = 128 * 32, SA = 256, SB = 256;  // one group: codes and scales of 128 + 128 rows
 constexpr int LSTAGE = 9216;                                     // 8,704 bytes used
 constexpr int HALF16 = 128 * 128;                                // 16 KB: 128 rows of 64 fp16 (or bf16)
@@ -78,7 +83,12 @@ constexpr int BAR_OFF = LOAD_OFF + LSTAGES * LSTAGE;
 constexpr int SMEM_BYTES = 1024 + BAR_OFF + 256;
 constexpr uint32_t TMEM_COLS = 512;                              // two 256-column accumulators
 static_assert(A4 + B4 + SA + SB <= LSTAGE, "a load slot holds one group");
-static_assert(HALF_ROWS % (NCONV * 32) == 0, "converters split the half rows evenly");
+static_assert(HALF_ROWS % (TEAM_WARPS * 32) == 0 && NCONV % TEAMS == 0, "a team splits the half rows evenly");
+static_assert(LSTAGES % TEAMS == 0, "a load slot always serves the same team");
+// A team that reaches group g finished g - TEAMS, which needs only the MMAs up to
+// g - TEAMS - CSTAGES; the slot of g must then be at most one phase behind the
+// one the team waits for (an mbarrier parity wait cannot tell phases two apart).
+static_assert(TEAMS <= CSTAGES, "no converter team runs two phases ahead of a slot");
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 // instruction descriptors: f32 accumulate (bit 4), A/B fp16 (0) or bf16 (1) at bits 7 and 10,
 // N >> 3 at bit 17, M >> 4 at bit 24 (M 256: the pair), both operands K-major
@@ -149,10 +159,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < LSTAGES; ++s) {
       dev::mbar_init(&load_full[s], 1);
-      dev::mbar_init(&load_empty[s], NCONV);
+      dev::mbar_init(&load_empty[s], TEAM_WARPS);
     }
     for (int c = 0; c < CSTAGES; ++c) {
-      dev::mbar_init(&conv_full[c], 2 * NCONV);
+      dev::mbar_init(&conv_full[c], 2 * TEAM_WARPS);
       dev::mbar_init(&conv_empty[c], 1);
     }
     dev::mbar_init(lr_local, 1);
@@ -295,13 +305,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   } else if (warp >= CONV_WARP0 && warp < EPI_WARP0) {
     // ------------------------------------------------------------ converters (both CTAs)
-    const int ct = (warp - CONV_WARP0) * 32 + lane;
+    const int team = (warp - CONV_WARP0) / TEAM_WARPS;
+    const int ct = ((warp - CONV_WARP0) % TEAM_WARPS) * 32 + lane;
     int gi = 0;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
       const PairTile pt = pair_tile(t, tiles_m);
       const bool a_live = (2 * pt.m2 + static_cast<int>(h)) * 128 < p.ld_sa;
       for (int g = 0; g < G; ++g, ++gi) {
+        if (gi % TEAMS != team) continue;            // the other teams' groups
         const int s = gi % LSTAGES, c = gi % CSTAGES;
         if (!dev::mbar_wait_warp(&load_full[s], (gi / LSTAGES) & 1, p.limit_ns, abort_flag) ||
             !dev::mbar_wait_warp(&conv_empty[c], ((gi / CSTAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
@@ -315,7 +327,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int j = 0; j < HR_PER_THREAD; ++j) {
           // half row hr of the 256 rows (activations 0..127, weights 128..255): 32 codes, k 32 hh .. 32 hh + 31
-          const int hr = ct + NCONV * 32 * j, row = hr >> 1, hh = hr & 1;
+          const int hr = ct + TEAM_WARPS * 32 * j, row = hr >> 1, hh = hr & 1;
           const uint4 q = *reinterpret_cast<const uint4 *>(st + row * 32 + hh * 16);
           const uint16_t sbits = (row < 128 && !a_live) ? 0 : sc[row];
           const __half s16 = __float2half_rn(__uint_as_float(static_cast<uint32_t>(sbits) << 16));

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -67,34 +68,97 @@ EncodeTiledFn encode_fn() {
 }
 }  // namespace
 
-int encode_tmap_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
-                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+namespace {
+// Encoded tensor maps, cached by every argument of the encode: a map is a pure
+// function of them (base address, extents, strides, box, swizzle, element
+// type), so a hit returns exactly what the driver would encode again.  The
+// per-call cost of a layer's GEMM (seven maps) and activation kernel (two)
+// then shrinks to lookups once its buffers have been seen.  Direct-mapped; a
+// colliding entry is simply replaced.
+struct TmapKey {
+  uint64_t dims[3], strides[2];
+  const void *base;
+  uint32_t box[3];
+  int dtype, rank, swizzle;
+};
+struct TmapEntry {
+  CUtensorMap map;
+  TmapKey key;
+  bool valid;
+};
+constexpr size_t kTmapCacheSize = 1024;
+std::mutex g_tmap_mutex;
+TmapEntry g_tmap_cache[kTmapCacheSize];
+
+TmapKey make_key(int rank, CUtensorMapDataType dtype, const void *base, const uint64_t *dims, const uint64_t *strides,
+                 const uint32_t *box, CUtensorMapSwizzle swizzle) {
+  TmapKey k;
+  std::memset(&k, 0, sizeof(k));   // padding bytes take part in the comparison
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+  k.base = base;
+  k.dtype = static_cast<int>(dtype);
+  k.rank = rank;
+  k.swizzle = static_cast<int>(swizzle);
+  return k;
+}
+
+size_t key_slot(const TmapKey &k) {
+  uint64_t h = 1469598103934665603ull;   // FNV-1a over the key's bytes
+  const unsigned char *b = reinterpret_cast<const unsigned char *>(&k);
+  for (size_t i = 0; i < sizeof(k); ++i) h = (h ^ b[i]) * 1099511628211ull;
+  return static_cast<size_t>(h % kTmapCacheSize);
+}
+
+int encode_tiled(int rank, CUtensorMap *out, CUtensorMapDataType dtype, const void *base, const uint64_t *dims,
+                 const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swizzle) {
+  const TmapKey key = make_key(rank, dtype, base, dims, strides, box, swizzle);
+  const size_t slot = key_slot(key);
+  {
+    std::lock_guard<std::mutex> lock(g_tmap_mutex);
+    const TmapEntry &e = g_tmap_cache[slot];
+    if (e.valid && std::memcmp(&e.key, &key, sizeof(key)) == 0) {
+      *out = e.map;
+      return SVDQ_OK;
+    }
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_stride_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = fn(out, dtype, 2, const_cast<void *>(base), dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cuuint64_t d[3] = {0, 0, 0}, st[2] = {0, 0};
+  cuuint32_t bx[3] = {0, 0, 0}, estride[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+  CUresult r = fn(out, dtype, static_cast<cuuint32_t>(rank), const_cast<void *>(base), d, st, bx, estride,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
-    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string(static_cast<int>(r)) + ")");
+    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (" + std::to_string(rank) + "-D) failed (code " +
+                                   std::to_string(static_cast<int>(r)) + ")");
+  std::lock_guard<std::mutex> lock(g_tmap_mutex);
+  TmapEntry &e = g_tmap_cache[slot];
+  e.map = *out;
+  e.key = key;
+  e.valid = true;
   return SVDQ_OK;
+}
+}  // namespace
+
+int encode_tmap_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, uint64_t inner, uint64_t outer,
+                   uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  const uint64_t dims[2] = {inner, outer}, strides[1] = {row_stride_bytes};
+  const uint32_t box[2] = {box_inner, box_outer};
+  return encode_tiled(2, out, dtype, base, dims, strides, box, swizzle);
 }
 
 int encode_tmap_3d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, const uint64_t (&dims)[3],
                    const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swizzle) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
-  cuuint64_t st[2] = {strides[0], strides[1]};
-  cuuint32_t bx[3] = {box[0], box[1], box[2]};
-  cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = fn(out, dtype, 3, const_cast<void *>(base), d, st, bx, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS)
-    return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (code " + std::to_string(static_cast<int>(r)) + ")");
-  return SVDQ_OK;
+  return encode_tiled(3, out, dtype, base, dims, strides, box, swizzle);
 }
 
 namespace {

@@ -249,3 +249,33 @@ def test_layer_and_binding_reject_mismatched_buffers():
                              layer.bias, c.m, c.n, c.k, c.rank, 0, 0,
                              torch.empty((c.m, c.n), dtype=torch.bfloat16, device=G.DEV))
     G.check_ok()
+
+
+def test_layer_repeated_calls_match_checked_path():
+    """A layer's later calls on the same buffers (pointers, shapes, strides, stream) go straight to
+    the C entry points with the arguments marshalled on the first call: their outputs are bit-identical
+    to those of the fully checked path on the same inputs, also after X's contents change in place
+    and for another row count (a new set of buffers)."""
+    from bit_w4a4_diffusion_smooth_b200.layer import SVDQLinear
+    c = synthetic.TINY
+    xb, wb, bb = c.make()
+    x = formats.bf16_bits_to_float(xb)
+    amax = np.max(np.abs(x), axis=0).astype(np.float32)
+    layer = SVDQLinear.from_weight(wb, amax, c.rank, bb, epilogue=lib.EPILOGUE_GELU_ERF)
+    fresh = lambda: SVDQLinear.from_weight(wb, amax, c.rank, bb, epilogue=lib.EPILOGUE_GELU_ERF)
+    X = G.bf16_dev(xb)
+    Y = torch.empty((c.m, c.n), dtype=torch.bfloat16, device=G.DEV)
+    y1 = G.bf16_host(layer(X, Y))                        # first call: checked path, plan recorded
+    xb2 = synthetic.activation(c.m, c.k, c.seed + 7, synthetic.count(0.01, c.k), 50.0)[0]
+    X.copy_(G.bf16_dev(xb2))                             # same buffer, new contents
+    y2 = G.bf16_host(layer(X, Y))                        # repeated call: the recorded plan
+    G.check_ok()
+    np.testing.assert_array_equal(y1, G.bf16_host(fresh()(G.bf16_dev(xb))))
+    np.testing.assert_array_equal(y2, G.bf16_host(fresh()(G.bf16_dev(xb2))))
+    m2 = c.m - 5                                         # another row count: new buffers, new plan
+    Y2 = torch.empty((m2, c.n), dtype=torch.bfloat16, device=G.DEV)
+    y3 = G.bf16_host(layer(X[:m2], Y2))
+    y4 = G.bf16_host(layer(X[:m2], Y2))
+    G.check_ok()
+    np.testing.assert_array_equal(y3, G.bf16_host(fresh()(G.bf16_dev(xb2[:m2]))))
+    np.testing.assert_array_equal(y4, y3)

@@ -108,17 +108,25 @@ struct TcMaps {
 };
 
 // Four fp16 pairs of one word of eight codes (element i at bits 4i), in the
-// permuted k order (i, i + 4): pair i = (q_i s, q_{i+4} s), exact.
+// permuted k order (i, i + 4): pair i = (q_i s, q_{i+4} s), exact.  One
+// mask-and-xor per pair puts the offset-binary code u = q + 8 (the nibble with
+// its top bit flipped) into an fp16 mantissa: at bits 0..3 under the exponent
+// of 1024 (value 1024 + u), at bits 4..7 under the exponent of 64 (whose
+// mantissa bit 4 weighs 1: value 64 + u), so one shift by 8 serves the four
+// pairs; subtracting 1032 or 72 gives q exactly, and the multiply q s.
 __device__ __forceinline__ uint4 dequant8(uint32_t x, __half2 s2) {
-  const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
+  const __half2 b1024 = __floats2half2_rn(1032.0f, 1032.0f), b64 = __floats2half2_rn(72.0f, 72.0f);
+  const uint32_t y = x >> 8;
+  uint32_t t[4];
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[0]) : "r"(x), "r"(0x000F000Fu), "r"(0x64086408u));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[1]) : "r"(x), "r"(0x00F000F0u), "r"(0x54805480u));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[2]) : "r"(y), "r"(0x000F000Fu), "r"(0x64086408u));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t[3]) : "r"(y), "r"(0x00F000F0u), "r"(0x54805480u));
   uint32_t o[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // nibble -> fp16 1024 + (q + 8): the offset-binary code (q xor 8 on the low 4 bits) in the mantissa
-    uint32_t t;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(t) : "r"(x >> (4 * i)), "r"(0x000F000Fu), "r"(0x64086408u));
-    const __half2 q = __hsub2(*reinterpret_cast<__half2 *>(&t), bias);       // q, exact
-    const __half2 v = __hmul2(q, s2);                                         // q s, exact
+    const __half2 q = __hsub2(*reinterpret_cast<__half2 *>(&t[i]), (i & 1) ? b64 : b1024);   // q, exact
+    const __half2 v = __hmul2(q, s2);                                                       // q s, exact
     o[i] = *reinterpret_cast<const uint32_t *>(&v);
   }
   return make_uint4(o[0], o[1], o[2], o[3]);

@@ -8,9 +8,11 @@ against the oracle (oracle/int4.py), through the C ABI.
     tests/layouts.py): Y within the parity bar (excess error over the row RMS
     <= 1e-2, as for the NVFP4 GEMM); ragged M, K up to 3072, GELU from inside
     the output, no bias, rank 0.
-  * The chain K1 -> K2 at the MLP fc1 size (4608 x 3072 -> 12288, erf GELU)
-    with the library's host pack: codes and scales of sampled rows bit-exact,
-    and Y of those rows against the oracle on the GPU's own operands.
+  * The chain K1 -> K2 at full size on the MLP fc1 (4608 x 3072 -> 12288, erf
+    GELU), the single block's fused QKV + MLP-in (-> 21504, GELU from column
+    9216) and its output projection (K = 15360), with the library's host pack:
+    codes and scales of sampled rows bit-exact, and Y of those rows against the
+    oracle on the GPU's own operands.
 """
 import numpy as np
 import pytest
@@ -129,30 +131,39 @@ def test_int4_gemm_many_tiles_sampled():
     G.parity("INT4 K2 Y many tiles (sampled rows)", y[rows], want, TOL)
 
 
-def test_int4_chain_mlp_fc1_full_size():
-    """4608 x 3072 -> 12288 with the erf GELU: the library's host pack, K1 then K2 on the GPU."""
-    m, k, n, rank = 4608, 3072, 12288, 32
-    xb, x, wb, amax = _data(m, k, n, 90)
+@pytest.mark.parametrize("name,m,k,n,epilogue,begin,seed", [
+    ("mlp fc1", 4608, 3072, 12288, svdquant.EPILOGUE_GELU_ERF, 0, 90),
+    ("single qkv_mlp", 4608, 3072, 21504, svdquant.EPILOGUE_GELU_ERF, 9216, 93),
+    ("single out", 4608, 15360, 3072, svdquant.EPILOGUE_NONE, 0, 96)])
+def test_int4_chain_full_size(name, m, k, n, epilogue, begin, seed):
+    """The layer shapes of a 12B-class DiT at full size (the MLP fc1 with the erf GELU; the single
+    block's fused QKV + MLP-in with GELU on columns 9216.. only; its output projection at K =
+    15360): the library's host pack, K1 then K2 on the GPU, in the benchmark's launch
+    configuration.  Codes and scales of sampled rows bit-exact, Y of those rows against the oracle
+    on the GPU's own operands."""
+    rank = 32
+    xb, x, wb, amax = _data(m, k, n, seed)
     pk = lib.svdq_pack_weights_int4(wb, amax, rank)
-    bb = synthetic.bias(n, 91)
+    bb = synthetic.bias(n, seed + 1)
     l1 = L.bf16_bits_to_f64(pk["l1t"]).T
     codes, scales, U = _k1(xb, m, k, rank, pk["inv_lambda"], l1)
     Y = G.poisoned_bf16(m, n)
     lib.svdq_linear_int4(codes, scales, U, G.dev(pk["w_codes"]), G.dev(pk["w_scales"]), G.dev(pk["l2t"]),
-                         G.bf16_dev(bb), m, n, k, rank, svdquant.EPILOGUE_GELU_ERF, 0, Y)
+                         G.bf16_dev(bb), m, n, k, rank, epilogue, begin, Y)
     G.check_ok()
-    rows = np.sort(np.random.default_rng(92).choice(m, 24, replace=False))
+    rows = np.sort(np.random.default_rng(seed + 2).choice(m, 24, replace=False))
+    rows[0], rows[-1] = 0, m - 1
     q, s, u = _unpack_k1(codes, scales, U, m, k)
     oq, osf, ou = int4.quantize_act(x[rows], pk["inv_lambda"], l1)
     np.testing.assert_array_equal(q[rows], oq)
     np.testing.assert_array_equal(s[rows], osf)
-    G.parity("INT4 chain U", L.bf16_bits_to_f64(u[rows, :rank]), ou, TOL)
+    G.parity(f"INT4 {name} U", L.bf16_bits_to_f64(u[rows, :rank]), ou, TOL)
     qw = L.int4_unpack(pk["w_codes"], n, k)
     sw = L.int4_scales_unpack(pk["w_scales"], n, k // 64, n)
     l2 = L.bf16_bits_to_f64(L.lowrank_unpack(pk["l2t"], n, 256))[:, :rank].T
     want = int4.int4_linear(q[rows], s[rows], qw, sw, L.bf16_bits_to_f64(u[rows, :rank]), l2,
-                            formats.bf16_bits_to_float(bb), svdquant.EPILOGUE_GELU_ERF, 0)
-    G.parity("INT4 chain Y (GPU operands)", G.bf16_host(Y)[rows], want, TOL)
+                            formats.bf16_bits_to_float(bb), epilogue, begin)
+    G.parity(f"INT4 {name} Y (GPU operands)", G.bf16_host(Y)[rows], want, TOL)
 
 
 def test_int4_layer_from_weight():

@@ -136,3 +136,20 @@ def test_pack_argument_checks():
         lib.awq_pack_weights(np.zeros((64, 48), np.uint16), np.ones(64, np.float32))
     with pytest.raises(lib.SvdqError):
         lib.awq_pack_weights(np.zeros((64, 64), np.uint16), np.zeros(64, np.float32))
+
+
+def test_empty_inputs_are_rejected_as_shapes():
+    """M = 0 (an empty batch) and a zero width are shape errors of every device call and size query,
+    reported before anything touches a GPU."""
+    so = lib.load()
+    p = ctypes.c_void_p(16)  # never dereferenced: the shape check fails first
+    assert so.svdq_quantize_act(p, 0, 256, 256, p, p, 16, p, p, p, p, None) == lib.ERR_SHAPE
+    assert so.svdq_linear_w4a4(p, p, p, p, p, p, None, 0, 256, 256, 16, 0, 0, p, 256, None) == lib.ERR_SHAPE
+    assert so.svdq_linear_w4a4(p, p, p, p, p, p, None, 64, 0, 256, 16, 0, 0, p, 256, None) == lib.ERR_SHAPE
+    assert so.svdq_quantize_act_int4(p, 0, 256, 256, p, p, 16, p, p, p, None) == lib.ERR_SHAPE
+    assert so.svdq_linear_int4(p, p, p, p, p, p, None, 0, 256, 256, 16, 0, 0, p, 256, None) == lib.ERR_SHAPE
+    for call in (lambda: lib.svdq_act_sizes(0, 256), lambda: lib.svdq_int4_act_sizes(0, 256),
+                 lambda: lib.svdq_weight_sizes(256, 0, 16), lambda: lib.svdq_int4_weight_sizes(256, 0)):
+        with pytest.raises(lib.SvdqError) as e:
+            call()
+        assert e.value.status == lib.ERR_SHAPE

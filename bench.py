@@ -955,11 +955,14 @@ def run_dit_step(args):
     one_t = torch.ones(1, device=device)
     s_w = torch.full((1,), 1e-3, device=device)
     pools, act, layers = {}, {}, []
+    cond = {}     # the modulation projections all read the step's conditioning vector
     for kind, name, m, k, n, gbeg in plan:
         if kind == "awq":
             g_n = k // 64
+            if (m, k) not in cond:
+                cond[(m, k)] = rand_bf16(m, k)
             layers.append(dict(kind=kind, m=m, k=k, n=n,
-                               X=rand_bf16(m, k), inv=torch.ones(k, device=device),
+                               X=cond[(m, k)], inv=torch.ones(k, device=device),
                                qw=torch.randint(0, 2 ** 31, (k // 8 * n,), dtype=torch.int32, device=device,
                                                 generator=gen),
                                sc=(torch.rand(g_n * n, device=device, generator=gen) * 1e-3).to(torch.bfloat16),
@@ -993,9 +996,16 @@ def run_dit_step(args):
             prev_fc1[L["name"].rsplit(".", 1)[0]] = L["Y"]
 
     # launch units: with --group-streams on, the image and text instances of a dual-stream block's
-    # projection run as one grouped K1 and one grouped K2 launch (adjacent in the plan)
+    # projection run as one grouped K1 and one grouped K2 launch (adjacent in the plan); with
+    # --group-awq on, every modulation projection of the step (they depend only on the conditioning
+    # vector) runs in one grouped AWQ launch at the start of the step
     units = []
+    awq_layers = [L for L in layers if L["kind"] == "awq"]
+    if args.group_awq == "on" and awq_layers:
+        units.append(awq_layers)
     for L in layers:
+        if args.group_awq == "on" and L["kind"] == "awq":
+            continue
         prev = units[-1] if units else None
         if (args.group_streams == "on" and L["kind"] == "w4a4" and L["name"].startswith("dual.txt.") and prev
                 and prev[0]["kind"] == "w4a4" and prev[0]["name"] == L["name"].replace(".txt.", ".img.")):
@@ -1005,6 +1015,11 @@ def run_dit_step(args):
 
     def run_unit(unit):
         L = unit[0]
+        if L["kind"] == "awq" and len(unit) > 1:
+            lib.awq_linear_w4a16_grouped([dict(X=u["X"], inv_awq=u["inv"], qweight=u["qw"], scales=u["sc"],
+                                               zeros=u["z"], bias=u["b"], N=u["n"], Y=u["Y"]) for u in unit],
+                                         L["m"], L["k"])
+            return
         if L["kind"] == "awq":
             lib.awq_linear_w4a16(L["X"], L["inv"], L["qw"], L["sc"], L["z"], L["b"], L["n"], L["Y"])
             return
@@ -1092,6 +1107,21 @@ def run_dit_step(args):
         breakdown.append({"layer": name if kind == "w4a4" else f"{name} (AWQ)", "m": m, "k": k, "n": n,
                           "count": cnt, "us_each": round(us, 2), "TFLOP/s": round(fl / (us * 1e-6) / 1e12, 1),
                           "ms_per_step": round(us * cnt / 1e3, 3)})
+    if args.group_awq == "on" and awq_layers:  # the grouped modulation launch alone
+        for _ in range(3):
+            run_unit(awq_layers)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            run_unit(awq_layers)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) / 10 * 1e3
+        wbytes = sum(L["n"] * L["k"] // 2 + 2 * 2 * L["n"] * (L["k"] // 64) for L in awq_layers)
+        breakdown.append({"layer": f"all {len(awq_layers)} modulation projections (AWQ, one grouped launch)",
+                          "us_each": round(us, 2), "count": 1, "ms_per_step": round(us / 1e3, 3),
+                          "weight_GB/s": round(wbytes / (us * 1e-6) / 1e9, 1)})
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -1118,6 +1148,9 @@ def run_dit_step(args):
                    "group_streams": (f"{args.group_streams}: a dual-stream block's image and text instances of "
                                      "each projection run as one grouped K1 and one grouped K2 launch"
                                      if args.group_streams == "on" else "off: every layer its own launches"),
+                   "group_awq": ("on: the step's modulation projections (one shared conditioning vector) run as "
+                                 "one grouped AWQ launch" if args.group_awq == "on" else
+                                 "off: every modulation projection its own launch"),
                    "layers": {"w4a4": n_w4a4, "awq": n_awq}, "flops_per_step": flops},
         "breakdown": breakdown,
         "gpu_launches": args.steps * sum(1 if u[0]["kind"] == "awq" else 2 for u in units),
@@ -1144,6 +1177,8 @@ def main():
                     help="layers: QKV + MLP pair + AWQ projection (default); dit-step: one whole DiT step")
     ap.add_argument("--group-streams", choices=("on", "off"), default="on",
                     help="dit-step: image and text instances of a dual-stream projection as one grouped launch")
+    ap.add_argument("--group-awq", choices=("on", "off"), default="on",
+                    help="dit-step: the step's modulation projections (one shared input) as one grouped AWQ launch")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = {"reference": 10}.get(args.impl, 300 if args.workload == "layers" else 200)

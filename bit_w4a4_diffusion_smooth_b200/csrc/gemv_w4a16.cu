@@ -32,6 +32,11 @@
 // More than 16 rows (a batch of modulation vectors) run as blocks of 16 rows
 // on the grid's second dimension; each block is one more pass over the
 // weights, mostly from L2.
+// A grouped launch runs several projections of the same input shape (the
+// modulation layers of a DiT step all read the same conditioning vector):
+// their quads form one sequence on the grid's first dimension, problem after
+// problem, and each CTA finds its problem by a binary search over the prefix
+// sums of the quad counts.  A single call is a group of one (no search).
 // The weight layout (qweight) is the MMA fragment order; see svdq.h.
 #include <cuda_runtime.h>
 
@@ -69,6 +74,16 @@ struct Params {
   uint16_t *Y;
   unsigned int *status;
   unsigned long long limit_ns;
+};
+
+// Up to C problems of the same M and K in one launch; quad_end holds the prefix sums of
+// their quad counts (N / 64).
+constexpr int kAwqMaxGroup = SVDQ_AWQ_MAX_GROUP;
+template <int C>
+struct AwqGroup {
+  Params p[C];
+  int quad_end[C];
+  int count;
 };
 
 // The raw X words and inv_awq pairs a lane needs for the four k16 steps of
@@ -154,15 +169,25 @@ constexpr int SMEM_BYTES = BAR_OFF + 2 * RING * 8 + 16;
 static_assert(S_WARPS * 4 * 2 * 32 * 4 * 4 <= BAR_OFF, "the partial sums fit the drained ring");
 
 // MERGED: up to 4 rows, the hi and lo parts of X^ in one MMA (NT = 1).
-template <int NT, bool MERGED>
-__global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
+template <int NT, bool MERGED, int C>
+__global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(const __grid_constant__ AwqGroup<C> grp) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + BAR_OFF);
   uint64_t *empty = full + RING;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + RING);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, t = lane & 3;
-  const int quad = blockIdx.x;
+  int pi = 0;                                     // this CTA's problem
+  if constexpr (C > 1) {
+    int lo = 0, hi = grp.count - 1;
+    while (lo < hi) {                             // the first problem whose quads end past blockIdx.x
+      const int mid = (lo + hi) >> 1;
+      if (static_cast<int>(blockIdx.x) < grp.quad_end[mid]) hi = mid; else lo = mid + 1;
+    }
+    pi = lo;
+  }
+  Params p = grp.p[pi];
+  const int quad = static_cast<int>(blockIdx.x) - (pi > 0 ? grp.quad_end[pi - 1] : 0);
   const int nchunks = (p.G + CHUNK_G - 1) / CHUNK_G;
   {  // this CTA's block of 8 NT rows
     const int r0 = static_cast<int>(blockIdx.y) * 8 * NT;
@@ -355,15 +380,53 @@ __global__ void __launch_bounds__(S_THREADS, 2) awq_gemv_kernel(Params p) {
   }
 }
 
-template <int NT, bool MERGED>
-int launch(const Params &p, cudaStream_t stream) {
-  const int rc = smem_optin_once<awq_gemv_kernel<NT, MERGED>>(SMEM_BYTES, "awq_linear_w4a16");
+template <int NT, bool MERGED, int C>
+int launch(const AwqGroup<C> &g, int total_quads, int M, cudaStream_t stream, const char *fn) {
+  const int rc = smem_optin_once<awq_gemv_kernel<NT, MERGED, C>>(SMEM_BYTES, fn);
   if (rc != SVDQ_OK) return rc;
-  DependentLaunch dl(dim3(p.N / 64, (p.M + 8 * NT - 1) / (8 * NT)), dim3(S_THREADS), SMEM_BYTES, stream);
-  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT, MERGED>, p);
+  DependentLaunch dl(dim3(total_quads, (M + 8 * NT - 1) / (8 * NT)), dim3(S_THREADS), SMEM_BYTES, stream);
+  cudaError_t e = cudaLaunchKernelEx(&dl.cfg, awq_gemv_kernel<NT, MERGED, C>, g);
   if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string("awq_linear_w4a16 launch: ") + cudaGetErrorString(e));
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, std::string(fn) + " launch: " + cudaGetErrorString(e));
   return ok();
+}
+
+// up to 4 rows: hi and lo parts in one MMA; up to 8: one block of rows; more: blocks of 16
+// rows, one pass over the weights each
+template <int C>
+int launch_rows(const AwqGroup<C> &g, int total_quads, int M, cudaStream_t s, const char *fn) {
+  if (M <= 4) return launch<1, true, C>(g, total_quads, M, s, fn);
+  return M > 8 ? launch<2, false, C>(g, total_quads, M, s, fn) : launch<1, false, C>(g, total_quads, M, s, fn);
+}
+
+// Checks one problem and fills its parameter block (all but the status word).
+int make_problem(const char *fn, const void *X, int M, int K, int ldx, const float *inv_awq, const uint32_t *qweight,
+                 const void *scales, const void *zeros, const void *bias, int N, void *Y, int ldy, Params *p) {
+  const std::string name(fn);
+  if (!X || !qweight || !scales || !zeros || !Y) return fail(SVDQ_ERR_INVALID_ARG, name + ": null pointer");
+  if (M < 1 || M > 65535 * 16 || K < 64 || K % 64 || N < 64 || N % 64 || ldx < K || ldx % 8 || ldy < N ||
+      ldy % 8)
+    return fail(SVDQ_ERR_SHAPE, name + ": need 1 <= M <= 1048560, K % 64 == 0, N % 64 == 0, ldx >= K, "
+                                       "ldy >= N, ldx/ldy % 8 == 0");
+  if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+      (inv_awq && !aligned16(inv_awq)) || !aligned16(Y))
+    return fail(SVDQ_ERR_ALIGNMENT, name + ": pointers must be 16-byte aligned");
+  *p = Params{};
+  p->M = M;
+  p->K = K;
+  p->N = N;
+  p->ldx = ldx;
+  p->ldy = ldy;
+  p->G = K / 64;
+  p->X = static_cast<const uint16_t *>(X);
+  p->inv = inv_awq;
+  p->qw = reinterpret_cast<const uint4 *>(qweight);
+  p->scales = static_cast<const uint16_t *>(scales);
+  p->zeros = static_cast<const uint16_t *>(zeros);
+  p->bias = static_cast<const uint16_t *>(bias);
+  p->Y = static_cast<uint16_t *>(Y);
+  p->limit_ns = kWaitLimitNs;
+  return SVDQ_OK;
 }
 
 }  // namespace
@@ -374,38 +437,42 @@ using namespace svdq;
 extern "C" int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq, const uint32_t *qweight,
                                 const void *scales, const void *zeros, int group, const void *bias, int N, void *Y,
                                 int ldy, svdq_stream_t stream) {
+  const char *fn = "awq_linear_w4a16";
   if (!X || !qweight || !scales || !zeros || !Y) return fail(SVDQ_ERR_INVALID_ARG, "awq_linear_w4a16: null pointer");
   if (group != 64) return fail(SVDQ_ERR_SHAPE, "awq_linear_w4a16: group must be 64");
-  if (M < 1 || M > 65535 * 16 || K < 64 || K % 64 || N < 64 || N % 64 || ldx < K || ldx % 8 || ldy < N ||
-      ldy % 8)
-    return fail(SVDQ_ERR_SHAPE, "awq_linear_w4a16: need 1 <= M <= 1048560, K % 64 == 0, N % 64 == 0, ldx >= K, "
-                                "ldy >= N, ldx/ldy % 8 == 0");
-  if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
-      (inv_awq && !aligned16(inv_awq)) || !aligned16(Y))
-    return fail(SVDQ_ERR_ALIGNMENT, "awq_linear_w4a16: pointers must be 16-byte aligned");
+  AwqGroup<1> g;
+  // shapes and alignment first (no device needed), then the device state
+  int rc = make_problem(fn, X, M, K, ldx, inv_awq, qweight, scales, zeros, bias, N, Y, ldy, &g.p[0]);
+  if (rc != SVDQ_OK) return rc;
   DeviceState *st = current_device_state();
   if (!st) return SVDQ_ERR_NOT_INITIALIZED;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int G = K / 64;
+  g.p[0].status = st->status_word;
+  g.quad_end[0] = N / 64;
+  g.count = 1;
+  return launch_rows<1>(g, N / 64, M, reinterpret_cast<cudaStream_t>(stream), fn);
+}
 
-  Params p;
-  p.M = M;
-  p.K = K;
-  p.N = N;
-  p.ldx = ldx;
-  p.ldy = ldy;
-  p.G = G;
-  p.X = static_cast<const uint16_t *>(X);
-  p.inv = inv_awq;
-  p.qw = reinterpret_cast<const uint4 *>(qweight);
-  p.scales = static_cast<const uint16_t *>(scales);
-  p.zeros = static_cast<const uint16_t *>(zeros);
-  p.bias = static_cast<const uint16_t *>(bias);
-  p.Y = static_cast<uint16_t *>(Y);
-  p.status = st->status_word;
-  p.limit_ns = kWaitLimitNs;
-  // up to 4 rows: hi and lo parts in one MMA; up to 8: one block of rows; more: blocks of 16
-  // rows, one pass over the weights each
-  if (M <= 4) return launch<1, true>(p, s);
-  return M > 8 ? launch<2, false>(p, s) : launch<1, false>(p, s);
+extern "C" int awq_linear_w4a16_grouped(const awq_problem_t *problems, int count, int M, int K, int group,
+                                        svdq_stream_t stream) {
+  const char *fn = "awq_linear_w4a16_grouped";
+  if (!problems || count < 1 || count > kAwqMaxGroup)
+    return fail(SVDQ_ERR_INVALID_ARG, std::string(fn) + ": need 1 <= count <= " + std::to_string(kAwqMaxGroup));
+  if (group != 64) return fail(SVDQ_ERR_SHAPE, std::string(fn) + ": group must be 64");
+  static thread_local AwqGroup<kAwqMaxGroup> g;   // ~13 KB: kept off the stack
+  int total = 0;
+  for (int i = 0; i < count; ++i) {
+    const awq_problem_t &q = problems[i];
+    const int rc = make_problem(fn, q.X, M, K, q.ldx, q.inv_awq, q.qweight, q.scales, q.zeros, q.bias, q.N, q.Y,
+                                q.ldy, &g.p[i]);
+    if (rc != SVDQ_OK) return rc;
+    if (total > (1 << 30) - q.N / 64) return fail(SVDQ_ERR_SHAPE, std::string(fn) + ": too many columns in one launch");
+    total += q.N / 64;
+    g.quad_end[i] = total;
+  }
+  DeviceState *st = current_device_state();
+  if (!st) return SVDQ_ERR_NOT_INITIALIZED;
+  for (int i = 0; i < count; ++i) g.p[i].status = st->status_word;
+  for (int i = count; i < kAwqMaxGroup; ++i) g.quad_end[i] = total;
+  g.count = count;
+  return launch_rows<kAwqMaxGroup>(g, total, M, reinterpret_cast<cudaStream_t>(stream), fn);
 }

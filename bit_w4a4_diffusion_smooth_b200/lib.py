@@ -50,6 +50,15 @@ class W4A4Problem(ctypes.Structure):
                 ("gelu_col_begin", ctypes.c_int), ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int)]
 
 
+class AwqProblem(ctypes.Structure):
+    """awq_problem of include/svdq.h."""
+    _fields_ = [("X", ctypes.c_void_p), ("ldx", ctypes.c_int), ("inv_awq", ctypes.c_void_p),
+                ("qweight", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("N", ctypes.c_int), ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int)]
+
+
+AWQ_MAX_GROUP = 128
+
 _SIGNATURES = {
     "svdq_version": (_I, []),
     "svdq_last_error_string": (ctypes.c_char_p, []),
@@ -80,6 +89,7 @@ _SIGNATURES = {
     "awq_packed_sizes": (_I, [_I, _I, _I, _SZ, _SZ, _SZ, _SZ]),
     "awq_pack_weights": (_I, [_P, _I, _I, _P, _I, _P, _P, _P, _P]),
     "awq_linear_w4a16": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P]),
+    "awq_linear_w4a16_grouped": (_I, [ctypes.POINTER(AwqProblem), _I, _I, _I, _I, _P]),
     "awq_gemm_workspace_size": (_I, [_I, _I, _I, _SZ]),
     "awq_linear_w4a16_gemm": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _I, _P, _I, _P, _I, _P, _P]),
     "awq_expand_weights": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
@@ -578,6 +588,31 @@ def awq_linear_w4a16(X, inv_awq, qweight, scales, zeros, bias, N, Y, group=64, M
         _dptr(bias, "bias", allow_none=True), N, _dptr(Y, "Y", torch.bfloat16), Y.stride(0),
         _stream(stream)))
 
+
+
+def awq_linear_w4a16_grouped(problems, M, K, group=64, stream=None):
+    """One launch of the W4A16 GEMV over several projections of the same M and K (dicts of
+    awq_linear_w4a16's arguments X, inv_awq, qweight, scales, zeros, bias, N, Y); outputs are
+    bit-identical to separate calls."""
+    import torch
+    if not 1 <= len(problems) <= AWQ_MAX_GROUP:
+        raise ValueError(f"a grouped AWQ launch takes 1..{AWQ_MAX_GROUP} problems, got {len(problems)}")
+    arr = (AwqProblem * len(problems))()
+    for i, d in enumerate(problems):
+        X, Y, N = d["X"], d["Y"], d["N"]
+        _need_2d(X, M, K, "X")
+        _need_2d(Y, M, N, "Y")
+        _need_bytes(d["qweight"], N * K // 2, "qweight")
+        _need_bytes(d["scales"], 2 * N * (K // group), "scales")
+        _need_bytes(d["zeros"], 2 * N * (K // group), "zeros")
+        _need_bytes(d.get("inv_awq"), 4 * K, "inv_awq")
+        _need_bytes(d.get("bias"), 2 * N, "bias")
+        arr[i] = AwqProblem(_dptr(X, "X", torch.bfloat16), X.stride(0), _dptr(d.get("inv_awq"), "inv_awq", allow_none=True),
+                            _dptr(d["qweight"], "qweight"), _dptr(d["scales"], "scales"), _dptr(d["zeros"], "zeros"),
+                            _dptr(d.get("bias"), "bias", allow_none=True), N, _dptr(Y, "Y", torch.bfloat16),
+                            Y.stride(0))
+    _check("awq_linear_w4a16_grouped", load().awq_linear_w4a16_grouped(arr, len(problems), M, K, group,
+                                                                       _stream(stream)))
 
 def awq_gemm_workspace_size(M, K, N):
     n = ctypes.c_size_t()

@@ -404,6 +404,34 @@ int awq_linear_w4a16(const void *X, int M, int K, int ldx, const float *inv_awq,
                      const void *bias, int N, void *Y, int ldy, svdq_stream_t stream);
 
 /*
+ * Several AWQ projections of the same input shape in one launch (the
+ * modulation / adaLN layers of a DiT step all read the same conditioning
+ * vector).  Each problem is computed exactly as awq_linear_w4a16 computes it
+ * (the same kernel per 64-column quad; outputs bit-identical to separate
+ * calls); the problems' quads form one grid, problem after problem.
+ * `problems` is a HOST array of `count` (1..SVDQ_AWQ_MAX_GROUP) descriptors,
+ * read during the call; M, K and group are shared; every descriptor obeys the
+ * rules of awq_linear_w4a16 (its own X, ldx, inv_awq, weights, bias, N, Y,
+ * ldy).  Errors as awq_linear_w4a16, checked for every problem before
+ * anything is launched; SVDQ_ERR_INVALID_ARG for count outside the range.
+ */
+#define SVDQ_AWQ_MAX_GROUP 128
+typedef struct awq_problem {
+  const void *X;              /* [M][ldx] bf16 */
+  int ldx;
+  const float *inv_awq;       /* [K] f32 or NULL */
+  const uint32_t *qweight;    /* N*K/2 bytes, layout of awq_pack_weights */
+  const void *scales;         /* bf16 */
+  const void *zeros;          /* bf16 */
+  const void *bias;           /* [N] bf16 or NULL */
+  int N;
+  void *Y;                    /* [M][ldy] bf16 */
+  int ldy;
+} awq_problem_t;
+int awq_linear_w4a16_grouped(const awq_problem_t *problems, int count, int M, int K, int group,
+                             svdq_stream_t stream);
+
+/*
  * AWQ W4A16 for many rows (the GEMM path; awq_linear_w4a16 reads the packed
  * weights once per block of 16 rows, which suits the few rows of a
  * modulation layer).  Same result definition as awq_linear_w4a16,

@@ -153,3 +153,16 @@ def test_empty_inputs_are_rejected_as_shapes():
         with pytest.raises(lib.SvdqError) as e:
             call()
         assert e.value.status == lib.ERR_SHAPE
+
+
+def test_grouped_awq_rejects_bad_groups_before_touching_a_gpu():
+    so = lib.load()
+    p = ctypes.c_void_p(16)  # never dereferenced
+    arr = (lib.AwqProblem * 2)()
+    arr[0] = lib.AwqProblem(p, 256, None, p, p, p, None, 128, p, 128)
+    arr[1] = lib.AwqProblem(p, 256, None, p, p, p, None, 96, p, 96)      # N % 64
+    assert so.awq_linear_w4a16_grouped(arr, 0, 2, 256, 64, None) == lib.ERR_INVALID_ARG
+    assert so.awq_linear_w4a16_grouped(arr, lib.AWQ_MAX_GROUP + 1, 2, 256, 64, None) == lib.ERR_INVALID_ARG
+    assert so.awq_linear_w4a16_grouped(arr, 2, 2, 256, 64, None) == lib.ERR_SHAPE
+    assert so.awq_linear_w4a16_grouped(arr, 1, 2, 256, 32, None) == lib.ERR_SHAPE   # group 32
+    assert so.awq_linear_w4a16_grouped(arr, 1, 0, 256, 64, None) == lib.ERR_SHAPE   # M = 0

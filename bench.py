@@ -506,6 +506,61 @@ def int4_variant(W, device, pk, reps=20):
                     "16-bit tensor peak"}
 
 
+def host_path_point(device, m=512, k=3072, n=9216, reps=100):
+    """Host cost of a layer call: a 512-row text-stream projection (m x k -> n, rank 32) through
+    SVDQLinear's repeated calls (the marshalled arguments of its first call with these buffers),
+    launched from the host back to back, against the same calls replayed from a CUDA graph.
+    Random-valid packed bytes (speed only)."""
+    import time
+
+    import torch
+
+    from bit_w4a4_diffusion_smooth_b200 import lib
+    from bit_w4a4_diffusion_smooth_b200.layer import SVDQLinear
+    rng = np.random.default_rng(5)
+    ws = lib.svdq_weight_sizes(k, n, RANK)
+    packed = dict(inv_lambda=np.ones(k, np.float32), l1t=np.zeros((RANK, k), np.uint16),
+                  l2t=rng.integers(0, 256, ws["l2t"], dtype=np.uint8) & 0x3F,
+                  w_bundle=rng.integers(0, 256, ws["w_bundle"], dtype=np.uint8) & 0x77, s_w=1e-3, s_a=1.0)
+    layer = SVDQLinear(packed, k, n, RANK, device=device)
+    X = (torch.randn(m, k, device=device) * 0.5).to(torch.bfloat16)
+    Y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+    for _ in range(5):
+        layer(X, Y)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        layer(X, Y)
+    e1.record()
+    torch.cuda.synchronize()
+    launched = e0.elapsed_time(e1) / reps * 1e3
+    t = time.perf_counter()
+    for _ in range(reps):
+        layer(X, Y)
+    host = (time.perf_counter() - t) / reps * 1e6
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(10):
+            layer(X, Y)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps // 10):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    replayed = e0.elapsed_time(e1) / reps * 1e3
+    del graph
+    return {"layer": f"SVDQLinear {m}x{k}->{n} r{RANK}, repeated calls on the same buffers",
+            "host_launched_us": round(launched, 2), "graph_us": round(replayed, 2),
+            "host_us_per_call": round(host, 2),
+            "what": "GPU time per call (K1 + K2) of 100 calls launched from the host back to back, against the "
+                    "same calls replayed from a CUDA graph; host_us_per_call is the host's own time per call"}
+
+
 def copy_floor(device, nbytes, reps=24):
     """A library copy of `nbytes` (torch, device to device) with L2 flushed before it, timed like the
     kernels: the HBM rate a plain stream of this size reaches on this GPU, as (GB/s counting read +
@@ -677,6 +732,7 @@ def run_ours(args):
     awq_batch = awq_many_rows(W, device)
     pk_local, _ = peaks()
     int4_pass = int4_variant(W, device, pk_local)
+    host_path = host_path_point(device)
     fp4_lib = fp4_library_point(device, *LAYERS["fc1"][:3]) if not args.no_library_points else "skipped"
 
     # ---- max over ranks
@@ -764,6 +820,7 @@ def run_ours(args):
         "kernels": ktab,
         "awq_many_rows": awq_batch,
         "int4_w4a4": int4_pass,
+        "host_path": host_path,
         "reference_points": {
             "hbm_copy_same_bytes": {"GB/s": round(floor_gbs, 1), "us": round(floor_us, 2),
                                     "what": f"torch copy of {TOKENS}x{HIDDEN} bf16, timed like the kernels "

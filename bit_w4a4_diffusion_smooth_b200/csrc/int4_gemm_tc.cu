@@ -1,5 +1,6 @@
 // INT4 W4A4 GEMM on the 5th-generation tensor cores (tcgen05), for N a
-// multiple of 256.
+// multiple of 128 (256-column tiles; a last tile of 128 columns when N % 256
+// is 128).
 //
 // The layer is the INT4 variant of the pages' W4A4 layer (donmalab.com,
 // "Diffusers × Nunchaku 4-bit", section "實務上的影響與硬體要求"; this library
@@ -94,6 +95,9 @@ static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 // N >> 3 at bit 17, M >> 4 at bit 24 (M 256: the pair), both operands K-major
 constexpr uint32_t IDESC_F16 = (1u << 4) | ((256 >> 3) << 17) | ((256 >> 4) << 24);
 constexpr uint32_t IDESC_BF16 = IDESC_F16 | (1u << 7) | (1u << 10);
+// a last tile of 128 columns (N % 256 == 128): N 128, each CTA serving 64 weight rows
+constexpr uint32_t IDESC_F16_HALF = (1u << 4) | ((128 >> 3) << 17) | ((256 >> 4) << 24);
+constexpr uint32_t IDESC_BF16_HALF = IDESC_F16_HALF | (1u << 7) | (1u << 10);
 
 struct TcParams {
   const uint16_t *a_scales, *w_scales, *bias;
@@ -132,11 +136,20 @@ __device__ __forceinline__ uint4 dequant8(uint32_t x, __half2 s2) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Pair tile t: its 256-row block of activations (m fastest) and 256-column block of weights.
+// Pair tile t: its 256-row block of activations (m fastest) and 256-column block of weights; a
+// last block of 128 columns (N % 256 == 128) is a half tile, whose CTAs serve 64 weight rows each.
 struct PairTile {
   int m2, nt;
+  bool half;
 };
-__device__ __forceinline__ PairTile pair_tile(int t, int tiles_m) { return PairTile{t % tiles_m, t / tiles_m}; }
+__device__ __forceinline__ PairTile pair_tile(int t, int tiles_m, int N) {
+  const int nt = t / tiles_m;
+  return PairTile{t % tiles_m, nt, (nt + 1) * BN > N};
+}
+// this CTA's first weight row of the tile
+__device__ __forceinline__ int weight_row0(const PairTile &pt, uint32_t h) {
+  return pt.nt * BN + (pt.half ? 64 : 128) * static_cast<int>(h);
+}
 
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -160,7 +173,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   const uint32_t h = dev::cluster_ctarank();
   const int G = p.K / 64;
   const int tiles_m = (p.ld_sa + 255) / 256;
-  const int total = tiles_m * (p.N / BN);
+  const int total = tiles_m * ((p.N + BN - 1) / BN);
   const int pair = static_cast<int>(dev::cluster_id_x()), num_pairs = static_cast<int>(dev::num_clusters_x());
   const int t_begin = static_cast<int>((static_cast<long long>(pair) * total) / num_pairs);
   const int t_end = static_cast<int>((static_cast<long long>(pair + 1) * total) / num_pairs);
@@ -210,9 +223,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int gi = 0;
       bool ok = true;
       for (int t = t_begin; t < t_end && ok; ++t) {
-        const PairTile pt = pair_tile(t, tiles_m);
-        const int m0 = (2 * pt.m2 + static_cast<int>(h)) * 128, nb0 = pt.nt * BN + 128 * static_cast<int>(h);
+        const PairTile pt = pair_tile(t, tiles_m, p.N);
+        const int m0 = (2 * pt.m2 + static_cast<int>(h)) * 128, nb0 = weight_row0(pt, h);
         const bool a_live = m0 < p.ld_sa;    // the odd CTA of a last, half pair has no rows
+        // weight rows past N read as zeros (the tensor map's bounds); their scales are not copied
+        const int sb_bytes = pt.half ? SB / 2 : SB;
         for (int g = 0; g < G; ++g, ++gi) {
           const int s = gi % LSTAGES;
           if (!dev::mbar_wait(&load_empty[s], ((gi / LSTAGES) & 1) ^ 1, p.limit_ns, abort_flag)) {
@@ -222,13 +237,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           }
           uint8_t *st = smem + LOAD_OFF + s * LSTAGE;
           // a CTA without rows loads no activation codes or scales: its converters use scale 0
-          dev::mbar_arrive_expect_tx(&load_full[s], (a_live ? A4 + SA : 0) + B4 + SB);
+          dev::mbar_arrive_expect_tx(&load_full[s], (a_live ? A4 + SA : 0) + B4 + sb_bytes);
           if (a_live) {
             dev::tma_load_2d(st, &maps.a, &load_full[s], g * 32, m0);
             dev::bulk_load(st + A4 + B4, p.a_scales + static_cast<size_t>(g) * p.ld_sa + m0, SA, &load_full[s]);
           }
           dev::tma_load_2d(st + A4, &maps.b, &load_full[s], g * 32, nb0);
-          dev::bulk_load(st + A4 + B4 + SA, p.w_scales + static_cast<size_t>(g) * p.N + nb0, SB, &load_full[s]);
+          dev::bulk_load(st + A4 + B4 + SA, p.w_scales + static_cast<size_t>(g) * p.N + nb0, sb_bytes, &load_full[s]);
         }
       }
       // every copy issued lands before the block leaves
@@ -240,8 +255,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (lane == 0 && p.rank > 0) {
       int lt = 0;
       for (int t = t_begin; t < t_end; ++t, ++lt) {
-        const PairTile pt = pair_tile(t, tiles_m);
-        const int m0 = (2 * pt.m2 + static_cast<int>(h)) * 128, nb0 = pt.nt * BN + 128 * static_cast<int>(h);
+        const PairTile pt = pair_tile(t, tiles_m, p.N);
+        const int m0 = (2 * pt.m2 + static_cast<int>(h)) * 128, nb0 = weight_row0(pt, h);
         const bool a_live = m0 < p.ld_sa;
         if (!dev::mbar_wait(lr_empty, (lt & 1) ^ 1, p.limit_ns, abort_flag)) {
           fail_wait();
@@ -265,6 +280,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int gi = 0, lt = 0;
       for (int t = t_begin; t < t_end && ok; ++t, ++lt) {
         const int b = lt & 1;
+        const bool half = pair_tile(t, tiles_m, p.N).half;
+        const uint32_t idesc_bf16 = half ? IDESC_BF16_HALF : IDESC_BF16, idesc_f16 = half ? IDESC_F16_HALF : IDESC_F16;
         if (!dev::mbar_wait_cluster(&tmem_empty[b], ((lt >> 1) & 1) ^ 1, p.limit_ns, abort_flag)) {
           fail_wait();
           break;
@@ -280,7 +297,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           dev::tc_fence_after();
           const uint32_t ua = dev::smem_u32(smem + LR_OFF), lb = ua + HALF16;
           for (int j = 0; j < p.rank / 16; ++j) {   // K = 16 bf16 = 32 bytes per MMA
-            dev::umma_bf16_pair(acc, dev::desc_sw128(ua + 32 * j), dev::desc_sw128(lb + 32 * j), IDESC_BF16,
+            dev::umma_bf16_pair(acc, dev::desc_sw128(ua + 32 * j), dev::desc_sw128(lb + 32 * j), idesc_bf16,
                                 accumulate);
             accumulate = 1;
           }
@@ -297,7 +314,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
           dev::tc_fence_after();
           const uint32_t sa = dev::smem_u32(smem + CONV_OFF + c * CSTAGE), sb = sa + HALF16;
           for (int j = 0; j < 4; ++j) {               // K = 16 fp16 = 32 bytes per MMA
-            dev::umma_bf16_pair(acc, dev::desc_sw128(sa + 32 * j), dev::desc_sw128(sb + 32 * j), IDESC_F16,
+            dev::umma_bf16_pair(acc, dev::desc_sw128(sa + 32 * j), dev::desc_sw128(sb + 32 * j), idesc_f16,
                                 accumulate);
             accumulate = 1;
           }
@@ -318,7 +335,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     int gi = 0;
     bool ok = true;
     for (int t = t_begin; t < t_end && ok; ++t) {
-      const PairTile pt = pair_tile(t, tiles_m);
+      const PairTile pt = pair_tile(t, tiles_m, p.N);
       const bool a_live = (2 * pt.m2 + static_cast<int>(h)) * 128 < p.ld_sa;
       for (int g = 0; g < G; ++g, ++gi) {
         if (gi % TEAMS != team) continue;            // the other teams' groups
@@ -362,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     int lt = 0;
     for (int t = t_begin; t < t_end; ++t, ++lt) {
-      const PairTile pt = pair_tile(t, tiles_m);
+      const PairTile pt = pair_tile(t, tiles_m, p.N);
       const int b = lt & 1;
       if (!dev::mbar_wait_warp(&tmem_full[b], (lt >> 1) & 1, p.limit_ns, abort_flag)) {
         fail_wait();
@@ -371,13 +388,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       dev::tc_fence_after();
       const int m0 = (2 * pt.m2 + static_cast<int>(h)) * 128, n0 = pt.nt * BN;
       const int row = 32 * q + lane, grow = m0 + row;
+      const int nchunk = pt.half ? BN / 64 : BN / 32;   // 32-column chunks of the tile
 #pragma unroll 1
-      for (int cb = 0; cb < BN / 32; ++cb) {
+      for (int cb = 0; cb < nchunk; ++cb) {
         uint32_t v[32];
         dev::tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(BN * b + 32 * cb),
                                 v);
         dev::tmem_wait_ld();
-        if (cb == BN / 32 - 1) {                       // the accumulator is read: hand it back to the MMA thread
+        if (cb == nchunk - 1) {                        // the accumulator is read: hand it back to the MMA thread
           dev::tc_fence_before();
           __syncwarp();
           if (lane == 0) dev::mbar_arrive_cluster(dev::mapa(dev::smem_u32(&tmem_empty[b]), 0));
@@ -459,7 +477,7 @@ int launch(const TcMaps &maps, const TcParams &p, cudaStream_t stream) {
   int resident = 0;
   const int rc = prepare_device<EPI>(&resident);
   if (rc != SVDQ_OK) return rc;
-  const int tiles = (p.ld_sa + 255) / 256 * (p.N / BN);
+  const int tiles = (p.ld_sa + 255) / 256 * ((p.N + BN - 1) / BN);
   const int pairs = tiles < resident ? tiles : resident;
   DependentLaunch dl(dim3(2 * pairs), dim3(THREADS), SMEM_BYTES, stream);
   cudaError_t e = cudaLaunchKernelEx(&dl.cfg, int4_gemm_tc_kernel<EPI>, maps, p);

@@ -166,7 +166,7 @@ int encode_tmap_2d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base
 int encode_tmap_3d(CUtensorMap *out, CUtensorMapDataType dtype, const void *base, const uint64_t (&dims)[3],
                    const uint64_t (&strides)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
 
-// The INT4 W4A4 GEMM on tcgen05 (int4_gemm_tc.cu), for N % 256 == 0; svdq_linear_int4 checks the
+// The INT4 W4A4 GEMM on tcgen05 (int4_gemm_tc.cu), for N % 128 == 0; svdq_linear_int4 checks the
 // arguments and dispatches here.
 int launch_int4_tc(const uint8_t *a_codes, const void *a_scales, const void *U, const uint8_t *w_codes,
                    const void *w_scales, const void *l2t, const void *bias, int M, int N, int K, int rank, int epilogue,

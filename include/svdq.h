@@ -521,13 +521,12 @@ int svdq_quantize_act_int4(const void *X, int M, int K, int ldx, const float *in
  * The INT4 GEMM with the low-rank up-projection fused in:
  *   Y = bf16( epilogue( sum_g (s_a[m,g] s_w[n,g]) sum_{k in g} q_a q_w
  *                       + U . L2T^T + bias ) )
- * B200 has no 4-bit integer MMA.  For N % 256 == 0 the codes become exact
- * fp16 operands q * s (4 + 8 significant bits fit fp16's 11; exact while
- * |q s| lies in fp16's normal range, i.e. activation and weight magnitudes
- * below ~57,000 and group scales above 2^-14) multiplied on the tensor cores
- * (tcgen05 kind::f16, fp32 accumulation, no per-group rescale) by
- * persistent SM pairs over 256 x 256 tiles; other widths run 8-bit warp MMAs
- * (exact int32 per group) with a per-group fp32 rescale.
+ * B200 has no 4-bit integer MMA.  The codes become exact fp16 operands q * s
+ * (4 + 8 significant bits fit fp16's 11; exact while |q s| lies in fp16's
+ * normal range, i.e. activation and weight magnitudes below ~57,000 and group
+ * scales above 2^-14) multiplied on the tensor cores (tcgen05 kind::f16, fp32
+ * accumulation, no per-group rescale) by persistent SM pairs over 256 x 256
+ * tiles, with a last tile of 128 columns when N % 256 == 128.
  * Args: a_codes, a_scales, U from svdq_quantize_act_int4; w_codes,
  * w_scales from svdq_quantize_int4_host, l2t from svdq_pack_weights
  * (uploaded); bias [N] bf16 or NULL; Y [M][ldy] bf16.

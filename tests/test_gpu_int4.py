@@ -7,7 +7,7 @@ against the oracle (oracle/int4.py), through the C ABI.
   * GEMM on the oracle's own operands (uploaded in the test-side layouts of
     tests/layouts.py): Y within the parity bar (excess error over the row RMS
     <= 1e-2, as for the NVFP4 GEMM); ragged M, K up to 3072, GELU from inside
-    the output, no bias, rank 0.
+    the output, no bias, rank 0, widths with a last block of 128 columns.
   * The chain K1 -> K2 at full size on the MLP fc1 (4608 x 3072 -> 12288, erf
     GELU), the single block's fused QKV + MLP-in (-> 21504, GELU from column
     9216) and its output projection (K = 15360), with the library's host pack:
@@ -115,9 +115,10 @@ def test_int4_gemm_matches_oracle(m, k, n, rank, epilogue, begin, with_bias):
 
 
 def test_int4_gemm_many_tiles_sampled():
-    """Several 256 x 256 tiles per SM pair (both accumulators in turn), a last half pair, rank 16, tanh GELU
-    from column 1000: sampled rows against the oracle on the same operands."""
-    m, k, n, rank = 4480, 1024, 5120, 16
+    """Several 256 x 256 tiles per SM pair (both accumulators in turn), a last half pair, a last column
+    block of 128 (N % 256 == 128), rank 16, tanh GELU from column 1000: sampled rows against the oracle
+    on the same operands."""
+    m, k, n, rank = 4480, 1024, 5248, 16
     xb, x, wb, amax = _data(m, k, n, 55)
     p = int4.pack(formats.bf16_bits_to_float(wb), amax, rank)
     qa, sa, u = int4.quantize_act(x, p["inv_lambda"], p["l1"])

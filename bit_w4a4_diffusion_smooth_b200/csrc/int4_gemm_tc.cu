@@ -488,7 +488,7 @@ int launch(const TcMaps &maps, const TcParams &p, cudaStream_t stream) {
 
 }  // namespace
 
-// The tcgen05 INT4 GEMM (N % 256 == 0); arguments already checked by svdq_linear_int4.
+// The tcgen05 INT4 GEMM (N % 128 == 0); arguments already checked by svdq_linear_int4.
 int launch_int4_tc(const uint8_t *a_codes, const void *a_scales, const void *U, const uint8_t *w_codes,
                    const void *w_scales, const void *l2t, const void *bias, int M, int N, int K, int rank, int epilogue,
                    int gelu_col_begin, void *Y, int ldy, unsigned int *status, cudaStream_t stream) {
